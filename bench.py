@@ -1,0 +1,395 @@
+"""Benchmark of the GDN mixer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extra]
+
+Headline (``value``): prefill token-heads/s (B x T x H per second) of gdn_chunk_fwd on the
+prefill workload B=2, H=16, T=4096, dk=dv=128, bf16 q/k/v, fp32 g/beta/state, S0 = 0,
+chunk 64 -- one launch of the tensor-core chunked kernel per step, inputs resident in HBM,
+three input sets rotated so that every step reads from DRAM (3 x 137 MB > 126 MB L2).
+Secondary workloads measured in the same run (``other_workloads``): decode (256 x 32
+heads, 100 in-place steps), long prefill (T=32768, H=32, S0 != 0), full mixer (4 packed
+sequences, prep -> chunk -> out gate).
+
+N > 1: one process per GPU (torchrun), every rank runs its own batch (independent
+sequences, no data-path collective: weak scaling); time = max over ranks.
+``--impl reference``: the fp64 CPU oracle on the host cores, same metric and workload,
+each step a bounded sample; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s (B×T×H, dk=dv=128) + decode state-updates/s; % roofline"
+UNIT = "token-heads/s"
+
+
+def env_rank():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d.get("bf16_tflops"), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") if os.path.isdir(
+            os.path.join(ROOT, "gpurun_out")) else f"/tmp/gdn_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        sm = [float(r[1]) for r in rows]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def prefill_bytes(N, H, nseq, dk=128, dv=128, in_bytes=2, y_bytes=2, S0=False, S_T=True):
+    """Algorithmic HBM bytes of one gdn_chunk_fwd launch: read q, k, v, g, beta (+S0),
+    write y (+S_T), each exactly once."""
+    b = N * H * ((2 * dk + dv) * in_bytes + 8 + dv * y_bytes)
+    state = nseq * H * dk * dv * 4
+    return b + (state if S0 else 0) + (state if S_T else 0)
+
+
+def timed(torch, fn, steps, warmup, stream):
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3  # seconds
+
+
+def max_over_ranks(torch, dist, x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(torch, dist, world):
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ----------------------------------------------------------------------------- CPU baseline
+
+def cpu_baseline(cfg_idx=1, target_s=12.0):
+    """The fp64 oracle (unmodified) on the host cores, on a bounded sample of the prefill
+    workload: the first `nh` heads of every sequence, nh sized so the run takes ~target_s."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from linear_attention_token_gdn_b200 import inputs
+
+    c = inputs.CONFIGS[cfg_idx]
+    x = inputs.make_prefill(cfg_idx, "cpu")
+    ncores = os.cpu_count() or 1
+    # calibrate: one (sequence, head) unit single-threaded on a 512-token slice
+    T = c["T"]
+    sl = slice(0, 512)
+    t0 = time.perf_counter()
+    oracle.recurrence(x["q"][sl, :1], x["k"][sl, :1], x["v"][sl, :1], x["g"][sl, :1], x["beta"][sl, :1], nthreads=1)
+    per_tok = (time.perf_counter() - t0) / 512
+    units_budget = max(1, int(target_s * ncores / (per_tok * T)))
+    nh = max(1, min(c["H"], units_budget // c["B"]))
+    hs = slice(0, nh)
+    t0 = time.perf_counter()
+    oracle.recurrence(x["q"][:, hs], x["k"][:, hs], x["v"][:, hs], x["g"][:, hs], x["beta"][:, hs], None,
+                      x["cu_seqlens"], nthreads=0)
+    dt = time.perf_counter() - t0
+    used = oracle.threads_used(0, c["B"] * nh)
+    work = c["B"] * T * nh
+    return {"value": work / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": f"prefill B={c['B']} T={T} heads 0..{nh - 1} of {c['H']} (dk=dv=128, fp64 C oracle, "
+                      f"{dt:.1f} s wall on {used} threads)"}
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    cb = None
+    times = []
+    work = 0
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(1, target_s=args.ref_step_s)
+        if i >= args.warmup:
+            times.append(1.0 / r["value"])
+            cb = r
+    value = cb["value"] if len(times) == 1 else len(times) / sum(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill_B2_H16_T4096_d128", "global_batch": 2, "seq_len": 4096, "heads": 16,
+                       "dk": 128, "dv": 128, "parallelism": "host threads"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                             "sample": cb["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from linear_attention_token_gdn_b200 import build as gbuild
+    from linear_attention_token_gdn_b200 import gdn, inputs
+
+    rank, world, local = env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if rank == 0:
+        gbuild.build()
+    if world > 1:
+        dist.barrier()
+    gdn.lib()
+    stream = torch.cuda.current_stream()
+    hbm_peak, tf_peak, peak_src = peaks()
+
+    # ---- headline: prefill workload, three rotating input sets --------------------------
+    c = inputs.CONFIGS[1]
+    sets = [inputs.make_prefill(1, "cuda", seed=inputs.SEED_BASE + 1 + 1000 * rank + s) for s in range(3)]
+    N, H = sets[0]["N"], sets[0]["H"]
+    nseq = sets[0]["num_seqs"]
+    outs = [(torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16),
+             torch.empty(nseq, H, 128, 128, device="cuda")) for _ in range(3)]
+    ws_bytes = gdn.workspace_size(N, nseq, H, 128, 128, 64)
+    ws = torch.empty(max(ws_bytes, 16), device="cuda", dtype=torch.uint8)
+
+    def step(i):
+        x = sets[i % 3]
+        y, S_T = outs[i % 3]
+        gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64, y=y, S_T=S_T,
+                      workspace=ws)
+
+    barrier(torch, dist, world)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        dt = timed(torch, step, args.steps, args.warmup, stream)
+        barrier(torch, dist, world)
+        if dt < 0.5:  # keep the GPU busy long enough for the clock sampler to see it
+            soak = timed(torch, step, max(1, int(args.steps * 0.6 / max(dt, 1e-6))), 0, stream)
+    dt = max_over_ranks(torch, dist, dt, world)
+    gdn.check_device_error()
+    per_step = dt / args.steps
+    work = N * H  # token-heads per rank per step
+    value = work * world / per_step
+    alg_bytes = prefill_bytes(N, H, nseq)
+    achieved = alg_bytes / per_step / 1e9
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prefill_B2_H16_T4096_d128", "global_batch": 2 * world, "seq_len": 4096,
+                       "heads": 16, "dk": 128, "dv": 128, "chunk": 64, "state": "fp32, S0=0",
+                       "parallelism": f"dp{world}",
+                       "l2": "3 rotating input sets (3 x 137 MB > 126 MB L2)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None, "kernel": "chunk_fwd_tc_kernel",
+                         "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": alg_bytes},
+            "gpu_launches": args.steps, "clocks": clk.summary()}
+
+    # ---- end to end through the public API with pinned host buffers ----------------------
+    hx = {k: sets[0][k].cpu().pin_memory() for k in ("q", "k", "v", "g", "beta")}
+    dx = {k: torch.empty_like(sets[0][k]) for k in hx}
+    hy = torch.empty(N, H, 128, dtype=torch.bfloat16).pin_memory()
+    hS = torch.empty(nseq, H, 128, 128).pin_memory()
+    cu = sets[0]["cu_seqlens"]
+
+    def e2e_step(i):
+        for k in hx:
+            dx[k].copy_(hx[k], non_blocking=True)
+        y, S_T = gdn.chunk_fwd(dx["q"], dx["k"], dx["v"], dx["g"], dx["beta"], None, cu, chunk=64, y=outs[0][0],
+                               S_T=outs[0][1], workspace=ws)
+        hy.copy_(y, non_blocking=True)
+        hS.copy_(S_T, non_blocking=True)
+
+    barrier(torch, dist, world)
+    e2e_steps = max(3, min(args.steps, 20))
+    dte = timed(torch, e2e_step, e2e_steps, 2, stream)
+    dte = max_over_ranks(torch, dist, dte, world)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hy.numel() * 2 + hS.numel() * 4
+    line["e2e"] = {"value": work * world * e2e_steps / dte, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                   "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    if not args.no_extra:
+        line["other_workloads"] = extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak)
+    if rank == 0:
+        if args.impl_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(1, target_s=args.cpu_s)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    res = []
+
+    # decode: 256 x 32 heads, 100 in-place steps per "step"
+    c = inputs.CONFIGS[3]
+    state = inputs.make_decode_state(3, "cuda", seed=inputs.SEED_BASE + 3 + 1000 * rank)
+    steps_in = [inputs.make_decode_step(3, "cuda", step=s, seed=inputs.SEED_BASE + 3 + 1000 * rank)
+                for s in range(c["steps"])]
+    y = torch.empty(c["B"], c["H"], 128, device="cuda", dtype=torch.bfloat16)
+
+    def dec(i):
+        for x in steps_in:
+            gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, y=y)
+
+    barrier(torch, dist, world)
+    dt = max_over_ranks(torch, dist, timed(torch, dec, 3, 1, stream), world)
+    per_launch = dt / (3 * c["steps"])
+    upd = c["B"] * c["H"]
+    bytes_l = upd * (2 * 128 * 128 * 4 + 3 * 128 * 2 + 8 + 128 * 2)
+    res.append({"workload": c["name"], "value": upd * world / per_launch, "unit": "state-updates/s",
+                "us_per_step": per_launch * 1e6,
+                "roofline": {"bound": "hbm", "achieved": bytes_l / per_launch / 1e9, "peak": hbm_peak,
+                             "unit": "GB/s", "frac": bytes_l / per_launch / 1e9 / hbm_peak,
+                             "kernel": "decode_step_kernel", "alg_bytes_per_launch": bytes_l},
+                "gpu_launches": 3 * c["steps"]})
+    del state, steps_in
+
+    # long prefill: B=1, H=32, T=32768, S0 != 0
+    x = inputs.make_prefill(2, "cuda", seed=inputs.SEED_BASE + 2 + 1000 * rank)
+    N, H, nseq = x["N"], x["H"], x["num_seqs"]
+    yb = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)
+    ST = torch.empty(nseq, H, 128, 128, device="cuda")
+    ws = torch.empty(max(gdn.workspace_size(N, nseq, H, 128, 128, 64), 16), device="cuda", dtype=torch.uint8)
+
+    def lp(i):
+        gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64, y=yb, S_T=ST,
+                      workspace=ws)
+
+    barrier(torch, dist, world)
+    n_lp = 3
+    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 1, stream), world) / n_lp
+    bl = prefill_bytes(N, H, nseq, S0=True)
+    res.append({"workload": inputs.CONFIGS[2]["name"], "value": N * H * world / dt, "unit": UNIT,
+                "ms_per_step": dt * 1e3,
+                "roofline": {"bound": "hbm", "achieved": bl / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": bl / dt / 1e9 / hbm_peak, "kernel": "chunk_fwd_tc_kernel",
+                             "alg_bytes_per_launch": bl}, "gpu_launches": n_lp,
+                "l2": "1.1 GB working set > L2"})
+    del x, yb, ST
+
+    # full mixer: prep -> chunk -> out gate on 4 packed sequences
+    m = inputs.make_mixer(4, "cuda", seed=inputs.SEED_BASE + 4 + 1000 * rank)
+    N, H = m["N"], m["H"]
+    bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
+    gbuf = torch.empty(N, H, device="cuda")
+    bbuf = torch.empty(N, H, device="cuda")
+    ym = torch.empty(N, H, 128, device="cuda")
+    out = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)
+    nsq = m["num_seqs"]
+    wsm = torch.empty(max(gdn.workspace_size(N, nsq, H, 128, 128, 64), 16), device="cuda", dtype=torch.uint8)
+
+    def mix(i):
+        gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"], m["alpha_logit"],
+                 m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"], out=(*bufs, gbuf, bbuf))
+        gdn.chunk_fwd(bufs[0], bufs[1], bufs[2], gbuf, bbuf, None, m["cu_seqlens"], chunk=64, y=ym,
+                      final_state=False, workspace=wsm)
+        gdn.out_gate(ym, m["z"], m["norm_w"], m["eps"], out=out)
+
+    barrier(torch, dist, world)
+    n_m = 5
+    dt = max_over_ranks(torch, dist, timed(torch, mix, n_m, 1, stream), world) / n_m
+    fused_min = N * (H * 3 * 128 * 2 + H * 2 * 2 + H * 128 * 2 + H * 128 * 2)
+    res.append({"workload": inputs.CONFIGS[4]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
+                "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
+                "roofline": {"bound": "hbm", "achieved": fused_min / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": fused_min / dt / 1e9 / hbm_peak, "kernel": "prep+chunk+out_gate",
+                             "alg_bytes_per_step": fused_min,
+                             "note": "bytes = fused minimum (read projections, logits, z; write out)"},
+                "gpu_launches": 3 * n_m})
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--cpu-s", type=float, default=12.0, help="target seconds of the CPU-baseline sample")
+    ap.add_argument("--ref-step-s", type=float, default=8.0)
+    ap.add_argument("--no-cpu-baseline", dest="impl_cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,165 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, a B200 (sm_100a) implementation of the Gated
+ * DeltaNet (GDN) token mixer.
+ *
+ * The operations follow "On the design of Qwen3.8-Next architecture: evaluation,
+ * efficiency and training stability" (paper-archivist reading of arXiv
+ * 2608.30320), section 2.1.1:
+ *   "Gated Delta recurrence", eqs. (1)-(5):
+ *       S~_{t-1} = alpha_t S_{t-1}                  (1)
+ *       e_t      = v_t - S~_{t-1}^T k_t             (2)
+ *       S_t      = S~_{t-1} + beta_t k_t e_t^T      (3)
+ *       y_t      = S_t^T q_t                        (4)
+ *     with S_t in R^{dk x dv} (the transpose of the original GDN convention).
+ *   "GDN parameterisation", eqs. (6)-(11): ShortConv -> SiLU -> L2Norm for q and
+ *     k, ShortConv -> SiLU for v, beta = sigmoid(.), alpha = exp(-exp(A)
+ *     softplus(. + b)), and the sigmoid output gate over a zero-centred RMSNorm.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.   Token-major, head-minor: q, k are [N, H, dk], v, y, z are [N, H, dv],
+ *           per-token scalars (g, beta, logits) are [N, H]; the innermost index
+ *           is contiguous.  A state is [rows, H, dk, dv] fp32, dv contiguous.
+ *           N counts all tokens of all packed sequences.
+ * Sequences. cu_seqlens (int32, [num_seqs+1], cu[0] = 0, non-decreasing,
+ *           cu[num_seqs] <= N) gives packed variable-length sequences; NULL means
+ *           num_seqs sequences of N/num_seqs tokens each.  Every sequence starts
+ *           from its own initial state row and a zero convolution history.
+ * Decay.    alpha is passed as g = log(alpha) (fp32): the chunked algorithm works
+ *           with cumulative log-decays, and alpha itself can underflow in fp32.
+ * Memory.   Every pointer is a DEVICE pointer owned by the caller, 16-byte
+ *           aligned.  The library allocates nothing and keeps no per-call state;
+ *           calls are re-entrant from several host threads.
+ * Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *           only enqueues work on it and returns; nothing synchronises.
+ * Errors.   Argument errors are detected on the host before anything is enqueued
+ *           and return GDN_ERR_INVALID_ARG (bad value) or GDN_ERR_UNSUPPORTED
+ *           (valid but not implemented).  A failed launch returns GDN_ERR_CUDA.
+ *           Device-side bounded waits that run out record a code in a device error
+ *           word, read by gdn_check_device_error.  gdn_last_error_message gives a
+ *           one-line reason for the calling thread's last failure.  No C++
+ *           exception crosses this interface.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* gdn_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,
+    GDN_ERR_UNSUPPORTED = 2,
+    GDN_ERR_CUDA = 3,
+    GDN_ERR_TIMEOUT = 4
+} gdn_status_t;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 } gdn_dtype_t;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gdn_version(void);
+
+/* Static string naming a status code. */
+const char* gdn_status_string(gdn_status_t status);
+
+/* One-line reason for the calling thread's most recent non-OK return ("" if none). */
+const char* gdn_last_error_message(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error word.
+ * Returns GDN_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check,
+ * GDN_ERR_INVALID_ARG if a kernel found cu_seqlens out of order / range or a state
+ * slot out of range, GDN_ERR_CUDA if the stream reports a CUDA error, else GDN_OK.
+ */
+gdn_status_t gdn_check_device_error(gdn_stream_t stream);
+
+/*
+ * Test knob: the clock64 budget of every device-side wait (0 restores the default
+ * of about one second).  Process-wide; affects kernels launched after the call.
+ */
+void gdn_set_wait_budget(uint64_t cycles);
+
+/*
+ * gdn_prep -- eqs. (6)-(10): the input side of the mixer.
+ *   q = L2Norm(SiLU(ShortConv(x_q)))   (6)     k = L2Norm(SiLU(ShortConv(x_k)))   (7)
+ *   v = SiLU(ShortConv(x_v))           (8)     beta = sigmoid(beta_logit)         (9)
+ *   g = log alpha = -exp(A_log[h]) * softplus(alpha_logit + alpha_bias[h])         (10)
+ * ShortConv is causal and depthwise with conv_width taps and no bias:
+ *   conv[t, c] = sum_{j<W} w[c][j] * x[t-(W-1)+j, c], zero before the sequence start,
+ * with channel c = h*d + i and w stored [H*d, W] fp32 (tap W-1 meets token t).
+ * L2Norm(x) = x / sqrt(sum_i x_i^2 + l2_eps) over the head dimension.
+ *   x_q, x_k [N,H,dk], x_v [N,H,dv], beta_logit, alpha_logit [N,H]: in_dtype.
+ *   A_log, alpha_bias [H] fp32.   q, k [N,H,dk], v [N,H,dv]: out_dtype.
+ *   g_out, beta_out [N,H] fp32.   conv_width in [1, 8].  dk, dv in {16,32,64,128}.
+ * Tokens at index >= cu_seqlens[num_seqs] are left untouched.
+ */
+gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
+                      const float* conv_w_k, const float* conv_w_v, int conv_width,
+                      const void* beta_logit, const void* alpha_logit, const float* A_log,
+                      const float* alpha_bias, const int32_t* cu_seqlens, int num_seqs, int N, int H,
+                      int dk, int dv, float l2_eps, gdn_dtype_t in_dtype, gdn_dtype_t out_dtype,
+                      void* q, void* k, void* v, float* g_out, float* beta_out, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_fwd -- prefill: eqs. (1)-(4) over every token of every packed sequence.
+ *   q, k [N,H,dk], v [N,H,dv]: in_dtype.  g = log alpha, beta [N,H]: fp32.
+ *   S0 [num_seqs,H,dk,dv] fp32 or NULL (zero initial state).
+ *   y [N,H,dv]: y_dtype.  S_T [num_seqs,H,dk,dv] fp32 (final state) or NULL.
+ *   scale multiplies the readout (y_t = scale * S_t^T q_t); 1.0 is eq. (4) as printed.
+ * chunk selects the algorithm:
+ *   chunk = 0: token-sequential fp32 recurrence on CUDA cores (any supported
+ *              shape and dtype; exact up to fp32 rounding order).
+ *   chunk = 64 or 128: chunkwise-parallel form on the tcgen05 tensor cores
+ *              (requires dk = dv = 128 and in_dtype BF16 or F16).  It is derived
+ *              from eq. (5): within a chunk, the UT transform T = (I + A)^-1 with
+ *              A[r,s] = beta_r exp(gamma_r - gamma_s) k_r.k_s turns the token loop
+ *              into dense products; between chunks the state is carried in fp32.
+ * workspace: device scratch of at least gdn_chunk_fwd_workspace_size(...) bytes
+ * (may be NULL when that size is 0).  Tokens at index >= cu_seqlens[num_seqs] are
+ * neither read nor written.
+ */
+size_t gdn_chunk_fwd_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk);
+
+gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* S0, const int32_t* cu_seqlens,
+                           int num_seqs, int N, int H, int dk, int dv, int chunk, float scale,
+                           gdn_dtype_t in_dtype, gdn_dtype_t y_dtype, void* y, float* S_T,
+                           void* workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/*
+ * gdn_decode_step -- one token per row against a resident state, eqs. (1)-(4):
+ *   S <- alpha S + beta k e^T with e = v - alpha S^T k, y = scale * S^T q (new S).
+ *   q, k [B,H,dk], v [B,H,dv]: in_dtype.  g, beta [B,H] fp32.
+ *   state [num_slots,H,dk,dv] fp32, read and written in place; row b uses
+ *   state[state_slot[b]] (int32 [B], NULL = row b uses slot b, which needs
+ *   num_slots >= B).  Two rows must not name the same slot.  A row whose slot is
+ *   outside [0, num_slots) is skipped and flagged in the device error word
+ *   (gdn_check_device_error then returns GDN_ERR_INVALID_ARG).  y [B,H,dv]: y_dtype.
+ */
+gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                             const float* beta, float* state, const int32_t* state_slot,
+                             int num_slots, int B, int H, int dk, int dv, float scale,
+                             gdn_dtype_t in_dtype,
+                             gdn_dtype_t y_dtype, void* y, gdn_stream_t stream);
+
+/*
+ * gdn_out_gate -- eq. (11) without the output projection W_o:
+ *   out = sigmoid(z) * y / sqrt(mean_dv(y^2) + eps) * (1 + norm_w)
+ * per (token, head) over dv; norm_w [dv] fp32 is shared by all heads (the
+ * zero-centred RMSNorm weight).  y [N,H,dv]: y_dtype; z, out [N,H,dv]: io_dtype.
+ */
+gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, float eps, int N, int H,
+                          int dv, gdn_dtype_t y_dtype, gdn_dtype_t io_dtype, void* out,
+                          gdn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,271 @@
+// gdn_lib.cu -- the C ABI of libgdn.so (declared in include/gdn.h): argument validation,
+// launch configuration and error reporting around the device kernels.
+//
+// Every entry point validates on the host and returns before enqueuing anything when an
+// argument is wrong; it never synchronises and never allocates.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/gdn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "out_gate.cuh"
+#include "prep.cuh"
+#include "recurrent.cuh"
+#include "chunk_tc.cuh"
+
+namespace {
+
+thread_local char g_msg[256] = "";
+std::atomic<unsigned long long> g_wait_budget{0};
+
+gdn_status_t fail(gdn_status_t s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+gdn_status_t launched(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool dtype_ok(int t) { return t == GDN_F32 || t == GDN_BF16 || t == GDN_F16; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, ...)                                            \
+    do {                                                              \
+        if (!(cond)) return fail(GDN_ERR_INVALID_ARG, __VA_ARGS__);   \
+    } while (0)
+
+#define REQUIRE_PTR(p, name)                                                            \
+    do {                                                                                \
+        if ((p) == nullptr) return fail(GDN_ERR_INVALID_ARG, "%s is NULL", name);       \
+        if (!aligned16(p)) return fail(GDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+    } while (0)
+
+#define OPT_PTR(p, name)                                                                \
+    do {                                                                                \
+        if ((p) != nullptr && !aligned16(p))                                            \
+            return fail(GDN_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);       \
+    } while (0)
+
+// Dispatch a <DK, DV> template over the 16 supported head-size pairs.
+template <template <int, int> class F, typename... Args>
+gdn_status_t dispatch_dims(int dk, int dv, Args&&... args) {
+#define GDN_DV_CASES(DKV)                                                        \
+    switch (dv) {                                                                \
+        case 16: return F<DKV, 16>::run(args...);                                \
+        case 32: return F<DKV, 32>::run(args...);                                \
+        case 64: return F<DKV, 64>::run(args...);                                \
+        case 128: return F<DKV, 128>::run(args...);                              \
+    }                                                                            \
+    break;
+    switch (dk) {
+        case 16: GDN_DV_CASES(16)
+        case 32: GDN_DV_CASES(32)
+        case 64: GDN_DV_CASES(64)
+        case 128: GDN_DV_CASES(128)
+    }
+#undef GDN_DV_CASES
+    return fail(GDN_ERR_INVALID_ARG, "unsupported head sizes dk=%d dv=%d", dk, dv);
+}
+
+unsigned long long wait_budget() {
+    unsigned long long b = g_wait_budget.load(std::memory_order_relaxed);
+    return b ? b : 2000000000ull;  // ~1 s at the B200's boost clock
+}
+
+// ---------------------------------------------------------------- launchers
+
+template <int DK, int DV>
+struct DecodeLaunch {
+    static gdn_status_t run(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                            float* state, const int32_t* slot, int num_slots, int B, int H, float scale,
+                            int in_dt, int y_dt, void* y, cudaStream_t st) {
+        using Sh = gdn::DecodeShape<DK, DV>;
+        gdn::decode_step_kernel<DK, DV><<<(unsigned)(B * H), Sh::THREADS, 0, st>>>(
+            q, k, v, g, beta, state, slot, num_slots, H, scale, in_dt, y_dt, y);
+        return launched("decode_step_kernel");
+    }
+};
+
+template <int DK, int DV>
+struct RecurrentLaunch {
+    static gdn_status_t run(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                            const float* S0, const int32_t* cu, int num_seqs, int N, int H, float scale,
+                            int in_dt, int y_dt, void* y, float* S_T, cudaStream_t st) {
+        using Sh = gdn::RecShape<DK, DV>;
+        const unsigned grid = (unsigned)(num_seqs * H * (DV / Sh::SLAB));
+        gdn::recurrent_fwd_kernel<DK, DV><<<grid, Sh::THREADS, 0, st>>>(
+            q, k, v, g, beta, S0, cu, num_seqs, N, H, scale, in_dt, y_dt, y, S_T);
+        return launched("recurrent_fwd_kernel");
+    }
+};
+
+template <int DK, int DV>
+struct PrepLaunch {
+    static gdn_status_t run(const void* xq, const void* xk, const void* xv, const float* wq, const float* wk,
+                            const float* wv, int W, const void* bl, const void* al, const float* A,
+                            const float* ba, const int32_t* cu, int num_seqs, int N, int H, float eps,
+                            int in_dt, int out_dt, void* q, void* k, void* v, float* g, float* beta,
+                            cudaStream_t st) {
+        const long long rows = (long long)N * H;
+        const unsigned grid = (unsigned)((rows + gdn::kPrepWarps - 1) / gdn::kPrepWarps);
+        if (DK >= 32 && DV >= 32) {
+            gdn::prep_kernel<(DK >= 32 ? DK : 32), (DV >= 32 ? DV : 32)><<<grid, 32 * gdn::kPrepWarps, 0, st>>>(
+                xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g,
+                beta);
+        } else {
+            gdn::prep_small_kernel<DK, DV><<<grid, 32 * gdn::kPrepWarps, 0, st>>>(
+                xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g,
+                beta);
+        }
+        return launched("prep_kernel");
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return 100; }
+
+const char* gdn_status_string(gdn_status_t s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+const char* gdn_last_error_message(void) { return g_msg; }
+
+void gdn_set_wait_budget(uint64_t cycles) { g_wait_budget.store(cycles, std::memory_order_relaxed); }
+
+gdn_status_t gdn_check_device_error(gdn_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    unsigned word = 0;
+    e = cudaMemcpyFromSymbol(&word, gdn::g_error_word, sizeof(word));
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "error word: %s", cudaGetErrorString(e));
+    if (word) {
+        const unsigned zero = 0;
+        cudaMemcpyToSymbol(gdn::g_error_word, &zero, sizeof(zero));
+        if (word & gdn::kErrTimeout) return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (word 0x%x)", word);
+        if (word & gdn::kErrSeqlens) return fail(GDN_ERR_INVALID_ARG, "cu_seqlens out of order or range (word 0x%x)", word);
+        if (word & gdn::kErrSlot) return fail(GDN_ERR_INVALID_ARG, "state_slot out of range (word 0x%x)", word);
+        return fail(GDN_ERR_CUDA, "device error word 0x%x", word);
+    }
+    g_msg[0] = 0;
+    return GDN_OK;
+}
+
+gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                             float* state, const int32_t* state_slot, int num_slots, int B, int H, int dk,
+                             int dv, float scale, gdn_dtype_t in_dtype, gdn_dtype_t y_dtype, void* y,
+                             gdn_stream_t stream) {
+    REQUIRE(B >= 0 && H >= 1 && num_slots >= 0, "bad sizes B=%d H=%d num_slots=%d", B, H, num_slots);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(y_dtype), "bad dtype");
+    REQUIRE(state_slot != nullptr || num_slots >= B, "num_slots=%d < B=%d without state_slot", num_slots, B);
+    REQUIRE((long long)B * H <= 0x7fffffffLL, "B*H too large");
+    if (B == 0) return GDN_OK;
+    REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k"); REQUIRE_PTR(v, "v"); REQUIRE_PTR(g, "g");
+    REQUIRE_PTR(beta, "beta"); REQUIRE_PTR(state, "state"); REQUIRE_PTR(y, "y"); OPT_PTR(state_slot, "state_slot");
+    return dispatch_dims<DecodeLaunch>(dk, dv, q, k, v, g, beta, state, state_slot, num_slots, B, H, scale,
+                                       (int)in_dtype, (int)y_dtype, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t gdn_chunk_fwd_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk) {
+    return gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+}
+
+gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
+                           int dv, int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t y_dtype, void* y,
+                           float* S_T, void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(y_dtype), "bad dtype");
+    REQUIRE(chunk == 0 || chunk == 64 || chunk == 128, "chunk=%d not in {0, 64, 128}", chunk);
+    REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
+    REQUIRE((long long)N * H * (dk > dv ? dk : dv) < (1LL << 40), "problem too large");
+    if (N == 0 && S_T == nullptr) return GDN_OK;
+    REQUIRE_PTR(g, "g"); REQUIRE_PTR(beta, "beta"); REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k");
+    REQUIRE_PTR(v, "v"); REQUIRE_PTR(y, "y");
+    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens"); OPT_PTR(workspace, "workspace");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (chunk == 0)
+        return dispatch_dims<RecurrentLaunch>(dk, dv, q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, scale,
+                                              (int)in_dtype, (int)y_dtype, y, S_T, st);
+    if (dk != 128 || dv != 128 || in_dtype == GDN_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "chunked path needs dk=dv=128 and bf16/f16 inputs (use chunk=0)");
+    const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+    REQUIRE(workspace_bytes >= need && (need == 0 || workspace != nullptr), "workspace of %zu bytes < %zu",
+            workspace_bytes, need);
+    gdn::ChunkArgs a{q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, chunk, scale, (int)in_dtype,
+                     (int)y_dtype, y, S_T, workspace, wait_budget()};
+    const char* why = nullptr;
+    cudaError_t e = gdn::chunk_tc_launch(a, st, &why);
+    if (why) return fail(GDN_ERR_CUDA, "chunk_tc: %s", why);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "chunk_tc: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
+gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
+                      const float* conv_w_k, const float* conv_w_v, int conv_width, const void* beta_logit,
+                      const void* alpha_logit, const float* A_log, const float* alpha_bias,
+                      const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk, int dv, float l2_eps,
+                      gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* q, void* k, void* v, float* g_out,
+                      float* beta_out, gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(out_dtype), "bad dtype");
+    REQUIRE(conv_width >= 1 && conv_width <= 8, "conv_width=%d not in [1, 8]", conv_width);
+    REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
+    REQUIRE(l2_eps >= 0.f, "l2_eps < 0");
+    if (N == 0) return GDN_OK;
+    REQUIRE_PTR(x_q, "x_q"); REQUIRE_PTR(x_k, "x_k"); REQUIRE_PTR(x_v, "x_v");
+    REQUIRE_PTR(conv_w_q, "conv_w_q"); REQUIRE_PTR(conv_w_k, "conv_w_k"); REQUIRE_PTR(conv_w_v, "conv_w_v");
+    REQUIRE_PTR(beta_logit, "beta_logit"); REQUIRE_PTR(alpha_logit, "alpha_logit");
+    REQUIRE_PTR(A_log, "A_log"); REQUIRE_PTR(alpha_bias, "alpha_bias");
+    REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k"); REQUIRE_PTR(v, "v"); REQUIRE_PTR(g_out, "g_out");
+    REQUIRE_PTR(beta_out, "beta_out"); OPT_PTR(cu_seqlens, "cu_seqlens");
+    return dispatch_dims<PrepLaunch>(dk, dv, x_q, x_k, x_v, conv_w_q, conv_w_k, conv_w_v, conv_width, beta_logit,
+                                     alpha_logit, A_log, alpha_bias, cu_seqlens, num_seqs, N, H, l2_eps,
+                                     (int)in_dtype, (int)out_dtype, q, k, v, g_out, beta_out,
+                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, float eps, int N, int H, int dv,
+                          gdn_dtype_t y_dtype, gdn_dtype_t io_dtype, void* out, gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1, "bad sizes N=%d H=%d", N, H);
+    REQUIRE(head_dim_ok(dv), "dv=%d not in {16,32,64,128}", dv);
+    REQUIRE(dtype_ok(y_dtype) && dtype_ok(io_dtype), "bad dtype");
+    REQUIRE(eps >= 0.f, "eps < 0");
+    if (N == 0) return GDN_OK;
+    REQUIRE_PTR(y, "y"); REQUIRE_PTR(z, "z"); REQUIRE_PTR(norm_w, "norm_w"); REQUIRE_PTR(out, "out");
+    const long long rows = (long long)N * H;
+    const unsigned grid = (unsigned)((rows + gdn::kGateWarps - 1) / gdn::kGateWarps);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (dv) {
+        case 16: gdn::out_gate_kernel<16><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
+        case 32: gdn::out_gate_kernel<32><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
+        case 64: gdn::out_gate_kernel<64><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
+        default: gdn::out_gate_kernel<128><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
+    }
+    return launched("out_gate_kernel");
+}
+
+}  // extern "C"

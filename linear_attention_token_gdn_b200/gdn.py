@@ -1,0 +1,181 @@
+"""Thin ctypes binding of libgdn.so with the C ABI's entry-point names.
+
+Argument marshalling only: every step of the mixer runs in the CUDA kernels behind
+``include/gdn.h``.  PyTorch provides device memory and the current stream; output
+tensors are allocated here with ``torch.empty`` when the caller passes none.
+There is no fallback: if ``libgdn.so`` is missing or no CUDA device is present, the
+compute calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
+F32, BF16, F16 = 0, 1, 2
+_DT = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}
+
+# Every symbol include/gdn.h declares, with its ctypes signature.
+_P, _I, _F, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+SIGNATURES = {
+    "gdn_version": ([], _I),
+    "gdn_status_string": ([_I], ctypes.c_char_p),
+    "gdn_last_error_message": ([], ctypes.c_char_p),
+    "gdn_check_device_error": ([_P], _I),
+    "gdn_set_wait_budget": ([_U64], None),
+    "gdn_prep": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I,
+                  _P, _P, _P, _P, _P, _P], _I),
+    "gdn_chunk_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
+    "gdn_chunk_fwd": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P,
+                       _Z, _P], _I),
+    "gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P], _I),
+    "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
+}
+
+_lib = None
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{status_string(status)}: {msg}")
+        self.status = status
+
+
+def lib():
+    """The loaded libgdn.so (ctypes.CDLL with argtypes set).  Raises if it was never built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m linear_attention_token_gdn_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().gdn_status_string(s).decode()
+
+
+def last_error_message() -> str:
+    return lib().gdn_last_error_message().decode()
+
+
+def _check(status: int):
+    if status != GDN_OK:
+        raise GDNError(status, last_error_message())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libgdn takes device tensors only")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dt(t):
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise ValueError(f"unsupported dtype {t.dtype}") from None
+
+
+def version() -> int:
+    return lib().gdn_version()
+
+
+def set_wait_budget(cycles: int):
+    lib().gdn_set_wait_budget(int(cycles))
+
+
+def check_device_error(stream=None):
+    """Synchronise the stream and raise if a kernel flagged an error since the last check."""
+    _check(lib().gdn_check_device_error(_stream(stream)))
+
+
+def workspace_size(N, num_seqs, H, dk, dv, chunk) -> int:
+    return int(lib().gdn_chunk_fwd_workspace_size(N, num_seqs, H, dk, dv, chunk))
+
+
+def prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bias, cu_seqlens=None,
+         num_seqs=1, eps=1e-6, out_dtype=None, out=None, stream=None):
+    """gdn_prep: eqs. (6)-(10).  Returns (q, k, v, g, beta)."""
+    N, H, dk = x_q.shape
+    dv = x_v.shape[2]
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    out_dtype = x_q.dtype if out_dtype is None else out_dtype
+    if out is None:
+        dev = x_q.device
+        out = (torch.empty(N, H, dk, device=dev, dtype=out_dtype), torch.empty(N, H, dk, device=dev, dtype=out_dtype),
+               torch.empty(N, H, dv, device=dev, dtype=out_dtype), torch.empty(N, H, device=dev),
+               torch.empty(N, H, device=dev))
+    q, k, v, g, beta = out
+    _check(lib().gdn_prep(_ptr(x_q), _ptr(x_k), _ptr(x_v), _ptr(w_q), _ptr(w_k), _ptr(w_v), w_q.shape[1],
+                          _ptr(beta_logit), _ptr(alpha_logit), _ptr(A_log), _ptr(alpha_bias), _ptr(cu_seqlens),
+                          num_seqs, N, H, dk, dv, float(eps), _dt(x_q), _DT[out_dtype], _ptr(q), _ptr(k),
+                          _ptr(v), _ptr(g), _ptr(beta), _stream(stream)))
+    return q, k, v, g, beta
+
+
+def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=None, chunk=64, scale=1.0, y_dtype=None,
+              final_state=True, y=None, S_T=None, workspace=None, stream=None):
+    """gdn_chunk_fwd: prefill over packed sequences.  Returns (y, S_T or None)."""
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    elif num_seqs is None:
+        num_seqs = 1
+    y_dtype = q.dtype if y_dtype is None else y_dtype
+    if y is None:
+        y = torch.empty(N, H, dv, device=q.device, dtype=y_dtype)
+    if S_T is None and final_state:
+        S_T = torch.empty(num_seqs, H, dk, dv, device=q.device, dtype=torch.float32)
+    ws_bytes = workspace_size(N, num_seqs, H, dk, dv, chunk)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    _check(lib().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                               num_seqs, N, H, dk, dv, int(chunk), float(scale), _dt(q), _DT[y.dtype], _ptr(y),
+                               _ptr(S_T), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                               _stream(stream)))
+    return y, S_T
+
+
+def decode_step(q, k, v, g, beta, state, state_slot=None, scale=1.0, y_dtype=None, y=None, stream=None):
+    """gdn_decode_step: one token per row; ``state`` is updated in place.  Returns y."""
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    if y is None:
+        y = torch.empty(B, H, dv, device=q.device, dtype=q.dtype if y_dtype is None else y_dtype)
+    _check(lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(state_slot),
+                                 state.shape[0], B, H, dk, dv, float(scale), _dt(q), _DT[y.dtype], _ptr(y),
+                                 _stream(stream)))
+    return y
+
+
+def out_gate(y, z, norm_w, eps=1e-6, out=None, stream=None):
+    """gdn_out_gate: eq. (11) without W_o.  Returns out (dtype of z)."""
+    N, H, dv = y.shape
+    if out is None:
+        out = torch.empty(N, H, dv, device=z.device, dtype=z.dtype)
+    _check(lib().gdn_out_gate(_ptr(y), _ptr(z), _ptr(norm_w), float(eps), N, H, dv, _dt(y), _dt(z), _ptr(out),
+                              _stream(stream)))
+    return out

@@ -1,0 +1,107 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol include/gdn.h declares,
+and rejects bad arguments on the host before enqueuing anything (no device needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_token_gdn_b200 import build as gbuild
+from linear_attention_token_gdn_b200 import gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported_and_bound(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in gdn.SIGNATURES, n
+    assert set(gdn.SIGNATURES) == set(names)
+
+
+def test_status_strings_and_version(L):
+    assert gdn.version() >= 100
+    assert gdn.status_string(gdn.GDN_OK) == "GDN_OK"
+    assert gdn.status_string(gdn.GDN_ERR_TIMEOUT) == "GDN_ERR_TIMEOUT"
+
+
+A = ctypes.c_void_p(0x10000)      # an aligned fake address: validation never dereferences it
+MIS = ctypes.c_void_p(0x10004)    # misaligned
+
+
+def chunk_call(L, **over):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, S0=None, cu=None, num_seqs=2, N=64, H=2, dk=128, dv=128, chunk=64,
+             scale=1.0, in_dt=gdn.BF16, y_dt=gdn.BF16, y=A, S_T=None, ws=A, ws_bytes=1 << 30, stream=None)
+    a.update(over)
+    return L.gdn_chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["cu"], a["num_seqs"], a["N"],
+                           a["H"], a["dk"], a["dv"], a["chunk"], a["scale"], a["in_dt"], a["y_dt"], a["y"],
+                           a["S_T"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=None), dict(k=MIS), dict(dk=48), dict(dv=256), dict(chunk=32), dict(chunk=-1), dict(N=-1),
+    dict(H=0), dict(num_seqs=0), dict(N=63), dict(in_dt=7), dict(y_dt=-1), dict(S0=MIS),
+])
+def test_chunk_fwd_rejects_bad_arguments(L, over):
+    assert chunk_call(L, **over) == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.last_error_message() != ""
+
+
+@pytest.mark.parametrize("over", [dict(dk=64, dv=64), dict(in_dt=gdn.F32), dict(dk=128, dv=64)])
+def test_chunk_fwd_tensor_core_path_limits(L, over):
+    assert chunk_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_zero_tokens_is_a_no_op(L):
+    assert chunk_call(L, N=0, q=None, y=None) == gdn.GDN_OK
+    assert L.gdn_decode_step(None, None, None, None, None, None, None, 0, 0, 4, 128, 128, 1.0, 1, 1, None,
+                             None) == gdn.GDN_OK
+    assert L.gdn_out_gate(None, None, None, 1e-6, 0, 4, 128, 1, 1, None, None) == gdn.GDN_OK
+
+
+@pytest.mark.parametrize("over", [
+    dict(state=None), dict(num_slots=3), dict(dk=8), dict(y=MIS), dict(in_dt=5), dict(slot=MIS),
+])
+def test_decode_rejects_bad_arguments(L, over):
+    a = dict(state=A, slot=None, num_slots=4, B=4, H=2, dk=128, dv=128, in_dt=1, y=A)
+    a.update(over)
+    st = L.gdn_decode_step(A, A, A, A, A, a["state"], a["slot"], a["num_slots"], a["B"], a["H"], a["dk"], a["dv"],
+                           1.0, a["in_dt"], 1, a["y"], None)
+    assert st == gdn.GDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(W=0), dict(W=9), dict(x_q=None), dict(eps=-1.0), dict(dk=100)])
+def test_prep_rejects_bad_arguments(L, over):
+    a = dict(W=4, x_q=A, eps=1e-6, dk=128)
+    a.update(over)
+    st = L.gdn_prep(a["x_q"], A, A, A, A, A, a["W"], A, A, A, A, None, 1, 16, 2, a["dk"], 128, a["eps"], 1, 1,
+                    A, A, A, A, A, None)
+    assert st == gdn.GDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(dv=96), dict(eps=-1.0), dict(out=None), dict(io=3)])
+def test_out_gate_rejects_bad_arguments(L, over):
+    a = dict(dv=128, eps=1e-6, out=A, io=1)
+    a.update(over)
+    assert L.gdn_out_gate(A, A, A, a["eps"], 16, 2, a["dv"], 1, a["io"], a["out"], None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        gdn._ptr(torch.zeros(4))

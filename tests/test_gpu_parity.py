@@ -1,0 +1,225 @@
+"""GPU parity: every entry point of libgdn.so (called through the C ABI via the ctypes
+binding) against the fp64 oracle on the same seeded inputs.
+
+Error metric (per output tensor): max |gpu - oracle| / max |oracle|.  Bounds:
+  * 1e-4 for fp32 inputs (fp32 arithmetic on CUDA cores);
+  * 3e-3 for bf16/fp16 inputs with the fp32 state (tensor-core path: fp16 operands,
+    fp32 accumulation and state), and for any bf16/fp16 output (which alone adds up to
+    2^-9 of the largest element).
+The oracle receives the exact values the GPU receives (16-bit inputs upcast exactly).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_token_gdn_b200 import build as gbuild
+from linear_attention_token_gdn_b200 import gdn, inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_16 = 3e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    gbuild.build()
+    gdn.lib()
+
+
+def err(gpu, ref):
+    g = gpu.detach().double().cpu().numpy() if hasattr(gpu, "detach") else np.asarray(gpu)
+    ref = np.asarray(ref)
+    assert np.all(np.isfinite(g))
+    return float(np.max(np.abs(g - ref)) / max(np.max(np.abs(ref)), 1e-30))
+
+
+def to_dev(d):
+    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in d.items()}
+
+
+# --------------------------------------------------------------- recurrent (chunk=0)
+
+def test_recurrent_tiny_fp32_workload():
+    """The tiny workload: B=1, H=2, T=64, dk=dv=16, fp32, S0 = 0."""
+    x = inputs.make_prefill(0, "cuda")
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=0)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+    assert err(y, y_ref) < TOL_F32
+    assert err(S_T, S_ref) < TOL_F32
+    gdn.check_device_error()
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 32), (64, 16), (128, 128), (32, 64)])
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16, torch.float16])
+def test_recurrent_varlen_shapes_dtypes(dk, dv, dt):
+    lengths = [37, 1, 0, 70]
+    x = inputs.make_prefill(1, "cuda", seed=11 + dk + dv, lengths=lengths, H=3, dk=dk, dv=dv, dtype=dt,
+                            S0_std=0.3)
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=0,
+                           y_dtype=torch.float32)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
+    assert err(y, y_ref) < TOL_F32
+    assert err(S_T, S_ref) < TOL_F32
+    gdn.check_device_error()
+
+
+# --------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (16, 16), (64, 32), (32, 128)])
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_decode_steps_with_slots(dk, dv, dt):
+    B, H, slots = 5, 3, 9
+    state = inputs.make_decode_state(3, "cuda", seed=5, B=slots, H=H, dk=dk, dv=dv)
+    slot = torch.tensor([7, 0, 3, 8, 1], dtype=torch.int32, device="cuda")
+    ref_state = state.double().cpu().numpy()
+    for step in range(3):
+        x = inputs.make_decode_step(3, "cuda", step=step, seed=5, B=B, H=H, dk=dk, dv=dv, dtype=dt)
+        y = gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, slot, y_dtype=torch.float32)
+        y_ref, ref_state = oracle.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], ref_state, slot)
+        assert err(y, y_ref) < TOL_F32
+        assert err(state, ref_state) < TOL_F32
+    gdn.check_device_error()
+
+
+def test_decode_full_workload_sampled_heads():
+    """256 x 32 heads, dk = dv = 128, 100 in-place steps (bf16 q/k/v, bf16 y): check sampled
+    (row, head) pairs against the oracle run on those heads alone, every step."""
+    c = inputs.CONFIGS[3]
+    state = inputs.make_decode_state(3, "cuda")
+    picks = [(0, 0), (17, 5), (255, 31), (128, 16)]
+    ref = {p: state[p[0], p[1]].double().cpu().numpy()[None, None] for p in picks}
+    for step in range(c["steps"]):
+        x = inputs.make_decode_step(3, "cuda", step=step)
+        y = gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state)
+        if step % 11 == 0 or step == c["steps"] - 1:
+            for (b, h) in picks:
+                sl = lambda t: t[b:b + 1, h:h + 1]
+                y_ref, ref[(b, h)] = oracle.decode_step(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
+                                                        sl(x["beta"]), ref[(b, h)])
+                assert err(y[b, h], y_ref[0, 0]) < TOL_16
+        else:
+            for (b, h) in picks:
+                sl = lambda t: t[b:b + 1, h:h + 1]
+                _, ref[(b, h)] = oracle.decode_step(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
+                                                    sl(x["beta"]), ref[(b, h)])
+    for (b, h) in picks:
+        assert err(state[b, h], ref[(b, h)][0, 0]) < TOL_F32
+    gdn.check_device_error()
+
+
+def test_decode_rejects_out_of_range_slot_on_device():
+    state = torch.zeros(2, 1, 16, 16, device="cuda")
+    x = inputs.make_decode_step(3, "cuda", B=1, H=1, dk=16, dv=16, dtype=torch.float32)
+    gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state,
+                    torch.tensor([5], dtype=torch.int32, device="cuda"))
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.check_device_error()
+    assert e.value.status == gdn.GDN_ERR_INVALID_ARG
+    assert torch.all(state == 0)
+
+
+# ------------------------------------------------------------- prep / out gate
+
+@pytest.mark.parametrize("d", [128, 16])
+@pytest.mark.parametrize("out_dt", [torch.float32, torch.bfloat16])
+def test_prep_matches_oracle(d, out_dt):
+    m = inputs.make_mixer(4, "cuda", lengths=[33, 5, 64], d=d, H=3)
+    q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
+                                m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
+                                out_dtype=out_dt)
+    ref = oracle.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
+                      m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"])
+    tol = TOL_F32 if out_dt == torch.float32 else TOL_16
+    for got, want in zip((q, k, v), ref[:3]):
+        assert err(got, want) < tol
+    assert err(g, ref[3]) < TOL_F32
+    assert err(beta, ref[4]) < TOL_F32
+    gdn.check_device_error()
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_out_gate_matches_oracle(io):
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    y = torch.randn(300, 4, 128, device="cuda", generator=gen) * 2
+    z = torch.randn(300, 4, 128, device="cuda", generator=gen).to(io)
+    w = torch.randn(128, device="cuda", generator=gen) * 0.02
+    out = gdn.out_gate(y, z, w, 1e-6)
+    ref = oracle.out_gate(y, z, w, 1e-6)
+    assert err(out, ref) < (TOL_F32 if io == torch.float32 else TOL_16)
+
+
+# ---------------------------------------------------------- tensor-core chunked path
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("y_dt", [torch.float32, torch.bfloat16])
+def test_chunk_tc_small_ragged(dt, y_dt):
+    """Several chunks per sequence, ragged tails, an empty and a one-token sequence, S0 != 0."""
+    lengths = [3 * 64 + 17, 64, 1, 0, 130]
+    x = inputs.make_prefill(2, "cuda", seed=21, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64,
+                           y_dtype=y_dt)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
+    assert err(y, y_ref) < TOL_16
+    assert err(S_T, S_ref) < TOL_16
+    gdn.check_device_error()
+
+
+def test_chunk_tc_matches_recurrent_path_no_initial_state():
+    x = inputs.make_prefill(1, "cuda", seed=22, T=256, H=4)
+    y1, S1 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
+                           y_dtype=torch.float32)
+    y0, S0 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=0,
+                           y_dtype=torch.float32)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+    assert err(y0, y_ref) < TOL_F32
+    assert err(y1, y_ref) < TOL_16 and err(S1, S_ref) < TOL_16
+
+
+def test_chunk_tc_prefill_workload_full():
+    """B=2, H=16, T=4096, dk=dv=128, bf16, S0 = 0, chunk 64: every output checked."""
+    x = inputs.make_prefill(1, "cuda")
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+    assert err(y, y_ref) < TOL_16
+    assert err(S_T, S_ref) < TOL_16
+    gdn.check_device_error()
+
+
+def test_chunk_tc_long_prefill_sampled_heads():
+    """B=1, H=32, T=32768, S0 ~ N(0, 0.02), exp(A) up to 64: heads checked one by one
+    (slowest- and fastest-decaying heads included)."""
+    x = inputs.make_prefill(2, "cuda")
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64)
+    mean_g = x["g"].mean(0)
+    heads = sorted({0, int(mean_g.argmin()), int(mean_g.argmax()), 19})
+    for h in heads:
+        sl = slice(h, h + 1)
+        y_ref, S_ref = oracle.recurrence(x["q"][:, sl], x["k"][:, sl], x["v"][:, sl], x["g"][:, sl],
+                                         x["beta"][:, sl], x["S0"][:, sl], x["cu_seqlens"])
+        assert err(y[:, sl], y_ref) < TOL_16, h
+        assert err(S_T[:, sl], S_ref) < TOL_16, h
+    gdn.check_device_error()
+
+
+def test_full_mixer_workload_sampled_heads():
+    """Packed variable-length sequences, H=16, d=128, bf16: prep -> chunked recurrence ->
+    out gate through the C ABI, against the fp64 oracle mixer on sampled heads."""
+    m = inputs.make_mixer(4, "cuda")
+    q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
+                                m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
+                                out_dtype=torch.float16)
+    y, S_T = gdn.chunk_fwd(q, k, v, g, beta, None, m["cu_seqlens"], chunk=64, y_dtype=torch.float32)
+    out = gdn.out_gate(y, m["z"], m["norm_w"], m["eps"])
+    d = m["d"]
+    for h in (0, 9):
+        hs = slice(h, h + 1)
+        cs = slice(h * d, (h + 1) * d)
+        ref_out, ref_y, _ = oracle.mixer(m["x_q"][:, hs], m["x_k"][:, hs], m["x_v"][:, hs], m["w_q"][cs],
+                                         m["w_k"][cs], m["w_v"][cs], m["beta_logit"][:, hs],
+                                         m["alpha_logit"][:, hs], m["A_log"][hs], m["alpha_bias"][hs],
+                                         m["z"][:, hs], m["norm_w"], m["cu_seqlens"], eps_l2=m["eps"],
+                                         eps_rms=m["eps"])
+        assert err(out[:, hs], ref_out) < TOL_16, h
+    gdn.check_device_error()
