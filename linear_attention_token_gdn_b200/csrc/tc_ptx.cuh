@@ -147,3 +147,28 @@ __device__ __forceinline__ uint32_t swz_off(int r, int c, int row_bytes) {
 
 }  // namespace tc
 }  // namespace gdn
+
+namespace gdn {
+namespace tc {
+
+// Named barrier over `n` threads (a multiple of 32, warp-uniform call sites).
+__device__ __forceinline__ void bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier that also ANDs a predicate across the participating threads.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+}  // namespace tc
+}  // namespace gdn

@@ -1,11 +1,14 @@
 """GPU parity: every entry point of libgdn.so (called through the C ABI via the ctypes
 binding) against the fp64 oracle on the same seeded inputs.
 
-Error metric (per output tensor): max |gpu - oracle| / max |oracle|.  Bounds:
+Error metric (per output tensor): max over elements of
+    max(|gpu - oracle| - u |oracle|, 0) / max |oracle|
+where u is the unit roundoff of the output's own storage type (0 for fp32, 2^-11 for
+fp16, 2^-8 for bf16): a 16-bit output is a rounding of the computed value, and that
+final rounding alone can exceed the arithmetic bounds below.  Bounds:
   * 1e-4 for fp32 inputs (fp32 arithmetic on CUDA cores);
   * 3e-3 for bf16/fp16 inputs with the fp32 state (tensor-core path: fp16 operands,
-    fp32 accumulation and state), and for any bf16/fp16 output (which alone adds up to
-    2^-9 of the largest element).
+    fp32 accumulation, fp32 state).
 The oracle receives the exact values the GPU receives (16-bit inputs upcast exactly).
 """
 import numpy as np
@@ -28,15 +31,16 @@ def _lib(cuda_device):
     gdn.lib()
 
 
+UNIT_ROUNDOFF = {torch.float32: 0.0, torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -8}
+
+
 def err(gpu, ref):
-    g = gpu.detach().double().cpu().numpy() if hasattr(gpu, "detach") else np.asarray(gpu)
+    u = UNIT_ROUNDOFF[gpu.dtype]
+    g = gpu.detach().double().cpu().numpy()
     ref = np.asarray(ref)
     assert np.all(np.isfinite(g))
-    return float(np.max(np.abs(g - ref)) / max(np.max(np.abs(ref)), 1e-30))
-
-
-def to_dev(d):
-    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in d.items()}
+    excess = np.maximum(np.abs(g - ref) - u * np.abs(ref), 0.0)
+    return float(np.max(excess) / max(np.max(np.abs(ref)), 1e-30))
 
 
 # --------------------------------------------------------------- recurrent (chunk=0)
@@ -98,7 +102,7 @@ def test_decode_full_workload_sampled_heads():
                 sl = lambda t: t[b:b + 1, h:h + 1]
                 y_ref, ref[(b, h)] = oracle.decode_step(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
                                                         sl(x["beta"]), ref[(b, h)])
-                assert err(y[b, h], y_ref[0, 0]) < TOL_16
+                assert err(y[b, h], y_ref[0, 0]) < TOL_F32
         else:
             for (b, h) in picks:
                 sl = lambda t: t[b:b + 1, h:h + 1]
@@ -131,9 +135,8 @@ def test_prep_matches_oracle(d, out_dt):
                                 out_dtype=out_dt)
     ref = oracle.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
                       m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"])
-    tol = TOL_F32 if out_dt == torch.float32 else TOL_16
     for got, want in zip((q, k, v), ref[:3]):
-        assert err(got, want) < tol
+        assert err(got, want) < TOL_F32
     assert err(g, ref[3]) < TOL_F32
     assert err(beta, ref[4]) < TOL_F32
     gdn.check_device_error()
@@ -147,7 +150,7 @@ def test_out_gate_matches_oracle(io):
     w = torch.randn(128, device="cuda", generator=gen) * 0.02
     out = gdn.out_gate(y, z, w, 1e-6)
     ref = oracle.out_gate(y, z, w, 1e-6)
-    assert err(out, ref) < (TOL_F32 if io == torch.float32 else TOL_16)
+    assert err(out, ref) < TOL_F32
 
 
 # ---------------------------------------------------------- tensor-core chunked path
@@ -182,8 +185,9 @@ def test_chunk_tc_prefill_workload_full():
     x = inputs.make_prefill(1, "cuda")
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
-    assert err(y, y_ref) < TOL_16
-    assert err(S_T, S_ref) < TOL_16
+    ey, es = err(y, y_ref), err(S_T, S_ref)
+    print(f"prefill workload: y err {ey:.2e}, S_T err {es:.2e}")
+    assert ey < TOL_16 and es < TOL_16
     gdn.check_device_error()
 
 
@@ -223,3 +227,23 @@ def test_full_mixer_workload_sampled_heads():
                                          eps_rms=m["eps"])
         assert err(out[:, hs], ref_out) < TOL_16, h
     gdn.check_device_error()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """Failure detection without a GPU fault: with a one-cycle wait budget every mbarrier
+    wait of the chunked kernel gives up, the kernel flags GDN_ERR_TIMEOUT, drains its MMAs,
+    frees TMEM and returns; the next call with the default budget is correct again."""
+    x = inputs.make_prefill(1, "cuda", seed=23, T=256, H=2)
+    try:
+        gdn.set_wait_budget(1)
+        gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
+        with pytest.raises(gdn.GDNError) as e:
+            gdn.check_device_error()
+        assert e.value.status == gdn.GDN_ERR_TIMEOUT
+    finally:
+        gdn.set_wait_budget(0)
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
+                           y_dtype=torch.float32)
+    gdn.check_device_error()
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+    assert err(y, y_ref) < TOL_16 and err(S_T, S_ref) < TOL_16
