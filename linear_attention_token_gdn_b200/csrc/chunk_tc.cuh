@@ -1,43 +1,38 @@
 // chunk_tc.cuh -- chunkwise-parallel GDN prefill on the sm_100a tensor cores.
 //
 // The recurrence is eqs. (1)-(4) of "On the design of Qwen3.8-Next architecture", section
-// 2.1.1.  Unrolling eqs. (1)-(3) over a chunk of C tokens that starts from state S (the
-// closed form eq. (5) applied C times), with gamma_r the inclusive prefix sum of
+// 2.1.1.  Unrolling eqs. (1)-(3) over a chunk of C = 64 tokens that starts from state S
+// (the closed form eq. (5) applied C times), with gamma_r the inclusive prefix sum of
 // g = log alpha inside the chunk and Gamma_r = exp(gamma_r), gives
 //     A[r,s] = beta_r exp(gamma_r - gamma_s) k_r.k_s   (s < r),   T = (I + A)^-1
 //     W  = T diag(beta Gamma) K,      U~ = T diag(beta) V,      U = U~ - W S
 //     M[r,s] = exp(gamma_r - gamma_s) q_r.k_s           (s <= r)
-//     Y  = diag(Gamma) Q S + M U,     S' = Gamma_C S + (diag(Gamma_C / Gamma) K)^T U
-// Every decay factor is exp(<= 0): masks are applied elementwise to the fp32 products in
-// the TMEM epilogue, never factored as Gamma_r / Gamma_s.  For s in an earlier 16-row
-// block than r the factor is split at the end e of s's block,
-//     exp(gamma_r - gamma_s) = exp(gamma_r - gamma_e) * exp(gamma_e - gamma_s),
-// both factors <= 1, so a row needs 4 + 16 exponentials instead of 64.
+//     Y  = diag(Gamma) Q S + M U,     S' = Gamma_C S + K^T diag(Gamma_C / Gamma) U
+// Every decay factor is exp(<= 0) and is applied elementwise to fp32 products, never
+// factored as Gamma_r / Gamma_s.  For s in an earlier 16-row block than r the factor is
+// split at the end e of s's block, exp(gamma_r - gamma_e) * exp(gamma_e - gamma_s), both
+// factors <= 1, so a row needs 4 + 16 exponentials instead of 64.
 //
-// Work decomposition.  The dv columns of S evolve independently (W and A do not depend
-// on V), so one CTA owns one (sequence, head, dv-slab of NS columns) and walks the
-// sequence chunk by chunk.  Its 256 threads form two warpgroups:
-//   * the intra group (warps 4-7) computes everything that does not depend on the state
-//     for chunk c+1 -- fp16 operand tiles, masks, the UT transform T, W and U~ -- into one
-//     of two shared-memory / TMEM slots, while its loads for chunk c+2 are in flight;
-//   * the chain group (warps 0-3) carries the fp32 state (one row per thread, in
-//     registers) through chunk c with two dependent tensor-core round trips:
-//         [W;Q] S                         -> U = U~ - W S (fp16 operand), Q S kept
-//         [T_w;M] U  and  Kg^T U          -> Y = Gamma (Q S) + M U,  S' = Gamma_C S + Kg^T U
-// Slots are handed over with mbarriers (full: intra -> chain, empty: chain -> intra).
-// Products on tcgen05 (fp16 operands, fp32 accumulation in TMEM):
-//     [K;Q] K^T            (M=128, N=64,  K=128)   -> A (rows 0-63) and M (rows 64-127)
-//     [T_u;T_w] V_slab     (M=128, N=NS,  K=64)    -> U~ (rows 0-63)
-//     [T_u;T_w] K          (M=128, N=128, K=64)    -> W  (rows 64-127)
-//     [W;Q] S              (M=128, N=NS,  K=128)   -> W S (rows 0-63), Q S (rows 64-127)
-//     [T_w;M] U            (M=128, N=NS,  K=64)    -> M U (rows 64-127)
-//     (diag(Gamma_C/Gamma)K)^T U (M=128, N=NS, K=64) -> state increment
-// with T_u = T diag(beta), T_w = T diag(beta Gamma).  The 64x64 unit-lower-triangular
-// inverse T is formed in fp32 on the CUDA cores (16x16 diagonal blocks by forward
-// substitution, then the off-diagonal blocks in three dependent rounds).
-// Operand tiles use the 128B (or 64B) swizzled canonical layouts, so one tile (K, or a
-// slab tile) serves both as a K-major and as an MN-major operand.
-//
+// Two kernels:
+//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, several CTAs per SM.
+//                       [K;Q] K^T on tcgen05 (the 16-bit inputs used directly as
+//                       operands), the decay masks, and the unit-lower-triangular inverse
+//                       T in fp32 on the CUDA cores.  Writes a 24 KB record per
+//                       (chunk, head): T_w = T diag(beta Gamma), T_u = T diag(beta) and M,
+//                       fp16, already in the 128B-swizzled operand layout.
+//   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
+//                       the chunks.  A producer warpgroup bulk-copies the next chunk's
+//                       K, Q, V rows and record into staging, converts them to fp16
+//                       operand tiles and computes W = T_w K and U~ = T_u V on the tensor
+//                       cores; a chain warpgroup carries the fp32 state (one row per
+//                       thread) through two dependent tensor-core round trips per chunk:
+//                           [Q;W] S                  -> Q S, W S;  U = U~ - W S
+//                           [M;.] U  and  K^T U'     -> Y = Gamma (Q S) + M U,
+//                                                       S' = Gamma_C S + K^T U'
+//                       with U' = diag(Gamma_C / Gamma) U.  Slots are double-buffered and
+//                       handed over with mbarriers; y rows leave through bulk stores.
+// All products use fp16 operands with fp32 accumulation in TMEM.  Operand tiles use the
+// 128B / 64B swizzled canonical layouts, so one tile serves as K-major or MN-major operand.
 // Every wait is bounded (ChunkArgs::budget clock cycles); a wait that runs out sets the
 // device error word, lets in-flight MMAs drain, and the CTA returns after freeing TMEM.
 #pragma once
@@ -59,38 +54,69 @@ struct ChunkArgs {
     unsigned long long budget;
 };
 
-inline size_t chunk_tc_workspace_bytes(int, int, int, int, int, int) { return 0; }
+constexpr int kChunk = 64;
+constexpr int kRecBytes = 24576;  // per (chunk, head): T_w, T_u, M as 3 x [64 rows x 128 B]
 
-template <int NS>
-struct TcCfg {
-    static constexpr int C = 64;
-    static constexpr int ROWB = NS * 2;  // bytes per row of a slab tile
-    static constexpr uint32_t SWZ = NS == 32 ? tc::kSw64 : tc::kSw128;
-    // shared memory (byte offsets from a 1024-aligned base); [2] = per chunk-parity slot
-    static constexpr int OFF_X = 0;                          // [2] [K->W ; Q]: 2 x [128 x 128 B]
-    static constexpr int OFF_TM = OFF_X + 2 * 32768;         // [2] [T_u; T_w; M]: [192 x 128 B]
-    static constexpr int OFF_KG = OFF_TM + 2 * 24576;        // [2] Kg: 2 x [64 x 128 B]
-    static constexpr int OFF_VS = OFF_KG + 2 * 16384;        // V slab [64 x ROWB]
-    static constexpr int OFF_SS = OFF_VS + 64 * ROWB;        // S operand [128 x ROWB]
-    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;       // U operand [64 x ROWB]
-    static constexpr int OFF_A = OFF_SU + 64 * ROWB;         // fp32 A [64][65]
-    static constexpr int OFF_TF = OFF_A + 64 * 65 * 4;       // fp32 T [64][65]
-    static constexpr int OFF_Z = OFF_TF + 64 * 65 * 4;       // fp32 scratch [3][16][17]
-    static constexpr int OFF_VEC = OFF_Z + 3 * 16 * 17 * 4;  // [2] gamma, Gamma, beta, colf: 4 x 64 floats
-    static constexpr int OFF_META = OFF_VEC + 2 * 1024;      // [2] {c0, L}
-    static constexpr int OFF_BAR = OFF_META + 64;            // mbarriers + TMEM base
-    static constexpr int BYTES = OFF_BAR + 128 + 1024;       // + alignment slack
-    // TMEM columns (fp32 accumulators, lane = output row)
-    static constexpr uint32_t COL_QK = 0;
-    static constexpr uint32_t COL_UT = 64;                   // [2] x NS
-    static constexpr uint32_t COL_W = 64 + 2 * NS;           // 128
-    static constexpr uint32_t COL_1 = COL_W + 128;           // NS
-    static constexpr uint32_t COL_MU = COL_1 + NS;           // NS
-    static constexpr uint32_t COL_DS = COL_MU + NS;          // NS
-    static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(COL_DS + NS <= TMEM_COLS, "TMEM budget");
-    static_assert(BYTES <= 232448, "shared memory budget");
-};
+// Upper bound of the number of 64-token chunks over all sequences.
+inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
+    if (!varlen) {
+        const long long L = N / num_seqs;
+        return (long long)num_seqs * ((L + kChunk - 1) / kChunk);
+    }
+    return (N + kChunk - 1) / kChunk + num_seqs;
+}
+
+inline size_t chunk_tc_workspace_bytes(int N, int num_seqs, int H, int, int, int chunk) {
+    if (chunk == 0 || N <= 0 || num_seqs <= 0 || H <= 0) return 0;
+    // the bound for packed sequences also covers equal lengths
+    return (size_t)chunk_count_bound(N, num_seqs, true) * H * kRecBytes;
+}
+
+// Chunks of sequence m (warp-uniform).
+__device__ __forceinline__ int seq_chunks(const int32_t* cu, int m, int num_seqs, int N) {
+    int a, b;
+    seq_bounds(cu, m, num_seqs, N, a, b);
+    return (b - a + kChunk - 1) / kChunk;
+}
+
+// Virtual chunk v -> (sequence n, chunk j of n).  Warp-collective; false if v is past the end.
+__device__ bool locate_chunk(const int32_t* cu, int num_seqs, int N, int v, int& n, int& j) {
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    for (int m0 = 0; m0 < num_seqs; m0 += 32) {
+        const int m = m0 + lane;
+        const int cnt = m < num_seqs ? seq_chunks(cu, m, num_seqs, N) : 0;
+        int inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += t;
+        }
+        const int total = __shfl_sync(0xffffffffu, inc, 31);
+        if (v < base + total) {
+            const unsigned hit = __ballot_sync(0xffffffffu, base + inc > v);
+            const int l = __ffs(hit) - 1;
+            n = m0 + l;
+            j = v - (base + __shfl_sync(0xffffffffu, inc, l) - __shfl_sync(0xffffffffu, cnt, l));
+            return true;
+        }
+        base += total;
+    }
+    return false;
+}
+
+// Number of chunks of sequences 0 .. n-1 (warp-collective).
+__device__ int chunks_before(const int32_t* cu, int num_seqs, int N, int n) {
+    const int lane = threadIdx.x & 31;
+    int s = 0;
+    for (int m0 = 0; m0 < n; m0 += 32) {
+        const int m = m0 + lane;
+        s += m < n ? seq_chunks(cu, m, num_seqs, N) : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    return s;
+}
 
 // 8 consecutive 16-bit input elements -> 8 fp16 values packed in a uint4.
 __device__ __forceinline__ uint4 to_f16x8(uint4 u, int in_dt) {
@@ -115,39 +141,290 @@ __device__ __forceinline__ uint4 pack_f16x8(const float* x) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ void unpack_f16x8(uint4 u, float* x) {
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 f = __half22float2(*reinterpret_cast<__half2*>(&w[i]));
-        x[2 * i] = f.x;
-        x[2 * i + 1] = f.y;
-    }
-}
-
 __device__ __forceinline__ uint4 ldg16(const void* p, size_t elem_off) {
     return __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p) + elem_off));
 }
 
-template <int NS>
-__global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_constant__ ChunkArgs a) {
-    using Cf = TcCfg<NS>;
-    constexpr int C = Cf::C;
-    constexpr int NSLAB = 128 / NS;
-    constexpr int VU = (64 * NS / 8) / 128;  // 16-byte V pieces per intra thread
+__device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+
+// =====================================================================================
+// chunk_ut_kernel: per (chunk, head) -- masks and the UT transform
+// =====================================================================================
+
+struct UtCfg {
+    static constexpr int LD = 68;                          // fp32 row stride of A and T
+    static constexpr int OFF_KQ = 0;                       // [K;Q] raw 16-bit: 2 x [128 x 128 B]
+    static constexpr int OFF_A = OFF_KQ + 32768;           // fp32 A [64][LD]
+    static constexpr int OFF_T = OFF_A + 64 * LD * 4;      // fp32 T [64][LD]
+    static constexpr int OFF_Z = OFF_T + 64 * LD * 4;      // fp32 Z [3][16][20]
+    static constexpr int OFF_VEC = OFF_Z + 3 * 16 * 20 * 4; // gamma, Gamma, beta, colf: 4 x 64
+    static constexpr int OFF_META = OFF_VEC + 1024;
+    static constexpr int OFF_BAR = OFF_META + 32;
+    static constexpr int BYTES = OFF_BAR + 32 + 1024;
+    static constexpr uint32_t TMEM_COLS = 64;
+};
+
+__global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ ChunkArgs a) {
+    using Cf = UtCfg;
+    constexpr int LD = Cf::LD;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = tc::smem_u32(smem);
     float* fA = reinterpret_cast<float*>(smem + Cf::OFF_A);
-    float* fT = reinterpret_cast<float*>(smem + Cf::OFF_TF);
+    float* fT = reinterpret_cast<float*>(smem + Cf::OFF_T);
     float* fZ = reinterpret_cast<float*>(smem + Cf::OFF_Z);
+    float* vb = reinterpret_cast<float*>(smem + Cf::OFF_VEC);  // gamma[0:64] Gamma[64:128] beta[128:192] colf[192:256]
+    int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 8);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int v = blockIdx.x, h = blockIdx.y, H = a.H;
+    if (warp == 0) {
+        int n = 0, j = 0;
+        const bool found = locate_chunk(a.cu, a.num_seqs, a.N, v, n, j);
+        if (lane == 0) {
+            meta[0] = found;
+            meta[1] = n;
+            meta[2] = j;
+        }
+    }
+    __syncthreads();
+    if (!meta[0]) return;
+    int t_begin, t_end;
+    seq_bounds(a.cu, meta[1], a.num_seqs, a.N, t_begin, t_end);
+    const int t0 = t_begin + meta[2] * kChunk, L = min(kChunk, t_end - t0);
+    uint8_t* rec = reinterpret_cast<uint8_t*>(a.workspace) + ((size_t)v * H + h) * kRecBytes;
+
+    // ---- K (rows 0-63) and Q (rows 64-127), raw 16-bit, swizzled; gates --------------------
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int idx = tid + 128 * u, r = idx >> 4, cc = idx & 15, hf = cc >> 3, c8 = cc & 7;
+        const size_t off = ((size_t)(t0 + r) * H + h) * 128 + cc * 8;
+        const uint4 kv = r < L ? ldg16(a.k, off) : make_uint4(0, 0, 0, 0);
+        const uint4 qv = r < L ? ldg16(a.q, off) : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + Cf::OFF_KQ + hf * 16384 + tc::swz_off(r, c8, 128)) = kv;
+        *reinterpret_cast<uint4*>(smem + Cf::OFF_KQ + hf * 16384 + tc::swz_off(r + 64, c8, 128)) = qv;
+    }
+    if (tid < 64) {
+        float gv = tid < L ? a.g[(size_t)(t0 + tid) * H + h] : 0.f;
+        vb[128 + tid] = tid < L ? a.beta[(size_t)(t0 + tid) * H + h] : 0.f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, gv, o);
+            if (lane >= o) gv += y;
+        }
+        vb[tid] = gv;
+    }
+    if (warp == 0) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid >= 32 && tid < 64) vb[tid] += vb[31];
+    __syncthreads();
+    if (tid < 64) {
+        vb[64 + tid] = __expf(vb[tid]);
+        vb[192 + tid] = __expf(vb[tid | 15] - vb[tid]);  // exp(gamma_e - gamma_s), e = end of s's block
+    }
+    tc::fence_async_smem();
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // ---- [K;Q] K^T ---------------------------------------------------------------------------
+    if (tid == 0) {
+        const uint32_t id = a.in_dt == kBF16 ? tc::idesc_bf16(128, 64, false, false) : tc::idesc_f16(128, 64, false, false);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t d = tc::smem_desc(sbase + Cf::OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, tc::kSw128);
+            tc::mma_f16(tmem, d, d, id, kk > 0);
+        }
+        tc::mma_commit(bar);
+    }
+    const bool ok = __syncthreads_and(tc::mbar_wait_bounded(bar, 0, a.budget)) != 0;
+    if (!ok) {
+        if (tid == 0) raise_error(kErrTimeout);
+        tc::mbar_wait_bounded(bar, 0, 4000000000ull);
+    }
+    tc::tc_fence_after();
+
+    if (ok) {
+        // ---- masks: A (fp32) for the solve; M (fp16) straight into the record -------------------
+        {
+            float x[64];
+            const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+            tc::tmem_ld32(trow, x);
+            tc::tmem_ld32(trow + 32, x + 32);
+            const int r = tid & 63, R = r >> 4, rl = r & 15;
+            const float gr = vb[r];
+            const bool isA = tid < 64;
+            float rowf[4], dg[16];
+#pragma unroll
+            for (int S = 0; S < 4; ++S) rowf[S] = S < R ? __expf(gr - vb[16 * S + 15]) : 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) dg[jj] = (isA ? jj < rl : jj <= rl) ? __expf(gr - vb[16 * R + jj]) : 0.f;
+            const float sc = isA ? vb[128 + r] : 1.f;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                float m[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int s = 8 * cc + e, S = s >> 4;
+                    const float f = S < R ? rowf[S] * vb[192 + s] : (S == R ? dg[s & 15] : 0.f);
+                    m[e] = sc * f * x[s];
+                }
+                if (isA) {
+                    sts4(fA + r * LD + 8 * cc, make_float4(m[0], m[1], m[2], m[3]));
+                    sts4(fA + r * LD + 8 * cc + 4, make_float4(m[4], m[5], m[6], m[7]));
+                } else {
+                    *reinterpret_cast<uint4*>(rec + 16384 + tc::swz_off(r, cc, 128)) = pack_f16x8(m);
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- T = (I + A)^-1: 16x16 diagonal blocks by forward substitution (lane = column) -----
+        if (lane < 16) {
+            const int b0 = warp * 16, jc = lane;
+            float xs[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float arow[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 t = lds4(fA + (b0 + r) * LD + b0 + 4 * q4);
+                    arow[4 * q4] = t.x; arow[4 * q4 + 1] = t.y; arow[4 * q4 + 2] = t.z; arow[4 * q4 + 3] = t.w;
+                }
+                float acc = (r == jc) ? 1.f : 0.f;
+#pragma unroll
+                for (int s = 0; s < r; ++s) acc -= arow[s] * xs[s];
+                xs[r] = acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) fT[(b0 + r) * LD + b0 + jc] = xs[r];
+        }
+        __syncthreads();
+        // off-diagonal blocks, d = i - j = 1, 2, 3:  T_ij = -T_ii sum_{m=j}^{i-1} A_im T_mj
+        // work item = (block, row rr, 4-column group cg)
+        for (int d = 1; d < 4; ++d) {
+            const int items = (4 - d) * 64;
+            for (int o = tid; o < items; o += 128) {
+                const int blk = o >> 6, i = d + blk, jb = i - d, rr = (o >> 2) & 15, cg = o & 3;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int m = jb; m < i; ++m) {
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4) {
+                        const float4 av = lds4(fA + (16 * i + rr) * LD + 16 * m + 4 * s4);
+                        const float a4[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float4 t = lds4(fT + (16 * m + 4 * s4 + e) * LD + 16 * jb + 4 * cg);
+                            acc.x += a4[e] * t.x; acc.y += a4[e] * t.y; acc.z += a4[e] * t.z; acc.w += a4[e] * t.w;
+                        }
+                    }
+                }
+                sts4(fZ + (blk * 16 + rr) * 20 + 4 * cg, acc);
+            }
+            __syncthreads();
+            for (int o = tid; o < items; o += 128) {
+                const int blk = o >> 6, i = d + blk, jb = i - d, rr = (o >> 2) & 15, cg = o & 3;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4) {
+                    const float4 tv = lds4(fT + (16 * i + rr) * LD + 16 * i + 4 * s4);
+                    const float t4[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int s = 4 * s4 + e;
+                        const float tt = s <= rr ? t4[e] : 0.f;
+                        const float4 z = lds4(fZ + (blk * 16 + s) * 20 + 4 * cg);
+                        acc.x -= tt * z.x; acc.y -= tt * z.y; acc.z -= tt * z.z; acc.w -= tt * z.w;
+                    }
+                }
+                sts4(fT + (16 * i + rr) * LD + 16 * jb + 4 * cg, acc);
+            }
+            __syncthreads();
+        }
+        // ---- T_w = T diag(beta Gamma) (rows 0-63), T_u = T diag(beta) (rows 64-127) -> record -----
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int idx = tid + 128 * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
+            const float4 t0v = lds4(fT + r * LD + 8 * cc), t1v = lds4(fT + r * LD + 8 * cc + 4);
+            const float4 b0v = lds4(vb + 128 + 8 * cc), b1v = lds4(vb + 128 + 8 * cc + 4);
+            float t8[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+            float s8[8] = {b0v.x, b0v.y, b0v.z, b0v.w, b1v.x, b1v.y, b1v.z, b1v.w};
+            if (which == 0) {
+                const float4 g0v = lds4(vb + 64 + 8 * cc), g1v = lds4(vb + 64 + 8 * cc + 4);
+                s8[0] *= g0v.x; s8[1] *= g0v.y; s8[2] *= g0v.z; s8[3] *= g0v.w;
+                s8[4] *= g1v.x; s8[5] *= g1v.y; s8[6] *= g1v.z; s8[7] *= g1v.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t8[e] = (8 * cc + e <= r) ? t8[e] * s8[e] : 0.f;
+            *reinterpret_cast<uint4*>(rec + which * 8192 + tc::swz_off(r, cc, 128)) = pack_f16x8(t8);
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, Cf::TMEM_COLS);
+    }
+}
+
+// =====================================================================================
+// chunk_chain_kernel: per (sequence, head, dv slab) -- the sequential pass over chunks
+// =====================================================================================
+
+template <int NS>
+struct ChainCfg {
+    static constexpr int ROWB = NS * 2;                      // bytes per row of a slab tile (fp16)
+    static constexpr uint32_t SWZ = NS == 32 ? tc::kSw64 : tc::kSw128;
+    static constexpr int XREG = 192 * 128;                    // one K-half region of [K;Q;W]
+    static constexpr int OFF_X = 0;                           // [2] [K;Q;W] fp16: 2 x [192 x 128 B]
+    static constexpr int OFF_TT = OFF_X + 2 * 2 * XREG;       // [T_w; T_u]: [128 x 128 B]
+    static constexpr int OFF_M = OFF_TT + 16384;              // [2] M: [64 x 128 B]
+    static constexpr int OFF_STG = OFF_M + 2 * 8192;          // staging (raw rows + record)
+    static constexpr int STG_Q = 16384, STG_V = 32768, STG_REC = STG_V + 64 * ROWB;
+    static constexpr int STG_BYTES = STG_REC + kRecBytes;
+    static constexpr int OFF_VS = OFF_STG + STG_BYTES;        // [2] V slab fp16 [64 x ROWB]
+    static constexpr int OFF_SS = OFF_VS + 2 * 64 * ROWB;     // S operand [128 x ROWB]
+    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;        // U operand [64 x ROWB]
+    static constexpr int OFF_SU2 = OFF_SU + 64 * ROWB;        // U' = diag(Gamma_C/Gamma) U
+    static constexpr int OFF_YS = OFF_SU2 + 64 * ROWB;        // y rows for bulk stores [64 x NS x 4 B]
+    static constexpr int OFF_VEC = OFF_YS + 64 * NS * 4;      // [2] gamma, Gamma, f: 3 x 64 floats (1 KB)
+    static constexpr int OFF_META = OFF_VEC + 2 * 1024;       // [2] {c0, L}
+    static constexpr int OFF_BAR = OFF_META + 64;
+    static constexpr int BYTES = OFF_BAR + 128 + 1024;
+    static constexpr uint32_t COL_UT = 0;                     // [2] x NS (rows 64-127)
+    static constexpr uint32_t COL_W = 2 * NS;                 // 128 (rows 0-63)
+    static constexpr uint32_t COL_1 = COL_W + 128;            // NS
+    static constexpr uint32_t COL_MU = COL_1 + NS;            // NS (rows 0-63)
+    static constexpr uint32_t COL_DS = COL_MU + NS;           // NS
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(COL_DS + NS <= TMEM_COLS, "TMEM budget");
+    static_assert(BYTES <= 232448, "shared memory budget");
+};
+
+template <int NS>
+__global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a) {
+    using Cf = ChainCfg<NS>;
+    constexpr int NSLAB = 128 / NS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = tc::smem_u32(smem);
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
-    uint64_t* bar_i = bars + 0;      // intra-issued MMAs complete
+    uint64_t* bar_p = bars + 0;      // producer-issued MMAs complete
     uint64_t* bar_c = bars + 1;      // chain-issued MMAs complete
-    uint64_t* bar_full = bars + 2;   // [2] slot filled by the intra group
-    uint64_t* bar_empty = bars + 4;  // [2] slot released by the chain group
+    uint64_t* bar_full = bars + 2;   // [2] slot filled by the producer
+    uint64_t* bar_empty = bars + 4;  // [2] slot released by the chain
+    uint64_t* bar_stage = bars + 6;  // staging landed (bulk-copy bytes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 64);
+    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 72);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slab = blockIdx.x % NSLAB;
@@ -156,23 +433,26 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
     const int H = a.H;
     int t_begin, t_end;
     seq_bounds(a.cu, n, a.num_seqs, a.N, t_begin, t_end);
-    const int nchunks = (t_end - t_begin + C - 1) / C;
+    const int nchunks = (t_end - t_begin + kChunk - 1) / kChunk;
 
+    if (warp == 0) {
+        const int base = chunks_before(a.cu, a.num_seqs, a.N, n);
+        if (lane == 0) *s_base = base;
+    }
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < 7; ++i) tc::mbar_init(bars + i, 1);
         tc::fence_mbar_init();
     }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
+    if (warp == 1) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lanes
-
+    const int rec_base = *s_base;
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     auto vec = [&](int b) { return reinterpret_cast<float*>(smem + Cf::OFF_VEC + b * 1024); };
-    auto Xoff = [&](int b) { return Cf::OFF_X + b * 32768; };
-    auto TMoff = [&](int b) { return Cf::OFF_TM + b * 24576; };
-    auto KGoff = [&](int b) { return Cf::OFF_KG + b * 16384; };
+    auto Xoff = [&](int b) { return Cf::OFF_X + b * 2 * Cf::XREG; };
+    uint8_t* stg = smem + Cf::OFF_STG;
 
     if (warp < 4) {
         // =============================== chain group ===================================
@@ -198,7 +478,8 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
         };
         const uint32_t id_slab = tc::idesc_f16(128, NS, false, true);
         const uint32_t id_ds = tc::idesc_f16(128, NS, true, true);
-        const uint32_t sSS = sbase + Cf::OFF_SS, sSU = sbase + Cf::OFF_SU;
+        const uint32_t sSS = sbase + Cf::OFF_SS, sSU = sbase + Cf::OFF_SU, sSU2 = sbase + Cf::OFF_SU2;
+        const int ybytes = a.y_dt == kF32 ? 4 : 2;
 
         const size_t st_base = ((size_t)n * H + h) * 128 * 128 + (size_t)tid * 128 + slab * NS;
         float S[NS];
@@ -212,7 +493,18 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
             *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB)) = pack_f16x8(S + 8 * c);
         operands_ready();
 
-        float keep[NS];  // rows 64-127: (Q S) row
+        int ys_c0 = -1, ys_L = 0;  // y rows staged in YS, not yet stored
+        auto flush_y = [&]() {     // warp 0 issues one bulk store per valid staged row
+            if (warp == 0 && ys_c0 >= 0) {
+                for (int r = lane; r < ys_L; r += 32)
+                    tc::bulk_s2g(reinterpret_cast<uint8_t*>(a.y) + (((size_t)(ys_c0 + r) * H + h) * 128 + slab * NS) * ybytes,
+                                 smem + Cf::OFF_YS + r * NS * ybytes, NS * ybytes);
+                tc::bulk_commit();
+            }
+            ys_c0 = -1;
+        };
+
+        float qs[NS];  // rows 0-63: (Q S) row
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (!(ok = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget)))) {
@@ -220,74 +512,78 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
                 break;
             }
             tc::tc_fence_after();
-            const float* vb = vec(b);
+            const float* vb = vec(b);  // gamma[0:64] Gamma[64:128] f[128:192]
             const int c0 = meta[2 * b], L = meta[2 * b + 1];
             const float gC = vb[64 + 63];
-            const float gR = tid >= 64 ? vb[64 + tid - 64] : 0.f;
-            const uint32_t sX = sbase + Xoff(b), sTM = sbase + TMoff(b), sKG = sbase + KGoff(b);
+            const float gR = tid < 64 ? vb[64 + tid] : 0.f;
+            const float fR = tid >= 64 ? vb[128 + tid - 64] : 0.f;
+            const uint32_t sX = sbase + Xoff(b), sM = sbase + Cf::OFF_M + b * 8192;
 
-            // [W;Q] S
+            // [Q;W] S  -> Q S (rows 0-63), W S (rows 64-127)
             if (tid == 0) {
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t aw = tc::smem_desc(sX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, tc::kSw128);
+                    const uint64_t aw = tc::smem_desc(sX + (kk >> 2) * Cf::XREG + 64 * 128 + (kk & 3) * 32, 16, 1024, tc::kSw128);
                     const uint64_t bs = tc::smem_desc(sSS + kk * 16 * Cf::ROWB, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
                     tc::mma_f16(tmem + Cf::COL_1, aw, bs, id_slab, kk > 0);
                 }
             }
+            flush_y();  // the previous chunk's y rows leave while the MMA runs
             if (!(ok = commit_wait())) break;
 
-            // U = U~ - W S (rows 0-63) ; Q S kept (rows 64-127)
             {
                 float d1[NS];
 #pragma unroll
                 for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_1 + 32 * q4, d1 + 32 * q4);
-                if (warp < 2) {
+                if (warp >= 2) {  // U = U~ - W S, U' = f U
+                    const int r = tid - 64;
                     float ut[NS];
 #pragma unroll
-                    for (int q4 = 0; q4 < NS / 32; ++q4)
-                        tc::tmem_ld32(trow + Cf::COL_UT + b * NS + 32 * q4, ut + 32 * q4);
+                    for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_UT + b * NS + 32 * q4, ut + 32 * q4);
 #pragma unroll
                     for (int j = 0; j < NS; ++j) ut[j] -= d1[j];
 #pragma unroll
-                    for (int cc = 0; cc < NS / 8; ++cc)
-                        *reinterpret_cast<uint4*>(smem + Cf::OFF_SU + tc::swz_off(tid, cc, Cf::ROWB)) =
-                            pack_f16x8(ut + 8 * cc);
+                    for (int cc = 0; cc < NS / 8; ++cc) {
+                        *reinterpret_cast<uint4*>(smem + Cf::OFF_SU + tc::swz_off(r, cc, Cf::ROWB)) = pack_f16x8(ut + 8 * cc);
+                        float u2[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
+                        *reinterpret_cast<uint4*>(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::ROWB)) = pack_f16x8(u2);
+                    }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < NS; ++j) keep[j] = d1[j];
+                    for (int j = 0; j < NS; ++j) qs[j] = d1[j];
                 }
             }
+            if (warp == 0) tc::bulk_wait_read0();  // YS may be rewritten below
             operands_ready();
 
-            // M U (rows 64-127) and Kg^T U
+            // [M;.] U -> M U (rows 0-63) ;  K^T U' -> state increment
             if (tid == 0) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bu = tc::smem_desc(sSU + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-                    const uint64_t am = tc::smem_desc(sTM + 64 * 128 + kk * 32, 16, 1024, tc::kSw128);
+                    const uint64_t am = tc::smem_desc(sM + kk * 32, 16, 1024, tc::kSw128);
                     tc::mma_f16(tmem + Cf::COL_MU, am, bu, id_slab, kk > 0);
-                    const uint64_t ak = tc::smem_desc(sKG + kk * 2048, 8192, 1024, tc::kSw128);
-                    tc::mma_f16(tmem + Cf::COL_DS, ak, bu, id_ds, kk > 0);
+                    const uint64_t bu2 = tc::smem_desc(sSU2 + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
+                    const uint64_t ak = tc::smem_desc(sX + kk * 2048, Cf::XREG, 1024, tc::kSw128);
+                    tc::mma_f16(tmem + Cf::COL_DS, ak, bu2, id_ds, kk > 0);
                 }
             }
             if (!(ok = commit_wait())) break;
-            if (tid == 0) tc::mbar_arrive(bar_empty + b);  // slot b (smem and U~ columns) is free
+            if (tid == 0) tc::mbar_arrive(bar_empty + b);  // slot b (X, M, U~ columns) is free
 
             {
                 float t[NS];
-                if (warp >= 2) {
-                    const int r = tid - 64;
+                if (warp < 2) {  // y = scale (Gamma_r (Q S) + M U) -> YS
 #pragma unroll
                     for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_MU + 32 * q4, t + 32 * q4);
-                    if (r < L) {
-                        const size_t yoff = ((size_t)(c0 + r) * H + h) * 128 + slab * NS;
+                    if (tid < L) {
 #pragma unroll
                         for (int j = 0; j < NS; j += 4)
-                            st4(a.y, a.y_dt, yoff + j,
-                                make_float4(a.scale * (gR * keep[j] + t[j]), a.scale * (gR * keep[j + 1] + t[j + 1]),
-                                            a.scale * (gR * keep[j + 2] + t[j + 2]),
-                                            a.scale * (gR * keep[j + 3] + t[j + 3])));
+                            st4(smem + Cf::OFF_YS + tid * NS * ybytes, a.y_dt, j,
+                                make_float4(a.scale * (gR * qs[j] + t[j]), a.scale * (gR * qs[j + 1] + t[j + 1]),
+                                            a.scale * (gR * qs[j + 2] + t[j + 2]), a.scale * (gR * qs[j + 3] + t[j + 3])));
                     }
                 }
 #pragma unroll
@@ -298,88 +594,93 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
                 for (int cc = 0; cc < NS / 8; ++cc)
                     *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB)) = pack_f16x8(S + 8 * cc);
             }
+            ys_c0 = c0;
+            ys_L = L;
             operands_ready();
         }
+        if (ok) flush_y();
+        if (warp == 0) tc::bulk_wait0();
         if (ok && a.S_T) {
 #pragma unroll
             for (int j = 0; j < NS; j += 4)
                 *reinterpret_cast<float4*>(a.S_T + st_base + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     } else {
-        // =============================== intra group ===================================
+        // =============================== producer group ================================
         constexpr int BID = 2;
         const int it = tid - 128;
         uint32_t ph = 0;
         bool ok = true;
-        auto commit_wait = [&]() -> bool {
-            if (it == 0) tc::mma_commit(bar_i);
-            bool w = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_i, ph, a.budget));
-            if (!w) {
-                if (it == 0) raise_error(kErrTimeout);
-                tc::mbar_wait_bounded(bar_i, ph, 4000000000ull);
-            }
-            ph ^= 1u;
-            tc::tc_fence_after();
-            return w;
-        };
-        auto operands_ready = [&]() {
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::bar_sync(BID, 128);
-            tc::tc_fence_after();
-        };
-        const uint32_t id_qk = tc::idesc_f16(128, 64, false, false);
         const uint32_t id_slab = tc::idesc_f16(128, NS, false, true);
         const uint32_t id_w = tc::idesc_f16(128, 128, false, true);
-        const uint32_t sVS = sbase + Cf::OFF_VS;
+        const uint32_t sTT = sbase + Cf::OFF_TT;
 
-        // register prefetch of one chunk's inputs (issued a chunk ahead of use)
-        uint4 pk[8], pq[8], pv[VU];
+        // bulk copies of chunk ci's rows and record into staging (warp 4)
+        auto issue_loads = [&](int ci) {
+            if (warp != 4) return;
+            const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
+            if (lane == 0) tc::mbar_arrive_expect_tx(bar_stage, (uint32_t)(L * (512 + Cf::ROWB) + kRecBytes));
+            __syncwarp();
+            for (int r = lane; r < L; r += 32) {
+                const size_t row = (size_t)(c0 + r) * H + h;
+                tc::bulk_g2s(stg + r * 256, reinterpret_cast<const uint16_t*>(a.k) + row * 128, 256, bar_stage);
+                tc::bulk_g2s(stg + Cf::STG_Q + r * 256, reinterpret_cast<const uint16_t*>(a.q) + row * 128, 256, bar_stage);
+                tc::bulk_g2s(stg + Cf::STG_V + r * Cf::ROWB, reinterpret_cast<const uint16_t*>(a.v) + row * 128 + slab * NS,
+                             Cf::ROWB, bar_stage);
+            }
+            if (lane == 0)
+                tc::bulk_g2s(stg + Cf::STG_REC,
+                             reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes,
+                             kRecBytes, bar_stage);
+        };
         float pg = 0.f, pb = 0.f;
-        auto prefetch = [&](int ci) {
-            const int c0 = t_begin + ci * C, L = min(C, t_end - c0);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int idx = it + 128 * u, r = idx >> 4, cc = idx & 15;
-                const size_t off = ((size_t)(c0 + r) * H + h) * 128 + cc * 8;
-                pk[u] = r < L ? ldg16(a.k, off) : make_uint4(0, 0, 0, 0);
-                pq[u] = r < L ? ldg16(a.q, off) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < VU; ++u) {
-                const int idx = it + 128 * u, r = idx / (NS / 8), cc = idx % (NS / 8);
-                pv[u] = r < L ? ldg16(a.v, ((size_t)(c0 + r) * H + h) * 128 + slab * NS + cc * 8) : make_uint4(0, 0, 0, 0);
-            }
+        auto load_gates = [&](int ci) {
+            const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
             if (it < 64) {
                 pg = it < L ? a.g[(size_t)(c0 + it) * H + h] : 0.f;
                 pb = it < L ? a.beta[(size_t)(c0 + it) * H + h] : 0.f;
             }
         };
-        if (nchunks > 0) prefetch(0);
+        if (nchunks > 0) {
+            issue_loads(0);
+            load_gates(0);
+        }
 
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
-            const int c0 = t_begin + c * C, L = min(C, t_end - c0);
-            float* vb = vec(b);  // gamma[0:64] Gamma[64:128] beta[128:192] colf[192:256]
-            const uint32_t sX = sbase + Xoff(b), sTM = sbase + TMoff(b);
-            // the chain group must be done with this slot (chunk c-2)
-            if (!(ok = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_empty + b, ((c >> 1) & 1) ^ 1, a.budget)))) {
+            const int c0 = t_begin + c * kChunk, L = min(kChunk, t_end - c0);
+            float* vb = vec(b);
+            // slot b must be free (chain done with chunk c-2) and staging must hold chunk c
+            bool w = tc::mbar_wait_bounded(bar_empty + b, ((c >> 1) & 1) ^ 1, a.budget);
+            w = w && tc::mbar_wait_bounded(bar_stage, c & 1, a.budget);
+            if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (it == 0) raise_error(kErrTimeout);
                 break;
             }
             tc::tc_fence_after();
 
-            // ---- operand tiles from the prefetched registers; gates ------------------------
+            // ---- fp16 operand tiles: K, Q rows of [K;Q;W], V slab; the record -------------------
+            uint8_t* X = smem + Xoff(b);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int idx = it + 128 * u, r = idx >> 4, cc = idx & 15, hf = cc >> 3, c8 = cc & 7;
-                *reinterpret_cast<uint4*>(smem + Xoff(b) + hf * 16384 + tc::swz_off(r, c8, 128)) = to_f16x8(pk[u], a.in_dt);
-                *reinterpret_cast<uint4*>(smem + Xoff(b) + hf * 16384 + tc::swz_off(r + 64, c8, 128)) = to_f16x8(pq[u], a.in_dt);
+            for (int u = 0; u < 16; ++u) {
+                const int idx = it + 128 * u, which = idx >> 10, r = (idx >> 4) & 63, cc = idx & 15;
+                uint4 val = make_uint4(0, 0, 0, 0);
+                if (r < L) val = to_f16x8(*reinterpret_cast<const uint4*>(stg + which * Cf::STG_Q + r * 256 + cc * 16), a.in_dt);
+                *reinterpret_cast<uint4*>(X + (cc >> 3) * Cf::XREG + tc::swz_off(which * 64 + r, cc & 7, 128)) = val;
             }
 #pragma unroll
-            for (int u = 0; u < VU; ++u) {
+            for (int u = 0; u < (64 * NS / 8) / 128; ++u) {
                 const int idx = it + 128 * u, r = idx / (NS / 8), cc = idx % (NS / 8);
-                *reinterpret_cast<uint4*>(smem + Cf::OFF_VS + tc::swz_off(r, cc, Cf::ROWB)) = to_f16x8(pv[u], a.in_dt);
+                uint4 val = make_uint4(0, 0, 0, 0);
+                if (r < L) val = to_f16x8(*reinterpret_cast<const uint4*>(stg + Cf::STG_V + r * Cf::ROWB + cc * 16), a.in_dt);
+                *reinterpret_cast<uint4*>(smem + Cf::OFF_VS + b * 64 * Cf::ROWB + tc::swz_off(r, cc, Cf::ROWB)) = val;
+            }
+#pragma unroll
+            for (int u = 0; u < 12; ++u) {
+                const int idx = it + 128 * u;  // 16-byte piece of the record
+                const uint4 val = *reinterpret_cast<const uint4*>(stg + Cf::STG_REC + idx * 16);
+                uint8_t* dst = idx < 1024 ? smem + Cf::OFF_TT + idx * 16 : smem + Cf::OFF_M + b * 8192 + (idx - 1024) * 16;
+                *reinterpret_cast<uint4*>(dst) = val;
             }
             if (it < 64) {
                 float gv = pg;
@@ -389,163 +690,58 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
                     if (lane >= o) gv += y;
                 }
                 vb[it] = gv;
-                vb[128 + it] = pb;
             }
             if (it == 0) {
                 meta[2 * b] = c0;
                 meta[2 * b + 1] = L;
             }
-            if (c + 1 < nchunks) prefetch(c + 1);  // next chunk's loads overlap this chunk's work
+            tc::fence_async_smem();  // staging reads precede the next bulk copies into it
             tc::bar_sync(BID, 128);
+            if (c + 1 < nchunks) issue_loads(c + 1);
             if (it >= 32 && it < 64) vb[it] += vb[31];
             tc::bar_sync(BID, 128);
             if (it < 64) {
-                vb[64 + it] = expf(vb[it]);
-                vb[192 + it] = expf(vb[(it | 15)] - vb[it]);  // exp(gamma_e - gamma_s), e = end of s's block
+                vb[64 + it] = __expf(vb[it]);
+                vb[128 + it] = __expf(vb[63] - vb[it]);
             }
-            operands_ready();
-
-            // ---- [K;Q] K^T -------------------------------------------------------------------
-            if (it == 0) {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t d = tc::smem_desc(sX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, tc::kSw128);
-                    tc::mma_f16(tmem + Cf::COL_QK, d, d, id_qk, kk > 0);
-                }
-            }
-            if (!(ok = commit_wait())) break;
-
-            // ---- masks: A (fp32) for the solve, M (fp16 operand); Kg -----------------------------
-            {
-                float x[64];
-                tc::tmem_ld32(trow + Cf::COL_QK, x);
-                tc::tmem_ld32(trow + Cf::COL_QK + 32, x + 32);
-                const int r = it & 63, R = r >> 4, rl = r & 15;
-                const float gr = vb[r];
-                const bool isA = it < 64;
-                float rowf[4], dg[16];
-#pragma unroll
-                for (int S = 0; S < 4; ++S) rowf[S] = S < R ? expf(gr - vb[16 * S + 15]) : 0.f;
-#pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    dg[j] = (isA ? j < rl : j <= rl) ? expf(gr - vb[16 * R + j]) : 0.f;
-                const float* colf = vb + 192;
-                if (isA) {
-                    const float br = vb[128 + r];
-#pragma unroll
-                    for (int s = 0; s < 64; ++s) {
-                        const int S = s >> 4;
-                        const float f = S < R ? rowf[S] * colf[s] : (S == R ? dg[s & 15] : 0.f);
-                        fA[r * 65 + s] = br * f * x[s];
-                    }
-                } else {
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        float m[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int s = 8 * cc + e, S = s >> 4;
-                            const float f = S < R ? rowf[S] * colf[s] : (S == R ? dg[s & 15] : 0.f);
-                            m[e] = f * x[s];
-                        }
-                        *reinterpret_cast<uint4*>(smem + TMoff(b) + tc::swz_off(128 + r, cc, 128)) = pack_f16x8(m);
-                    }
-                }
-                const float gl = vb[63];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int idx = it + 128 * u, rr = idx >> 4, cc = idx & 15, hf = cc >> 3, c8 = cc & 7;
-                    float kx[8];
-                    unpack_f16x8(*reinterpret_cast<const uint4*>(smem + Xoff(b) + hf * 16384 + tc::swz_off(rr, c8, 128)), kx);
-                    const float f = expf(gl - vb[rr]);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) kx[e] *= f;
-                    *reinterpret_cast<uint4*>(smem + KGoff(b) + hf * 8192 + tc::swz_off(rr, c8, 128)) = pack_f16x8(kx);
-                }
-            }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
             tc::bar_sync(BID, 128);
+            tc::tc_fence_after();
 
-            // ---- T = (I + A)^-1: 16x16 diagonal blocks by forward substitution ----------------
-            {
-                const int w4 = warp - 4;
-                if (lane < 16) {
-                    const int b0 = w4 * 16, j = lane;
-                    float xs[16];
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float acc = (r == j) ? 1.f : 0.f;
-#pragma unroll
-                        for (int s = 0; s < r; ++s) acc -= fA[(b0 + r) * 65 + b0 + s] * xs[s];
-                        xs[r] = acc;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) fT[(b0 + r) * 65 + b0 + j] = xs[r];
-                }
-            }
-            tc::bar_sync(BID, 128);
-            // off-diagonal blocks, d = i - j = 1, 2, 3:  T_ij = -T_ii sum_{m=j}^{i-1} A_im T_mj
-            for (int d = 1; d < 4; ++d) {
-                const int nblk = 4 - d;
-                for (int o = it; o < nblk * 256; o += 128) {
-                    const int blk = o >> 8, i = d + blk, j = i - d, e = o & 255, rr = e >> 4, cc = e & 15;
-                    float acc = 0.f;
-                    for (int m = j; m < i; ++m) {
-#pragma unroll
-                        for (int s = 0; s < 16; ++s) acc += fA[(16 * i + rr) * 65 + 16 * m + s] * fT[(16 * m + s) * 65 + 16 * j + cc];
-                    }
-                    fZ[(blk * 16 + rr) * 17 + cc] = acc;
-                }
-                tc::bar_sync(BID, 128);
-                for (int o = it; o < nblk * 256; o += 128) {
-                    const int blk = o >> 8, i = d + blk, j = i - d, e = o & 255, rr = e >> 4, cc = e & 15;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int s = 0; s < 16; ++s)
-                        if (s <= rr) acc -= fT[(16 * i + rr) * 65 + 16 * i + s] * fZ[(blk * 16 + s) * 17 + cc];
-                    fT[(16 * i + rr) * 65 + 16 * j + cc] = acc;
-                }
-                tc::bar_sync(BID, 128);
-            }
-            // T_u = T diag(beta), T_w = T diag(beta Gamma): fp16 rows 0-63 / 64-127 of [T_u; T_w; M]
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int idx = it + 128 * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
-                float t8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s = 8 * cc + e;
-                    const float sc = which ? vb[128 + s] * vb[64 + s] : vb[128 + s];
-                    t8[e] = s <= r ? fT[r * 65 + s] * sc : 0.f;
-                }
-                *reinterpret_cast<uint4*>(smem + TMoff(b) + tc::swz_off(which * 64 + r, cc, 128)) = pack_f16x8(t8);
-            }
-            operands_ready();
-
-            // ---- U~ = T_u V_slab (into this slot's TMEM columns) and W = T_w K ------------------
+            // ---- U~ = T_u V (rows 64-127 of this slot's columns) and W = T_w K (rows 0-63) ------
             if (it == 0) {
+                const uint32_t sV = sbase + Cf::OFF_VS + b * 64 * Cf::ROWB, sXb = sbase + Xoff(b);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t at = tc::smem_desc(sTM + kk * 32, 16, 1024, tc::kSw128);
-                    const uint64_t bv = tc::smem_desc(sVS + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
+                    const uint64_t at = tc::smem_desc(sTT + kk * 32, 16, 1024, tc::kSw128);
+                    const uint64_t bv = tc::smem_desc(sV + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
                     tc::mma_f16(tmem + Cf::COL_UT + b * NS, at, bv, id_slab, kk > 0);
-                    const uint64_t bk = tc::smem_desc(sX + kk * 2048, 16384, 1024, tc::kSw128);
+                    const uint64_t bk = tc::smem_desc(sXb + kk * 2048, Cf::XREG, 1024, tc::kSw128);
                     tc::mma_f16(tmem + Cf::COL_W, at, bk, id_w, kk > 0);
                 }
+                tc::mma_commit(bar_p);
             }
-            if (!(ok = commit_wait())) break;
+            w = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_p, ph, a.budget));
+            if (!w) {
+                if (it == 0) raise_error(kErrTimeout);
+                tc::mbar_wait_bounded(bar_p, ph, 4000000000ull);
+            }
+            ph ^= 1u;
+            tc::tc_fence_after();
+            if (!(ok = w)) break;
 
-            // ---- W -> rows 0-63 of this slot's [W;Q] ----------------------------------------------
-            if (it >= 64) {
-                const int r = it - 64;
+            // ---- W -> rows 128-191 of [K;Q;W] ----------------------------------------------------
+            if (it < 64) {
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    float w[32];
-                    tc::tmem_ld32(trow + Cf::COL_W + 32 * q4, w);
+                    float wv[32];
+                    tc::tmem_ld32(trow + Cf::COL_W + 32 * q4, wv);
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
                         const int ch = q4 * 4 + cc;
-                        *reinterpret_cast<uint4*>(smem + Xoff(b) + (ch >> 3) * 16384 + tc::swz_off(r, ch & 7, 128)) =
-                            pack_f16x8(w + 8 * cc);
+                        *reinterpret_cast<uint4*>(X + (ch >> 3) * Cf::XREG + tc::swz_off(128 + it, ch & 7, 128)) =
+                            pack_f16x8(wv + 8 * cc);
                     }
                 }
             }
@@ -553,39 +749,39 @@ __global__ void __launch_bounds__(256, 1) chunk_fwd_tc_kernel(const __grid_const
             tc::tc_fence_before();
             tc::bar_sync(BID, 128);
             if (it == 0) tc::mbar_arrive(bar_full + b);  // hand slot b to the chain group
+            if (c + 1 < nchunks) load_gates(c + 1);
         }
         (void)ok;
     }
 
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, Cf::TMEM_COLS);
     }
 }
 
-template <int NS>
-inline cudaError_t launch_chunk_tc(const ChunkArgs& a, cudaStream_t st) {
-    using Cf = TcCfg<NS>;
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::BYTES);
-    if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(a.num_seqs * a.H * (128 / NS));
-    chunk_fwd_tc_kernel<NS><<<grid, 256, Cf::BYTES, st>>>(a);
-    return cudaGetLastError();
-}
-
 inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const char** why) {
     *why = nullptr;
-    if (a.chunk != 64) {
+    if (a.chunk != kChunk) {
         *why = "only chunk = 64 is built";
         return cudaSuccess;
     }
-    // 32-column slabs give 4 CTAs per (sequence, head); use 64-column slabs when that
-    // would not fit the GPU's 148 SMs in one wave.
-    const long long units = (long long)a.num_seqs * a.H;
-    if (units * 4 <= 148) return launch_chunk_tc<32>(a, st);
-    return launch_chunk_tc<64>(a, st);
+    constexpr int NS = 32;
+    using Ch = ChainCfg<NS>;
+    cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, UtCfg::BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_chain_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
+    if (e != cudaSuccess) return e;
+    const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
+    if (nvc > 0) {
+        chunk_ut_kernel<<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    chunk_chain_kernel<NS><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace gdn

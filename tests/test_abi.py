@@ -56,6 +56,7 @@ def chunk_call(L, **over):
 @pytest.mark.parametrize("over", [
     dict(q=None), dict(k=MIS), dict(dk=48), dict(dv=256), dict(chunk=32), dict(chunk=-1), dict(N=-1),
     dict(H=0), dict(num_seqs=0), dict(N=63), dict(in_dt=7), dict(y_dt=-1), dict(S0=MIS),
+    dict(ws_bytes=0, ws=None),
 ])
 def test_chunk_fwd_rejects_bad_arguments(L, over):
     assert chunk_call(L, **over) == gdn.GDN_ERR_INVALID_ARG
@@ -65,6 +66,13 @@ def test_chunk_fwd_rejects_bad_arguments(L, over):
 @pytest.mark.parametrize("over", [dict(dk=64, dv=64), dict(in_dt=gdn.F32), dict(dk=128, dv=64)])
 def test_chunk_fwd_tensor_core_path_limits(L, over):
     assert chunk_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_workspace_size_covers_every_chunk(L):
+    # one 24 KB record per (64-token chunk, head); packed sequences add one partial chunk each
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 24576
+    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 24576
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0
 
 
 def test_zero_tokens_is_a_no_op(L):
