@@ -133,6 +133,37 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
                            void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate device memory.
+ * (An addition of this library; the paper has no counterpart.)
+ *
+ * Some callers cannot obtain scratch memory at call time: a serving loop whose device
+ * memory is fixed at start-up, a plugin whose host process owns every device
+ * allocation, or code on a path where cudaMalloc's implicit device synchronisation is
+ * not acceptable.  This entry point takes the same arguments as gdn_chunk_fwd minus the
+ * workspace, and uses instead a scratch array of GDN_NOALLOC_SCRATCH_BYTES (64 MiB)
+ * that is part of the library's device image: every GPU that loads the library holds
+ * it until the process exits.  It calls no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *   - A call whose scratch need, gdn_chunk_fwd_workspace_size(N, num_seqs, H, dk, dv,
+ *     chunk), exceeds GDN_NOALLOC_SCRATCH_BYTES returns GDN_ERR_INVALID_ARG with the
+ *     two sizes in gdn_last_error_message().  (chunk = 0 needs no scratch.)
+ *   - The first call on a device looks up that device's address of the array
+ *     (cudaGetSymbolAddress) with the device current; make that first call before any
+ *     stream capture.  Later calls reuse the address.
+ *   - All calls share the one array, which keeps the last call's contents; every
+ *     record a call reads was written earlier in the same call, so nothing needs
+ *     clearing.  Calls that overlap on the GPU (different streams, or devices sharing
+ *     a context) race on the array and give undefined results: serialise them.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (64ull << 20)
+
+gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g,
+                                   const float* beta, const float* S0, const int32_t* cu_seqlens,
+                                   int num_seqs, int N, int H, int dk, int dv, int chunk,
+                                   float scale, gdn_dtype_t in_dtype, gdn_dtype_t y_dtype,
+                                   void* y, float* S_T, gdn_stream_t stream);
+
+/*
  * gdn_decode_step -- one token per row against a resident state, eqs. (1)-(4):
  *   S <- alpha S + beta k e^T with e = v - alpha S^T k, y = scale * S^T q (new S).
  *   q, k [B,H,dk], v [B,H,dv]: in_dtype.  g, beta [B,H] fp32.

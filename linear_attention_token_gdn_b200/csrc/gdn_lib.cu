@@ -4,6 +4,7 @@
 // Every entry point validates on the host and returns before enqueuing anything when an
 // argument is wrong; it never synchronises and never allocates.
 #include <atomic>
+#include <mutex>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -131,6 +132,30 @@ struct PrepLaunch {
     }
 };
 
+// Scratch of gdn_chunk_fwd_noalloc: part of the device image, one copy per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[256] = {};  // device address of g_noalloc_scratch, per device ordinal
+
+// Device address of the scratch array on the current device; looked up once per device.
+gdn_status_t noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 256) return fail(GDN_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -221,6 +246,23 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     if (why) return fail(GDN_ERR_CUDA, "chunk_tc: %s", why);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "chunk_tc: %s", cudaGetErrorString(e));
     return GDN_OK;
+}
+
+gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                   const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
+                                   int dv, int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t y_dtype, void* y,
+                                   float* S_T, gdn_stream_t stream) {
+    const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+    if (need > GDN_NOALLOC_SCRATCH_BYTES)
+        return fail(GDN_ERR_INVALID_ARG, "needs %zu bytes of scratch; the no-allocation entry point holds %llu",
+                    need, (unsigned long long)GDN_NOALLOC_SCRATCH_BYTES);
+    void* ws = nullptr;
+    if (need > 0) {
+        const gdn_status_t st = noalloc_scratch(&ws);
+        if (st != GDN_OK) return st;
+    }
+    return gdn_chunk_fwd(q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, dk, dv, chunk, scale, in_dtype, y_dtype, y,
+                         S_T, ws, need, stream);
 }
 
 gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,

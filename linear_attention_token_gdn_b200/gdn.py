@@ -33,6 +33,7 @@ SIGNATURES = {
     "gdn_chunk_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
     "gdn_chunk_fwd": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P,
                        _Z, _P], _I),
+    "gdn_chunk_fwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P], _I),
     "gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
 }
@@ -156,6 +157,27 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=None, chunk=6
                                num_seqs, N, H, dk, dv, int(chunk), float(scale), _dt(q), _DT[y.dtype], _ptr(y),
                                _ptr(S_T), _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                _stream(stream)))
+    return y, S_T
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=None, chunk=64, scale=1.0,
+                      y_dtype=None, final_state=True, y=None, S_T=None, stream=None):
+    """gdn_chunk_fwd_noalloc: gdn_chunk_fwd with the library's built-in scratch instead of a
+    caller workspace (for callers that cannot allocate device memory).  Returns (y, S_T)."""
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    elif num_seqs is None:
+        num_seqs = 1
+    y_dtype = q.dtype if y_dtype is None else y_dtype
+    if y is None:
+        y = torch.empty(N, H, dv, device=q.device, dtype=y_dtype)
+    if S_T is None and final_state:
+        S_T = torch.empty(num_seqs, H, dk, dv, device=q.device, dtype=torch.float32)
+    _check(lib().gdn_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                                       num_seqs, N, H, dk, dv, int(chunk), float(scale), _dt(q), _DT[y.dtype],
+                                       _ptr(y), _ptr(S_T), _stream(stream)))
     return y, S_T
 
 
