@@ -21,21 +21,24 @@
 //                       (chunk, head): T_w = T diag(beta Gamma), T_u = T diag(beta) and M,
 //                       fp16, already in the 128B-swizzled operand layout.
 //   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
-//                       the chunks.  A producer warpgroup bulk-copies the next chunk's
-//                       K, Q, V rows and record into staging, converts them to fp16
-//                       operand tiles and computes W = T_w K and U~ = T_u V on the tensor
-//                       cores; a chain warpgroup carries the fp32 state (one row per
+//                       the chunks.  A producer warpgroup brings the next chunk's K, Q and
+//                       V tiles in with TMA and its record with a bulk copy, converts them
+//                       to fp16 operand tiles and computes W = T_w K and U~ = T_u V on the
+//                       tensor cores; a chain warpgroup carries the fp32 state (one row per
 //                       thread) through two dependent tensor-core round trips per chunk:
 //                           [Q;W] S                  -> Q S, W S;  U = U~ - W S
 //                           [M;.] U  and  K^T U'     -> Y = Gamma (Q S) + M U,
 //                                                       S' = Gamma_C S + K^T U'
 //                       with U' = diag(Gamma_C / Gamma) U.  Slots are double-buffered and
-//                       handed over with mbarriers; y rows leave through bulk stores.
+//                       handed over with mbarriers; full chunks of y leave through TMA stores.
 // All products use fp16 operands with fp32 accumulation in TMEM.  Operand tiles use the
 // 128B / 64B swizzled canonical layouts, so one tile serves as K-major or MN-major operand.
 // Every wait is bounded (ChunkArgs::budget clock cycles); a wait that runs out sets the
 // device error word, lets in-flight MMAs drain, and the CTA returns after freeing TMEM.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -52,6 +55,12 @@ struct ChunkArgs {
     float* S_T;
     void* workspace;
     unsigned long long budget;
+};
+
+// TMA descriptors of the chain kernel: [N, H, 128] views of k, q (64-column halves, 128B
+// swizzle), v (NS-column slab, 64B swizzle) and y (NS-column slab, no swizzle, stores).
+struct ChainMaps {
+    CUtensorMap k, q, v, y;
 };
 
 constexpr int kChunk = 64;
@@ -162,10 +171,12 @@ struct UtCfg {
     static constexpr int OFF_META = OFF_VEC + 1024;
     static constexpr int OFF_BAR = OFF_META + 32;
     static constexpr int BYTES = OFF_BAR + 32 + 1024;
+    static_assert(OFF_KQ % 1024 == 0, "swizzled TMA destination");
     static constexpr uint32_t TMEM_COLS = 64;
 };
 
-__global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ ChunkArgs a) {
+__global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
+                                                       const __grid_constant__ ChainMaps maps) {
     using Cf = UtCfg;
     constexpr int LD = Cf::LD;
     extern __shared__ uint8_t smem_raw[];
@@ -176,8 +187,9 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
     float* fZ = reinterpret_cast<float*>(smem + Cf::OFF_Z);
     float* vb = reinterpret_cast<float*>(smem + Cf::OFF_VEC);  // gamma[0:64] Gamma[64:128] beta[128:192] colf[192:256]
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 8);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);       // MMA done
+    uint64_t* bar_ld = bar + 1;                                            // K, Q tiles landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 16);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int v = blockIdx.x, h = blockIdx.y, H = a.H;
@@ -197,15 +209,19 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
     const int t0 = t_begin + meta[2] * kChunk, L = min(kChunk, t_end - t0);
     uint8_t* rec = reinterpret_cast<uint8_t*>(a.workspace) + ((size_t)v * H + h) * kRecBytes;
 
-    // ---- K (rows 0-63) and Q (rows 64-127), raw 16-bit, swizzled; gates --------------------
+    // ---- K (rows 0-63) and Q (rows 64-127) as they are stored (bf16 or fp16), by TMA into the
+    //      128B-swizzled operand layout.  Rows past the sequence end hold other tokens; they
+    //      only meet beta = 0 or the strictly-upper mask, so nothing needs clearing. ----------------
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::mbar_init(bar_ld, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(bar_ld, 4 * 8192);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const int idx = tid + 128 * u, r = idx >> 4, cc = idx & 15, hf = cc >> 3, c8 = cc & 7;
-        const size_t off = ((size_t)(t0 + r) * H + h) * 128 + cc * 8;
-        const uint4 kv = r < L ? ldg16(a.k, off) : make_uint4(0, 0, 0, 0);
-        const uint4 qv = r < L ? ldg16(a.q, off) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(smem + Cf::OFF_KQ + hf * 16384 + tc::swz_off(r, c8, 128)) = kv;
-        *reinterpret_cast<uint4*>(smem + Cf::OFF_KQ + hf * 16384 + tc::swz_off(r + 64, c8, 128)) = qv;
+        for (int hf = 0; hf < 2; ++hf) {
+            tc::tma_load_3d(smem + Cf::OFF_KQ + hf * 16384, &maps.k, 64 * hf, h, t0, bar_ld);
+            tc::tma_load_3d(smem + Cf::OFF_KQ + hf * 16384 + 8192, &maps.q, 64 * hf, h, t0, bar_ld);
+        }
     }
     if (tid < 64) {
         float gv = tid < L ? a.g[(size_t)(t0 + tid) * H + h] : 0.f;
@@ -218,10 +234,6 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
         vb[tid] = gv;
     }
     if (warp == 0) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
-    if (tid == 0) {
-        tc::mbar_init(bar, 1);
-        tc::fence_mbar_init();
-    }
     __syncthreads();
     if (tid >= 32 && tid < 64) vb[tid] += vb[31];
     __syncthreads();
@@ -229,14 +241,18 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
         vb[64 + tid] = __expf(vb[tid]);
         vb[192 + tid] = __expf(vb[tid | 15] - vb[tid]);  // exp(gamma_e - gamma_s), e = end of s's block
     }
-    tc::fence_async_smem();
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const bool landed = __syncthreads_and(tc::mbar_wait_bounded(bar_ld, 0, a.budget)) != 0;
+    if (!landed) {
+        if (tid == 0) raise_error(kErrTimeout);
+        tc::mbar_wait_bounded(bar_ld, 0, 4000000000ull);
+    }
 
     // ---- [K;Q] K^T ---------------------------------------------------------------------------
-    if (tid == 0) {
+    if (tid == 0 && landed) {
         const uint32_t id = a.in_dt == kBF16 ? tc::idesc_bf16(128, 64, false, false) : tc::idesc_f16(128, 64, false, false);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -245,14 +261,17 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
         }
         tc::mma_commit(bar);
     }
-    const bool ok = __syncthreads_and(tc::mbar_wait_bounded(bar, 0, a.budget)) != 0;
-    if (!ok) {
-        if (tid == 0) raise_error(kErrTimeout);
-        tc::mbar_wait_bounded(bar, 0, 4000000000ull);
+    bool done = false;
+    if (landed) {  // uniform
+        done = __syncthreads_and(tc::mbar_wait_bounded(bar, 0, a.budget)) != 0;
+        if (!done) {
+            if (tid == 0) raise_error(kErrTimeout);
+            tc::mbar_wait_bounded(bar, 0, 4000000000ull);
+        }
     }
     tc::tc_fence_after();
 
-    if (ok) {
+    if (landed && done) {
         // ---- masks: A (fp32) for the solve; M (fp16) straight into the record -------------------
         {
             float x[64];
@@ -387,9 +406,9 @@ struct ChainCfg {
     static constexpr int OFF_X = 0;                           // [2] [K;Q;W] fp16: 2 x [192 x 128 B]
     static constexpr int OFF_TT = OFF_X + 2 * 2 * XREG;       // [T_w; T_u]: [128 x 128 B]
     static constexpr int OFF_M = OFF_TT + 16384;              // [2] M: [64 x 128 B]
-    static constexpr int OFF_STG = OFF_M + 2 * 8192;          // staging (raw rows + record)
-    static constexpr int STG_Q = 16384, STG_V = 32768, STG_REC = STG_V + 64 * ROWB;
-    static constexpr int STG_BYTES = STG_REC + kRecBytes;
+    static constexpr int OFF_STG = OFF_M + 2 * 8192;          // staging: 2 x [K;Q] half [128 x 128 B]
+    static constexpr int STG_BYTES = 32768;
+    static constexpr uint32_t STAGE_TX = 32768 + 64 * ROWB;   // K, Q halves and the V slab, per chunk
     static constexpr int OFF_VS = OFF_STG + STG_BYTES;        // [2] V slab fp16 [64 x ROWB]
     static constexpr int OFF_SS = OFF_VS + 2 * 64 * ROWB;     // S operand [128 x ROWB]
     static constexpr int OFF_SU = OFF_SS + 128 * ROWB;        // U operand [64 x ROWB]
@@ -410,7 +429,8 @@ struct ChainCfg {
 };
 
 template <int NS>
-__global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a) {
+__global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a,
+                                                             const __grid_constant__ ChainMaps maps) {
     using Cf = ChainCfg<NS>;
     constexpr int NSLAB = 128 / NS;
     extern __shared__ uint8_t smem_raw[];
@@ -422,9 +442,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     uint64_t* bar_c = bars + 1;      // chain-issued MMAs complete
     uint64_t* bar_full = bars + 2;   // [2] slot filled by the producer
     uint64_t* bar_empty = bars + 4;  // [2] slot released by the chain
-    uint64_t* bar_stage = bars + 6;  // staging landed (bulk-copy bytes)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 64);
-    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 72);
+    uint64_t* bar_stage = bars + 6;  // K, Q staging and V slab landed (bytes)
+    uint64_t* bar_tt = bars + 7;     // [T_w; T_u] of the next chunk landed in TT
+    uint64_t* bar_m = bars + 8;      // M of the current chunk landed in M[b]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 96);
+    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 104);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slab = blockIdx.x % NSLAB;
@@ -440,7 +462,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (lane == 0) *s_base = base;
     }
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < 9; ++i) tc::mbar_init(bars + i, 1);
         tc::fence_mbar_init();
     }
     if (warp == 1) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
@@ -493,12 +515,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB)) = pack_f16x8(S + 8 * c);
         operands_ready();
 
-        int ys_c0 = -1, ys_L = 0;  // y rows staged in YS, not yet stored
-        auto flush_y = [&]() {     // warp 0 issues one bulk store per valid staged row
-            if (warp == 0 && ys_c0 >= 0) {
-                for (int r = lane; r < ys_L; r += 32)
-                    tc::bulk_s2g(reinterpret_cast<uint8_t*>(a.y) + (((size_t)(ys_c0 + r) * H + h) * 128 + slab * NS) * ybytes,
-                                 smem + Cf::OFF_YS + r * NS * ybytes, NS * ybytes);
+        int ys_c0 = -1;  // a full chunk of y rows staged in YS, not yet stored
+        auto flush_y = [&]() {
+            if (tid == 0 && ys_c0 >= 0) {
+                tc::tma_store_3d(&maps.y, slab * NS, h, ys_c0, smem + Cf::OFF_YS);
                 tc::bulk_commit();
             }
             ys_c0 = -1;
@@ -555,7 +575,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     for (int j = 0; j < NS; ++j) qs[j] = d1[j];
                 }
             }
-            if (warp == 0) tc::bulk_wait_read0();  // YS may be rewritten below
+            if (tid == 0) tc::bulk_wait_read0();  // YS may be rewritten below
             operands_ready();
 
             // [M;.] U -> M U (rows 0-63) ;  K^T U' -> state increment
@@ -575,13 +595,16 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
 
             {
                 float t[NS];
-                if (warp < 2) {  // y = scale (Gamma_r (Q S) + M U) -> YS
+                if (warp < 2) {  // y = scale (Gamma_r (Q S) + M U): staged for a TMA store, or stored directly
 #pragma unroll
                     for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_MU + 32 * q4, t + 32 * q4);
                     if (tid < L) {
+                        void* dst = L == kChunk ? static_cast<void*>(smem + Cf::OFF_YS + tid * NS * ybytes)
+                                                : static_cast<void*>(reinterpret_cast<uint8_t*>(a.y) +
+                                                                     (((size_t)(c0 + tid) * H + h) * 128 + slab * NS) * ybytes);
 #pragma unroll
                         for (int j = 0; j < NS; j += 4)
-                            st4(smem + Cf::OFF_YS + tid * NS * ybytes, a.y_dt, j,
+                            st4(dst, a.y_dt, j,
                                 make_float4(a.scale * (gR * qs[j] + t[j]), a.scale * (gR * qs[j + 1] + t[j + 1]),
                                             a.scale * (gR * qs[j + 2] + t[j + 2]), a.scale * (gR * qs[j + 3] + t[j + 3])));
                     }
@@ -594,12 +617,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 for (int cc = 0; cc < NS / 8; ++cc)
                     *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB)) = pack_f16x8(S + 8 * cc);
             }
-            ys_c0 = c0;
-            ys_L = L;
+            ys_c0 = L == kChunk ? c0 : -1;
             operands_ready();
         }
         if (ok) flush_y();
-        if (warp == 0) tc::bulk_wait0();
+        if (tid == 0) tc::bulk_wait0();
         if (ok && a.S_T) {
 #pragma unroll
             for (int j = 0; j < NS; j += 4)
@@ -615,23 +637,37 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         const uint32_t id_w = tc::idesc_f16(128, 128, false, true);
         const uint32_t sTT = sbase + Cf::OFF_TT;
 
-        // bulk copies of chunk ci's rows and record into staging (warp 4)
+        // TMA copies of chunk ci's K, Q halves (staging), V slab (its operand slot) and record
+        int issued = -1, landed = -1;        // last chunk whose staging copies were issued / waited for
+        int tt_issued = -1, tt_landed = -1;  // same for the [T_w; T_u] part of the records
+        int m_issued = -1, m_landed = -1;    // same for the M part
+        auto rec_ptr = [&](int ci) {
+            return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
+        };
+        // TMA copies of chunk ci's K, Q halves (staging) and V slab (its operand slot)
         auto issue_loads = [&](int ci) {
-            if (warp != 4) return;
-            const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
-            if (lane == 0) tc::mbar_arrive_expect_tx(bar_stage, (uint32_t)(L * (512 + Cf::ROWB) + kRecBytes));
-            __syncwarp();
-            for (int r = lane; r < L; r += 32) {
-                const size_t row = (size_t)(c0 + r) * H + h;
-                tc::bulk_g2s(stg + r * 256, reinterpret_cast<const uint16_t*>(a.k) + row * 128, 256, bar_stage);
-                tc::bulk_g2s(stg + Cf::STG_Q + r * 256, reinterpret_cast<const uint16_t*>(a.q) + row * 128, 256, bar_stage);
-                tc::bulk_g2s(stg + Cf::STG_V + r * Cf::ROWB, reinterpret_cast<const uint16_t*>(a.v) + row * 128 + slab * NS,
-                             Cf::ROWB, bar_stage);
+            issued = ci;
+            if (it != 0) return;
+            const int c0 = t_begin + ci * kChunk;
+            tc::mbar_arrive_expect_tx(bar_stage, Cf::STAGE_TX);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                tc::tma_load_3d(stg + hf * 16384, &maps.k, 64 * hf, h, c0, bar_stage);
+                tc::tma_load_3d(stg + hf * 16384 + 8192, &maps.q, 64 * hf, h, c0, bar_stage);
             }
-            if (lane == 0)
-                tc::bulk_g2s(stg + Cf::STG_REC,
-                             reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes,
-                             kRecBytes, bar_stage);
+            tc::tma_load_3d(smem + Cf::OFF_VS + (ci & 1) * 64 * Cf::ROWB, &maps.v, slab * NS, h, c0, bar_stage);
+        };
+        auto issue_tt = [&](int ci) {  // record bytes [0, 16 KB) -> TT
+            tt_issued = ci;
+            if (it != 0) return;
+            tc::mbar_arrive_expect_tx(bar_tt, 16384);
+            tc::bulk_g2s(smem + Cf::OFF_TT, rec_ptr(ci), 16384, bar_tt);
+        };
+        auto issue_m = [&](int ci) {  // record bytes [16 KB, 24 KB) -> M[ci & 1]
+            m_issued = ci;
+            if (it != 0) return;
+            tc::mbar_arrive_expect_tx(bar_m, 8192);
+            tc::bulk_g2s(smem + Cf::OFF_M + (ci & 1) * 8192, rec_ptr(ci) + 16384, 8192, bar_m);
         };
         float pg = 0.f, pb = 0.f;
         auto load_gates = [&](int ci) {
@@ -641,8 +677,14 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 pb = it < L ? a.beta[(size_t)(c0 + it) * H + h] : 0.f;
             }
         };
+        if (it == 0) {
+            tc::prefetch_tmap(&maps.k);
+            tc::prefetch_tmap(&maps.q);
+            tc::prefetch_tmap(&maps.v);
+        }
         if (nchunks > 0) {
             issue_loads(0);
+            issue_tt(0);
             load_gates(0);
         }
 
@@ -657,30 +699,26 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 if (it == 0) raise_error(kErrTimeout);
                 break;
             }
+            landed = c;
+            issue_m(c);  // slot b is free: its M rows can come in now
             tc::tc_fence_after();
 
-            // ---- fp16 operand tiles: K, Q rows of [K;Q;W], V slab; the record -------------------
+            // ---- fp16 operand tiles: K, Q rows of [K;Q;W] (same swizzled offsets as staged), V in
+            //      place, the record into TT and M[b]; rows past the sequence end are zeroed
             uint8_t* X = smem + Xoff(b);
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                const int idx = it + 128 * u, which = idx >> 10, r = (idx >> 4) & 63, cc = idx & 15;
+                const int idx = it + 128 * u, hf = idx >> 10, rem = idx & 1023, row = rem >> 3;  // row 0-63 K, 64-127 Q
                 uint4 val = make_uint4(0, 0, 0, 0);
-                if (r < L) val = to_f16x8(*reinterpret_cast<const uint4*>(stg + which * Cf::STG_Q + r * 256 + cc * 16), a.in_dt);
-                *reinterpret_cast<uint4*>(X + (cc >> 3) * Cf::XREG + tc::swz_off(which * 64 + r, cc & 7, 128)) = val;
+                if ((row & 63) < L) val = to_f16x8(*reinterpret_cast<const uint4*>(stg + idx * 16), a.in_dt);
+                *reinterpret_cast<uint4*>(X + hf * Cf::XREG + rem * 16) = val;
             }
+            uint8_t* VSb = smem + Cf::OFF_VS + b * 64 * Cf::ROWB;
 #pragma unroll
-            for (int u = 0; u < (64 * NS / 8) / 128; ++u) {
-                const int idx = it + 128 * u, r = idx / (NS / 8), cc = idx % (NS / 8);
-                uint4 val = make_uint4(0, 0, 0, 0);
-                if (r < L) val = to_f16x8(*reinterpret_cast<const uint4*>(stg + Cf::STG_V + r * Cf::ROWB + cc * 16), a.in_dt);
-                *reinterpret_cast<uint4*>(smem + Cf::OFF_VS + b * 64 * Cf::ROWB + tc::swz_off(r, cc, Cf::ROWB)) = val;
-            }
-#pragma unroll
-            for (int u = 0; u < 12; ++u) {
-                const int idx = it + 128 * u;  // 16-byte piece of the record
-                const uint4 val = *reinterpret_cast<const uint4*>(stg + Cf::STG_REC + idx * 16);
-                uint8_t* dst = idx < 1024 ? smem + Cf::OFF_TT + idx * 16 : smem + Cf::OFF_M + b * 8192 + (idx - 1024) * 16;
-                *reinterpret_cast<uint4*>(dst) = val;
+            for (int u = 0; u < (64 * Cf::ROWB / 16) / 128; ++u) {
+                const int idx = it + 128 * u, row = idx / (Cf::ROWB / 16);
+                uint4* p = reinterpret_cast<uint4*>(VSb + idx * 16);
+                *p = row < L ? to_f16x8(*p, a.in_dt) : make_uint4(0, 0, 0, 0);
             }
             if (it < 64) {
                 float gv = pg;
@@ -710,6 +748,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::tc_fence_after();
 
             // ---- U~ = T_u V (rows 64-127 of this slot's columns) and W = T_w K (rows 0-63) ------
+            if (!(ok = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_tt, c & 1, a.budget)))) {
+                if (it == 0) raise_error(kErrTimeout);
+                break;
+            }
+            tt_landed = c;
             if (it == 0) {
                 const uint32_t sV = sbase + Cf::OFF_VS + b * 64 * Cf::ROWB, sXb = sbase + Xoff(b);
 #pragma unroll
@@ -730,6 +773,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             ph ^= 1u;
             tc::tc_fence_after();
             if (!(ok = w)) break;
+            if (c + 1 < nchunks) issue_tt(c + 1);  // the MMAs have read TT
 
             // ---- W -> rows 128-191 of [K;Q;W] ----------------------------------------------------
             if (it < 64) {
@@ -747,10 +791,19 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
-            tc::bar_sync(BID, 128);
+            w = tc::mbar_wait_bounded(bar_m, c & 1, a.budget);  // M rows of slot b landed
+            if (!(ok = tc::bar_and(BID, 128, w))) {
+                if (it == 0) raise_error(kErrTimeout);
+                break;
+            }
+            m_landed = c;
             if (it == 0) tc::mbar_arrive(bar_full + b);  // hand slot b to the chain group
             if (c + 1 < nchunks) load_gates(c + 1);
         }
+        // never leave with copies into this CTA's shared memory in flight
+        if (issued > landed) tc::mbar_wait_bounded(bar_stage, issued & 1, 4000000000ull);
+        if (tt_issued > tt_landed) tc::mbar_wait_bounded(bar_tt, tt_issued & 1, 4000000000ull);
+        if (m_issued > m_landed) tc::mbar_wait_bounded(bar_m, m_issued & 1, 4000000000ull);
         (void)ok;
     }
 
@@ -762,6 +815,37 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     }
 }
 
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+inline EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// [N, H, 128] view of a token-major tensor; box = box_x columns x 1 head x box_z tokens.
+inline bool encode_map_3d(CUtensorMap* m, const void* base, int dt, int N, int H, uint32_t box_x, uint32_t box_z,
+                          CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    const int eb = dt == kF32 ? 4 : 2;
+    const CUtensorMapDataType t = dt == kF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                  : dt == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)N};
+    const cuuint64_t strides[2] = {(cuuint64_t)128 * eb, (cuuint64_t)H * 128 * eb};
+    const cuuint32_t box[3] = {box_x, 1, box_z};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const char** why) {
     *why = nullptr;
     if (a.chunk != kChunk) {
@@ -770,17 +854,25 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
     }
     constexpr int NS = 32;
     using Ch = ChainCfg<NS>;
+    ChainMaps maps;
+    if (!encode_map_3d(&maps.k, a.k, a.in_dt, a.N, a.H, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_3d(&maps.q, a.q, a.in_dt, a.N, a.H, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        *why = "cuTensorMapEncodeTiled failed";
+        return cudaSuccess;
+    }
     cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, UtCfg::BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_chain_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
     if (e != cudaSuccess) return e;
     const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
     if (nvc > 0) {
-        chunk_ut_kernel<<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a);
+        chunk_ut_kernel<<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a, maps);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    chunk_chain_kernel<NS><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a);
+    chunk_chain_kernel<NS><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a, maps);
     return cudaGetLastError();
 }
 
