@@ -86,6 +86,24 @@ gdn_status_t gdn_check_device_error(gdn_stream_t stream);
 void gdn_set_wait_budget(uint64_t cycles);
 
 /*
+ * Per-kernel launch timing (a measurement aid; the pages define no such call).
+ * gdn_timing_start: from now on every kernel launch of the library on the current
+ *   device is bracketed by two CUDA events recorded on the launch's stream, for at most
+ *   max_launches launches (later ones run untimed).  The event pool (2 * max_launches
+ *   events) is created here.  GDN_ERR_INVALID_ARG if timing is already on or
+ *   max_launches is outside [1, 2^20]; GDN_ERR_CUDA if the events cannot be created.
+ *   Do not start timing while a stream is being captured into a CUDA graph.
+ * gdn_timing_stop: waits for the recorded events, aggregates them per kernel name in
+ *   order of first launch, and turns timing off.  Up to cap entries are written:
+ *   names[i] (a static string owned by the library), launches[i], total_ms[i] (sum of
+ *   the launches' device durations).  *n_kernels (nullable) receives the number of
+ *   distinct kernels, which may exceed cap.  GDN_ERR_INVALID_ARG if timing is off.
+ */
+gdn_status_t gdn_timing_start(int max_launches);
+gdn_status_t gdn_timing_stop(int cap, const char** names, int* launches, double* total_ms,
+                             int* n_kernels);
+
+/*
  * gdn_prep -- eqs. (6)-(10): the input side of the mixer.
  *   q = L2Norm(SiLU(ShortConv(x_q)))   (6)     k = L2Norm(SiLU(ShortConv(x_k)))   (7)
  *   v = SiLU(ShortConv(x_v))           (8)     beta = sigmoid(beta_logit)         (9)

@@ -154,6 +154,17 @@ __device__ __forceinline__ uint4 ldg16(const void* p, size_t elem_off) {
     return __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p) + elem_off));
 }
 
+// The dynamic shared-memory base rounded up to 1024 bytes (the swizzle atom of the operand
+// tiles).  Offsetting the __shared__ array itself keeps the pointer in the shared address
+// space, so every access through it compiles to a shared-memory load or store.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* raw) {
+    return raw + ((1024u - (tc::smem_u32(raw) & 1023u)) & 1023u);
+}
+
+// Descriptor of the same operand advanced by byte_off (the start-address field holds
+// address >> 4 in its low 14 bits; operands stay below 256 KB, so no carry leaves the field).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t byte_off) { return d + (byte_off >> 4); }
+
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
@@ -180,7 +191,7 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
     using Cf = UtCfg;
     constexpr int LD = Cf::LD;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(smem);
     float* fA = reinterpret_cast<float*>(smem + Cf::OFF_A);
     float* fT = reinterpret_cast<float*>(smem + Cf::OFF_T);
@@ -254,9 +265,10 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
     // ---- [K;Q] K^T ---------------------------------------------------------------------------
     if (tid == 0 && landed) {
         const uint32_t id = a.in_dt == kBF16 ? tc::idesc_bf16(128, 64, false, false) : tc::idesc_f16(128, 64, false, false);
+        const uint64_t d0 = tc::smem_desc(sbase + Cf::OFF_KQ, 16, 1024, tc::kSw128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t d = tc::smem_desc(sbase + Cf::OFF_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, tc::kSw128);
+            const uint64_t d = desc_add(d0, (kk >> 2) * 16384 + (kk & 3) * 32);
             tc::mma_f16(tmem, d, d, id, kk > 0);
         }
         tc::mma_commit(bar);
@@ -434,7 +446,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     using Cf = ChainCfg<NS>;
     constexpr int NSLAB = 128 / NS;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(smem);
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
@@ -500,7 +512,13 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         };
         const uint32_t id_slab = tc::idesc_f16(128, NS, false, true);
         const uint32_t id_ds = tc::idesc_f16(128, NS, true, true);
-        const uint32_t sSS = sbase + Cf::OFF_SS, sSU = sbase + Cf::OFF_SU, sSU2 = sbase + Cf::OFF_SU2;
+        // operand descriptors at k-step 0 of slot 0; k-steps and slots are byte offsets from these
+        const uint64_t dX0 = tc::smem_desc(sbase + Cf::OFF_X, 16, 1024, tc::kSw128);        // K-major [Q;W] rows
+        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_X, Cf::XREG, 1024, tc::kSw128);  // MN-major K
+        const uint64_t dM0 = tc::smem_desc(sbase + Cf::OFF_M, 16, 1024, tc::kSw128);
+        const uint64_t dSS0 = tc::smem_desc(sbase + Cf::OFF_SS, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
+        const uint64_t dSU0 = tc::smem_desc(sbase + Cf::OFF_SU, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
+        const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const int ybytes = a.y_dt == kF32 ? 4 : 2;
 
         const size_t st_base = ((size_t)n * H + h) * 128 * 128 + (size_t)tid * 128 + slab * NS;
@@ -515,16 +533,36 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB)) = pack_f16x8(S + 8 * c);
         operands_ready();
 
-        int ys_c0 = -1;  // a full chunk of y rows staged in YS, not yet stored
-        auto flush_y = [&]() {
-            if (tid == 0 && ys_c0 >= 0) {
-                tc::tma_store_3d(&maps.y, slab * NS, h, ys_c0, smem + Cf::OFF_YS);
+        // y of chunk c-1 is formed while chunk c's first MMA runs; a full chunk leaves with one
+        // TMA store, a sequence's last partial chunk with plain stores.
+        int py_c0 = 0, py_L = 0;  // the chunk whose M U waits in TMEM (py_L = 0: none)
+        float py_g = 0.f;         // its Gamma_r (rows 0-63)
+        float qs[NS];             // its (Q S) row (rows 0-63)
+        auto y_epilogue = [&]() {  // warps 0-1: y = scale (Gamma_r (Q S) + M U) of chunk py
+            if (warp < 2 && py_L > 0) {
+                float t[NS];
+#pragma unroll
+                for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_MU + 32 * q4, t + 32 * q4);
+                if (tid < py_L) {
+                    void* dst = py_L == kChunk ? static_cast<void*>(smem + Cf::OFF_YS + tid * NS * ybytes)
+                                               : static_cast<void*>(reinterpret_cast<uint8_t*>(a.y) +
+                                                                    (((size_t)(py_c0 + tid) * H + h) * 128 + slab * NS) * ybytes);
+#pragma unroll
+                    for (int j = 0; j < NS; j += 4)
+                        st4(dst, a.y_dt, j,
+                            make_float4(a.scale * (py_g * qs[j] + t[j]), a.scale * (py_g * qs[j + 1] + t[j + 1]),
+                                        a.scale * (py_g * qs[j + 2] + t[j + 2]), a.scale * (py_g * qs[j + 3] + t[j + 3])));
+                }
+            }
+        };
+        auto y_store = [&]() {  // after a barrier that follows y_epilogue
+            if (tid == 0 && py_L == kChunk) {
+                tc::tma_store_3d(&maps.y, slab * NS, h, py_c0, smem + Cf::OFF_YS);
                 tc::bulk_commit();
             }
-            ys_c0 = -1;
+            py_L = 0;
         };
 
-        float qs[NS];  // rows 0-63: (Q S) row
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (!(ok = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget)))) {
@@ -537,18 +575,16 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const float gC = vb[64 + 63];
             const float gR = tid < 64 ? vb[64 + tid] : 0.f;
             const float fR = tid >= 64 ? vb[128 + tid - 64] : 0.f;
-            const uint32_t sX = sbase + Xoff(b), sM = sbase + Cf::OFF_M + b * 8192;
 
             // [Q;W] S  -> Q S (rows 0-63), W S (rows 64-127)
             if (tid == 0) {
+                const uint64_t aw0 = desc_add(dX0, b * 2 * Cf::XREG + 64 * 128);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t aw = tc::smem_desc(sX + (kk >> 2) * Cf::XREG + 64 * 128 + (kk & 3) * 32, 16, 1024, tc::kSw128);
-                    const uint64_t bs = tc::smem_desc(sSS + kk * 16 * Cf::ROWB, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-                    tc::mma_f16(tmem + Cf::COL_1, aw, bs, id_slab, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16(tmem + Cf::COL_1, desc_add(aw0, (kk >> 2) * Cf::XREG + (kk & 3) * 32),
+                                desc_add(dSS0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
             }
-            flush_y();  // the previous chunk's y rows leave while the MMA runs
+            y_epilogue();  // previous chunk's y while the MMA runs
             if (!(ok = commit_wait())) break;
 
             {
@@ -575,19 +611,16 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     for (int j = 0; j < NS; ++j) qs[j] = d1[j];
                 }
             }
-            if (tid == 0) tc::bulk_wait_read0();  // YS may be rewritten below
-            operands_ready();
+            operands_ready();  // also orders the staged y rows before their TMA store
+            y_store();
 
             // [M;.] U -> M U (rows 0-63) ;  K^T U' -> state increment
             if (tid == 0) {
+                const uint64_t am0 = desc_add(dM0, b * 8192), ak0 = desc_add(dK0, b * 2 * Cf::XREG);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bu = tc::smem_desc(sSU + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-                    const uint64_t am = tc::smem_desc(sM + kk * 32, 16, 1024, tc::kSw128);
-                    tc::mma_f16(tmem + Cf::COL_MU, am, bu, id_slab, kk > 0);
-                    const uint64_t bu2 = tc::smem_desc(sSU2 + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-                    const uint64_t ak = tc::smem_desc(sX + kk * 2048, Cf::XREG, 1024, tc::kSw128);
-                    tc::mma_f16(tmem + Cf::COL_DS, ak, bu2, id_ds, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(dSU0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::ROWB), id_ds, kk > 0);
                 }
             }
             if (!(ok = commit_wait())) break;
@@ -595,20 +628,6 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
 
             {
                 float t[NS];
-                if (warp < 2) {  // y = scale (Gamma_r (Q S) + M U): staged for a TMA store, or stored directly
-#pragma unroll
-                    for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_MU + 32 * q4, t + 32 * q4);
-                    if (tid < L) {
-                        void* dst = L == kChunk ? static_cast<void*>(smem + Cf::OFF_YS + tid * NS * ybytes)
-                                                : static_cast<void*>(reinterpret_cast<uint8_t*>(a.y) +
-                                                                     (((size_t)(c0 + tid) * H + h) * 128 + slab * NS) * ybytes);
-#pragma unroll
-                        for (int j = 0; j < NS; j += 4)
-                            st4(dst, a.y_dt, j,
-                                make_float4(a.scale * (gR * qs[j] + t[j]), a.scale * (gR * qs[j + 1] + t[j + 1]),
-                                            a.scale * (gR * qs[j + 2] + t[j + 2]), a.scale * (gR * qs[j + 3] + t[j + 3])));
-                    }
-                }
 #pragma unroll
                 for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_DS + 32 * q4, t + 32 * q4);
 #pragma unroll
@@ -617,10 +636,18 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 for (int cc = 0; cc < NS / 8; ++cc)
                     *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB)) = pack_f16x8(S + 8 * cc);
             }
-            ys_c0 = L == kChunk ? c0 : -1;
+            py_c0 = c0;
+            py_L = L;
+            py_g = gR;
+            if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next y_epilogue writes it
             operands_ready();
         }
-        if (ok) flush_y();
+        if (ok) {
+            y_epilogue();
+            tc::fence_async_smem();
+            tc::bar_sync(BID, 128);
+            y_store();
+        }
         if (tid == 0) tc::bulk_wait0();
         if (ok && a.S_T) {
 #pragma unroll
@@ -635,7 +662,9 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         bool ok = true;
         const uint32_t id_slab = tc::idesc_f16(128, NS, false, true);
         const uint32_t id_w = tc::idesc_f16(128, 128, false, true);
-        const uint32_t sTT = sbase + Cf::OFF_TT;
+        const uint64_t dTT0 = tc::smem_desc(sbase + Cf::OFF_TT, 16, 1024, tc::kSw128);
+        const uint64_t dV0 = tc::smem_desc(sbase + Cf::OFF_VS, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
+        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_X, Cf::XREG, 1024, tc::kSw128);  // MN-major K
 
         // TMA copies of chunk ci's K, Q halves (staging), V slab (its operand slot) and record
         int issued = -1, landed = -1;        // last chunk whose staging copies were issued / waited for
@@ -706,19 +735,25 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             // ---- fp16 operand tiles: K, Q rows of [K;Q;W] (same swizzled offsets as staged), V in
             //      place, the record into TT and M[b]; rows past the sequence end are zeroed
             uint8_t* X = smem + Xoff(b);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int idx = it + 128 * u, hf = idx >> 10, rem = idx & 1023, row = rem >> 3;  // row 0-63 K, 64-127 Q
-                uint4 val = make_uint4(0, 0, 0, 0);
-                if ((row & 63) < L) val = to_f16x8(*reinterpret_cast<const uint4*>(stg + idx * 16), a.in_dt);
-                *reinterpret_cast<uint4*>(X + hf * Cf::XREG + rem * 16) = val;
-            }
             uint8_t* VSb = smem + Cf::OFF_VS + b * 64 * Cf::ROWB;
+            constexpr int VU = (64 * Cf::ROWB / 16) / 128;
+            {
+                uint4 raw[16], vraw[VU];  // every load issued before the first store
 #pragma unroll
-            for (int u = 0; u < (64 * Cf::ROWB / 16) / 128; ++u) {
-                const int idx = it + 128 * u, row = idx / (Cf::ROWB / 16);
-                uint4* p = reinterpret_cast<uint4*>(VSb + idx * 16);
-                *p = row < L ? to_f16x8(*p, a.in_dt) : make_uint4(0, 0, 0, 0);
+                for (int u = 0; u < 16; ++u) raw[u] = *reinterpret_cast<const uint4*>(stg + (it + 128 * u) * 16);
+#pragma unroll
+                for (int u = 0; u < VU; ++u) vraw[u] = *reinterpret_cast<const uint4*>(VSb + (it + 128 * u) * 16);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int idx = it + 128 * u, hf = idx >> 10, rem = idx & 1023, row = rem >> 3;  // 0-63 K, 64-127 Q
+                    *reinterpret_cast<uint4*>(X + hf * Cf::XREG + rem * 16) =
+                        (row & 63) < L ? to_f16x8(raw[u], a.in_dt) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < VU; ++u) {
+                    const int idx = it + 128 * u, row = idx / (Cf::ROWB / 16);
+                    *reinterpret_cast<uint4*>(VSb + idx * 16) = row < L ? to_f16x8(vraw[u], a.in_dt) : make_uint4(0, 0, 0, 0);
+                }
             }
             if (it < 64) {
                 float gv = pg;
@@ -754,14 +789,12 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             tt_landed = c;
             if (it == 0) {
-                const uint32_t sV = sbase + Cf::OFF_VS + b * 64 * Cf::ROWB, sXb = sbase + Xoff(b);
+                const uint64_t bv0 = desc_add(dV0, b * 64 * Cf::ROWB), bk0 = desc_add(dK0, b * 2 * Cf::XREG);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t at = tc::smem_desc(sTT + kk * 32, 16, 1024, tc::kSw128);
-                    const uint64_t bv = tc::smem_desc(sV + kk * 16 * Cf::ROWB, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, at, bv, id_slab, kk > 0);
-                    const uint64_t bk = tc::smem_desc(sXb + kk * 2048, Cf::XREG, 1024, tc::kSw128);
-                    tc::mma_f16(tmem + Cf::COL_W, at, bk, id_w, kk > 0);
+                    const uint64_t at = desc_add(dTT0, kk * 32);
+                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, at, desc_add(bv0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_W, at, desc_add(bk0, kk * 2048), id_w, kk > 0);
                 }
                 tc::mma_commit(bar_p);
             }
@@ -868,10 +901,12 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
     if (e != cudaSuccess) return e;
     const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
     if (nvc > 0) {
+        LaunchScope timed(st, "chunk_ut_kernel");
         chunk_ut_kernel<<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a, maps);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+    LaunchScope timed(st, "chunk_chain_kernel");
     chunk_chain_kernel<NS><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a, maps);
     return cudaGetLastError();
 }

@@ -11,6 +11,7 @@
 
 #include "../../include/gdn.h"
 #include "common.cuh"
+#include "launch_timer.cuh"
 #include "decode.cuh"
 #include "out_gate.cuh"
 #include "prep.cuh"
@@ -91,6 +92,7 @@ struct DecodeLaunch {
                             float* state, const int32_t* slot, int num_slots, int B, int H, float scale,
                             int in_dt, int y_dt, void* y, cudaStream_t st) {
         using Sh = gdn::DecodeShape<DK, DV>;
+        gdn::LaunchScope timed(st, "decode_step_kernel");
         gdn::decode_step_kernel<DK, DV><<<(unsigned)(B * H), Sh::THREADS, 0, st>>>(
             q, k, v, g, beta, state, slot, num_slots, H, scale, in_dt, y_dt, y);
         return launched("decode_step_kernel");
@@ -104,6 +106,7 @@ struct RecurrentLaunch {
                             int in_dt, int y_dt, void* y, float* S_T, cudaStream_t st) {
         using Sh = gdn::RecShape<DK, DV>;
         const unsigned grid = (unsigned)(num_seqs * H * (DV / Sh::SLAB));
+        gdn::LaunchScope timed(st, "recurrent_fwd_kernel");
         gdn::recurrent_fwd_kernel<DK, DV><<<grid, Sh::THREADS, 0, st>>>(
             q, k, v, g, beta, S0, cu, num_seqs, N, H, scale, in_dt, y_dt, y, S_T);
         return launched("recurrent_fwd_kernel");
@@ -119,6 +122,7 @@ struct PrepLaunch {
                             cudaStream_t st) {
         const long long rows = (long long)N * H;
         const unsigned grid = (unsigned)((rows + gdn::kPrepWarps - 1) / gdn::kPrepWarps);
+        gdn::LaunchScope timed(st, "prep_kernel");
         if (DK >= 32 && DV >= 32) {
             gdn::prep_kernel<(DK >= 32 ? DK : 32), (DV >= 32 ? DV : 32)><<<grid, 32 * gdn::kPrepWarps, 0, st>>>(
                 xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g,
@@ -301,6 +305,7 @@ gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, flo
     const long long rows = (long long)N * H;
     const unsigned grid = (unsigned)((rows + gdn::kGateWarps - 1) / gdn::kGateWarps);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    gdn::LaunchScope timed(st, "out_gate_kernel");
     switch (dv) {
         case 16: gdn::out_gate_kernel<16><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
         case 32: gdn::out_gate_kernel<32><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
@@ -308,6 +313,74 @@ gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, flo
         default: gdn::out_gate_kernel<128><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
     }
     return launched("out_gate_kernel");
+}
+
+gdn_status_t gdn_timing_start(int max_launches) {
+    REQUIRE(max_launches >= 1 && max_launches <= (1 << 20), "max_launches=%d not in [1, 2^20]", max_launches);
+    gdn::LaunchTimer& t = gdn::launch_timer();
+    std::lock_guard<std::mutex> lock(t.mu);
+    REQUIRE(!t.on, "timing is already on");
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    t.pool.reserve(2 * (size_t)max_launches);
+    for (int i = 0; i < 2 * max_launches; ++i) {
+        cudaEvent_t ev = nullptr;
+        e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) {
+            for (cudaEvent_t x : t.pool) cudaEventDestroy(x);
+            t.pool.clear();
+            return fail(GDN_ERR_CUDA, "cudaEventCreate: %s", cudaGetErrorString(e));
+        }
+        t.pool.push_back(ev);
+    }
+    t.names.clear();
+    t.device = dev;
+    ++t.generation;
+    t.on = true;
+    return GDN_OK;
+}
+
+gdn_status_t gdn_timing_stop(int cap, const char** names, int* launches, double* total_ms, int* n_kernels) {
+    REQUIRE(cap >= 0 && (cap == 0 || (names && launches && total_ms)), "bad output arrays (cap=%d)", cap);
+    gdn::LaunchTimer& t = gdn::launch_timer();
+    std::lock_guard<std::mutex> lock(t.mu);
+    REQUIRE(t.on, "timing is not on");
+    gdn_status_t status = GDN_OK;
+    std::vector<const char*> kn;
+    std::vector<int> cnt;
+    std::vector<double> ms;
+    for (size_t i = 0; i < t.names.size(); ++i) {
+        float dt = 0.f;
+        cudaError_t e = cudaEventSynchronize(t.pool[2 * i + 1]);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&dt, t.pool[2 * i], t.pool[2 * i + 1]);
+        if (e != cudaSuccess) {
+            status = fail(GDN_ERR_CUDA, "timing event: %s", cudaGetErrorString(e));
+            break;
+        }
+        size_t j = 0;
+        while (j < kn.size() && std::strcmp(kn[j], t.names[i]) != 0) ++j;
+        if (j == kn.size()) {
+            kn.push_back(t.names[i]);
+            cnt.push_back(0);
+            ms.push_back(0.0);
+        }
+        cnt[j] += 1;
+        ms[j] += dt;
+    }
+    for (cudaEvent_t x : t.pool) cudaEventDestroy(x);
+    t.pool.clear();
+    t.names.clear();
+    ++t.generation;
+    t.on = false;
+    if (status != GDN_OK) return status;
+    for (size_t j = 0; j < kn.size() && (int)j < cap; ++j) {
+        names[j] = kn[j];
+        launches[j] = cnt[j];
+        total_ms[j] = ms[j];
+    }
+    if (n_kernels) *n_kernels = (int)kn.size();
+    return GDN_OK;
 }
 
 }  // extern "C"

@@ -36,6 +36,9 @@ SIGNATURES = {
     "gdn_chunk_fwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P], _I),
     "gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
+    "gdn_timing_start": ([_I], _I),
+    "gdn_timing_stop": ([_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double),
+                         ctypes.POINTER(_I)], _I),
 }
 
 _lib = None
@@ -109,6 +112,21 @@ def set_wait_budget(cycles: int):
 def check_device_error(stream=None):
     """Synchronise the stream and raise if a kernel flagged an error since the last check."""
     _check(lib().gdn_check_device_error(_stream(stream)))
+
+
+def timing_start(max_launches=4096):
+    """gdn_timing_start: time every library kernel launch with CUDA events from now on."""
+    _check(lib().gdn_timing_start(int(max_launches)))
+
+
+def timing_stop(cap=64):
+    """gdn_timing_stop: {kernel name: (launches, total device ms)} since timing_start."""
+    names = (ctypes.c_char_p * cap)()
+    launches = (_I * cap)()
+    total = (ctypes.c_double * cap)()
+    n = _I(0)
+    _check(lib().gdn_timing_stop(cap, names, launches, total, ctypes.byref(n)))
+    return {names[i].decode(): (launches[i], total[i]) for i in range(min(n.value, cap))}
 
 
 def workspace_size(N, num_seqs, H, dk, dv, chunk) -> int:

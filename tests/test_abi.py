@@ -113,3 +113,10 @@ def test_binding_refuses_host_tensors():
     import torch
     with pytest.raises(ValueError):
         gdn._ptr(torch.zeros(4))
+
+
+def test_timing_rejects_bad_use(L):
+    assert L.gdn_timing_start(0) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_timing_start(1 << 21) == gdn.GDN_ERR_INVALID_ARG
+    # stopping while timing is off is an argument error, with or without a device
+    assert L.gdn_timing_stop(0, None, None, None, None) == gdn.GDN_ERR_INVALID_ARG
