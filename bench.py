@@ -105,10 +105,12 @@ def prefill_bytes(N, H, nseq, dk=128, dv=128, in_bytes=2, y_bytes=2, S0=False, S
     return b + (state if S0 else 0) + (state if S_T else 0)
 
 
-def timed(torch, fn, steps, warmup, stream):
+def timed(torch, fn, steps, warmup, stream, on_start=None):
     for i in range(warmup):
         fn(i)
     torch.cuda.synchronize()
+    if on_start is not None:
+        on_start()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -117,6 +119,37 @@ def timed(torch, fn, steps, warmup, stream):
     e1.record(stream)
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / 1e3  # seconds
+
+
+def kernel_table(per_kernel, steps):
+    """{name: (launches, total ms)} from gdn.timing_stop -> per-kernel averages and shares."""
+    tot = sum(ms for _, ms in per_kernel.values()) or 1.0
+    return [{"name": n, "launches": c, "avg_us": ms * 1e3 / max(c, 1), "share": ms / tot}
+            for n, (c, ms) in per_kernel.items()]
+
+
+def traffic_per_call():
+    """DRAM bytes (read + write) of one gdn_chunk_fwd call on the headline workload, from the
+    ncu capture summarised in profiles/ -- or None when the kernel source has changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "chunk_fwd_prefill_B2_H16_T4096.md")
+    if not os.path.exists(path):
+        return None
+    src = b"".join(open(os.path.join(ROOT, "linear_attention_token_gdn_b200", "csrc", f), "rb").read()
+                   for f in ("chunk_tc.cuh", "tc_ptx.cuh", "common.cuh"))
+    digest = hashlib.sha256(src).hexdigest()[:16]
+    fields = {}
+    for line in open(path):
+        if line.startswith("traffic:"):
+            for kv in line.split()[1:]:
+                k, _, v = kv.partition("=")
+                fields[k] = v
+    if fields.get("source_sha256") != digest:
+        return None
+    try:
+        return int(fields["bytes_per_call"])
+    except (KeyError, ValueError):
+        return None
 
 
 def max_over_ranks(torch, dist, x, world):
@@ -232,7 +265,9 @@ def run_ours(args):
 
     barrier(torch, dist, world)
     with ClockSampler(torch.cuda.current_device()) as clk:
-        dt = timed(torch, step, args.steps, args.warmup, stream)
+        # every launch inside the timed region is bracketed by CUDA events on its stream
+        dt = timed(torch, step, args.steps, args.warmup, stream, on_start=lambda: gdn.timing_start(4 * args.steps + 8))
+        per_kernel = gdn.timing_stop()
         barrier(torch, dist, world)
         if dt < 0.5:  # keep the GPU busy long enough for the clock sampler to see it
             soak = timed(torch, step, max(1, int(args.steps * 0.6 / max(dt, 1e-6))), 0, stream)
@@ -242,7 +277,9 @@ def run_ours(args):
     work = N * H  # token-heads per rank per step
     value = work * world / per_step
     alg_bytes = prefill_bytes(N, H, nseq)
-    achieved = alg_bytes / per_step / 1e9
+    kern = kernel_table(per_kernel, args.steps)
+    op_s = sum(k["avg_us"] for k in kern) / 1e6  # device time of one gdn_chunk_fwd call
+    achieved = alg_bytes / op_s / 1e9
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -251,9 +288,11 @@ def run_ours(args):
                        "parallelism": f"dp{world}",
                        "l2": "3 rotating input sets (3 x 137 MB > 126 MB L2)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": None, "kernel": "chunk_fwd_tc_kernel",
-                         "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": alg_bytes},
-            "gpu_launches": args.steps, "clocks": clk.summary()}
+                         "frac": achieved / hbm_peak, "traffic": traffic_per_call(), "kernel":
+                         "gdn_chunk_fwd = chunk_ut_kernel + chunk_chain_kernel (per call)",
+                         "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": alg_bytes,
+                         "kernels": kern},
+            "gpu_launches": sum(k["launches"] for k in kern), "clocks": clk.summary()}
 
     # ---- end to end through the public API with pinned host buffers ----------------------
     hx = {k: sets[0][k].cpu().pin_memory() for k in ("q", "k", "v", "g", "beta")}
@@ -306,7 +345,8 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
             gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, y=y)
 
     barrier(torch, dist, world)
-    dt = max_over_ranks(torch, dist, timed(torch, dec, 3, 1, stream), world)
+    dt = max_over_ranks(torch, dist, timed(torch, dec, 3, 1, stream, on_start=lambda: gdn.timing_start(4096)), world)
+    kd = kernel_table(gdn.timing_stop(), 3)
     per_launch = dt / (3 * c["steps"])
     upd = c["B"] * c["H"]
     bytes_l = upd * (2 * 128 * 128 * 4 + 3 * 128 * 2 + 8 + 128 * 2)
@@ -314,8 +354,9 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
                 "us_per_step": per_launch * 1e6,
                 "roofline": {"bound": "hbm", "achieved": bytes_l / per_launch / 1e9, "peak": hbm_peak,
                              "unit": "GB/s", "frac": bytes_l / per_launch / 1e9 / hbm_peak,
-                             "kernel": "decode_step_kernel", "alg_bytes_per_launch": bytes_l},
-                "gpu_launches": 3 * c["steps"]})
+                             "kernel": "decode_step_kernel", "alg_bytes_per_launch": bytes_l,
+                             "kernel_avg_us": kd[0]["avg_us"] if kd else None},
+                "gpu_launches": sum(k["launches"] for k in kd)})
     del state, steps_in
 
     # long prefill: B=1, H=32, T=32768, S0 != 0
@@ -331,14 +372,18 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
 
     barrier(torch, dist, world)
     n_lp = 3
-    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 1, stream), world) / n_lp
+    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 1, stream, on_start=lambda: gdn.timing_start(64)),
+                        world) / n_lp
+    kl = kernel_table(gdn.timing_stop(), n_lp)
+    op_s = sum(k["avg_us"] for k in kl) / 1e6
     bl = prefill_bytes(N, H, nseq, S0=True)
     res.append({"workload": inputs.CONFIGS[2]["name"], "value": N * H * world / dt, "unit": UNIT,
                 "ms_per_step": dt * 1e3,
-                "roofline": {"bound": "hbm", "achieved": bl / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                             "frac": bl / dt / 1e9 / hbm_peak, "kernel": "chunk_fwd_tc_kernel",
-                             "alg_bytes_per_launch": bl}, "gpu_launches": n_lp,
-                "l2": "1.1 GB working set > L2"})
+                "roofline": {"bound": "hbm", "achieved": bl / op_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": bl / op_s / 1e9 / hbm_peak,
+                             "kernel": "gdn_chunk_fwd = chunk_ut_kernel + chunk_chain_kernel (per call)",
+                             "alg_bytes_per_launch": bl, "kernels": kl},
+                "gpu_launches": sum(k["launches"] for k in kl), "l2": "1.1 GB working set > L2"})
     del x, yb, ST
 
     # full mixer: prep -> chunk -> out gate on 4 packed sequences
@@ -361,15 +406,18 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
 
     barrier(torch, dist, world)
     n_m = 5
-    dt = max_over_ranks(torch, dist, timed(torch, mix, n_m, 1, stream), world) / n_m
+    dt = max_over_ranks(torch, dist, timed(torch, mix, n_m, 1, stream, on_start=lambda: gdn.timing_start(64)),
+                        world) / n_m
+    km = kernel_table(gdn.timing_stop(), n_m)
     fused_min = N * (H * 3 * 128 * 2 + H * 2 * 2 + H * 128 * 2 + H * 128 * 2)
     res.append({"workload": inputs.CONFIGS[4]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
                 "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
                 "roofline": {"bound": "hbm", "achieved": fused_min / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
                              "frac": fused_min / dt / 1e9 / hbm_peak, "kernel": "prep+chunk+out_gate",
                              "alg_bytes_per_step": fused_min,
-                             "note": "bytes = fused minimum (read projections, logits, z; write out)"},
-                "gpu_launches": 3 * n_m})
+                             "note": "bytes = fused minimum (read projections, logits, z; write out)",
+                             "kernels": km},
+                "gpu_launches": sum(k["launches"] for k in km)})
     return res
 
 

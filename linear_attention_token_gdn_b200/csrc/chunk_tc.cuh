@@ -14,27 +14,32 @@
 // factors <= 1, so a row needs 4 + 16 exponentials instead of 64.
 //
 // Two kernels:
-//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, several CTAs per SM.
+//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, four CTAs per SM.
 //                       [K;Q] K^T on tcgen05 (the 16-bit inputs used directly as
 //                       operands), the decay masks, and the unit-lower-triangular inverse
-//                       T in fp32 on the CUDA cores.  Writes a 24 KB record per
+//                       T in fp32 on the CUDA cores.  Writes a 40 KB record per
 //                       (chunk, head): T_w = T diag(beta Gamma), T_u = T diag(beta) and M,
-//                       fp16, already in the 128B-swizzled operand layout.
+//                       already in the 128B-swizzled operand layout.
 //   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
-//                       the chunks.  A producer warpgroup brings the next chunk's K, Q and
-//                       V tiles in with TMA and its record with a bulk copy, converts them
-//                       to fp16 operand tiles and computes W = T_w K and U~ = T_u V on the
-//                       tensor cores; a chain warpgroup carries the fp32 state (one row per
-//                       thread) through two dependent tensor-core round trips per chunk:
-//                           [Q;W] S                  -> Q S, W S;  U = U~ - W S
-//                           [M;.] U  and  K^T U'     -> Y = Gamma (Q S) + M U,
-//                                                       S' = Gamma_C S + K^T U'
-//                       with U' = diag(Gamma_C / Gamma) U.  Slots are double-buffered and
-//                       handed over with mbarriers; full chunks of y leave through TMA stores.
-// All products use fp16 operands with fp32 accumulation in TMEM.  Operand tiles use the
-// 128B / 64B swizzled canonical layouts, so one tile serves as K-major or MN-major operand.
-// Every wait is bounded (ChunkArgs::budget clock cycles); a wait that runs out sets the
-// device error word, lets in-flight MMAs drain, and the CTA returns after freeing TMEM.
+//                       the chunks.  A producer warpgroup brings each chunk's K, Q and V
+//                       tiles in with TMA, straight into operand slots, and computes
+//                       W = T_w K and U~ = T_u V on the tensor cores; a chain warpgroup
+//                       carries the fp32 state (one row per thread) through two dependent
+//                       tensor-core round trips per chunk:
+//                           [Q;W] S            -> Q S, W S;   U = U~ - W S
+//                           K^T U'             -> S' = Gamma_C S + K^T U'
+//                       with U' = diag(Gamma_C / Gamma) U, while M U, for
+//                       Y = Gamma (Q S) + M U, completes off the chain.  Q/W/M slots are
+//                       double-buffered, K/V stages triple-buffered, all handed over with
+//                       mbarriers; full chunks of y leave through swizzled TMA stores.
+// Operands are 16-bit in the inputs' own format (bf16 or fp16) with fp32 accumulation in
+// TMEM.  q, k, v enter the products exactly as stored.  A computed operand x whose rounding
+// would show in y or the state (T_u, M, U, U') enters as two products, hi = round(x) and
+// lo = round(x - hi), which carries 16 significant bits for bf16; T_w, W and S enter once.
+// Operand tiles use the 128B / 64B swizzled canonical layouts, so one tile serves as K-major
+// or MN-major operand.  Every wait is bounded (ChunkArgs::budget clock cycles); a wait that
+// runs out sets the device error word, lets in-flight MMAs and copies drain, and the CTA
+// returns after freeing TMEM.
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -64,7 +69,14 @@ struct ChainMaps {
 };
 
 constexpr int kChunk = 64;
-constexpr int kRecBytes = 24576;  // per (chunk, head): T_w, T_u, M as 3 x [64 rows x 128 B]
+// Record of one (chunk, head), written by chunk_ut_kernel: five [64 rows x 128 B] operand tiles
+// in the 128B-swizzled K-major layout, 16-bit in the input's format.
+constexpr int kRecTw = 0;          // T_w = T diag(beta Gamma)
+constexpr int kRecTuHi = 8192;     // T_u = T diag(beta), high half
+constexpr int kRecTuLo = 16384;    //   and the rounding remainder
+constexpr int kRecMHi = 24576;     // M, high half
+constexpr int kRecMLo = 32768;     //   and the rounding remainder
+constexpr int kRecBytes = 40960;
 
 // Upper bound of the number of 64-token chunks over all sequences.
 inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
@@ -127,33 +139,6 @@ __device__ int chunks_before(const int32_t* cu, int num_seqs, int N, int n) {
     return s;
 }
 
-// 8 consecutive 16-bit input elements -> 8 fp16 values packed in a uint4.
-__device__ __forceinline__ uint4 to_f16x8(uint4 u, int in_dt) {
-    if (in_dt == kF16) return u;
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[i]));
-        __half2 hv = __floats2half2_rn(f.x, f.y);
-        w[i] = *reinterpret_cast<uint32_t*>(&hv);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-__device__ __forceinline__ uint4 pack_f16x8(const float* x) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __half2 hv = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
-        w[i] = *reinterpret_cast<uint32_t*>(&hv);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-__device__ __forceinline__ uint4 ldg16(const void* p, size_t elem_off) {
-    return __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p) + elem_off));
-}
-
 // The dynamic shared-memory base rounded up to 1024 bytes (the swizzle atom of the operand
 // tiles).  Offsetting the __shared__ array itself keeps the pointer in the shared address
 // space, so every access through it compiles to a shared-memory load or store.
@@ -168,26 +153,74 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t byte_off) { re
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
+// 16-bit operands in the input's own format (bf16 or fp16), rounded to nearest.
+template <bool BF>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    if constexpr (BF) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&v);
+    } else {
+        __half2 v = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+}
+
+template <bool BF>
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+    if constexpr (BF) {
+        return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+    } else {
+        return __half22float2(*reinterpret_cast<__half2*>(&u));
+    }
+}
+
+template <bool BF>
+__device__ __forceinline__ uint4 pack8(const float* x) {
+    return make_uint4(pack2<BF>(x[0], x[1]), pack2<BF>(x[2], x[3]), pack2<BF>(x[4], x[5]), pack2<BF>(x[6], x[7]));
+}
+
+// x = hi + lo + O(2^-16 |x|) for bf16 (2^-22 for fp16): hi = round(x), lo = round(x - hi).
+template <bool BF>
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        h[i] = pack2<BF>(x[2 * i], x[2 * i + 1]);
+        const float2 f = unpack2<BF>(h[i]);
+        l[i] = pack2<BF>(x[2 * i] - f.x, x[2 * i + 1] - f.y);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+template <bool BF>
+__host__ __device__ constexpr uint32_t idesc16(int M, int N, bool a_mn, bool b_mn) {
+    return BF ? tc::idesc_bf16(M, N, a_mn, b_mn) : tc::idesc_f16(M, N, a_mn, b_mn);
+}
+
+__device__ __forceinline__ void st16(uint8_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+
 // =====================================================================================
 // chunk_ut_kernel: per (chunk, head) -- masks and the UT transform
 // =====================================================================================
 
 struct UtCfg {
-    static constexpr int LD = 68;                          // fp32 row stride of A and T
-    static constexpr int OFF_KQ = 0;                       // [K;Q] raw 16-bit: 2 x [128 x 128 B]
-    static constexpr int OFF_A = OFF_KQ + 32768;           // fp32 A [64][LD]
-    static constexpr int OFF_T = OFF_A + 64 * LD * 4;      // fp32 T [64][LD]
-    static constexpr int OFF_Z = OFF_T + 64 * LD * 4;      // fp32 Z [3][16][20]
-    static constexpr int OFF_VEC = OFF_Z + 3 * 16 * 20 * 4; // gamma, Gamma, beta, colf: 4 x 64
+    static constexpr int LD = 68;                           // fp32 row stride of A and T
+    static constexpr int OFF_KQ = 0;                        // [K;Q] as stored: 2 x [128 x 128 B]
+    static constexpr int OFF_A = 0;                         // fp32 A [64][LD], over [K;Q] once read
+    static constexpr int OFF_Z = OFF_A + 64 * LD * 4;       // fp32 Z [3][16][20], likewise
+    static constexpr int OFF_T = 32768;                     // fp32 T [64][LD]
+    static constexpr int OFF_VEC = OFF_T + 64 * LD * 4;     // gamma, Gamma, beta, colf: 4 x 64
     static constexpr int OFF_META = OFF_VEC + 1024;
     static constexpr int OFF_BAR = OFF_META + 32;
     static constexpr int BYTES = OFF_BAR + 32 + 1024;
-    static_assert(OFF_KQ % 1024 == 0, "swizzled TMA destination");
+    static_assert(OFF_Z + 3 * 16 * 20 * 4 <= OFF_T, "A and Z fit in the [K;Q] tiles");
     static constexpr uint32_t TMEM_COLS = 64;
 };
 
-__global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
-                                                       const __grid_constant__ ChainMaps maps) {
+template <bool BF>
+__global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
+                                                          const __grid_constant__ ChainMaps maps) {
     using Cf = UtCfg;
     constexpr int LD = Cf::LD;
     extern __shared__ uint8_t smem_raw[];
@@ -264,7 +297,7 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
 
     // ---- [K;Q] K^T ---------------------------------------------------------------------------
     if (tid == 0 && landed) {
-        const uint32_t id = a.in_dt == kBF16 ? tc::idesc_bf16(128, 64, false, false) : tc::idesc_f16(128, 64, false, false);
+        constexpr uint32_t id = idesc16<BF>(128, 64, false, false);
         const uint64_t d0 = tc::smem_desc(sbase + Cf::OFF_KQ, 16, 1024, tc::kSw128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -284,7 +317,8 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
     tc::tc_fence_after();
 
     if (landed && done) {
-        // ---- masks: A (fp32) for the solve; M (fp16) straight into the record -------------------
+        // ---- masks: A (fp32, over the consumed [K;Q] tiles) for the solve; M as hi + lo
+        //      16-bit halves straight into the record ---------------------------------------------
         {
             float x[64];
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
@@ -312,7 +346,10 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
                     sts4(fA + r * LD + 8 * cc, make_float4(m[0], m[1], m[2], m[3]));
                     sts4(fA + r * LD + 8 * cc + 4, make_float4(m[4], m[5], m[6], m[7]));
                 } else {
-                    *reinterpret_cast<uint4*>(rec + 16384 + tc::swz_off(r, cc, 128)) = pack_f16x8(m);
+                    uint4 hi, lo;
+                    split8<BF>(m, hi, lo);
+                    st16(rec + kRecMHi + tc::swz_off(r, cc, 128), hi);
+                    st16(rec + kRecMLo + tc::swz_off(r, cc, 128), lo);
                 }
             }
         }
@@ -380,7 +417,7 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
             }
             __syncthreads();
         }
-        // ---- T_w = T diag(beta Gamma) (rows 0-63), T_u = T diag(beta) (rows 64-127) -> record -----
+        // ---- T_w = T diag(beta Gamma) (one 16-bit copy), T_u = T diag(beta) (hi + lo) -> record -----
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int idx = tid + 128 * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
@@ -395,7 +432,14 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) t8[e] = (8 * cc + e <= r) ? t8[e] * s8[e] : 0.f;
-            *reinterpret_cast<uint4*>(rec + which * 8192 + tc::swz_off(r, cc, 128)) = pack_f16x8(t8);
+            if (which == 0) {
+                st16(rec + kRecTw + tc::swz_off(r, cc, 128), pack8<BF>(t8));
+            } else {
+                uint4 hi, lo;
+                split8<BF>(t8, hi, lo);
+                st16(rec + kRecTuHi + tc::swz_off(r, cc, 128), hi);
+                st16(rec + kRecTuLo + tc::swz_off(r, cc, 128), lo);
+            }
         }
     }
     tc::tc_fence_before();
@@ -412,35 +456,38 @@ __global__ void __launch_bounds__(128) chunk_ut_kernel(const __grid_constant__ C
 
 template <int NS>
 struct ChainCfg {
-    static constexpr int ROWB = NS * 2;                      // bytes per row of a slab tile (fp16)
+    static constexpr int ROWB = NS * 2;                        // bytes per row of a 16-bit slab tile
     static constexpr uint32_t SWZ = NS == 32 ? tc::kSw64 : tc::kSw128;
-    static constexpr int XREG = 192 * 128;                    // one K-half region of [K;Q;W]
-    static constexpr int OFF_X = 0;                           // [2] [K;Q;W] fp16: 2 x [192 x 128 B]
-    static constexpr int OFF_TT = OFF_X + 2 * 2 * XREG;       // [T_w; T_u]: [128 x 128 B]
-    static constexpr int OFF_M = OFF_TT + 16384;              // [2] M: [64 x 128 B]
-    static constexpr int OFF_STG = OFF_M + 2 * 8192;          // staging: 2 x [K;Q] half [128 x 128 B]
-    static constexpr int STG_BYTES = 32768;
-    static constexpr uint32_t STAGE_TX = 32768 + 64 * ROWB;   // K, Q halves and the V slab, per chunk
-    static constexpr int OFF_VS = OFF_STG + STG_BYTES;        // [2] V slab fp16 [64 x ROWB]
-    static constexpr int OFF_SS = OFF_VS + 2 * 64 * ROWB;     // S operand [128 x ROWB]
-    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;        // U operand [64 x ROWB]
-    static constexpr int OFF_SU2 = OFF_SU + 64 * ROWB;        // U' = diag(Gamma_C/Gamma) U
-    static constexpr int OFF_YS = OFF_SU2 + 64 * ROWB;        // y rows for bulk stores [64 x NS x 4 B]
-    static constexpr int OFF_VEC = OFF_YS + 64 * NS * 4;      // [2] gamma, Gamma, f: 3 x 64 floats (1 KB)
-    static constexpr int OFF_META = OFF_VEC + 2 * 1024;       // [2] {c0, L}
+    static constexpr int QW_HALF = 128 * 128;                  // one 64-column half of [Q;W]
+    static constexpr int K_HALF = 64 * 128;                    // one 64-column half of K
+    static constexpr int OFF_QW = 0;                           // [2 slots] [Q;W]: 2 halves x [128 x 128 B]
+    static constexpr int OFF_M = OFF_QW + 2 * 2 * QW_HALF;     // [2 slots] [M hi; M lo]: [128 x 128 B]
+    static constexpr int OFF_KS = OFF_M + 2 * 16384;           // [3 stages] K: 2 halves x [64 x 128 B]
+    static constexpr int OFF_TT = OFF_KS + 3 * 2 * K_HALF;     // [T_w; T_w; T_u hi; T_u lo]: [256 x 128 B]
+    static constexpr int OFF_VS = OFF_TT + 32768;              // [3 stages] V slab [64 x ROWB]
+    static constexpr int OFF_SS = OFF_VS + 3 * 64 * ROWB;      // S [128 x ROWB]
+    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // U hi, U lo: 2 x [64 x ROWB]
+    static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // U' hi, U' lo
+    static constexpr int OFF_YS = OFF_SU2 + 2 * 64 * ROWB;     // y rows for the TMA store [64 x NS x 4 B]
+    static constexpr int OFF_VEC = OFF_YS + 64 * NS * 4;       // [2 slots] gamma, Gamma, f: 3 x 64 floats
+    static constexpr int OFF_META = OFF_VEC + 2 * 1024;        // [2 slots] {c0, L}
     static constexpr int OFF_BAR = OFF_META + 64;
-    static constexpr int BYTES = OFF_BAR + 128 + 1024;
-    static constexpr uint32_t COL_UT = 0;                     // [2] x NS (rows 64-127)
-    static constexpr uint32_t COL_W = 2 * NS;                 // 128 (rows 0-63)
-    static constexpr uint32_t COL_1 = COL_W + 128;            // NS
-    static constexpr uint32_t COL_MU = COL_1 + NS;            // NS (rows 0-63)
-    static constexpr uint32_t COL_DS = COL_MU + NS;           // NS
+    static constexpr int BYTES = OFF_BAR + 256 + 1024;
+    static constexpr uint32_t KV_TX = 2 * K_HALF + 64 * ROWB;  // K and the V slab of one chunk
+    static constexpr uint32_t QM_TX = 2 * 8192 + 16384;        // Q and M hi/lo of one chunk
+    // TMEM columns
+    static constexpr uint32_t COL_UT = 0;                      // [2 slots] x NS: U~ (lanes 64-127)
+    static constexpr uint32_t COL_W = 2 * NS;                  // 128: W (both lane halves)
+    static constexpr uint32_t COL_1 = COL_W + 128;             // NS: Q S (lanes 0-63), W S (64-127)
+    static constexpr uint32_t COL_MU = COL_1 + NS;             // NS: M U (lanes 0-63)
+    static constexpr uint32_t COL_DS = COL_MU + NS;            // NS: K^T U'
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(COL_DS + NS <= TMEM_COLS, "TMEM budget");
     static_assert(BYTES <= 232448, "shared memory budget");
+    static_assert(OFF_YS % 1024 == 0 && OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0, "swizzle atoms");
 };
 
-template <int NS>
+template <int NS, bool BF>
 __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a,
                                                              const __grid_constant__ ChainMaps maps) {
     using Cf = ChainCfg<NS>;
@@ -450,15 +497,16 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     const uint32_t sbase = tc::smem_u32(smem);
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
-    uint64_t* bar_p = bars + 0;      // producer-issued MMAs complete
-    uint64_t* bar_c = bars + 1;      // chain-issued MMAs complete
-    uint64_t* bar_full = bars + 2;   // [2] slot filled by the producer
-    uint64_t* bar_empty = bars + 4;  // [2] slot released by the chain
-    uint64_t* bar_stage = bars + 6;  // K, Q staging and V slab landed (bytes)
-    uint64_t* bar_tt = bars + 7;     // [T_w; T_u] of the next chunk landed in TT
-    uint64_t* bar_m = bars + 8;      // M of the current chunk landed in M[b]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 96);
-    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 104);
+    uint64_t* bar_p = bars + 0;        // producer-issued MMAs complete
+    uint64_t* bar_c = bars + 1;        // chain-issued state MMAs complete
+    uint64_t* bar_y = bars + 2;        // chain-issued M U complete
+    uint64_t* bar_tt = bars + 3;       // [T_w; T_u] of the next chunk landed in TT
+    uint64_t* bar_full = bars + 4;     // [2 slots] W, U~, gates of a chunk ready (producer)
+    uint64_t* bar_empty = bars + 6;    // [2 slots] slot, its U~ columns and the K stage released (chain)
+    uint64_t* bar_qm = bars + 8;       // [2 slots] Q and M landed (bytes)
+    uint64_t* bar_kv = bars + 10;      // [3 stages] K and V landed (bytes)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 128);
+    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 136);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slab = blockIdx.x % NSLAB;
@@ -474,7 +522,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (lane == 0) *s_base = base;
     }
     if (tid == 0) {
-        for (int i = 0; i < 9; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < 13; ++i) tc::mbar_init(bars + i, 1);
         tc::fence_mbar_init();
     }
     if (warp == 1) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
@@ -485,20 +533,21 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     const int rec_base = *s_base;
     const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     auto vec = [&](int b) { return reinterpret_cast<float*>(smem + Cf::OFF_VEC + b * 1024); };
-    auto Xoff = [&](int b) { return Cf::OFF_X + b * 2 * Cf::XREG; };
-    uint8_t* stg = smem + Cf::OFF_STG;
+    auto QWoff = [&](int b) { return Cf::OFF_QW + b * 2 * Cf::QW_HALF; };
+    auto Koff = [&](int s) { return Cf::OFF_KS + s * 2 * Cf::K_HALF; };
+    auto Voff = [&](int s) { return Cf::OFF_VS + s * 64 * Cf::ROWB; };
 
     if (warp < 4) {
         // =============================== chain group ===================================
         constexpr int BID = 1;
-        uint32_t ph = 0;
-        bool ok = true;
-        auto commit_wait = [&]() -> bool {
-            if (tid == 0) tc::mma_commit(bar_c);
-            bool w = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_c, ph, a.budget));
+        uint32_t ph_c = 0, ph_y = 0;
+        bool ok = true, c_pending = false, mu_pending = false;
+        // wait for a tcgen05.commit; on a timeout flag the error and let the MMAs drain
+        auto wait_mma = [&](uint64_t* bar, uint32_t& ph) -> bool {
+            const bool w = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar, ph, a.budget));
             if (!w) {
                 if (tid == 0) raise_error(kErrTimeout);
-                tc::mbar_wait_bounded(bar_c, ph, 4000000000ull);
+                tc::mbar_wait_bounded(bar, ph, 4000000000ull);
             }
             ph ^= 1u;
             tc::tc_fence_after();
@@ -510,16 +559,17 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::bar_sync(BID, 128);
             tc::tc_fence_after();
         };
-        const uint32_t id_slab = tc::idesc_f16(128, NS, false, true);
-        const uint32_t id_ds = tc::idesc_f16(128, NS, true, true);
-        // operand descriptors at k-step 0 of slot 0; k-steps and slots are byte offsets from these
-        const uint64_t dX0 = tc::smem_desc(sbase + Cf::OFF_X, 16, 1024, tc::kSw128);        // K-major [Q;W] rows
-        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_X, Cf::XREG, 1024, tc::kSw128);  // MN-major K
+        constexpr uint32_t id_slab = idesc16<BF>(128, NS, false, true);
+        constexpr uint32_t id_ds = idesc16<BF>(128, NS, true, true);
+        // operand descriptors at k-step 0 of slot / stage 0; k-steps and slots are byte offsets
+        const uint64_t dQW0 = tc::smem_desc(sbase + Cf::OFF_QW, 16, 1024, tc::kSw128);      // K-major [Q;W]
+        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_KS, Cf::K_HALF, 1024, tc::kSw128);  // MN-major K^T
         const uint64_t dM0 = tc::smem_desc(sbase + Cf::OFF_M, 16, 1024, tc::kSw128);
         const uint64_t dSS0 = tc::smem_desc(sbase + Cf::OFF_SS, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dSU0 = tc::smem_desc(sbase + Cf::OFF_SU, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const int ybytes = a.y_dt == kF32 ? 4 : 2;
+        const int yrow = NS * ybytes;  // 64 or 128 B: the y tile's swizzle span
 
         const size_t st_base = ((size_t)n * H + h) * 128 * 128 + (size_t)tid * 128 + slab * NS;
         float S[NS];
@@ -529,12 +579,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
         }
 #pragma unroll
-        for (int c = 0; c < NS / 8; ++c)
-            *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB)) = pack_f16x8(S + 8 * c);
+        for (int c = 0; c < NS / 8; ++c) st16(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB), pack8<BF>(S + 8 * c));
         operands_ready();
 
         // y of chunk c-1 is formed while chunk c's first MMA runs; a full chunk leaves with one
-        // TMA store, a sequence's last partial chunk with plain stores.
+        // TMA store (swizzled staging rows), a sequence's last partial chunk with plain stores.
         int py_c0 = 0, py_L = 0;  // the chunk whose M U waits in TMEM (py_L = 0: none)
         float py_g = 0.f;         // its Gamma_r (rows 0-63)
         float qs[NS];             // its (Q S) row (rows 0-63)
@@ -543,15 +592,26 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 float t[NS];
 #pragma unroll
                 for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_MU + 32 * q4, t + 32 * q4);
-                if (tid < py_L) {
-                    void* dst = py_L == kChunk ? static_cast<void*>(smem + Cf::OFF_YS + tid * NS * ybytes)
-                                               : static_cast<void*>(reinterpret_cast<uint8_t*>(a.y) +
-                                                                    (((size_t)(py_c0 + tid) * H + h) * 128 + slab * NS) * ybytes);
 #pragma unroll
-                    for (int j = 0; j < NS; j += 4)
-                        st4(dst, a.y_dt, j,
-                            make_float4(a.scale * (py_g * qs[j] + t[j]), a.scale * (py_g * qs[j + 1] + t[j + 1]),
-                                        a.scale * (py_g * qs[j + 2] + t[j + 2]), a.scale * (py_g * qs[j + 3] + t[j + 3])));
+                for (int j = 0; j < NS; ++j) t[j] = a.scale * (py_g * qs[j] + t[j]);
+                if (py_L == kChunk) {
+                    uint8_t* ys = smem + Cf::OFF_YS;
+                    if (a.y_dt == kF32) {
+#pragma unroll
+                        for (int cc = 0; cc < NS / 4; ++cc)
+                            *reinterpret_cast<float4*>(ys + tc::swz_off(tid, cc, yrow)) =
+                                make_float4(t[4 * cc], t[4 * cc + 1], t[4 * cc + 2], t[4 * cc + 3]);
+                    } else if (a.y_dt == kBF16) {
+#pragma unroll
+                        for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, yrow), pack8<true>(t + 8 * cc));
+                    } else {
+#pragma unroll
+                        for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, yrow), pack8<false>(t + 8 * cc));
+                    }
+                } else if (tid < py_L) {
+                    void* dst = reinterpret_cast<uint8_t*>(a.y) + (((size_t)(py_c0 + tid) * H + h) * 128 + slab * NS) * ybytes;
+#pragma unroll
+                    for (int j = 0; j < NS; j += 4) st4(dst, a.y_dt, j, make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]));
                 }
             }
         };
@@ -564,8 +624,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         };
 
         for (int c = 0; c < nchunks; ++c) {
-            const int b = c & 1;
-            if (!(ok = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget)))) {
+            const int b = c & 1, kst = c % 3;
+            bool w = tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget);
+            w = w && tc::mbar_wait_bounded(bar_qm + b, (c >> 1) & 1, a.budget);
+            if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (tid == 0) raise_error(kErrTimeout);
                 break;
             }
@@ -576,22 +638,29 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const float gR = tid < 64 ? vb[64 + tid] : 0.f;
             const float fR = tid >= 64 ? vb[128 + tid - 64] : 0.f;
 
-            // [Q;W] S  -> Q S (rows 0-63), W S (rows 64-127)
+            // [Q;W] S -> Q S (lanes 0-63), W S (lanes 64-127)
             if (tid == 0) {
-                const uint64_t aw0 = desc_add(dX0, b * 2 * Cf::XREG + 64 * 128);
+                const uint64_t a0 = desc_add(dQW0, QWoff(b));
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(tmem + Cf::COL_1, desc_add(aw0, (kk >> 2) * Cf::XREG + (kk & 3) * 32),
+                    tc::mma_f16(tmem + Cf::COL_1, desc_add(a0, (kk >> 2) * Cf::QW_HALF + (kk & 3) * 32),
                                 desc_add(dSS0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
+                tc::mma_commit(bar_c);
             }
-            y_epilogue();  // previous chunk's y while the MMA runs
-            if (!(ok = commit_wait())) break;
+            c_pending = true;
+            if (mu_pending) {  // the previous chunk's M U, for its y
+                mu_pending = false;
+                if (!(ok = wait_mma(bar_y, ph_y))) break;
+            }
+            y_epilogue();
+            c_pending = false;
+            if (!(ok = wait_mma(bar_c, ph_c))) break;
 
             {
                 float d1[NS];
 #pragma unroll
                 for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_1 + 32 * q4, d1 + 32 * q4);
-                if (warp >= 2) {  // U = U~ - W S, U' = f U
+                if (warp >= 2) {  // U = U~ - W S (hi + lo), U' = f U (hi + lo)
                     const int r = tid - 64;
                     float ut[NS];
 #pragma unroll
@@ -600,11 +669,16 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     for (int j = 0; j < NS; ++j) ut[j] -= d1[j];
 #pragma unroll
                     for (int cc = 0; cc < NS / 8; ++cc) {
-                        *reinterpret_cast<uint4*>(smem + Cf::OFF_SU + tc::swz_off(r, cc, Cf::ROWB)) = pack_f16x8(ut + 8 * cc);
+                        uint4 hi, lo;
+                        split8<BF>(ut + 8 * cc, hi, lo);
+                        st16(smem + Cf::OFF_SU + tc::swz_off(r, cc, Cf::ROWB), hi);
+                        st16(smem + Cf::OFF_SU + 64 * Cf::ROWB + tc::swz_off(r, cc, Cf::ROWB), lo);
                         float u2[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
-                        *reinterpret_cast<uint4*>(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::ROWB)) = pack_f16x8(u2);
+                        split8<BF>(u2, hi, lo);
+                        st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::ROWB), hi);
+                        st16(smem + Cf::OFF_SU2 + 64 * Cf::ROWB + tc::swz_off(r, cc, Cf::ROWB), lo);
                     }
                 } else {
 #pragma unroll
@@ -614,17 +688,28 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             operands_ready();  // also orders the staged y rows before their TMA store
             y_store();
 
-            // [M;.] U -> M U (rows 0-63) ;  K^T U' -> state increment
+            // K^T U' -> state increment (waited on); then M U -> y (waited on with the next chunk)
             if (tid == 0) {
-                const uint64_t am0 = desc_add(dM0, b * 8192), ak0 = desc_add(dK0, b * 2 * Cf::XREG);
+                const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS), am0 = desc_add(dM0, b * 16384);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(dSU0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
                     tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::ROWB), id_ds, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048),
+                                desc_add(dSU20, 64 * Cf::ROWB + kk * 16 * Cf::ROWB), id_ds, 1);
                 }
+                tc::mma_commit(bar_c);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {  // [M hi; M lo] U hi + [M hi; M lo] U lo + [M lo; .] U hi
+                    const uint64_t bu = desc_add(dSU0, kk * 16 * Cf::ROWB);
+                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), bu, id_slab, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(bu, 64 * Cf::ROWB), id_slab, 1);
+                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, 8192 + kk * 32), bu, id_slab, 1);
+                }
+                tc::mma_commit(bar_y);
+                tc::mma_commit(bar_empty + b);  // slot b, its U~ columns and K stage kst are free
             }
-            if (!(ok = commit_wait())) break;
-            if (tid == 0) tc::mbar_arrive(bar_empty + b);  // slot b (X, M, U~ columns) is free
+            mu_pending = true;
+            if (!(ok = wait_mma(bar_c, ph_c))) break;
 
             {
                 float t[NS];
@@ -633,8 +718,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
 #pragma unroll
                 for (int j = 0; j < NS; ++j) S[j] = gC * S[j] + t[j];
 #pragma unroll
-                for (int cc = 0; cc < NS / 8; ++cc)
-                    *reinterpret_cast<uint4*>(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB)) = pack_f16x8(S + 8 * cc);
+                for (int cc = 0; cc < NS / 8; ++cc) st16(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB), pack8<BF>(S + 8 * cc));
             }
             py_c0 = c0;
             py_L = L;
@@ -642,12 +726,18 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next y_epilogue writes it
             operands_ready();
         }
-        if (ok) {
-            y_epilogue();
-            tc::fence_async_smem();
-            tc::bar_sync(BID, 128);
-            y_store();
+        if (ok && mu_pending) {
+            mu_pending = false;
+            if ((ok = wait_mma(bar_y, ph_y))) {
+                y_epilogue();
+                tc::fence_async_smem();
+                tc::bar_sync(BID, 128);
+                y_store();
+            }
         }
+        // never free TMEM under an MMA in flight
+        if (c_pending) tc::mbar_wait_bounded(bar_c, ph_c, 4000000000ull);
+        if (mu_pending) tc::mbar_wait_bounded(bar_y, ph_y, 4000000000ull);
         if (tid == 0) tc::bulk_wait0();
         if (ok && a.S_T) {
 #pragma unroll
@@ -660,51 +750,51 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         const int it = tid - 128;
         uint32_t ph = 0;
         bool ok = true;
-        const uint32_t id_slab = tc::idesc_f16(128, NS, false, true);
-        const uint32_t id_w = tc::idesc_f16(128, 128, false, true);
+        constexpr uint32_t id_v = idesc16<BF>(128, NS, false, true);
+        constexpr uint32_t id_w = idesc16<BF>(128, 128, false, true);
         const uint64_t dTT0 = tc::smem_desc(sbase + Cf::OFF_TT, 16, 1024, tc::kSw128);
         const uint64_t dV0 = tc::smem_desc(sbase + Cf::OFF_VS, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_X, Cf::XREG, 1024, tc::kSw128);  // MN-major K
+        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_KS, Cf::K_HALF, 1024, tc::kSw128);  // MN-major K
 
-        // TMA copies of chunk ci's K, Q halves (staging), V slab (its operand slot) and record
-        int issued = -1, landed = -1;        // last chunk whose staging copies were issued / waited for
-        int tt_issued = -1, tt_landed = -1;  // same for the [T_w; T_u] part of the records
-        int m_issued = -1, m_landed = -1;    // same for the M part
+        // copies in flight into this CTA's shared memory, for the exit drain
+        int kv_issued = -1, kv_landed = -1, tt_issued = -1, tt_landed = -1;
+        int qm_last0 = -1, qm_last1 = -1;  // last chunk whose Q/M copies went to slot 0 / 1
         auto rec_ptr = [&](int ci) {
             return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
         };
-        // TMA copies of chunk ci's K, Q halves (staging) and V slab (its operand slot)
-        auto issue_loads = [&](int ci) {
-            issued = ci;
+        auto issue_kv = [&](int ci) {  // K and the V slab of chunk ci -> stage ci % 3
+            kv_issued = ci;
+            if (it != 0) return;
+            const int c0 = t_begin + ci * kChunk, s = ci % 3;
+            uint64_t* bk = bar_kv + s;
+            tc::mbar_arrive_expect_tx(bk, Cf::KV_TX);
+            tc::tma_load_3d(smem + Koff(s), &maps.k, 0, h, c0, bk);
+            tc::tma_load_3d(smem + Koff(s) + Cf::K_HALF, &maps.k, 64, h, c0, bk);
+            tc::tma_load_3d(smem + Voff(s), &maps.v, slab * NS, h, c0, bk);
+        };
+        auto issue_qm = [&](int ci) {  // Q of chunk ci and its M hi/lo -> slot ci & 1
+            const int bb = ci & 1;
+            (bb ? qm_last1 : qm_last0) = ci;
             if (it != 0) return;
             const int c0 = t_begin + ci * kChunk;
-            tc::mbar_arrive_expect_tx(bar_stage, Cf::STAGE_TX);
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                tc::tma_load_3d(stg + hf * 16384, &maps.k, 64 * hf, h, c0, bar_stage);
-                tc::tma_load_3d(stg + hf * 16384 + 8192, &maps.q, 64 * hf, h, c0, bar_stage);
-            }
-            tc::tma_load_3d(smem + Cf::OFF_VS + (ci & 1) * 64 * Cf::ROWB, &maps.v, slab * NS, h, c0, bar_stage);
+            uint64_t* bq = bar_qm + bb;
+            uint8_t* qw = smem + QWoff(bb);
+            tc::mbar_arrive_expect_tx(bq, Cf::QM_TX);
+            tc::tma_load_3d(qw, &maps.q, 0, h, c0, bq);
+            tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bq);
+            tc::bulk_g2s(smem + Cf::OFF_M + bb * 16384, rec_ptr(ci) + kRecMHi, 16384, bq);
         };
-        auto issue_tt = [&](int ci) {  // record bytes [0, 16 KB) -> TT
+        auto issue_tt = [&](int ci) {  // [T_w; T_w; T_u hi; T_u lo] of chunk ci -> TT
             tt_issued = ci;
             if (it != 0) return;
-            tc::mbar_arrive_expect_tx(bar_tt, 16384);
-            tc::bulk_g2s(smem + Cf::OFF_TT, rec_ptr(ci), 16384, bar_tt);
+            tc::mbar_arrive_expect_tx(bar_tt, 32768);
+            tc::bulk_g2s(smem + Cf::OFF_TT, rec_ptr(ci) + kRecTw, 8192, bar_tt);
+            tc::bulk_g2s(smem + Cf::OFF_TT + 8192, rec_ptr(ci) + kRecTw, 24576, bar_tt);
         };
-        auto issue_m = [&](int ci) {  // record bytes [16 KB, 24 KB) -> M[ci & 1]
-            m_issued = ci;
-            if (it != 0) return;
-            tc::mbar_arrive_expect_tx(bar_m, 8192);
-            tc::bulk_g2s(smem + Cf::OFF_M + (ci & 1) * 8192, rec_ptr(ci) + 16384, 8192, bar_m);
-        };
-        float pg = 0.f, pb = 0.f;
+        float pg = 0.f;  // g of the next chunk (beta is already inside T_w, T_u)
         auto load_gates = [&](int ci) {
             const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
-            if (it < 64) {
-                pg = it < L ? a.g[(size_t)(c0 + it) * H + h] : 0.f;
-                pb = it < L ? a.beta[(size_t)(c0 + it) * H + h] : 0.f;
-            }
+            if (it < 64) pg = it < L ? a.g[(size_t)(c0 + it) * H + h] : 0.f;
         };
         if (it == 0) {
             tc::prefetch_tmap(&maps.k);
@@ -712,49 +802,25 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::prefetch_tmap(&maps.v);
         }
         if (nchunks > 0) {
-            issue_loads(0);
+            issue_kv(0);
             issue_tt(0);
             load_gates(0);
         }
 
         for (int c = 0; c < nchunks; ++c) {
-            const int b = c & 1;
+            const int b = c & 1, kst = c % 3;
             const int c0 = t_begin + c * kChunk, L = min(kChunk, t_end - c0);
             float* vb = vec(b);
-            // slot b must be free (chain done with chunk c-2) and staging must hold chunk c
+            // slot b, its U~ columns and K stage (c+1) % 3 are free once the chain is done with c-2
             bool w = tc::mbar_wait_bounded(bar_empty + b, ((c >> 1) & 1) ^ 1, a.budget);
-            w = w && tc::mbar_wait_bounded(bar_stage, c & 1, a.budget);
             if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (it == 0) raise_error(kErrTimeout);
                 break;
             }
-            landed = c;
-            issue_m(c);  // slot b is free: its M rows can come in now
-            tc::tc_fence_after();
+            issue_qm(c);
+            if (c + 1 < nchunks) issue_kv(c + 1);
 
-            // ---- fp16 operand tiles: K, Q rows of [K;Q;W] (same swizzled offsets as staged), V in
-            //      place, the record into TT and M[b]; rows past the sequence end are zeroed
-            uint8_t* X = smem + Xoff(b);
-            uint8_t* VSb = smem + Cf::OFF_VS + b * 64 * Cf::ROWB;
-            constexpr int VU = (64 * Cf::ROWB / 16) / 128;
-            {
-                uint4 raw[16], vraw[VU];  // every load issued before the first store
-#pragma unroll
-                for (int u = 0; u < 16; ++u) raw[u] = *reinterpret_cast<const uint4*>(stg + (it + 128 * u) * 16);
-#pragma unroll
-                for (int u = 0; u < VU; ++u) vraw[u] = *reinterpret_cast<const uint4*>(VSb + (it + 128 * u) * 16);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int idx = it + 128 * u, hf = idx >> 10, rem = idx & 1023, row = rem >> 3;  // 0-63 K, 64-127 Q
-                    *reinterpret_cast<uint4*>(X + hf * Cf::XREG + rem * 16) =
-                        (row & 63) < L ? to_f16x8(raw[u], a.in_dt) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < VU; ++u) {
-                    const int idx = it + 128 * u, row = idx / (Cf::ROWB / 16);
-                    *reinterpret_cast<uint4*>(VSb + idx * 16) = row < L ? to_f16x8(vraw[u], a.in_dt) : make_uint4(0, 0, 0, 0);
-                }
-            }
+            // ---- gates of chunk c: gamma (inclusive prefix sum), Gamma, f = exp(gamma_C - gamma) --
             if (it < 64) {
                 float gv = pg;
 #pragma unroll
@@ -768,33 +834,32 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 meta[2 * b] = c0;
                 meta[2 * b + 1] = L;
             }
-            tc::fence_async_smem();  // staging reads precede the next bulk copies into it
             tc::bar_sync(BID, 128);
-            if (c + 1 < nchunks) issue_loads(c + 1);
             if (it >= 32 && it < 64) vb[it] += vb[31];
             tc::bar_sync(BID, 128);
             if (it < 64) {
                 vb[64 + it] = __expf(vb[it]);
                 vb[128 + it] = __expf(vb[63] - vb[it]);
             }
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::bar_sync(BID, 128);
-            tc::tc_fence_after();
 
-            // ---- U~ = T_u V (rows 64-127 of this slot's columns) and W = T_w K (rows 0-63) ------
-            if (!(ok = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_tt, c & 1, a.budget)))) {
+            // ---- W = T_w K (both lane halves), U~ = T_u hi V + T_u lo V (lanes 64-127) -----------
+            w = tc::mbar_wait_bounded(bar_kv + kst, (c / 3) & 1, a.budget);
+            w = w && tc::mbar_wait_bounded(bar_tt, c & 1, a.budget);
+            if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (it == 0) raise_error(kErrTimeout);
                 break;
             }
+            kv_landed = c;
             tt_landed = c;
+            tc::tc_fence_after();
             if (it == 0) {
-                const uint64_t bv0 = desc_add(dV0, b * 64 * Cf::ROWB), bk0 = desc_add(dK0, b * 2 * Cf::XREG);
+                const uint64_t bv0 = desc_add(dV0, Voff(kst) - Cf::OFF_VS), bk0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t at = desc_add(dTT0, kk * 32);
-                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, at, desc_add(bv0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
-                    tc::mma_f16(tmem + Cf::COL_W, at, desc_add(bk0, kk * 2048), id_w, kk > 0);
+                    const uint64_t bv = desc_add(bv0, kk * 16 * Cf::ROWB);
+                    tc::mma_f16(tmem + Cf::COL_W, desc_add(dTT0, kk * 32), desc_add(bk0, kk * 2048), id_w, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, desc_add(dTT0, 8192 + kk * 32), bv, id_v, kk > 0);
+                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, desc_add(dTT0, 16384 + kk * 32), bv, id_v, 1);
                 }
                 tc::mma_commit(bar_p);
             }
@@ -808,35 +873,30 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             if (!(ok = w)) break;
             if (c + 1 < nchunks) issue_tt(c + 1);  // the MMAs have read TT
 
-            // ---- W -> rows 128-191 of [K;Q;W] ----------------------------------------------------
-            if (it < 64) {
+            // ---- W -> rows 64-127 of [Q;W] in slot b: lanes 0-63 write columns 0-63, lanes 64-127
+            //      columns 64-127 (each lane half of the accumulator holds all of W) ------------------
+            {
+                const int r = it & 63, hf = it >> 6;
+                float wv[64];
+                tc::tmem_ld32(trow + Cf::COL_W + 64 * hf, wv);
+                tc::tmem_ld32(trow + Cf::COL_W + 64 * hf + 32, wv + 32);
+                uint8_t* qw = smem + QWoff(b) + hf * Cf::QW_HALF;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float wv[32];
-                    tc::tmem_ld32(trow + Cf::COL_W + 32 * q4, wv);
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        const int ch = q4 * 4 + cc;
-                        *reinterpret_cast<uint4*>(X + (ch >> 3) * Cf::XREG + tc::swz_off(128 + it, ch & 7, 128)) =
-                            pack_f16x8(wv + 8 * cc);
-                    }
-                }
+                for (int cc = 0; cc < 8; ++cc) st16(qw + tc::swz_off(64 + r, cc, 128), pack8<BF>(wv + 8 * cc));
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
-            w = tc::mbar_wait_bounded(bar_m, c & 1, a.budget);  // M rows of slot b landed
-            if (!(ok = tc::bar_and(BID, 128, w))) {
-                if (it == 0) raise_error(kErrTimeout);
-                break;
-            }
-            m_landed = c;
+            tc::bar_sync(BID, 128);
             if (it == 0) tc::mbar_arrive(bar_full + b);  // hand slot b to the chain group
             if (c + 1 < nchunks) load_gates(c + 1);
         }
         // never leave with copies into this CTA's shared memory in flight
-        if (issued > landed) tc::mbar_wait_bounded(bar_stage, issued & 1, 4000000000ull);
+        if (kv_issued > kv_landed) tc::mbar_wait_bounded(bar_kv + kv_issued % 3, (kv_issued / 3) & 1, 4000000000ull);
+        if (kv_issued > kv_landed + 1)
+            tc::mbar_wait_bounded(bar_kv + (kv_issued - 1) % 3, ((kv_issued - 1) / 3) & 1, 4000000000ull);
         if (tt_issued > tt_landed) tc::mbar_wait_bounded(bar_tt, tt_issued & 1, 4000000000ull);
-        if (m_issued > m_landed) tc::mbar_wait_bounded(bar_m, m_issued & 1, 4000000000ull);
+        if (qm_last0 >= 0) tc::mbar_wait_bounded(bar_qm + 0, (qm_last0 >> 1) & 1, 4000000000ull);
+        if (qm_last1 >= 0) tc::mbar_wait_bounded(bar_qm + 1, (qm_last1 >> 1) & 1, 4000000000ull);
         (void)ok;
     }
 
@@ -879,6 +939,28 @@ inline bool encode_map_3d(CUtensorMap* m, const void* base, int dt, int N, int H
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <bool BF>
+inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, cudaStream_t st) {
+    constexpr int NS = 32;
+    using Ch = ChainCfg<NS>;
+    cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel<BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, UtCfg::BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_chain_kernel<NS, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
+    if (e != cudaSuccess) return e;
+    const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
+    if (nvc > 0) {
+        LaunchScope timed(st, "chunk_ut_kernel");
+        chunk_ut_kernel<BF><<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a, maps);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    LaunchScope timed(st, "chunk_chain_kernel");
+    chunk_chain_kernel<NS, BF><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a, maps);
+    return cudaGetLastError();
+}
+
+// Both kernels of the chunked path on stream st.  *why is set (and nothing launched) when the
+// configuration is not built or a tensor map cannot be encoded.
 inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const char** why) {
     *why = nullptr;
     if (a.chunk != kChunk) {
@@ -886,29 +968,17 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
         return cudaSuccess;
     }
     constexpr int NS = 32;
-    using Ch = ChainCfg<NS>;
+    // y tiles are NS columns = 64 B (16-bit) or 128 B (fp32) per row, stored with the matching swizzle
+    const CUtensorMapSwizzle yswz = a.y_dt == kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     ChainMaps maps;
     if (!encode_map_3d(&maps.k, a.k, a.in_dt, a.N, a.H, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.q, a.q, a.in_dt, a.N, a.H, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, NS, kChunk, yswz)) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaSuccess;
     }
-    cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, UtCfg::BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_chain_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
-    if (e != cudaSuccess) return e;
-    const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
-    if (nvc > 0) {
-        LaunchScope timed(st, "chunk_ut_kernel");
-        chunk_ut_kernel<<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a, maps);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    LaunchScope timed(st, "chunk_chain_kernel");
-    chunk_chain_kernel<NS><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a, maps);
-    return cudaGetLastError();
+    return a.in_dt == kBF16 ? chunk_tc_launch_t<true>(a, maps, st) : chunk_tc_launch_t<false>(a, maps, st);
 }
 
 }  // namespace gdn
