@@ -32,10 +32,13 @@
 //                       Y = Gamma (Q S) + M U, completes off the chain.  Q/W/M slots are
 //                       double-buffered, K/V stages triple-buffered, all handed over with
 //                       mbarriers; full chunks of y leave through swizzled TMA stores.
-// Operands are 16-bit in the inputs' own format (bf16 or fp16) with fp32 accumulation in
-// TMEM.  q, k, v enter the products exactly as stored.  A computed operand x whose rounding
-// would show in y or the state (T_u, M, U, U') enters as two products, hi = round(x) and
-// lo = round(x - hi), which carries 16 significant bits for bf16; T_w, W and S enter once.
+// Operands are 16-bit with fp32 accumulation in TMEM.  q, k, v enter the products exactly as
+// stored (bf16 or fp16), so their partners take the same format.  A computed partner whose
+// rounding would show in y or the state (T_u, U') enters as two products, hi = round(x) and
+// lo = round(x - hi), which carries 16 significant bits for bf16; T_w, W and S enter once.  M U
+// pairs two computed operands, so it runs in fp16 (11 significant bits) whatever the input
+// format.  Records and [hi | lo] pairs are side by side in one operand (N = 2 x 32), so each
+// pair costs one MMA per k-step.
 // Operand tiles use the 128B / 64B swizzled canonical layouts, so one tile serves as K-major
 // or MN-major operand.  Every wait is bounded (ChunkArgs::budget clock cycles); a wait that
 // runs out sets the device error word, lets in-flight MMAs and copies drain, and the CTA
@@ -69,14 +72,13 @@ struct ChainMaps {
 };
 
 constexpr int kChunk = 64;
-// Record of one (chunk, head), written by chunk_ut_kernel: five [64 rows x 128 B] operand tiles
-// in the 128B-swizzled K-major layout, 16-bit in the input's format.
-constexpr int kRecTw = 0;          // T_w = T diag(beta Gamma)
-constexpr int kRecTuHi = 8192;     // T_u = T diag(beta), high half
+// Record of one (chunk, head), written by chunk_ut_kernel: four [64 rows x 128 B] operand tiles
+// in the 128B-swizzled K-major layout.
+constexpr int kRecTw = 0;          // T_w = T diag(beta Gamma), 16-bit in the input's format
+constexpr int kRecTuHi = 8192;     // T_u = T diag(beta), high half (input's format)
 constexpr int kRecTuLo = 16384;    //   and the rounding remainder
-constexpr int kRecMHi = 24576;     // M, high half
-constexpr int kRecMLo = 32768;     //   and the rounding remainder
-constexpr int kRecBytes = 40960;
+constexpr int kRecM = 24576;       // M, fp16 (it only meets U, another computed operand)
+constexpr int kRecBytes = 32768;
 
 // Upper bound of the number of 64-token chunks over all sequences.
 inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
@@ -236,7 +238,8 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 16);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int v = blockIdx.x, h = blockIdx.y, H = a.H;
+    // heads vary fastest across the grid, so CTAs resident together read whole token rows
+    const int H = a.H, v = (int)(blockIdx.x / (unsigned)H), h = (int)(blockIdx.x % (unsigned)H);
     if (warp == 0) {
         int n = 0, j = 0;
         const bool found = locate_chunk(a.cu, a.num_seqs, a.N, v, n, j);
@@ -317,8 +320,8 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
     tc::tc_fence_after();
 
     if (landed && done) {
-        // ---- masks: A (fp32, over the consumed [K;Q] tiles) for the solve; M as hi + lo
-        //      16-bit halves straight into the record ---------------------------------------------
+        // ---- masks: A (fp32, over the consumed [K;Q] tiles) for the solve; M (fp16) straight
+        //      into the record ---------------------------------------------------------------------
         {
             float x[64];
             const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
@@ -346,10 +349,7 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
                     sts4(fA + r * LD + 8 * cc, make_float4(m[0], m[1], m[2], m[3]));
                     sts4(fA + r * LD + 8 * cc + 4, make_float4(m[4], m[5], m[6], m[7]));
                 } else {
-                    uint4 hi, lo;
-                    split8<BF>(m, hi, lo);
-                    st16(rec + kRecMHi + tc::swz_off(r, cc, 128), hi);
-                    st16(rec + kRecMLo + tc::swz_off(r, cc, 128), lo);
+                    st16(rec + kRecM + tc::swz_off(r, cc, 128), pack8<false>(m));
                 }
             }
         }
@@ -461,30 +461,33 @@ struct ChainCfg {
     static constexpr int QW_HALF = 128 * 128;                  // one 64-column half of [Q;W]
     static constexpr int K_HALF = 64 * 128;                    // one 64-column half of K
     static constexpr int OFF_QW = 0;                           // [2 slots] [Q;W]: 2 halves x [128 x 128 B]
-    static constexpr int OFF_M = OFF_QW + 2 * 2 * QW_HALF;     // [2 slots] [M hi; M lo]: [128 x 128 B]
-    static constexpr int OFF_KS = OFF_M + 2 * 16384;           // [3 stages] K: 2 halves x [64 x 128 B]
+    static constexpr int OFF_M = OFF_QW + 2 * 2 * QW_HALF;     // [2 slots] M fp16: [64 x 128 B]
+    static constexpr int OFF_KS = OFF_M + 2 * 8192;            // [3 stages] K: 2 halves x [64 x 128 B]
     static constexpr int OFF_TT = OFF_KS + 3 * 2 * K_HALF;     // [T_w; T_w; T_u hi; T_u lo]: [256 x 128 B]
     static constexpr int OFF_VS = OFF_TT + 32768;              // [3 stages] V slab [64 x ROWB]
     static constexpr int OFF_SS = OFF_VS + 3 * 64 * ROWB;      // S [128 x ROWB]
-    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // U hi, U lo: 2 x [64 x ROWB]
-    static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // U' hi, U' lo
+    static constexpr int UROWB = 2 * ROWB;                      // [hi | lo] rows of U': 128 B
+    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // U fp16: [64 x ROWB]
+    static constexpr int OFF_SU2 = OFF_SU + 64 * ROWB;         // [U' hi | U' lo]: [64 x UROWB]
     static constexpr int OFF_YS = OFF_SU2 + 2 * 64 * ROWB;     // y rows for the TMA store [64 x NS x 4 B]
     static constexpr int OFF_VEC = OFF_YS + 64 * NS * 4;       // [2 slots] gamma, Gamma, f: 3 x 64 floats
     static constexpr int OFF_META = OFF_VEC + 2 * 1024;        // [2 slots] {c0, L}
     static constexpr int OFF_BAR = OFF_META + 64;
     static constexpr int BYTES = OFF_BAR + 256 + 1024;
     static constexpr uint32_t KV_TX = 2 * K_HALF + 64 * ROWB;  // K and the V slab of one chunk
-    static constexpr uint32_t QM_TX = 2 * 8192 + 16384;        // Q and M hi/lo of one chunk
+    static constexpr uint32_t QM_TX = 2 * 8192 + 8192;         // Q and M of one chunk
     // TMEM columns
     static constexpr uint32_t COL_UT = 0;                      // [2 slots] x NS: U~ (lanes 64-127)
     static constexpr uint32_t COL_W = 2 * NS;                  // 128: W (both lane halves)
     static constexpr uint32_t COL_1 = COL_W + 128;             // NS: Q S (lanes 0-63), W S (64-127)
     static constexpr uint32_t COL_MU = COL_1 + NS;             // NS: M U (lanes 0-63)
-    static constexpr uint32_t COL_DS = COL_MU + NS;            // NS: K^T U'
+    static constexpr uint32_t COL_DS = COL_MU + NS;            // 2 NS: [K^T U' hi | K^T U' lo]
     static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(COL_DS + NS <= TMEM_COLS, "TMEM budget");
+    static_assert(COL_DS + 2 * NS <= TMEM_COLS, "TMEM budget");
+    static_assert(NS == 32, "[hi | lo] operand rows are one 128-byte swizzle atom");
     static_assert(BYTES <= 232448, "shared memory budget");
-    static_assert(OFF_YS % 1024 == 0 && OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0, "swizzle atoms");
+    static_assert(OFF_YS % 1024 == 0 && OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0 && OFF_SU2 % 1024 == 0,
+                  "swizzle atoms");
 };
 
 template <int NS, bool BF>
@@ -542,32 +545,37 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         constexpr int BID = 1;
         uint32_t ph_c = 0, ph_y = 0;
         bool ok = true, c_pending = false, mu_pending = false;
-        // wait for a tcgen05.commit; on a timeout flag the error and let the MMAs drain
+        // each thread waits for a tcgen05.commit on its own; a timeout flags the error, lets the
+        // MMAs drain, and is combined over the group at the next barrier
         auto wait_mma = [&](uint64_t* bar, uint32_t& ph) -> bool {
-            const bool w = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar, ph, a.budget));
+            const bool w = tc::mbar_wait_bounded(bar, ph, a.budget);
             if (!w) {
-                if (tid == 0) raise_error(kErrTimeout);
+                raise_error(kErrTimeout);
                 tc::mbar_wait_bounded(bar, ph, 4000000000ull);
             }
             ph ^= 1u;
             tc::tc_fence_after();
             return w;
         };
-        auto operands_ready = [&]() {
+        // smem operands written by this group become visible to the tensor cores and TMA;
+        // returns the AND of v over the group
+        auto operands_ready = [&](bool v) -> bool {
             tc::fence_async_smem();
             tc::tc_fence_before();
-            tc::bar_sync(BID, 128);
+            const bool all = tc::bar_and(BID, 128, v);
             tc::tc_fence_after();
+            return all;
         };
         constexpr uint32_t id_slab = idesc16<BF>(128, NS, false, true);
-        constexpr uint32_t id_ds = idesc16<BF>(128, NS, true, true);
+        constexpr uint32_t id_ds = idesc16<BF>(128, 2 * NS, true, true);  // K^T [U' hi | U' lo]
+        constexpr uint32_t id_mu = idesc16<false>(128, NS, false, true);  // M U, both fp16
         // operand descriptors at k-step 0 of slot / stage 0; k-steps and slots are byte offsets
         const uint64_t dQW0 = tc::smem_desc(sbase + Cf::OFF_QW, 16, 1024, tc::kSw128);      // K-major [Q;W]
         const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_KS, Cf::K_HALF, 1024, tc::kSw128);  // MN-major K^T
         const uint64_t dM0 = tc::smem_desc(sbase + Cf::OFF_M, 16, 1024, tc::kSw128);
         const uint64_t dSS0 = tc::smem_desc(sbase + Cf::OFF_SS, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dSU0 = tc::smem_desc(sbase + Cf::OFF_SU, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-        const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
+        const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::UROWB, 8 * Cf::UROWB, tc::kSw128);
         const int ybytes = a.y_dt == kF32 ? 4 : 2;
         const int yrow = NS * ybytes;  // 64 or 128 B: the y tile's swizzle span
 
@@ -580,7 +588,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         }
 #pragma unroll
         for (int c = 0; c < NS / 8; ++c) st16(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB), pack8<BF>(S + 8 * c));
-        operands_ready();
+        operands_ready(true);
 
         // y of chunk c-1 is formed while chunk c's first MMA runs; a full chunk leaves with one
         // TMA store (swizzled staging rows), a sequence's last partial chunk with plain stores.
@@ -590,8 +598,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         auto y_epilogue = [&]() {  // warps 0-1: y = scale (Gamma_r (Q S) + M U) of chunk py
             if (warp < 2 && py_L > 0) {
                 float t[NS];
-#pragma unroll
-                for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_MU + 32 * q4, t + 32 * q4);
+                tc::tmem_ld32(trow + Cf::COL_MU, t);
 #pragma unroll
                 for (int j = 0; j < NS; ++j) t[j] = a.scale * (py_g * qs[j] + t[j]);
                 if (py_L == kChunk) {
@@ -648,19 +655,21 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 tc::mma_commit(bar_c);
             }
             c_pending = true;
-            if (mu_pending) {  // the previous chunk's M U, for its y
+            bool w_y = true;
+            if (mu_pending) {  // the previous chunk's M U, for its y (warps 0-1 only)
                 mu_pending = false;
-                if (!(ok = wait_mma(bar_y, ph_y))) break;
+                if (warp < 2) w_y = wait_mma(bar_y, ph_y);
+                else ph_y ^= 1u;
             }
-            y_epilogue();
+            if (w_y) y_epilogue();
+            const bool w1 = wait_mma(bar_c, ph_c);
             c_pending = false;
-            if (!(ok = wait_mma(bar_c, ph_c))) break;
 
             {
                 float d1[NS];
 #pragma unroll
                 for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_1 + 32 * q4, d1 + 32 * q4);
-                if (warp >= 2) {  // U = U~ - W S (hi + lo), U' = f U (hi + lo)
+                if (warp >= 2) {  // U = U~ - W S (fp16, for M U), U' = f U (hi + lo, for K^T U')
                     const int r = tid - 64;
                     float ut[NS];
 #pragma unroll
@@ -670,53 +679,44 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
 #pragma unroll
                     for (int cc = 0; cc < NS / 8; ++cc) {
                         uint4 hi, lo;
-                        split8<BF>(ut + 8 * cc, hi, lo);
-                        st16(smem + Cf::OFF_SU + tc::swz_off(r, cc, Cf::ROWB), hi);
-                        st16(smem + Cf::OFF_SU + 64 * Cf::ROWB + tc::swz_off(r, cc, Cf::ROWB), lo);
+                        st16(smem + Cf::OFF_SU + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(ut + 8 * cc));
                         float u2[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
                         split8<BF>(u2, hi, lo);
-                        st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::ROWB), hi);
-                        st16(smem + Cf::OFF_SU2 + 64 * Cf::ROWB + tc::swz_off(r, cc, Cf::ROWB), lo);
+                        st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::UROWB), hi);
+                        st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc + NS / 8, Cf::UROWB), lo);
                     }
                 } else {
 #pragma unroll
                     for (int j = 0; j < NS; ++j) qs[j] = d1[j];
                 }
             }
-            operands_ready();  // also orders the staged y rows before their TMA store
+            if (!(ok = operands_ready(w_y && w1))) break;  // also orders the staged y rows before their store
             y_store();
 
             // K^T U' -> state increment (waited on); then M U -> y (waited on with the next chunk)
             if (tid == 0) {
-                const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS), am0 = desc_add(dM0, b * 16384);
+                const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS), am0 = desc_add(dM0, b * 8192);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::ROWB), id_ds, kk > 0);
-                    tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048),
-                                desc_add(dSU20, 64 * Cf::ROWB + kk * 16 * Cf::ROWB), id_ds, 1);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::UROWB), id_ds, kk > 0);
                 tc::mma_commit(bar_c);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {  // [M hi; M lo] U hi + [M hi; M lo] U lo + [M lo; .] U hi
-                    const uint64_t bu = desc_add(dSU0, kk * 16 * Cf::ROWB);
-                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), bu, id_slab, kk > 0);
-                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(bu, 64 * Cf::ROWB), id_slab, 1);
-                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, 8192 + kk * 32), bu, id_slab, 1);
-                }
+                for (int kk = 0; kk < 4; ++kk)  // rows 0-63: M U (rows 64-127 read the next tile: unused)
+                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(dSU0, kk * 16 * Cf::ROWB), id_mu, kk > 0);
                 tc::mma_commit(bar_y);
                 tc::mma_commit(bar_empty + b);  // slot b, its U~ columns and K stage kst are free
             }
             mu_pending = true;
-            if (!(ok = wait_mma(bar_c, ph_c))) break;
+            const bool w2 = wait_mma(bar_c, ph_c);
 
             {
-                float t[NS];
+                float t[NS], t2[NS];
+                tc::tmem_ld32(trow + Cf::COL_DS, t);
+                tc::tmem_ld32(trow + Cf::COL_DS + NS, t2);
 #pragma unroll
-                for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_DS + 32 * q4, t + 32 * q4);
-#pragma unroll
-                for (int j = 0; j < NS; ++j) S[j] = gC * S[j] + t[j];
+                for (int j = 0; j < NS; ++j) S[j] = gC * S[j] + (t[j] + t2[j]);
 #pragma unroll
                 for (int cc = 0; cc < NS / 8; ++cc) st16(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB), pack8<BF>(S + 8 * cc));
             }
@@ -724,16 +724,13 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             py_L = L;
             py_g = gR;
             if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next y_epilogue writes it
-            operands_ready();
+            if (!(ok = operands_ready(w2))) break;
         }
         if (ok && mu_pending) {
             mu_pending = false;
-            if ((ok = wait_mma(bar_y, ph_y))) {
-                y_epilogue();
-                tc::fence_async_smem();
-                tc::bar_sync(BID, 128);
-                y_store();
-            }
+            const bool w = wait_mma(bar_y, ph_y);
+            if (w) y_epilogue();
+            if ((ok = operands_ready(w))) y_store();
         }
         // never free TMEM under an MMA in flight
         if (c_pending) tc::mbar_wait_bounded(bar_c, ph_c, 4000000000ull);
@@ -762,9 +759,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         auto rec_ptr = [&](int ci) {
             return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
         };
+        // copies are issued by one thread of warp 6, which has no part in the gate arithmetic
+        constexpr int kIssuer = 64;
         auto issue_kv = [&](int ci) {  // K and the V slab of chunk ci -> stage ci % 3
             kv_issued = ci;
-            if (it != 0) return;
+            if (it != kIssuer) return;
             const int c0 = t_begin + ci * kChunk, s = ci % 3;
             uint64_t* bk = bar_kv + s;
             tc::mbar_arrive_expect_tx(bk, Cf::KV_TX);
@@ -772,21 +771,21 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::tma_load_3d(smem + Koff(s) + Cf::K_HALF, &maps.k, 64, h, c0, bk);
             tc::tma_load_3d(smem + Voff(s), &maps.v, slab * NS, h, c0, bk);
         };
-        auto issue_qm = [&](int ci) {  // Q of chunk ci and its M hi/lo -> slot ci & 1
+        auto issue_qm = [&](int ci) {  // Q of chunk ci and its M -> slot ci & 1
             const int bb = ci & 1;
             (bb ? qm_last1 : qm_last0) = ci;
-            if (it != 0) return;
+            if (it != kIssuer) return;
             const int c0 = t_begin + ci * kChunk;
             uint64_t* bq = bar_qm + bb;
             uint8_t* qw = smem + QWoff(bb);
             tc::mbar_arrive_expect_tx(bq, Cf::QM_TX);
             tc::tma_load_3d(qw, &maps.q, 0, h, c0, bq);
             tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bq);
-            tc::bulk_g2s(smem + Cf::OFF_M + bb * 16384, rec_ptr(ci) + kRecMHi, 16384, bq);
+            tc::bulk_g2s(smem + Cf::OFF_M + bb * 8192, rec_ptr(ci) + kRecM, 8192, bq);
         };
         auto issue_tt = [&](int ci) {  // [T_w; T_w; T_u hi; T_u lo] of chunk ci -> TT
             tt_issued = ci;
-            if (it != 0) return;
+            if (it != kIssuer) return;
             tc::mbar_arrive_expect_tx(bar_tt, 32768);
             tc::bulk_g2s(smem + Cf::OFF_TT, rec_ptr(ci) + kRecTw, 8192, bar_tt);
             tc::bulk_g2s(smem + Cf::OFF_TT + 8192, rec_ptr(ci) + kRecTw, 24576, bar_tt);
@@ -796,7 +795,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
             if (it < 64) pg = it < L ? a.g[(size_t)(c0 + it) * H + h] : 0.f;
         };
-        if (it == 0) {
+        if (it == kIssuer) {
             tc::prefetch_tmap(&maps.k);
             tc::prefetch_tmap(&maps.q);
             tc::prefetch_tmap(&maps.v);
@@ -820,8 +819,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             issue_qm(c);
             if (c + 1 < nchunks) issue_kv(c + 1);
 
-            // ---- gates of chunk c: gamma (inclusive prefix sum), Gamma, f = exp(gamma_C - gamma) --
+            // ---- gates of chunk c (warps 4-5): gamma (inclusive prefix sum), Gamma,
+            //      f = exp(gamma_C - gamma) -----------------------------------------------------------
             if (it < 64) {
+                constexpr int BID_G = 3;
                 float gv = pg;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -829,15 +830,13 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     if (lane >= o) gv += y;
                 }
                 vb[it] = gv;
-            }
-            if (it == 0) {
-                meta[2 * b] = c0;
-                meta[2 * b + 1] = L;
-            }
-            tc::bar_sync(BID, 128);
-            if (it >= 32 && it < 64) vb[it] += vb[31];
-            tc::bar_sync(BID, 128);
-            if (it < 64) {
+                if (it == 0) {
+                    meta[2 * b] = c0;
+                    meta[2 * b + 1] = L;
+                }
+                tc::bar_sync(BID_G, 64);
+                if (it >= 32) vb[it] += vb[31];
+                tc::bar_sync(BID_G, 64);
                 vb[64 + it] = __expf(vb[it]);
                 vb[128 + it] = __expf(vb[63] - vb[it]);
             }
@@ -950,7 +949,7 @@ inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, 
     const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
     if (nvc > 0) {
         LaunchScope timed(st, "chunk_ut_kernel");
-        chunk_ut_kernel<BF><<<dim3((unsigned)nvc, (unsigned)a.H), 128, UtCfg::BYTES, st>>>(a, maps);
+        chunk_ut_kernel<BF><<<(unsigned)(nvc * a.H), 128, UtCfg::BYTES, st>>>(a, maps);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -120,18 +120,14 @@ struct PrepLaunch {
                             const float* ba, const int32_t* cu, int num_seqs, int N, int H, float eps,
                             int in_dt, int out_dt, void* q, void* k, void* v, float* g, float* beta,
                             cudaStream_t st) {
-        const long long rows = (long long)N * H;
-        const unsigned grid = (unsigned)((rows + gdn::kPrepWarps - 1) / gdn::kPrepWarps);
+        const unsigned grid = (unsigned)((N + gdn::kPrepRun - 1) / gdn::kPrepRun) * (unsigned)H;
         gdn::LaunchScope timed(st, "prep_kernel");
-        if (DK >= 32 && DV >= 32) {
-            gdn::prep_kernel<(DK >= 32 ? DK : 32), (DV >= 32 ? DV : 32)><<<grid, 32 * gdn::kPrepWarps, 0, st>>>(
-                xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g,
-                beta);
-        } else {
-            gdn::prep_small_kernel<DK, DV><<<grid, 32 * gdn::kPrepWarps, 0, st>>>(
-                xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g,
-                beta);
-        }
+        if (W <= 4)
+            gdn::prep_kernel<DK, DV, 4><<<grid, 128, 0, st>>>(xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs,
+                                                               N, H, eps, in_dt, out_dt, q, k, v, g, beta);
+        else
+            gdn::prep_kernel<DK, DV, 8><<<grid, 128, 0, st>>>(xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs,
+                                                               N, H, eps, in_dt, out_dt, q, k, v, g, beta);
         return launched("prep_kernel");
     }
 };
@@ -303,7 +299,8 @@ gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, flo
     if (N == 0) return GDN_OK;
     REQUIRE_PTR(y, "y"); REQUIRE_PTR(z, "z"); REQUIRE_PTR(norm_w, "norm_w"); REQUIRE_PTR(out, "out");
     const long long rows = (long long)N * H;
-    const unsigned grid = (unsigned)((rows + gdn::kGateWarps - 1) / gdn::kGateWarps);
+    const long long per_block = (long long)gdn::kGateWarps * gdn::kGateRows;
+    const unsigned grid = (unsigned)((rows + per_block - 1) / per_block);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     gdn::LaunchScope timed(st, "out_gate_kernel");
     switch (dv) {

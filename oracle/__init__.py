@@ -14,7 +14,8 @@ Every function follows "On the design of Qwen3.8-Next architecture"
   against a state updated in place.
 * :func:`prep`        -- eqs. (6)-(10) ("GDN parameterisation").
 * :func:`out_gate`    -- eq. (11) without the output projection W_o.
-* :func:`mixer`       -- prep -> recurrence -> out_gate, all in fp64.
+* :func:`mixer`       -- prep -> recurrence -> out_gate in fp64 (optionally with q, k, v
+  rounded once to a 16-bit storage format between prep and the recurrence).
 
 The pins that tie these functions to the page (closed form eq. (5), pure decay,
 exact retrieval, brute-force products, textbook special cases, a hand-worked
@@ -182,12 +183,20 @@ def out_gate(y, z, w, eps=1e-6):
 
 
 def mixer(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bias, z, norm_w,
-          cu_seqlens=None, num_seqs=1, S0=None, eps_l2=1e-6, eps_rms=1e-6, nthreads=0):
+          cu_seqlens=None, num_seqs=1, S0=None, eps_l2=1e-6, eps_rms=1e-6, nthreads=0, inter_dtype=None):
     """The full post-projection mixer in fp64: eqs. (6)-(10), (1)-(4), (11) without W_o.
+
+    inter_dtype (None, torch.bfloat16 or torch.float16): the storage format of q, k, v between
+    the input side (6)-(8) and the recurrence.  The pages leave it open; a mixer that keeps
+    them in 16-bit memory rounds each value once to the nearest representable number, which
+    this models with torch's round-to-nearest-even conversion.  None keeps fp64.
 
     Returns (out [N, H, dv], y [N, H, dv], S_T).
     """
     q, k, v, g, beta = prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log,
                             alpha_bias, cu_seqlens, num_seqs, eps_l2, nthreads)
+    if inter_dtype is not None:
+        import torch  # its dtype conversion is the rounding step; no other torch arithmetic here
+        q, k, v = (torch.from_numpy(np.ascontiguousarray(t)).to(inter_dtype).double().numpy() for t in (q, k, v))
     y, S_T = recurrence(q, k, v, g, beta, S0, cu_seqlens, num_seqs, 1.0, nthreads)
     return out_gate(y, z, norm_w, eps_rms), y, S_T
