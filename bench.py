@@ -246,6 +246,14 @@ def run_ours(args):
     gdn.lib()
     stream = torch.cuda.current_stream()
     hbm_peak, tf_peak, peak_src = peaks()
+    if args.only:  # one secondary workload alone (for profiling), its own JSON line
+        line = WORKLOADS[args.only](torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     # ---- headline: prefill workload, three rotating input sets --------------------------
     c = inputs.CONFIGS[1]
@@ -330,10 +338,8 @@ def run_ours(args):
     return 0
 
 
-def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
-    res = []
-
-    # decode: 256 x 32 heads, 100 in-place steps per "step"
+def wl_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    """decode: 256 x 32 heads, 100 in-place steps per "step"."""
     c = inputs.CONFIGS[3]
     state = inputs.make_decode_state(3, "cuda", seed=inputs.SEED_BASE + 3 + 1000 * rank)
     steps_in = [inputs.make_decode_step(3, "cuda", step=s, seed=inputs.SEED_BASE + 3 + 1000 * rank)
@@ -350,16 +356,17 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
     per_launch = dt / (3 * c["steps"])
     upd = c["B"] * c["H"]
     bytes_l = upd * (2 * 128 * 128 * 4 + 3 * 128 * 2 + 8 + 128 * 2)
-    res.append({"workload": c["name"], "value": upd * world / per_launch, "unit": "state-updates/s",
+    return {"workload": c["name"], "value": upd * world / per_launch, "unit": "state-updates/s",
                 "us_per_step": per_launch * 1e6,
                 "roofline": {"bound": "hbm", "achieved": bytes_l / per_launch / 1e9, "peak": hbm_peak,
                              "unit": "GB/s", "frac": bytes_l / per_launch / 1e9 / hbm_peak,
                              "kernel": "decode_step_kernel", "alg_bytes_per_launch": bytes_l,
                              "kernel_avg_us": kd[0]["avg_us"] if kd else None},
-                "gpu_launches": sum(k["launches"] for k in kd)})
-    del state, steps_in
+                "gpu_launches": sum(k["launches"] for k in kd)}
 
-    # long prefill: B=1, H=32, T=32768, S0 != 0
+
+def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    """long prefill: B=1, H=32, T=32768, S0 != 0."""
     x = inputs.make_prefill(2, "cuda", seed=inputs.SEED_BASE + 2 + 1000 * rank)
     N, H, nseq = x["N"], x["H"], x["num_seqs"]
     yb = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)
@@ -377,16 +384,17 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
     kl = kernel_table(gdn.timing_stop(), n_lp)
     op_s = sum(k["avg_us"] for k in kl) / 1e6
     bl = prefill_bytes(N, H, nseq, S0=True)
-    res.append({"workload": inputs.CONFIGS[2]["name"], "value": N * H * world / dt, "unit": UNIT,
+    return {"workload": inputs.CONFIGS[2]["name"], "value": N * H * world / dt, "unit": UNIT,
                 "ms_per_step": dt * 1e3,
                 "roofline": {"bound": "hbm", "achieved": bl / op_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                              "frac": bl / op_s / 1e9 / hbm_peak,
                              "kernel": "gdn_chunk_fwd = chunk_ut_kernel + chunk_chain_kernel (per call)",
                              "alg_bytes_per_launch": bl, "kernels": kl},
-                "gpu_launches": sum(k["launches"] for k in kl), "l2": "1.1 GB working set > L2"})
-    del x, yb, ST
+                "gpu_launches": sum(k["launches"] for k in kl), "l2": "1.1 GB working set > L2"}
 
-    # full mixer: prep -> chunk -> out gate on 4 packed sequences
+
+def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    """full mixer: prep -> chunk -> out gate on 4 packed sequences."""
     m = inputs.make_mixer(4, "cuda", seed=inputs.SEED_BASE + 4 + 1000 * rank)
     N, H = m["N"], m["H"]
     bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
@@ -410,14 +418,24 @@ def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
                         world) / n_m
     km = kernel_table(gdn.timing_stop(), n_m)
     fused_min = N * (H * 3 * 128 * 2 + H * 2 * 2 + H * 128 * 2 + H * 128 * 2)
-    res.append({"workload": inputs.CONFIGS[4]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
+    return {"workload": inputs.CONFIGS[4]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
                 "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
                 "roofline": {"bound": "hbm", "achieved": fused_min / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
                              "frac": fused_min / dt / 1e9 / hbm_peak, "kernel": "prep+chunk+out_gate",
                              "alg_bytes_per_step": fused_min,
                              "note": "bytes = fused minimum (read projections, logits, z; write out)",
                              "kernels": km},
-                "gpu_launches": sum(k["launches"] for k in km)})
+                "gpu_launches": sum(k["launches"] for k in km)}
+
+
+WORKLOADS = {"decode": wl_decode, "long": wl_long, "mixer": wl_mixer}
+
+
+def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    res = []
+    for fn in WORKLOADS.values():
+        res.append(fn(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak))
+        torch.cuda.empty_cache()
     return res
 
 
@@ -428,6 +446,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--only", choices=["decode", "long", "mixer"], default=None,
+                    help="run one secondary workload alone and print its line (profiling aid)")
     ap.add_argument("--cpu-s", type=float, default=12.0, help="target seconds of the CPU-baseline sample")
     ap.add_argument("--ref-step-s", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", dest="impl_cpu_baseline", action="store_false")
