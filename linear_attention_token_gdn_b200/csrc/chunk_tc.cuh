@@ -17,28 +17,29 @@
 //   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, four CTAs per SM.
 //                       [K;Q] K^T on tcgen05 (the 16-bit inputs used directly as
 //                       operands), the decay masks, and the unit-lower-triangular inverse
-//                       T in fp32 on the CUDA cores.  Writes a 40 KB record per
+//                       T in fp32 on the CUDA cores.  Writes a 24 KB record per
 //                       (chunk, head): T_w = T diag(beta Gamma), T_u = T diag(beta) and M,
 //                       already in the 128B-swizzled operand layout.
 //   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
 //                       the chunks.  A producer warpgroup brings each chunk's K, Q and V
 //                       tiles in with TMA, straight into operand slots, and computes
-//                       W = T_w K and U~ = T_u V on the tensor cores; a chain warpgroup
-//                       carries the fp32 state (one row per thread) through two dependent
-//                       tensor-core round trips per chunk:
-//                           [Q;W] S            -> Q S, W S;   U = U~ - W S
-//                           K^T U'             -> S' = Gamma_C S + K^T U'
+//                       W = T_w K and [0; U~] = [0; T_u] V on the tensor cores; a chain
+//                       warpgroup carries the fp32 state (one row per thread) through two
+//                       dependent tensor-core round trips per chunk:
+//                           [0; U~] + [Q; -W] S -> Q S and U = U~ - W S in one accumulator
+//                           K^T U'              -> S' = Gamma_C S + K^T U'
 //                       with U' = diag(Gamma_C / Gamma) U, while M U, for
-//                       Y = Gamma (Q S) + M U, completes off the chain.  Q/W/M slots are
-//                       double-buffered, K/V stages triple-buffered, all handed over with
-//                       mbarriers; full chunks of y leave through swizzled TMA stores.
-// Operands are 16-bit with fp32 accumulation in TMEM.  q, k, v enter the products exactly as
-// stored (bf16 or fp16), so their partners take the same format.  A computed partner whose
-// rounding would show in y or the state (T_u, U') enters as two products, hi = round(x) and
-// lo = round(x - hi), which carries 16 significant bits for bf16; T_w, W and S enter once.  M U
-// pairs two computed operands, so it runs in fp16 (11 significant bits) whatever the input
-// format.  Records and [hi | lo] pairs are side by side in one operand (N = 2 x 32), so each
-// pair costs one MMA per k-step.
+//                       Y = Gamma (Q S) + M U, is issued with the next chunk's first MMAs.
+//                       Q/W/M slots are double-buffered, K/V stages triple-buffered, all
+//                       handed over with mbarriers; full chunks of y leave through swizzled
+//                       TMA stores.
+// Operands are 16-bit with fp32 accumulation in TMEM.  Each tcgen05.mma instruction costs
+// the SM's MMA front end about as much below N = 128 as at N = 128, so products are shaped
+// to use few instructions.  q and k enter exactly as stored (bf16 or fp16), so their partners
+// (T_w, W, S, U') take the same format; U' enters as a rounded high half plus its remainder,
+// side by side in one N = 64 operand, because its rounding would show in the state.  Products
+// between values we compute -- T_u V (V converted to fp16 in place) and M U -- run in fp16
+// (11 significant bits).
 // Operand tiles use the 128B / 64B swizzled canonical layouts, so one tile serves as K-major
 // or MN-major operand.  Every wait is bounded (ChunkArgs::budget clock cycles); a wait that
 // runs out sets the device error word, lets in-flight MMAs and copies drain, and the CTA
@@ -72,13 +73,12 @@ struct ChainMaps {
 };
 
 constexpr int kChunk = 64;
-// Record of one (chunk, head), written by chunk_ut_kernel: four [64 rows x 128 B] operand tiles
+// Record of one (chunk, head), written by chunk_ut_kernel: three [64 rows x 128 B] operand tiles
 // in the 128B-swizzled K-major layout.
-constexpr int kRecTw = 0;          // T_w = T diag(beta Gamma), 16-bit in the input's format
-constexpr int kRecTuHi = 8192;     // T_u = T diag(beta), high half (input's format)
-constexpr int kRecTuLo = 16384;    //   and the rounding remainder
-constexpr int kRecM = 24576;       // M, fp16 (it only meets U, another computed operand)
-constexpr int kRecBytes = 32768;
+constexpr int kRecTw = 0;          // T_w = T diag(beta Gamma), 16-bit in the input's format (meets K)
+constexpr int kRecTu = 8192;       // T_u = T diag(beta), fp16 (meets V converted to fp16)
+constexpr int kRecM = 16384;       // M, fp16 (meets U, another computed operand)
+constexpr int kRecBytes = 24576;
 
 // Upper bound of the number of 64-token chunks over all sequences.
 inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
             }
             __syncthreads();
         }
-        // ---- T_w = T diag(beta Gamma) (one 16-bit copy), T_u = T diag(beta) (hi + lo) -> record -----
+        // ---- T_w = T diag(beta Gamma) (input's format), T_u = T diag(beta) (fp16) -> record ------
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int idx = tid + 128 * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
@@ -432,14 +432,8 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) t8[e] = (8 * cc + e <= r) ? t8[e] * s8[e] : 0.f;
-            if (which == 0) {
-                st16(rec + kRecTw + tc::swz_off(r, cc, 128), pack8<BF>(t8));
-            } else {
-                uint4 hi, lo;
-                split8<BF>(t8, hi, lo);
-                st16(rec + kRecTuHi + tc::swz_off(r, cc, 128), hi);
-                st16(rec + kRecTuLo + tc::swz_off(r, cc, 128), lo);
-            }
+            if (which == 0) st16(rec + kRecTw + tc::swz_off(r, cc, 128), pack8<BF>(t8));
+            else st16(rec + kRecTu + tc::swz_off(r, cc, 128), pack8<false>(t8));
         }
     }
     tc::tc_fence_before();
@@ -457,39 +451,51 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
 template <int NS>
 struct ChainCfg {
     static constexpr int ROWB = NS * 2;                        // bytes per row of a 16-bit slab tile
+    static constexpr int UROWB = 2 * ROWB;                     // [hi | lo] rows of U': 128 B
     static constexpr uint32_t SWZ = NS == 32 ? tc::kSw64 : tc::kSw128;
     static constexpr int QW_HALF = 128 * 128;                  // one 64-column half of [Q;W]
     static constexpr int K_HALF = 64 * 128;                    // one 64-column half of K
     static constexpr int OFF_QW = 0;                           // [2 slots] [Q;W]: 2 halves x [128 x 128 B]
     static constexpr int OFF_M = OFF_QW + 2 * 2 * QW_HALF;     // [2 slots] M fp16: [64 x 128 B]
     static constexpr int OFF_KS = OFF_M + 2 * 8192;            // [3 stages] K: 2 halves x [64 x 128 B]
-    static constexpr int OFF_TT = OFF_KS + 3 * 2 * K_HALF;     // [T_w; T_w; T_u hi; T_u lo]: [256 x 128 B]
+    static constexpr int OFF_TT = OFF_KS + 3 * 2 * K_HALF;     // [T_w; T_w; 0; T_u]: [256 x 128 B]
     static constexpr int OFF_VS = OFF_TT + 32768;              // [3 stages] V slab [64 x ROWB]
     static constexpr int OFF_SS = OFF_VS + 3 * 64 * ROWB;      // S [128 x ROWB]
-    static constexpr int UROWB = 2 * ROWB;                      // [hi | lo] rows of U': 128 B
-    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // U fp16: [64 x ROWB]
-    static constexpr int OFF_SU2 = OFF_SU + 64 * ROWB;         // [U' hi | U' lo]: [64 x UROWB]
-    static constexpr int OFF_YS = OFF_SU2 + 2 * 64 * ROWB;     // y rows for the TMA store [64 x NS x 4 B]
+    static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // [2 slots] U fp16: [64 x ROWB]
+    static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // [U' hi | U' lo]: [64 x UROWB]
+    static constexpr int OFF_YS = OFF_SU2 + 64 * UROWB;        // y rows for the TMA store [64 x NS x 4 B]
     static constexpr int OFF_VEC = OFF_YS + 64 * NS * 4;       // [2 slots] gamma, Gamma, f: 3 x 64 floats
     static constexpr int OFF_META = OFF_VEC + 2 * 1024;        // [2 slots] {c0, L}
     static constexpr int OFF_BAR = OFF_META + 64;
+    static constexpr int NBARS = 20;
     static constexpr int BYTES = OFF_BAR + 256 + 1024;
     static constexpr uint32_t KV_TX = 2 * K_HALF + 64 * ROWB;  // K and the V slab of one chunk
-    static constexpr uint32_t QM_TX = 2 * 8192 + 8192;         // Q and M of one chunk
+    static constexpr uint32_t Q_TX = 2 * 8192;                 // Q of one chunk
+    static constexpr uint32_t M_TX = 8192;                     // M of one chunk
     // TMEM columns
-    static constexpr uint32_t COL_UT = 0;                      // [2 slots] x NS: U~ (lanes 64-127)
+    static constexpr uint32_t COL_U = 0;                       // [2 slots] x NS: [0; U~] + [Q; -W] S over dk 0-63
     static constexpr uint32_t COL_W = 2 * NS;                  // 128: W (both lane halves)
-    static constexpr uint32_t COL_1 = COL_W + 128;             // NS: Q S (lanes 0-63), W S (64-127)
-    static constexpr uint32_t COL_MU = COL_1 + NS;             // NS: M U (lanes 0-63)
+    static constexpr uint32_t COL_1B = COL_W + 128;            // NS: [Q; -W] S over dk 64-127
+    static constexpr uint32_t COL_MU = COL_1B + NS;            // NS: M U (lanes 0-63)
     static constexpr uint32_t COL_DS = COL_MU + NS;            // 2 NS: [K^T U' hi | K^T U' lo]
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(COL_DS + 2 * NS <= TMEM_COLS, "TMEM budget");
     static_assert(NS == 32, "[hi | lo] operand rows are one 128-byte swizzle atom");
+    static_assert(NBARS * 8 <= 192, "barrier area");
     static_assert(BYTES <= 232448, "shared memory budget");
-    static_assert(OFF_YS % 1024 == 0 && OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0 && OFF_SU2 % 1024 == 0,
+    static_assert(OFF_M % 1024 == 0 && OFF_KS % 1024 == 0 && OFF_TT % 1024 == 0 && OFF_YS % 1024 == 0 &&
+                      OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0 && OFF_SU % 1024 == 0 && OFF_SU2 % 1024 == 0,
                   "swizzle atoms");
 };
 
+// Synchronisation of one chunk c in slot b = c & 1 (stage c % 3 for K and V):
+//   producer -> chain   full[b]      W(c) in [Q;W] slot b, U~(c) in TMEM, gates and bounds of c
+//                       q[b], m[b]   Q(c), M(c) landed (TMA / bulk copy bytes)
+//   chain -> producer   ds_done[b]   the state MMA of c completed: [Q;W] slot b, U~ columns b and
+//                                    K stage c % 3 are free (everything else of c was read before)
+//                       m_empty[b]   M U of c completed: M slot b and U slot b are free
+// The chain issues M U of chunk c at the start of chunk c + 1, right after that chunk's first
+// MMAs, and forms y of c while they run.
 template <int NS, bool BF>
 __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a,
                                                              const __grid_constant__ ChainMaps maps) {
@@ -500,16 +506,21 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     const uint32_t sbase = tc::smem_u32(smem);
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
-    uint64_t* bar_p = bars + 0;        // producer-issued MMAs complete
-    uint64_t* bar_c = bars + 1;        // chain-issued state MMAs complete
-    uint64_t* bar_y = bars + 2;        // chain-issued M U complete
-    uint64_t* bar_tt = bars + 3;       // [T_w; T_u] of the next chunk landed in TT
-    uint64_t* bar_full = bars + 4;     // [2 slots] W, U~, gates of a chunk ready (producer)
-    uint64_t* bar_empty = bars + 6;    // [2 slots] slot, its U~ columns and the K stage released (chain)
-    uint64_t* bar_qm = bars + 8;       // [2 slots] Q and M landed (bytes)
-    uint64_t* bar_kv = bars + 10;      // [3 stages] K and V landed (bytes)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 128);
-    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 136);
+    uint64_t* bar_p = bars + 0;        // producer: W = T_w K complete
+    uint64_t* bar_p2 = bars + 1;       // producer: U~ = T_u V complete
+    uint64_t* bar_c1 = bars + 2;       // chain: [Q;W] S over dk 0-63 complete
+    uint64_t* bar_c2 = bars + 3;       // chain: [Q;W] S over dk 64-127 complete
+    uint64_t* bar_ds = bars + 4;       // chain: K^T U' complete
+    uint64_t* bar_y = bars + 5;        // chain: M U complete
+    uint64_t* bar_tt = bars + 6;       // T_w, T_u of the next chunk landed in TT
+    uint64_t* bar_full = bars + 7;     // [2 slots]
+    uint64_t* bar_dsd = bars + 9;      // [2 slots] ds_done
+    uint64_t* bar_mfree = bars + 11;   // [2 slots] m_empty
+    uint64_t* bar_q = bars + 13;       // [2 slots]
+    uint64_t* bar_m = bars + 15;       // [2 slots]
+    uint64_t* bar_kv = bars + 17;      // [3 stages] K and V landed (bytes)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 192);
+    int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 200);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slab = blockIdx.x % NSLAB;
@@ -525,7 +536,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (lane == 0) *s_base = base;
     }
     if (tid == 0) {
-        for (int i = 0; i < 13; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < Cf::NBARS; ++i) tc::mbar_init(bars + i, 1);
         tc::fence_mbar_init();
     }
     if (warp == 1) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
@@ -543,8 +554,8 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     if (warp < 4) {
         // =============================== chain group ===================================
         constexpr int BID = 1;
-        uint32_t ph_c = 0, ph_y = 0;
-        bool ok = true, c_pending = false, mu_pending = false;
+        uint32_t ph_c1 = 0, ph_c2 = 0, ph_ds = 0, ph_y = 0;
+        bool ok = true, c1_pending = false, c2_pending = false, ds_pending = false, mu_pending = false;
         // each thread waits for a tcgen05.commit on its own; a timeout flags the error, lets the
         // MMAs drain, and is combined over the group at the next barrier
         auto wait_mma = [&](uint64_t* bar, uint32_t& ph) -> bool {
@@ -566,9 +577,9 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::tc_fence_after();
             return all;
         };
-        constexpr uint32_t id_slab = idesc16<BF>(128, NS, false, true);
-        constexpr uint32_t id_ds = idesc16<BF>(128, 2 * NS, true, true);  // K^T [U' hi | U' lo]
-        constexpr uint32_t id_mu = idesc16<false>(128, NS, false, true);  // M U, both fp16
+        constexpr uint32_t id_slab = idesc16<BF>(128, NS, false, true);    // [Q;W] S
+        constexpr uint32_t id_ds = idesc16<BF>(128, 2 * NS, true, true);   // K^T [U' hi | U' lo]
+        constexpr uint32_t id_mu = idesc16<false>(128, NS, false, true);   // M U, both fp16
         // operand descriptors at k-step 0 of slot / stage 0; k-steps and slots are byte offsets
         const uint64_t dQW0 = tc::smem_desc(sbase + Cf::OFF_QW, 16, 1024, tc::kSw128);      // K-major [Q;W]
         const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_KS, Cf::K_HALF, 1024, tc::kSw128);  // MN-major K^T
@@ -590,12 +601,36 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         for (int c = 0; c < NS / 8; ++c) st16(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB), pack8<BF>(S + 8 * c));
         operands_ready(true);
 
-        // y of chunk c-1 is formed while chunk c's first MMA runs; a full chunk leaves with one
-        // TMA store (swizzled staging rows), a sequence's last partial chunk with plain stores.
-        int py_c0 = 0, py_L = 0;  // the chunk whose M U waits in TMEM (py_L = 0: none)
+        // M U of chunk ci (slot bb) -> COL_MU; by thread 0 once M(ci) has landed.  A wait that runs
+        // out is flagged and then completed (the copy always lands), so the MMA is always issued
+        // and every commit below arrives.
+        auto issue_mu = [&](int ci) -> bool {
+            bool w = true;
+            if (tid == 0) {
+                const int bb = ci & 1;
+                w = tc::mbar_wait_bounded(bar_m + bb, (ci >> 1) & 1, a.budget);
+                if (!w) {
+                    raise_error(kErrTimeout);
+                    tc::mbar_wait_bounded(bar_m + bb, (ci >> 1) & 1, 4000000000ull);
+                }
+                const uint64_t am0 = desc_add(dM0, bb * 8192), bu0 = desc_add(dSU0, bb * 64 * Cf::ROWB);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // rows 0-63: M U (rows 64-127 read the next tile: unused)
+                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(bu0, kk * 16 * Cf::ROWB), id_mu,
+                                kk > 0);
+                tc::mma_commit(bar_y);
+                tc::mma_commit(bar_mfree + bb);
+            }
+            mu_pending = true;
+            return w;
+        };
+
+        // y of chunk py (warps 0-1): y = scale (Gamma_r (Q S) + M U); a full chunk is staged in
+        // swizzled rows for one TMA store, a sequence's last partial chunk goes out with plain stores.
+        int py_c0 = 0, py_L = 0;
         float py_g = 0.f;         // its Gamma_r (rows 0-63)
         float qs[NS];             // its (Q S) row (rows 0-63)
-        auto y_epilogue = [&]() {  // warps 0-1: y = scale (Gamma_r (Q S) + M U) of chunk py
+        auto y_epilogue = [&]() {
             if (warp < 2 && py_L > 0) {
                 float t[NS];
                 tc::tmem_ld32(trow + Cf::COL_MU, t);
@@ -629,11 +664,19 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             py_L = 0;
         };
+        // wait for M U of the previous chunk (warps 0-1 need it; all threads keep the phase)
+        auto wait_mu = [&]() -> bool {
+            bool w = true;
+            if (warp < 2) w = wait_mma(bar_y, ph_y);
+            else ph_y ^= 1u;
+            mu_pending = false;
+            return w;
+        };
 
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1, kst = c % 3;
             bool w = tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget);
-            w = w && tc::mbar_wait_bounded(bar_qm + b, (c >> 1) & 1, a.budget);
+            w = w && tc::mbar_wait_bounded(bar_q + b, (c >> 1) & 1, a.budget);
             if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (tid == 0) raise_error(kErrTimeout);
                 break;
@@ -645,41 +688,43 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const float gR = tid < 64 ? vb[64 + tid] : 0.f;
             const float fR = tid >= 64 ? vb[128 + tid - 64] : 0.f;
 
-            // [Q;W] S -> Q S (lanes 0-63), W S (lanes 64-127)
-            if (tid == 0) {
-                const uint64_t a0 = desc_add(dQW0, QWoff(b));
+            // [Q; -W] S over dk 0-63 (thread 0) is added onto [0; U~] already in COL_U[b]; dk 64-127
+            // (thread 32) goes to COL_1B.  Their sum: Q S in lanes 0-63, U = U~ - W S in lanes 64-127.
+            if (tid == 0 || tid == 32) {
+                const int hf = tid >> 5;
+                const uint64_t a0 = desc_add(dQW0, QWoff(b) + hf * Cf::QW_HALF);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16(tmem + Cf::COL_1, desc_add(a0, (kk >> 2) * Cf::QW_HALF + (kk & 3) * 32),
-                                desc_add(dSS0, kk * 16 * Cf::ROWB), id_slab, kk > 0);
-                tc::mma_commit(bar_c);
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16(tmem + (hf ? Cf::COL_1B : Cf::COL_U + b * NS), desc_add(a0, kk * 32),
+                                desc_add(dSS0, (hf * 4 + kk) * 16 * Cf::ROWB), id_slab, hf == 0 || kk > 0);
+                tc::mma_commit(hf ? bar_c2 : bar_c1);
             }
-            c_pending = true;
-            bool w_y = true;
-            if (mu_pending) {  // the previous chunk's M U, for its y (warps 0-1 only)
-                mu_pending = false;
-                if (warp < 2) w_y = wait_mma(bar_y, ph_y);
-                else ph_y ^= 1u;
+            c1_pending = c2_pending = true;
+            bool wm = true, wy = true;
+            if (c > 0) {  // the previous chunk's M U, then its y while [Q;W] S runs
+                wm = issue_mu(c - 1);
+                wy = wait_mu();
+                if (wy) y_epilogue();
             }
-            if (w_y) y_epilogue();
-            const bool w1 = wait_mma(bar_c, ph_c);
-            c_pending = false;
+            c1_pending = false;
+            const bool w1 = wait_mma(bar_c1, ph_c1);
+            c2_pending = false;
+            const bool w2 = wait_mma(bar_c2, ph_c2);
 
             {
-                float d1[NS];
-#pragma unroll
-                for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_1 + 32 * q4, d1 + 32 * q4);
-                if (warp >= 2) {  // U = U~ - W S (fp16, for M U), U' = f U (hi + lo, for K^T U')
+                float d1[NS], d2[NS];
+                tc::tmem_ld32(trow + Cf::COL_U + b * NS, d1);
+                tc::tmem_ld32(trow + Cf::COL_1B, d2);
+                if (warp >= 2) {  // U (fp16, for M U), U' = f U (hi + lo, for K^T U')
                     const int r = tid - 64;
                     float ut[NS];
 #pragma unroll
-                    for (int q4 = 0; q4 < NS / 32; ++q4) tc::tmem_ld32(trow + Cf::COL_UT + b * NS + 32 * q4, ut + 32 * q4);
-#pragma unroll
-                    for (int j = 0; j < NS; ++j) ut[j] -= d1[j];
+                    for (int j = 0; j < NS; ++j) ut[j] = d1[j] + d2[j];
+                    uint8_t* su = smem + Cf::OFF_SU + b * 64 * Cf::ROWB;
 #pragma unroll
                     for (int cc = 0; cc < NS / 8; ++cc) {
                         uint4 hi, lo;
-                        st16(smem + Cf::OFF_SU + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(ut + 8 * cc));
+                        st16(su + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(ut + 8 * cc));
                         float u2[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
@@ -689,27 +734,23 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < NS; ++j) qs[j] = d1[j];
+                    for (int j = 0; j < NS; ++j) qs[j] = d1[j] + d2[j];
                 }
             }
-            if (!(ok = operands_ready(w_y && w1))) break;  // also orders the staged y rows before their store
+            if (!(ok = operands_ready(wm && wy && w1 && w2))) break;  // also orders the staged y rows
             y_store();
 
-            // K^T U' -> state increment (waited on); then M U -> y (waited on with the next chunk)
+            // K^T U' -> state increment; its completion also releases slot b and K stage kst
             if (tid == 0) {
-                const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS), am0 = desc_add(dM0, b * 8192);
+                const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::UROWB), id_ds, kk > 0);
-                tc::mma_commit(bar_c);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // rows 0-63: M U (rows 64-127 read the next tile: unused)
-                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(dSU0, kk * 16 * Cf::ROWB), id_mu, kk > 0);
-                tc::mma_commit(bar_y);
-                tc::mma_commit(bar_empty + b);  // slot b, its U~ columns and K stage kst are free
+                tc::mma_commit(bar_ds);
+                tc::mma_commit(bar_dsd + b);
             }
-            mu_pending = true;
-            const bool w2 = wait_mma(bar_c, ph_c);
+            ds_pending = false;
+            const bool w3 = wait_mma(bar_ds, ph_ds);
 
             {
                 float t[NS], t2[NS];
@@ -724,16 +765,18 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             py_L = L;
             py_g = gR;
             if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next y_epilogue writes it
-            if (!(ok = operands_ready(w2))) break;
+            if (!(ok = operands_ready(w3))) break;
         }
-        if (ok && mu_pending) {
-            mu_pending = false;
-            const bool w = wait_mma(bar_y, ph_y);
-            if (w) y_epilogue();
-            if ((ok = operands_ready(w))) y_store();
+        if (ok && nchunks > 0) {  // the last chunk's M U and y
+            const bool wm = issue_mu(nchunks - 1);
+            const bool wy = wait_mu();
+            if (wy) y_epilogue();
+            if ((ok = operands_ready(wm && wy))) y_store();
         }
         // never free TMEM under an MMA in flight
-        if (c_pending) tc::mbar_wait_bounded(bar_c, ph_c, 4000000000ull);
+        if (c1_pending) tc::mbar_wait_bounded(bar_c1, ph_c1, 4000000000ull);
+        if (c2_pending) tc::mbar_wait_bounded(bar_c2, ph_c2, 4000000000ull);
+        if (ds_pending) tc::mbar_wait_bounded(bar_ds, ph_ds, 4000000000ull);
         if (mu_pending) tc::mbar_wait_bounded(bar_y, ph_y, 4000000000ull);
         if (tid == 0) tc::bulk_wait0();
         if (ok && a.S_T) {
@@ -745,22 +788,22 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         // =============================== producer group ================================
         constexpr int BID = 2;
         const int it = tid - 128;
-        uint32_t ph = 0;
+        uint32_t ph_w = 0, ph_u = 0;
         bool ok = true;
-        constexpr uint32_t id_v = idesc16<BF>(128, NS, false, true);
+        constexpr uint32_t id_v = idesc16<false>(128, NS, false, true);  // T_u V in fp16
         constexpr uint32_t id_w = idesc16<BF>(128, 128, false, true);
         const uint64_t dTT0 = tc::smem_desc(sbase + Cf::OFF_TT, 16, 1024, tc::kSw128);
         const uint64_t dV0 = tc::smem_desc(sbase + Cf::OFF_VS, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_KS, Cf::K_HALF, 1024, tc::kSw128);  // MN-major K
 
+        // copies are issued by one thread of warp 6, which has no part in the gate arithmetic
+        constexpr int kIssuer = 64;
         // copies in flight into this CTA's shared memory, for the exit drain
         int kv_issued = -1, kv_landed = -1, tt_issued = -1, tt_landed = -1;
-        int qm_last0 = -1, qm_last1 = -1;  // last chunk whose Q/M copies went to slot 0 / 1
+        int q_last0 = -1, q_last1 = -1, m_last0 = -1, m_last1 = -1;
         auto rec_ptr = [&](int ci) {
             return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
         };
-        // copies are issued by one thread of warp 6, which has no part in the gate arithmetic
-        constexpr int kIssuer = 64;
         auto issue_kv = [&](int ci) {  // K and the V slab of chunk ci -> stage ci % 3
             kv_issued = ci;
             if (it != kIssuer) return;
@@ -771,30 +814,40 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::tma_load_3d(smem + Koff(s) + Cf::K_HALF, &maps.k, 64, h, c0, bk);
             tc::tma_load_3d(smem + Voff(s), &maps.v, slab * NS, h, c0, bk);
         };
-        auto issue_qm = [&](int ci) {  // Q of chunk ci and its M -> slot ci & 1
+        auto issue_q = [&](int ci) {  // Q of chunk ci -> rows 0-63 of [Q;W] slot ci & 1
             const int bb = ci & 1;
-            (bb ? qm_last1 : qm_last0) = ci;
+            (bb ? q_last1 : q_last0) = ci;
             if (it != kIssuer) return;
             const int c0 = t_begin + ci * kChunk;
-            uint64_t* bq = bar_qm + bb;
             uint8_t* qw = smem + QWoff(bb);
-            tc::mbar_arrive_expect_tx(bq, Cf::QM_TX);
-            tc::tma_load_3d(qw, &maps.q, 0, h, c0, bq);
-            tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bq);
-            tc::bulk_g2s(smem + Cf::OFF_M + bb * 8192, rec_ptr(ci) + kRecM, 8192, bq);
+            tc::mbar_arrive_expect_tx(bar_q + bb, Cf::Q_TX);
+            tc::tma_load_3d(qw, &maps.q, 0, h, c0, bar_q + bb);
+            tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bar_q + bb);
         };
-        auto issue_tt = [&](int ci) {  // [T_w; T_w; T_u hi; T_u lo] of chunk ci -> TT
+        auto issue_m = [&](int ci) {  // M of chunk ci -> M slot ci & 1 (issuer thread only)
+            const int bb = ci & 1;
+            (bb ? m_last1 : m_last0) = ci;
+            tc::mbar_arrive_expect_tx(bar_m + bb, Cf::M_TX);
+            tc::bulk_g2s(smem + Cf::OFF_M + bb * 8192, rec_ptr(ci) + kRecM, 8192, bar_m + bb);
+        };
+        auto issue_tt = [&](int ci) {  // T_w (twice) and T_u of chunk ci -> TT rows 0-127, 192-255
             tt_issued = ci;
             if (it != kIssuer) return;
-            tc::mbar_arrive_expect_tx(bar_tt, 32768);
+            tc::mbar_arrive_expect_tx(bar_tt, 3 * 8192);
             tc::bulk_g2s(smem + Cf::OFF_TT, rec_ptr(ci) + kRecTw, 8192, bar_tt);
-            tc::bulk_g2s(smem + Cf::OFF_TT + 8192, rec_ptr(ci) + kRecTw, 24576, bar_tt);
+            tc::bulk_g2s(smem + Cf::OFF_TT + 8192, rec_ptr(ci) + kRecTw, 8192, bar_tt);
+            tc::bulk_g2s(smem + Cf::OFF_TT + 24576, rec_ptr(ci) + kRecTu, 8192, bar_tt);
         };
         float pg = 0.f;  // g of the next chunk (beta is already inside T_w, T_u)
         auto load_gates = [&](int ci) {
             const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
             if (it < 64) pg = it < L ? a.g[(size_t)(c0 + it) * H + h] : 0.f;
         };
+        // TT rows 128-191 stay zero: A = [0; T_u] leaves lanes 0-63 of the U~ accumulator at zero
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            st16(smem + Cf::OFF_TT + 16384 + (it + 128 * i) * 16, make_uint4(0, 0, 0, 0));
+        tc::fence_async_smem();
         if (it == kIssuer) {
             tc::prefetch_tmap(&maps.k);
             tc::prefetch_tmap(&maps.q);
@@ -810,13 +863,13 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const int b = c & 1, kst = c % 3;
             const int c0 = t_begin + c * kChunk, L = min(kChunk, t_end - c0);
             float* vb = vec(b);
-            // slot b, its U~ columns and K stage (c+1) % 3 are free once the chain is done with c-2
-            bool w = tc::mbar_wait_bounded(bar_empty + b, ((c >> 1) & 1) ^ 1, a.budget);
+            // slot b, U~ columns b and K stage (c + 1) % 3 are free once the state MMA of c - 2 is done
+            bool w = tc::mbar_wait_bounded(bar_dsd + b, ((c >> 1) & 1) ^ 1, a.budget);
             if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (it == 0) raise_error(kErrTimeout);
                 break;
             }
-            issue_qm(c);
+            issue_q(c);
             if (c + 1 < nchunks) issue_kv(c + 1);
 
             // ---- gates of chunk c (warps 4-5): gamma (inclusive prefix sum), Gamma,
@@ -841,7 +894,8 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 vb[128 + it] = __expf(vb[63] - vb[it]);
             }
 
-            // ---- W = T_w K (both lane halves), U~ = T_u hi V + T_u lo V (lanes 64-127) -----------
+            // ---- W = T_w K (thread 0; both lane halves) and U~ = T_u V (thread 32; lanes 64-127),
+            //      two issuers with their own commits ---------------------------------------------------
             w = tc::mbar_wait_bounded(bar_kv + kst, (c / 3) & 1, a.budget);
             w = w && tc::mbar_wait_bounded(bar_tt, c & 1, a.budget);
             if (!(ok = tc::bar_and(BID, 128, w))) {
@@ -850,35 +904,64 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             kv_landed = c;
             tt_landed = c;
+            if constexpr (BF) {  // V slab bf16 -> fp16 in place (exact for every normal value)
+                uint8_t* vs = smem + Voff(kst);
+#pragma unroll
+                for (int i = 0; i < (64 * Cf::ROWB) / (16 * 128); ++i) {
+                    uint4* p16 = reinterpret_cast<uint4*>(vs + (it + 128 * i) * 16);
+                    const uint4 u = *p16;
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t o4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = unpack2<true>(w4[e]);
+                        o4[e] = pack2<false>(f.x, f.y);
+                    }
+                    *p16 = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                }
+                tc::fence_async_smem();
+                tc::bar_sync(BID, 128);
+            }
             tc::tc_fence_after();
             if (it == 0) {
-                const uint64_t bv0 = desc_add(dV0, Voff(kst) - Cf::OFF_VS), bk0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
+                const uint64_t bk0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bv = desc_add(bv0, kk * 16 * Cf::ROWB);
+                for (int kk = 0; kk < 4; ++kk)
                     tc::mma_f16(tmem + Cf::COL_W, desc_add(dTT0, kk * 32), desc_add(bk0, kk * 2048), id_w, kk > 0);
-                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, desc_add(dTT0, 8192 + kk * 32), bv, id_v, kk > 0);
-                    tc::mma_f16(tmem + Cf::COL_UT + b * NS, desc_add(dTT0, 16384 + kk * 32), bv, id_v, 1);
-                }
                 tc::mma_commit(bar_p);
+            } else if (it == 32) {  // [0; T_u] V (fp16): lanes 0-63 zero, lanes 64-127 U~
+                const uint64_t bv0 = desc_add(dV0, Voff(kst) - Cf::OFF_VS);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16(tmem + Cf::COL_U + b * NS, desc_add(dTT0, 16384 + kk * 32),
+                                desc_add(bv0, kk * 16 * Cf::ROWB), id_v, kk > 0);
+                tc::mma_commit(bar_p2);
             }
-            w = tc::bar_and(BID, 128, tc::mbar_wait_bounded(bar_p, ph, a.budget));
-            if (!w) {
-                if (it == 0) raise_error(kErrTimeout);
-                tc::mbar_wait_bounded(bar_p, ph, 4000000000ull);
+            bool ww = tc::mbar_wait_bounded(bar_p, ph_w, a.budget);
+            if (!ww) {
+                raise_error(kErrTimeout);
+                tc::mbar_wait_bounded(bar_p, ph_w, 4000000000ull);
             }
-            ph ^= 1u;
+            ph_w ^= 1u;
+            bool wu = tc::mbar_wait_bounded(bar_p2, ph_u, a.budget);
+            if (!wu) {
+                raise_error(kErrTimeout);
+                tc::mbar_wait_bounded(bar_p2, ph_u, 4000000000ull);
+            }
+            ph_u ^= 1u;
             tc::tc_fence_after();
-            if (!(ok = w)) break;
+            if (!(ok = tc::bar_and(BID, 128, ww && wu))) break;
             if (c + 1 < nchunks) issue_tt(c + 1);  // the MMAs have read TT
 
-            // ---- W -> rows 64-127 of [Q;W] in slot b: lanes 0-63 write columns 0-63, lanes 64-127
+            // ---- -W -> rows 64-127 of [Q; -W] in slot b: lanes 0-63 write columns 0-63, lanes 64-127
             //      columns 64-127 (each lane half of the accumulator holds all of W) ------------------
             {
                 const int r = it & 63, hf = it >> 6;
                 float wv[64];
                 tc::tmem_ld32(trow + Cf::COL_W + 64 * hf, wv);
                 tc::tmem_ld32(trow + Cf::COL_W + 64 * hf + 32, wv + 32);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) wv[j] = -wv[j];
                 uint8_t* qw = smem + QWoff(b) + hf * Cf::QW_HALF;
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) st16(qw + tc::swz_off(64 + r, cc, 128), pack8<BF>(wv + 8 * cc));
@@ -886,7 +969,13 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::fence_async_smem();
             tc::tc_fence_before();
             tc::bar_sync(BID, 128);
-            if (it == 0) tc::mbar_arrive(bar_full + b);  // hand slot b to the chain group
+            if (it == 0) tc::mbar_arrive(bar_full + b);  // hand chunk c to the chain group
+
+            // ---- M of chunk c, once M U of c - 2 has read the slot ---------------------------------
+            if (it == kIssuer) {
+                if (tc::mbar_wait_bounded(bar_mfree + b, ((c >> 1) & 1) ^ 1, a.budget)) issue_m(c);
+                else raise_error(kErrTimeout);
+            }
             if (c + 1 < nchunks) load_gates(c + 1);
         }
         // never leave with copies into this CTA's shared memory in flight
@@ -894,8 +983,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (kv_issued > kv_landed + 1)
             tc::mbar_wait_bounded(bar_kv + (kv_issued - 1) % 3, ((kv_issued - 1) / 3) & 1, 4000000000ull);
         if (tt_issued > tt_landed) tc::mbar_wait_bounded(bar_tt, tt_issued & 1, 4000000000ull);
-        if (qm_last0 >= 0) tc::mbar_wait_bounded(bar_qm + 0, (qm_last0 >> 1) & 1, 4000000000ull);
-        if (qm_last1 >= 0) tc::mbar_wait_bounded(bar_qm + 1, (qm_last1 >> 1) & 1, 4000000000ull);
+        if (q_last0 >= 0) tc::mbar_wait_bounded(bar_q + 0, (q_last0 >> 1) & 1, 4000000000ull);
+        if (q_last1 >= 0) tc::mbar_wait_bounded(bar_q + 1, (q_last1 >> 1) & 1, 4000000000ull);
+        if (m_last0 >= 0) tc::mbar_wait_bounded(bar_m + 0, (m_last0 >> 1) & 1, 4000000000ull);
+        if (m_last1 >= 0) tc::mbar_wait_bounded(bar_m + 1, (m_last1 >> 1) & 1, 4000000000ull);
         (void)ok;
     }
 

@@ -70,8 +70,8 @@ def test_chunk_fwd_tensor_core_path_limits(L, over):
 
 def test_workspace_size_covers_every_chunk(L):
     # one 24 KB record per (64-token chunk, head); packed sequences add one partial chunk each
-    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 32768
-    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 32768
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 24576
+    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 24576
     assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0
 
 
