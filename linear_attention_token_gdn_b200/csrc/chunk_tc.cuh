@@ -50,6 +50,7 @@
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace gdn {
 
@@ -154,27 +155,6 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t byte_off) { re
 
 __device__ __forceinline__ float4 lds4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ void sts4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
-
-// 16-bit operands in the input's own format (bf16 or fp16), rounded to nearest.
-template <bool BF>
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-    if constexpr (BF) {
-        __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-        return *reinterpret_cast<uint32_t*>(&v);
-    } else {
-        __half2 v = __floats2half2_rn(a, b);
-        return *reinterpret_cast<uint32_t*>(&v);
-    }
-}
-
-template <bool BF>
-__device__ __forceinline__ float2 unpack2(uint32_t u) {
-    if constexpr (BF) {
-        return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
-    } else {
-        return __half22float2(*reinterpret_cast<__half2*>(&u));
-    }
-}
 
 template <bool BF>
 __device__ __forceinline__ uint4 pack8(const float* x) {
@@ -998,37 +978,6 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     }
 }
 
-using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
-
-inline EncodeTiledFn encode_tiled_fn() {
-    static EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        return reinterpret_cast<EncodeTiledFn>(p);
-    }();
-    return fn;
-}
-
-// [N, H, 128] view of a token-major tensor; box = box_x columns x 1 head x box_z tokens.
-inline bool encode_map_3d(CUtensorMap* m, const void* base, int dt, int N, int H, uint32_t box_x, uint32_t box_z,
-                          CUtensorMapSwizzle swz) {
-    EncodeTiledFn enc = encode_tiled_fn();
-    if (!enc) return false;
-    const int eb = dt == kF32 ? 4 : 2;
-    const CUtensorMapDataType t = dt == kF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                  : dt == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    const cuuint64_t dims[3] = {128, (cuuint64_t)H, (cuuint64_t)N};
-    const cuuint64_t strides[2] = {(cuuint64_t)128 * eb, (cuuint64_t)H * 128 * eb};
-    const cuuint32_t box[3] = {box_x, 1, box_z};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <bool BF>
 inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, cudaStream_t st) {
     constexpr int NS = 32;
@@ -1061,10 +1010,10 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
     // y tiles are NS columns = 64 B (16-bit) or 128 B (fp32) per row, stored with the matching swizzle
     const CUtensorMapSwizzle yswz = a.y_dt == kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     ChainMaps maps;
-    if (!encode_map_3d(&maps.k, a.k, a.in_dt, a.N, a.H, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_map_3d(&maps.q, a.q, a.in_dt, a.N, a.H, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, NS, kChunk, yswz)) {
+    if (!encode_map_3d(&maps.k, a.k, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_3d(&maps.q, a.q, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, 128, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, 128, NS, kChunk, yswz)) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaSuccess;
     }

@@ -73,6 +73,27 @@ __device__ __forceinline__ void st4(void* p, int dt, size_t i, float4 x) {
     *reinterpret_cast<uint2*>(reinterpret_cast<char*>(p) + 2 * i) = u;
 }
 
+// 16-bit operands in the input's own format (bf16 or fp16), rounded to nearest.
+template <bool BF>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    if constexpr (BF) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&v);
+    } else {
+        __half2 v = __floats2half2_rn(a, b);
+        return *reinterpret_cast<uint32_t*>(&v);
+    }
+}
+
+template <bool BF>
+__device__ __forceinline__ float2 unpack2(uint32_t u) {
+    if constexpr (BF) {
+        return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+    } else {
+        return __half22float2(*reinterpret_cast<__half2*>(&u));
+    }
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

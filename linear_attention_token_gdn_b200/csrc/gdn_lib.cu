@@ -115,20 +115,38 @@ struct RecurrentLaunch {
 
 template <int DK, int DV>
 struct PrepLaunch {
+    template <int TAPS>
+    static gdn_status_t go(const gdn::PrepMaps& maps, const float* wq, const float* wk, const float* wv, int W,
+                           const void* bl, const void* al, const float* A, const float* ba, const int32_t* cu,
+                           int num_seqs, int N, int H, float eps, int in_dt, int out_dt, void* q, void* k, void* v,
+                           float* g, float* beta, cudaStream_t st) {
+        const int esz = in_dt == GDN_F32 ? 4 : 2;
+        const int bytes = 2 * gdn::prep_tile_bytes(DK, TAPS, esz) + gdn::prep_tile_bytes(DV, TAPS, esz) + 16 + 128;
+        cudaError_t e = cudaFuncSetAttribute(gdn::prep_kernel<DK, DV, TAPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             bytes);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "prep_kernel smem: %s", cudaGetErrorString(e));
+        const unsigned grid = (unsigned)((N + gdn::kPrepRun - 1) / gdn::kPrepRun) * (unsigned)H;
+        gdn::LaunchScope timed(st, "prep_kernel");
+        gdn::prep_kernel<DK, DV, TAPS><<<grid, 128, bytes, st>>>(maps, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N,
+                                                                  H, eps, in_dt, out_dt, q, k, v, g, beta,
+                                                                  wait_budget());
+        return launched("prep_kernel");
+    }
     static gdn_status_t run(const void* xq, const void* xk, const void* xv, const float* wq, const float* wk,
                             const float* wv, int W, const void* bl, const void* al, const float* A,
                             const float* ba, const int32_t* cu, int num_seqs, int N, int H, float eps,
                             int in_dt, int out_dt, void* q, void* k, void* v, float* g, float* beta,
                             cudaStream_t st) {
-        const unsigned grid = (unsigned)((N + gdn::kPrepRun - 1) / gdn::kPrepRun) * (unsigned)H;
-        gdn::LaunchScope timed(st, "prep_kernel");
-        if (W <= 4)
-            gdn::prep_kernel<DK, DV, 4><<<grid, 128, 0, st>>>(xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs,
-                                                               N, H, eps, in_dt, out_dt, q, k, v, g, beta);
-        else
-            gdn::prep_kernel<DK, DV, 8><<<grid, 128, 0, st>>>(xq, xk, xv, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs,
-                                                               N, H, eps, in_dt, out_dt, q, k, v, g, beta);
-        return launched("prep_kernel");
+        const int taps = W <= 4 ? 4 : 8;
+        const uint32_t rows = (uint32_t)(gdn::kPrepRun + taps - 1);
+        gdn::PrepMaps maps;
+        if (!gdn::encode_map_3d(&maps.q, xq, in_dt, N, H, DK, DK, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !gdn::encode_map_3d(&maps.k, xk, in_dt, N, H, DK, DK, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !gdn::encode_map_3d(&maps.v, xv, in_dt, N, H, DV, DV, rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return fail(GDN_ERR_CUDA, "prep: cuTensorMapEncodeTiled failed");
+        if (taps == 4)
+            return go<4>(maps, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g, beta, st);
+        return go<8>(maps, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N, H, eps, in_dt, out_dt, q, k, v, g, beta, st);
     }
 };
 

@@ -2,14 +2,16 @@
 // ("GDN parameterisation"): causal depthwise ShortConv -> SiLU (-> L2Norm for q, k) on the
 // projection outputs, and the per-head beta / log-alpha gates.
 //
-// One CTA per (run of kPrepRun tokens, head), heads fastest across the grid, four warps: q, k, v and the gates.  A tensor's
-// warp walks its run; each lane owns d/32 adjacent channels (one 8-byte load per row for
-// 16-bit inputs), keeps their conv taps and the last W-1 input rows in registers, so every
-// input row is read from memory once (plus the history rows of each run).  L2Norm is a
-// warp reduction.  Rows are read and computed in batches of 8 independent tokens, which keeps
-// loads and reductions in flight.  HBM-bound: 3 x d inputs and outputs per (token, head).
+// One CTA per (run of kPrepRun tokens, head), heads fastest across the grid.  One TMA copy per
+// tensor brings the run's q, k, v input rows and the conv history before it into shared memory
+// (about 50 KB in flight per CTA for bf16, so the SM keeps enough bytes moving to stream at HBM
+// speed).  Warps 0-2 each take one tensor: a lane owns d/32 adjacent channels, keeps their taps
+// and the last W-1 rows in registers and computes 8 independent tokens at a time (L2Norm is a
+// warp reduction); warp 3 forms the gates.  HBM-bound: 3 x d inputs and outputs per (token, head).
 #pragma once
 #include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tmap.cuh"
 
 namespace gdn {
 
@@ -82,18 +84,48 @@ struct SeqWalk {
     }
 };
 
-// One tensor (q, k or v) of one head over tokens [t0, t1): ShortConv -> SiLU (-> L2Norm).
-// TAPS >= conv width; the taps are zero-padded in front.  The tokens of a batch are computed
-// independently (their reductions interleave), so each warp keeps 8 rows of work in flight.
-template <int D, int TAPS, bool NORM>
-__device__ __forceinline__ void prep_tensor(const void* __restrict__ x, const float* __restrict__ w, int W,
-                                            void* __restrict__ out, int in_dt, int out_dt, float eps, int t0,
-                                            int t1, int H, int h, int lane, SeqWalk sw) {
+// `per` adjacent channels of one input row held in shared memory (input format IDT).
+template <int PER, int IDT>
+__device__ __forceinline__ void lds_row(const uint8_t* p, float (&x)[PER]) {
+    if constexpr (IDT == kF32) {
+        if constexpr (PER == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(p);
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < PER; ++u) x[u] = reinterpret_cast<const float*>(p)[u];
+        }
+    } else {
+        constexpr bool BF = IDT == kBF16;
+        if constexpr (PER == 4) {
+            const uint2 v = *reinterpret_cast<const uint2*>(p);
+            const float2 a = unpack2<BF>(v.x), b = unpack2<BF>(v.y);
+            x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+        } else if constexpr (PER == 2) {
+            const float2 a = unpack2<BF>(*reinterpret_cast<const uint32_t*>(p));
+            x[0] = a.x; x[1] = a.y;
+        } else {
+            const uint16_t v = *reinterpret_cast<const uint16_t*>(p);
+            x[0] = unpack2<BF>((uint32_t)v).x;
+        }
+    }
+}
+
+// One tensor (q, k or v) of one head over tokens [t0, t1): ShortConv -> SiLU (-> L2Norm), read
+// from the CTA's tile, whose row r holds token t0 - (TAPS - 1) + r (rows before a sequence
+// start are masked, rows before token 0 or past N are zero-filled by the copy).  The tokens of
+// a batch are computed independently, so their reductions interleave.
+template <int D, int TAPS, bool NORM, int IDT>
+__device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, const float* __restrict__ w, int W,
+                                            void* __restrict__ out, int out_dt, float eps, int t0, int t1, int H,
+                                            int h, int lane, SeqWalk sw) {
     constexpr int PER = D >= 32 ? D / 32 : 1;
     constexpr int HIST = TAPS - 1;
     constexpr int B = kPrepBatch;
+    constexpr int ESZ = IDT == kF32 ? 4 : 2;
     const bool active = D >= 32 || lane < D;
     const int c0 = (D >= 32 ? lane * PER : lane);
+    const uint8_t* row0 = tile + c0 * ESZ;  // row r at row0 + r * D * ESZ
     float wp[TAPS][PER];  // wp[TAPS - W + j] = w[c][j]
 #pragma unroll
     for (int i = 0; i < TAPS; ++i) {
@@ -103,21 +135,24 @@ __device__ __forceinline__ void prep_tensor(const void* __restrict__ x, const fl
             wp[i][u] = (active && j >= 0) ? w[((size_t)h * D + c0 + u) * W + j] : 0.f;
         }
     }
-    // xb[0 .. HIST-1]: the rows before the batch; xb[HIST ..]: the batch
-    float xb[HIST + B][PER];
+    float xb[HIST + B][PER];  // [0, HIST): the rows before the batch; then the batch
 #pragma unroll
     for (int i = 0; i < HIST; ++i) {
-        const int s = t0 - HIST + i;
+        if (active) lds_row<PER, IDT>(row0 + i * D * ESZ, xb[i]);
+        else {
 #pragma unroll
-        for (int u = 0; u < PER; ++u) xb[i][u] = 0.f;
-        if (active && s >= 0) ld_row<PER>(x, in_dt, ((size_t)s * H + h) * D + c0, xb[i]);
+            for (int u = 0; u < PER; ++u) xb[i][u] = 0.f;
+        }
     }
     for (int tb = t0; tb < t1; tb += B) {
+        const int rb = tb - t0 + HIST;  // tile row of token tb
 #pragma unroll
         for (int k = 0; k < B; ++k) {
+            if (active && tb + k < t1) lds_row<PER, IDT>(row0 + (rb + k) * D * ESZ, xb[HIST + k]);
+            else {
 #pragma unroll
-            for (int u = 0; u < PER; ++u) xb[HIST + k][u] = 0.f;
-            if (active && tb + k < t1) ld_row<PER>(x, in_dt, ((size_t)(tb + k) * H + h) * D + c0, xb[HIST + k]);
+                for (int u = 0; u < PER; ++u) xb[HIST + k][u] = 0.f;
+            }
         }
         int lim[B];  // previous tokens of the same sequence (-1: past t1)
 #pragma unroll
@@ -159,9 +194,11 @@ __device__ __forceinline__ void prep_tensor(const void* __restrict__ x, const fl
                 for (int u = 0; u < PER; ++u) y[k][u] *= inv;
             }
         }
+        size_t e = ((size_t)tb * H + h) * D + c0;
+        const size_t step = (size_t)H * D;
 #pragma unroll
-        for (int k = 0; k < B; ++k)
-            if (active && tb + k < t1) st_row<PER>(out, out_dt, ((size_t)(tb + k) * H + h) * D + c0, y[k]);
+        for (int k = 0; k < B; ++k, e += step)
+            if (active && tb + k < t1) st_row<PER>(out, out_dt, e, y[k]);
 #pragma unroll
         for (int i = 0; i < HIST; ++i) {
 #pragma unroll
@@ -170,30 +207,51 @@ __device__ __forceinline__ void prep_tensor(const void* __restrict__ x, const fl
     }
 }
 
+// TMA descriptors of the three projection outputs, [N, H, d] each; box = d x 1 x (run + taps - 1).
+struct PrepMaps {
+    CUtensorMap q, k, v;
+};
+
+// Bytes of one tensor's tile (rows padded to a 128-byte multiple per tile).
+__host__ __device__ constexpr int prep_tile_bytes(int D, int taps, int esz) {
+    return ((kPrepRun + taps - 1) * D * esz + 127) / 128 * 128;
+}
+
 template <int DK, int DV, int TAPS>
 __global__ void __launch_bounds__(128)
-prep_kernel(const void* __restrict__ xq, const void* __restrict__ xk, const void* __restrict__ xv,
-            const float* __restrict__ wq, const float* __restrict__ wk, const float* __restrict__ wv, int W,
-            const void* __restrict__ beta_logit, const void* __restrict__ alpha_logit,
-            const float* __restrict__ A_log, const float* __restrict__ alpha_bias,
-            const int32_t* __restrict__ cu, int num_seqs, int N, int H, float eps, int in_dt, int out_dt,
-            void* __restrict__ q, void* __restrict__ k, void* __restrict__ v, float* __restrict__ g_out,
-            float* __restrict__ beta_out) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+prep_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ wq, const float* __restrict__ wk,
+            const float* __restrict__ wv, int W, const void* __restrict__ beta_logit,
+            const void* __restrict__ alpha_logit, const float* __restrict__ A_log,
+            const float* __restrict__ alpha_bias, const int32_t* __restrict__ cu, int num_seqs, int N, int H,
+            float eps, int in_dt, int out_dt, void* __restrict__ q, void* __restrict__ k, void* __restrict__ v,
+            float* __restrict__ g_out, float* __restrict__ beta_out, unsigned long long budget) {
+    constexpr int HIST = TAPS - 1;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // heads vary fastest across the grid, so CTAs resident together read whole token rows
     const int h = (int)(blockIdx.x % (unsigned)H);
     const int t0 = (int)(blockIdx.x / (unsigned)H) * kPrepRun;
     SeqWalk sw;
     sw.init(cu, num_seqs, N, t0);
     const int t1 = min(t0 + kPrepRun, sw.stop);  // tokens past the last sequence stay untouched
-    if (t0 >= t1) return;
-    if (warp == 0) {
-        prep_tensor<DK, TAPS, true>(xq, wq, W, q, in_dt, out_dt, eps, t0, t1, H, h, lane, sw);   // eq. (6)
-    } else if (warp == 1) {
-        prep_tensor<DK, TAPS, true>(xk, wk, W, k, in_dt, out_dt, eps, t0, t1, H, h, lane, sw);   // eq. (7)
-    } else if (warp == 2) {
-        prep_tensor<DV, TAPS, false>(xv, wv, W, v, in_dt, out_dt, eps, t0, t1, H, h, lane, sw);  // eq. (8)
-    } else {
+    if (t0 >= t1) return;  // uniform over the CTA
+    const int esz = in_dt == kF32 ? 4 : 2;
+    const int tqk = prep_tile_bytes(DK, TAPS, esz), tv = prep_tile_bytes(DV, TAPS, esz);
+    uint8_t* tile_q = smem;
+    uint8_t* tile_k = smem + tqk;
+    uint8_t* tile_v = smem + 2 * tqk;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * tqk + tv);
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)((kPrepRun + HIST) * (2 * DK + DV) * esz));
+        tc::tma_load_3d(tile_q, &maps.q, 0, h, t0 - HIST, bar);
+        tc::tma_load_3d(tile_k, &maps.k, 0, h, t0 - HIST, bar);
+        tc::tma_load_3d(tile_v, &maps.v, 0, h, t0 - HIST, bar);
+    }
+    __syncthreads();
+    if (warp == 3) {  // the gates need no tile
         const float ea = expf(A_log[h]), bias = alpha_bias[h];
         for (int t = t0 + lane; t < t1; t += 32) {
             const size_t th = (size_t)t * H + h;
@@ -201,6 +259,27 @@ prep_kernel(const void* __restrict__ xq, const void* __restrict__ xk, const void
             g_out[th] = -ea * softplusf_(ld1(alpha_logit, in_dt, th) + bias);      // eq. (10)
         }
     }
+    if (!tc::mbar_wait_bounded(bar, 0, budget)) {  // flag, let the copies land, skip the work
+        if (lane == 0) raise_error(kErrTimeout);
+        tc::mbar_wait_bounded(bar, 0, 4000000000ull);
+        return;
+    }
+    if (warp == 3) return;
+    const uint8_t* tile = warp == 0 ? tile_q : warp == 1 ? tile_k : tile_v;
+    const float* w = warp == 0 ? wq : warp == 1 ? wk : wv;
+    void* out = warp == 0 ? q : warp == 1 ? k : v;
+    // eqs. (6), (7): q and k are normalised; eq. (8): v is not
+#define GDN_PREP_TENSOR(IDT)                                                                          \
+    if (warp < 2) prep_tensor<DK, TAPS, true, IDT>(tile, w, W, out, out_dt, eps, t0, t1, H, h, lane, sw); \
+    else prep_tensor<DV, TAPS, false, IDT>(tile, w, W, out, out_dt, eps, t0, t1, H, h, lane, sw);
+    if (in_dt == kBF16) {
+        GDN_PREP_TENSOR(kBF16)
+    } else if (in_dt == kF16) {
+        GDN_PREP_TENSOR(kF16)
+    } else {
+        GDN_PREP_TENSOR(kF32)
+    }
+#undef GDN_PREP_TENSOR
 }
 
 }  // namespace gdn
