@@ -33,8 +33,8 @@ METRIC = "GDN prefill tokens/s (B×T×H, dk=dv=128) + decode state-updates/s; % 
 UNIT = "token-heads/s"
 
 
-def env_rank():
-    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+from linear_attention_token_gdn_b200.dist import aggregate, env_rank, rank_seed  # noqa: E402
+from linear_attention_token_gdn_b200 import dist as gdist  # noqa: E402
 
 
 def peaks():
@@ -153,17 +153,11 @@ def traffic_per_call():
 
 
 def max_over_ranks(torch, dist, x, world):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return gdist.max_over_ranks(x, world, device="cuda")
 
 
 def barrier(torch, dist, world):
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    gdist.barrier(world, cuda=True)
 
 
 # ----------------------------------------------------------------------------- CPU baseline
@@ -257,7 +251,7 @@ def run_ours(args):
 
     # ---- headline: prefill workload, three rotating input sets --------------------------
     c = inputs.CONFIGS[1]
-    sets = [inputs.make_prefill(1, "cuda", seed=inputs.SEED_BASE + 1 + 1000 * rank + s) for s in range(3)]
+    sets = [inputs.make_prefill(1, "cuda", seed=rank_seed(inputs.SEED_BASE + 1, rank) + s) for s in range(3)]
     N, H = sets[0]["N"], sets[0]["H"]
     nseq = sets[0]["num_seqs"]
     outs = [(torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16),
@@ -283,7 +277,7 @@ def run_ours(args):
     gdn.check_device_error()
     per_step = dt / args.steps
     work = N * H  # token-heads per rank per step
-    value = work * world / per_step
+    value = aggregate(work, world, per_step)
     alg_bytes = prefill_bytes(N, H, nseq)
     kern = kernel_table(per_kernel, args.steps)
     op_s = sum(k["avg_us"] for k in kern) / 1e6  # device time of one gdn_chunk_fwd call
@@ -341,8 +335,8 @@ def run_ours(args):
 def wl_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     """decode: 256 x 32 heads, 100 in-place steps per "step"."""
     c = inputs.CONFIGS[3]
-    state = inputs.make_decode_state(3, "cuda", seed=inputs.SEED_BASE + 3 + 1000 * rank)
-    steps_in = [inputs.make_decode_step(3, "cuda", step=s, seed=inputs.SEED_BASE + 3 + 1000 * rank)
+    state = inputs.make_decode_state(3, "cuda", seed=rank_seed(inputs.SEED_BASE + 3, rank))
+    steps_in = [inputs.make_decode_step(3, "cuda", step=s, seed=rank_seed(inputs.SEED_BASE + 3, rank))
                 for s in range(c["steps"])]
     y = torch.empty(c["B"], c["H"], 128, device="cuda", dtype=torch.bfloat16)
 
@@ -367,7 +361,7 @@ def wl_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
 def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     """long prefill: B=1, H=32, T=32768, S0 != 0."""
-    x = inputs.make_prefill(2, "cuda", seed=inputs.SEED_BASE + 2 + 1000 * rank)
+    x = inputs.make_prefill(2, "cuda", seed=rank_seed(inputs.SEED_BASE + 2, rank))
     N, H, nseq = x["N"], x["H"], x["num_seqs"]
     yb = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)
     ST = torch.empty(nseq, H, 128, 128, device="cuda")
@@ -395,7 +389,7 @@ def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
 def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     """full mixer: prep -> chunk -> out gate on 4 packed sequences."""
-    m = inputs.make_mixer(4, "cuda", seed=inputs.SEED_BASE + 4 + 1000 * rank)
+    m = inputs.make_mixer(4, "cuda", seed=rank_seed(inputs.SEED_BASE + 4, rank))
     N, H = m["N"], m["H"]
     bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
     gbuf = torch.empty(N, H, device="cuda")

@@ -1,0 +1,63 @@
+"""The multi-GPU path on CPU: two gloo ranks exercise the rank plumbing the benchmark uses
+(rank discovery, per-rank seeds, the barrier and the max-over-ranks time) and show that the
+replicas are independent: each rank's result equals a single process run on its seed."""
+import multiprocessing as mp
+import os
+import socket
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import dist_worker  # noqa: E402
+import oracle  # noqa: E402
+from linear_attention_token_gdn_b200 import dist as gd  # noqa: E402
+from linear_attention_token_gdn_b200 import inputs  # noqa: E402
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=dist_worker.run, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted((q.get(timeout=120) for _ in procs), key=lambda d: d["rank"])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [d["rank"] for d in out] == [0, 1] and all(d["world"] == 2 and d["local"] == d["rank"] for d in out)
+    assert all(d["t"] == 1.0 for d in out)            # every rank sees the slowest rank's time
+    assert all(d["value"] == 64 * 2 / 1.0 for d in out)
+    assert out[0]["seed"] != out[1]["seed"]
+    for d in out:                                      # replica r == one process on rank r's seed
+        x = inputs.make_prefill(0, "cpu", seed=d["seed"])
+        y, _ = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+        assert np.isclose(float(np.abs(y).sum()), d["y_sum"], rtol=0, atol=0)
+    assert out[0]["y_sum"] != out[1]["y_sum"]
+
+
+def test_single_process_defaults(monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert gd.env_rank() == (0, 1, 0)
+    assert gd.max_over_ranks(3.5, 1) == 3.5
+    assert gd.rank_seed(10, 0) == 10 and gd.rank_seed(10, 2) == 2010
+
+
+def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = bench.argparse.Namespace(steps=1, warmup=3, ref_step_s=1.0)
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
