@@ -127,7 +127,7 @@ struct PrepLaunch {
         if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "prep_kernel smem: %s", cudaGetErrorString(e));
         const unsigned grid = (unsigned)((N + gdn::kPrepRun - 1) / gdn::kPrepRun) * (unsigned)H;
         gdn::LaunchScope timed(st, "prep_kernel");
-        gdn::prep_kernel<DK, DV, TAPS><<<grid, 128, bytes, st>>>(maps, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N,
+        gdn::prep_kernel<DK, DV, TAPS><<<grid, gdn::kPrepThreads, bytes, st>>>(maps, wq, wk, wv, W, bl, al, A, ba, cu, num_seqs, N,
                                                                   H, eps, in_dt, out_dt, q, k, v, g, beta,
                                                                   wait_budget());
         return launched("prep_kernel");

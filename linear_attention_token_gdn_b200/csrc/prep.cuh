@@ -5,9 +5,9 @@
 // One CTA per (run of kPrepRun tokens, head), heads fastest across the grid.  One TMA copy per
 // tensor brings the run's q, k, v input rows and the conv history before it into shared memory
 // (about 50 KB in flight per CTA for bf16, so the SM keeps enough bytes moving to stream at HBM
-// speed).  Warps 0-2 each take one tensor: a lane owns d/32 adjacent channels, keeps their taps
-// and the last W-1 rows in registers and computes 8 independent tokens at a time (L2Norm is a
-// warp reduction); warp 3 forms the gates.  HBM-bound: 3 x d inputs and outputs per (token, head).
+// speed).  Two warps take each tensor, one per half of the run: a lane owns d/32 adjacent
+// channels, keeps their taps and the last W-1 rows in registers and computes 8 independent
+// tokens at a time (L2Norm is a warp reduction); warp 6 forms the gates.  HBM-bound: 3 x d inputs and outputs per (token, head).
 #pragma once
 #include "common.cuh"
 #include "tc_ptx.cuh"
@@ -16,7 +16,7 @@
 namespace gdn {
 
 constexpr int kPrepRun = 64;    // tokens per CTA
-constexpr int kPrepBatch = 8;   // input rows loaded per batch
+constexpr int kPrepBatch = 4;   // input rows loaded per batch
 
 // `per` adjacent channels of one row, starting at element i.
 template <int PER>
@@ -112,20 +112,20 @@ __device__ __forceinline__ void lds_row(const uint8_t* p, float (&x)[PER]) {
 }
 
 // One tensor (q, k or v) of one head over tokens [t0, t1): ShortConv -> SiLU (-> L2Norm), read
-// from the CTA's tile, whose row r holds token t0 - (TAPS - 1) + r (rows before a sequence
+// from the CTA's tile, whose row r holds token tt - (TAPS - 1) + r (rows before a sequence
 // start are masked, rows before token 0 or past N are zero-filled by the copy).  The tokens of
 // a batch are computed independently, so their reductions interleave.
 template <int D, int TAPS, bool NORM, int IDT>
-__device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, const float* __restrict__ w, int W,
-                                            void* __restrict__ out, int out_dt, float eps, int t0, int t1, int H,
-                                            int h, int lane, SeqWalk sw) {
+__device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, int tt, const float* __restrict__ w,
+                                            int W, void* __restrict__ out, int out_dt, float eps, int t0, int t1,
+                                            int H, int h, int lane, SeqWalk sw) {
     constexpr int PER = D >= 32 ? D / 32 : 1;
     constexpr int HIST = TAPS - 1;
     constexpr int B = kPrepBatch;
     constexpr int ESZ = IDT == kF32 ? 4 : 2;
     const bool active = D >= 32 || lane < D;
     const int c0 = (D >= 32 ? lane * PER : lane);
-    const uint8_t* row0 = tile + c0 * ESZ;  // row r at row0 + r * D * ESZ
+    const uint8_t* row0 = tile + (t0 - tt) * D * ESZ + c0 * ESZ;  // row of token t0 - HIST + r at row0 + r * D * ESZ
     float wp[TAPS][PER];  // wp[TAPS - W + j] = w[c][j]
 #pragma unroll
     for (int i = 0; i < TAPS; ++i) {
@@ -217,8 +217,10 @@ __host__ __device__ constexpr int prep_tile_bytes(int D, int taps, int esz) {
     return ((kPrepRun + taps - 1) * D * esz + 127) / 128 * 128;
 }
 
+constexpr int kPrepThreads = 224;  // 2 warps per tensor + 1 for the gates
+
 template <int DK, int DV, int TAPS>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kPrepThreads, 4)
 prep_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ wq, const float* __restrict__ wk,
             const float* __restrict__ wv, int W, const void* __restrict__ beta_logit,
             const void* __restrict__ alpha_logit, const float* __restrict__ A_log,
@@ -251,7 +253,7 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ wq,
         tc::tma_load_3d(tile_v, &maps.v, 0, h, t0 - HIST, bar);
     }
     __syncthreads();
-    if (warp == 3) {  // the gates need no tile
+    if (warp == 6) {  // the gates need no tile
         const float ea = expf(A_log[h]), bias = alpha_bias[h];
         for (int t = t0 + lane; t < t1; t += 32) {
             const size_t th = (size_t)t * H + h;
@@ -264,14 +266,19 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ wq,
         tc::mbar_wait_bounded(bar, 0, 4000000000ull);
         return;
     }
-    if (warp == 3) return;
-    const uint8_t* tile = warp == 0 ? tile_q : warp == 1 ? tile_k : tile_v;
-    const float* w = warp == 0 ? wq : warp == 1 ? wk : wv;
-    void* out = warp == 0 ? q : warp == 1 ? k : v;
+    if (warp == 6) return;
+    const int ten = warp >> 1;  // 0 q, 1 k, 2 v
+    const uint8_t* tile = ten == 0 ? tile_q : ten == 1 ? tile_k : tile_v;
+    const float* w = ten == 0 ? wq : ten == 1 ? wk : wv;
+    void* out = ten == 0 ? q : ten == 1 ? k : v;
+    const int ta = t0 + (warp & 1) * (kPrepRun / 2), tb = min(ta + kPrepRun / 2, t1);
+    if (ta >= tb) return;
+    SeqWalk swh;
+    swh.init(cu, num_seqs, N, ta);
     // eqs. (6), (7): q and k are normalised; eq. (8): v is not
-#define GDN_PREP_TENSOR(IDT)                                                                          \
-    if (warp < 2) prep_tensor<DK, TAPS, true, IDT>(tile, w, W, out, out_dt, eps, t0, t1, H, h, lane, sw); \
-    else prep_tensor<DV, TAPS, false, IDT>(tile, w, W, out, out_dt, eps, t0, t1, H, h, lane, sw);
+#define GDN_PREP_TENSOR(IDT)                                                                                     \
+    if (ten < 2) prep_tensor<DK, TAPS, true, IDT>(tile, t0, w, W, out, out_dt, eps, ta, tb, H, h, lane, swh);   \
+    else prep_tensor<DV, TAPS, false, IDT>(tile, t0, w, W, out, out_dt, eps, ta, tb, H, h, lane, swh);
     if (in_dt == kBF16) {
         GDN_PREP_TENSOR(kBF16)
     } else if (in_dt == kF16) {
