@@ -133,8 +133,9 @@ gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const f
  * chunk selects the algorithm:
  *   chunk = 0: token-sequential fp32 recurrence on CUDA cores (any supported
  *              shape and dtype; exact up to fp32 rounding order).
- *   chunk = 64 or 128: chunkwise-parallel form on the tcgen05 tensor cores
- *              (requires dk = dv = 128 and in_dtype BF16 or F16).  It is derived
+ *   chunk = 64: chunkwise-parallel form on the tcgen05 tensor cores
+ *              (requires dk = dv = 128 and in_dtype BF16 or F16; other shapes and
+ *              chunk sizes return GDN_ERR_UNSUPPORTED).  It is derived
  *              from eq. (5): within a chunk, the UT transform T = (I + A)^-1 with
  *              A[r,s] = beta_r exp(gamma_r - gamma_s) k_r.k_s turns the token loop
  *              into dense products; between chunks the state is carried in fp32.

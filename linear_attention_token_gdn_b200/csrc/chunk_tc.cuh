@@ -91,7 +91,7 @@ inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
 }
 
 inline size_t chunk_tc_workspace_bytes(int N, int num_seqs, int H, int, int, int chunk) {
-    if (chunk == 0 || N <= 0 || num_seqs <= 0 || H <= 0) return 0;
+    if (chunk != kChunk || N <= 0 || num_seqs <= 0 || H <= 0) return 0;
     // the bound for packed sequences also covers equal lengths
     return (size_t)chunk_count_bound(N, num_seqs, true) * H * kRecBytes;
 }

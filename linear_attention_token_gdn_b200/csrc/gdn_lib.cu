@@ -241,7 +241,7 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
     REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
     REQUIRE(dtype_ok(in_dtype) && dtype_ok(y_dtype), "bad dtype");
-    REQUIRE(chunk == 0 || chunk == 64 || chunk == 128, "chunk=%d not in {0, 64, 128}", chunk);
+    REQUIRE(chunk >= 0, "chunk=%d < 0", chunk);
     REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
     REQUIRE((long long)N * H * (dk > dv ? dk : dv) < (1LL << 40), "problem too large");
     if (N == 0 && S_T == nullptr) return GDN_OK;
@@ -252,6 +252,8 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     if (chunk == 0)
         return dispatch_dims<RecurrentLaunch>(dk, dv, q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, scale,
                                               (int)in_dtype, (int)y_dtype, y, S_T, st);
+    if (chunk != 64)
+        return fail(GDN_ERR_UNSUPPORTED, "chunk=%d: the tensor-core path is built for chunk 64 (chunk 0 for the recurrence)", chunk);
     if (dk != 128 || dv != 128 || in_dtype == GDN_F32)
         return fail(GDN_ERR_UNSUPPORTED, "chunked path needs dk=dv=128 and bf16/f16 inputs (use chunk=0)");
     const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);

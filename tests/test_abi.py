@@ -54,7 +54,7 @@ def chunk_call(L, **over):
 
 
 @pytest.mark.parametrize("over", [
-    dict(q=None), dict(k=MIS), dict(dk=48), dict(dv=256), dict(chunk=32), dict(chunk=-1), dict(N=-1),
+    dict(q=None), dict(k=MIS), dict(dk=48), dict(dv=256), dict(chunk=-1), dict(N=-1),
     dict(H=0), dict(num_seqs=0), dict(N=63), dict(in_dt=7), dict(y_dt=-1), dict(S0=MIS),
     dict(ws_bytes=0, ws=None),
 ])
@@ -63,9 +63,15 @@ def test_chunk_fwd_rejects_bad_arguments(L, over):
     assert gdn.last_error_message() != ""
 
 
-@pytest.mark.parametrize("over", [dict(dk=64, dv=64), dict(in_dt=gdn.F32), dict(dk=128, dv=64)])
+@pytest.mark.parametrize("over", [dict(dk=64, dv=64), dict(in_dt=gdn.F32), dict(dk=128, dv=64), dict(chunk=32),
+                                  dict(chunk=128)])
 def test_chunk_fwd_tensor_core_path_limits(L, over):
     assert chunk_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_workspace_size_is_zero_without_records(L):
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0     # token recurrence
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 128) == 0   # not built
 
 
 def test_workspace_size_covers_every_chunk(L):

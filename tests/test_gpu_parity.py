@@ -276,3 +276,20 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     gdn.check_device_error()
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
     assert err(y, y_ref) < TOL_16 and err(S_T, S_ref) < TOL_16
+
+
+def test_launch_timing_reports_each_kernel():
+    """gdn_timing_start/stop bracket every library launch with events on its stream."""
+    x = inputs.make_prefill(1, "cuda", seed=31, T=512, H=2)
+    gdn.timing_start(16)
+    for _ in range(2):
+        gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
+    gdn.decode_step(*(inputs.make_decode_step(3, "cuda", B=2, H=2)[k] for k in ("q", "k", "v", "g", "beta")),
+                    inputs.make_decode_state(3, "cuda", B=2, H=2))
+    t = gdn.timing_stop()
+    assert list(t) == ["chunk_ut_kernel", "chunk_chain_kernel", "decode_step_kernel"]
+    assert [c for c, _ in t.values()] == [2, 2, 1]
+    assert all(ms > 0 for _, ms in t.values())
+    with pytest.raises(gdn.GDNError):
+        gdn.timing_stop()  # timing is off again
+    gdn.check_device_error()
