@@ -416,7 +416,8 @@ def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
 
 def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
-    """full mixer: prep -> chunk -> out gate on 4 packed sequences."""
+    """full mixer on 4 packed sequences: prep -> chunk -> out gate (the variant with the gate
+    fused into the chunked pass is timed beside it)."""
     m = inputs.make_mixer(4, "cuda", seed=rank_seed(inputs.SEED_BASE + 4, rank))
     N, H = m["N"], m["H"]
     bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
@@ -427,21 +428,29 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     nsq = m["num_seqs"]
     wsm = torch.empty(max(gdn.workspace_size(N, nsq, H, 128, 128, 64), 16), device="cuda", dtype=torch.uint8)
 
-    def mix(i):
+    def mix(i):  # prep -> chunk -> out gate: three launches
         gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"], m["alpha_logit"],
                  m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"], out=(*bufs, gbuf, bbuf))
         gdn.chunk_fwd(bufs[0], bufs[1], bufs[2], gbuf, bbuf, None, m["cu_seqlens"], chunk=64, y=ym,
                       final_state=False, workspace=wsm)
         gdn.out_gate(ym, m["z"], m["norm_w"], m["eps"], out=out)
 
+    def mix_fused(i):  # the gate fused into the chunked pass (gdn_chunk_fwd_gated)
+        gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"], m["alpha_logit"],
+                 m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"], out=(*bufs, gbuf, bbuf))
+        gdn.chunk_fwd_gated(bufs[0], bufs[1], bufs[2], gbuf, bbuf, m["z"], m["norm_w"], m["eps"], None,
+                            m["cu_seqlens"], final_state=False, out=out, workspace=wsm)
+
     barrier(torch, dist, world)
     n_m = 5
+    dt_fused = max_over_ranks(torch, dist, timed(torch, mix_fused, n_m, 1, stream), world) / n_m
     dt = max_over_ranks(torch, dist, timed(torch, mix, n_m, 1, stream, on_start=lambda: gdn.timing_start(64)),
                         world) / n_m
     km = kernel_table(gdn.timing_stop(), n_m)
     fused_min = N * (H * 3 * 128 * 2 + H * 2 * 2 + H * 128 * 2 + H * 128 * 2)
     return {"workload": inputs.CONFIGS[4]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
                 "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
+                "ms_per_step_gate_fused_into_chunk": dt_fused * 1e3,
                 "roofline": {"bound": "hbm", "achieved": fused_min / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
                              "frac": fused_min / dt / 1e9 / hbm_peak, "kernel": "prep+chunk+out_gate",
                              "alg_bytes_per_step": fused_min,

@@ -152,6 +152,24 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
                            void* workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_fwd_gated -- gdn_chunk_fwd (chunk = 64) with eq. (11)'s output gate, without
+ * the projection W_o, fused into the chunked pass, so y never goes to memory:
+ *   out[t,h,:] = sigmoid(z[t,h,:]) * y[t,h,:] / sqrt(mean_i y[t,h,i]^2 + eps) * (1 + norm_w)
+ * Arguments as gdn_chunk_fwd, except: no y / y_dtype; z and out [N,H,dv] in io_dtype
+ * (BF16 or F16); norm_w [dv] fp32, shared by all heads; eps >= 0.  Tensor-core path only:
+ * chunk = 64, dk = dv = 128, in_dtype BF16 or F16 (anything else returns
+ * GDN_ERR_UNSUPPORTED; use gdn_chunk_fwd followed by gdn_out_gate).  The four 32-column dv slabs of a (sequence,
+ * head) run as one thread-block cluster and exchange each row's partial sum of squares
+ * through distributed shared memory.  Same workspace as gdn_chunk_fwd.
+ */
+gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* g,
+                                 const float* beta, const float* S0, const int32_t* cu_seqlens,
+                                 int num_seqs, int N, int H, int dk, int dv, int chunk, float scale,
+                                 gdn_dtype_t in_dtype, const void* z, const float* norm_w, float eps,
+                                 gdn_dtype_t io_dtype, void* out, float* S_T, void* workspace,
+                                 size_t workspace_bytes, gdn_stream_t stream);
+
+/*
  * gdn_chunk_fwd_noalloc -- gdn_chunk_fwd for callers that cannot allocate device memory.
  * (An addition of this library; the paper has no counterpart.)
  *

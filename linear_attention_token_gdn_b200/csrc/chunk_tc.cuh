@@ -65,12 +65,20 @@ struct ChunkArgs {
     float* S_T;
     void* workspace;
     unsigned long long budget;
+    // fused output gate (gdn_chunk_fwd_gated): out = sigmoid(z) y / rms(y) (1 + norm_w), and y
+    // is not written.  Unused (out == nullptr) by gdn_chunk_fwd.
+    const void* z;
+    const float* norm_w;
+    float eps;
+    int z_dt;
+    void* out;
 };
 
 // TMA descriptors of the chain kernel: [N, H, 128] views of k, q (64-column halves, 128B
-// swizzle), v (NS-column slab, 64B swizzle) and y (NS-column slab, no swizzle, stores).
+// swizzle), v and z (NS-column slab, 64B swizzle) and y -- or out, when the gate is fused --
+// (NS-column slab stores, swizzled to the row width).
 struct ChainMaps {
-    CUtensorMap k, q, v, y;
+    CUtensorMap k, q, v, y, z;
 };
 
 constexpr int kChunk = 64;
@@ -444,14 +452,19 @@ struct ChainCfg {
     static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // [2 slots] U fp16: [64 x ROWB]
     static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // [U' hi | U' lo]: [64 x UROWB]
     static constexpr int OFF_YS = OFF_SU2 + 64 * UROWB;        // y rows for the TMA store [64 x NS x 4 B]
-    static constexpr int OFF_VEC = OFF_YS + 64 * NS * 4;       // [2 slots] gamma, Gamma, f: 3 x 64 floats
+    static constexpr int OFF_ZS = OFF_YS + 64 * NS * 4;        // [2 slots] z slab [64 x ROWB] (gated)
+    static constexpr int OFF_GZ = OFF_ZS + 2 * 64 * ROWB;      // sigmoid(z) (1 + w) rows, fp32 [64 x NS] (gated)
+    static constexpr int OFF_VEC = OFF_GZ + 64 * NS * 4;       // [2 slots] gamma, Gamma, f: 3 x 64 floats
     static constexpr int OFF_META = OFF_VEC + 2 * 1024;        // [2 slots] {c0, L}
-    static constexpr int OFF_BAR = OFF_META + 64;
-    static constexpr int NBARS = 20;
+    static constexpr int OFF_RS = OFF_META + 64;               // [2] [4 slabs] [64 rows] y^2 sums (gated)
+    static constexpr int OFF_NW = OFF_RS + 2 * 4 * 64 * 4;     // 1 + norm_w of this slab (gated)
+    static constexpr int OFF_BAR = OFF_NW + NS * 4;
+    static constexpr int NBARS = 22;
     static constexpr int BYTES = OFF_BAR + 256 + 1024;
     static constexpr uint32_t KV_TX = 2 * K_HALF + 64 * ROWB;  // K and the V slab of one chunk
     static constexpr uint32_t Q_TX = 2 * 8192;                 // Q of one chunk
     static constexpr uint32_t M_TX = 8192;                     // M of one chunk
+    static constexpr uint32_t Z_TX = 64 * ROWB;                // z slab of one chunk (gated)
     // TMEM columns
     static constexpr uint32_t COL_U = 0;                       // [2 slots] x NS: [0; U~] + [Q; -W] S over dk 0-63
     static constexpr uint32_t COL_W = 2 * NS;                  // 128: W (both lane halves)
@@ -464,7 +477,8 @@ struct ChainCfg {
     static_assert(NBARS * 8 <= 192, "barrier area");
     static_assert(BYTES <= 232448, "shared memory budget");
     static_assert(OFF_M % 1024 == 0 && OFF_KS % 1024 == 0 && OFF_TT % 1024 == 0 && OFF_YS % 1024 == 0 &&
-                      OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0 && OFF_SU % 1024 == 0 && OFF_SU2 % 1024 == 0,
+                      OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0 && OFF_SU % 1024 == 0 && OFF_SU2 % 1024 == 0 && OFF_ZS % 1024 == 0 &&
+                      OFF_GZ % 1024 == 0,
                   "swizzle atoms");
 };
 
@@ -476,7 +490,7 @@ struct ChainCfg {
 //                       m_empty[b]   M U of c completed: M slot b and U slot b are free
 // The chain issues M U of chunk c at the start of chunk c + 1, right after that chunk's first
 // MMAs, and forms y of c while they run.
-template <int NS, bool BF>
+template <int NS, bool BF, bool GATED>
 __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a,
                                                              const __grid_constant__ ChainMaps maps) {
     using Cf = ChainCfg<NS>;
@@ -499,6 +513,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     uint64_t* bar_q = bars + 13;       // [2 slots]
     uint64_t* bar_m = bars + 15;       // [2 slots]
     uint64_t* bar_kv = bars + 17;      // [3 stages] K and V landed (bytes)
+    uint64_t* bar_rs = bars + 20;      // [2] the 4 slab CTAs' y^2 sums of a chunk landed (gated, bytes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 192);
     int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 200);
 
@@ -522,6 +537,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     if (warp == 1) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
     tc::tc_fence_before();
     __syncthreads();
+    if constexpr (GATED) tc::cluster_sync();  // peers' barriers exist before anyone stores to them
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int rec_base = *s_base;
@@ -567,8 +583,6 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         const uint64_t dSS0 = tc::smem_desc(sbase + Cf::OFF_SS, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dSU0 = tc::smem_desc(sbase + Cf::OFF_SU, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::UROWB, 8 * Cf::UROWB, tc::kSw128);
-        const int ybytes = a.y_dt == kF32 ? 4 : 2;
-        const int yrow = NS * ybytes;  // 64 or 128 B: the y tile's swizzle span
 
         const size_t st_base = ((size_t)n * H + h) * 128 * 128 + (size_t)tid * 128 + slab * NS;
         float S[NS];
@@ -579,6 +593,8 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         }
 #pragma unroll
         for (int c = 0; c < NS / 8; ++c) st16(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB), pack8<BF>(S + 8 * c));
+        float* nw = reinterpret_cast<float*>(smem + Cf::OFF_NW);
+        if (GATED && tid < NS) nw[tid] = 1.f + a.norm_w[slab * NS + tid];
         operands_ready(true);
 
         // M U of chunk ci (slot bb) -> COL_MU; by thread 0 once M(ci) has landed.  A wait that runs
@@ -599,7 +615,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(bu0, kk * 16 * Cf::ROWB), id_mu,
                                 kk > 0);
                 tc::mma_commit(bar_y);
-                tc::mma_commit(bar_mfree + bb);
+                if constexpr (!GATED) tc::mma_commit(bar_mfree + bb);  // gated: gate_out frees it
             }
             mu_pending = true;
             return w;
@@ -610,34 +626,129 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         int py_c0 = 0, py_L = 0;
         float py_g = 0.f;         // its Gamma_r (rows 0-63)
         float qs[NS];             // its (Q S) row (rows 0-63)
+        int py_x = -1;            // its index in the sequence (gated: selects buffers and phases)
+        bool gated_ok = true;
+        // Gated: out = sigmoid(z) y / sqrt(mean_dv(y^2) + eps) (1 + w).  The four slab CTAs of the
+        // cluster each hold 32 of the 128 columns of y.  For every chunk each CTA stores every row's
+        // partial sum of squares into all four CTAs' shared memory with st.async, whose bytes
+        // complete on the receiver's own bar_rs phase (armed by the receiver: 4 x 64 x 4 bytes).
+        // y_epilogue sends and keeps y in yt; gate_out, after the next MMA wait, waits for the phase,
+        // forms the full mean and gates yt with the z tile the producer loaded beside M.  Every CTA
+        // sends and receives exactly nchunks times, also after an error (see the drain below), so
+        // no store is still in flight towards a CTA when it exits.
+        float yt[NS];
+        bool yt_pending = false;
+        int n_sent = 0, n_recv = 0;  // chunks sent to the cluster / phases of bar_rs waited for
+        constexpr uint32_t RS_TX = NSLAB * 64 * 4;
+        auto send_sums = [&](int x, float ss) {  // warps 0-1
+            const int bb = x & 1;
+            if (tid == 0) tc::mbar_arrive_expect_tx(bar_rs + bb, RS_TX);
+            const uint32_t rs = tc::smem_u32(smem + Cf::OFF_RS) + (uint32_t)((bb * 4 + slab) * 64 + tid) * 4;
+            const uint32_t br = tc::smem_u32(bar_rs + bb);
+#pragma unroll
+            for (int p = 0; p < NSLAB; ++p) tc::st_async_f32(tc::mapa(rs, (uint32_t)p), ss, tc::mapa(br, (uint32_t)p));
+            n_sent = x + 1;
+        };
+        auto stage_rows = [&](const float* t, int dt) {  // a finished row -> YS (full chunk) or memory
+            if (py_L == kChunk) {
+                uint8_t* ys = smem + Cf::OFF_YS;
+                if (dt == kF32) {
+#pragma unroll
+                    for (int cc = 0; cc < NS / 4; ++cc)
+                        *reinterpret_cast<float4*>(ys + tc::swz_off(tid, cc, 4 * NS)) =
+                            make_float4(t[4 * cc], t[4 * cc + 1], t[4 * cc + 2], t[4 * cc + 3]);
+                } else if (dt == kBF16) {
+#pragma unroll
+                    for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, 2 * NS), pack8<true>(t + 8 * cc));
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, 2 * NS), pack8<false>(t + 8 * cc));
+                }
+            } else if (tid < py_L) {
+                void* dst = reinterpret_cast<uint8_t*>(GATED ? a.out : a.y) +
+                            (((size_t)(py_c0 + tid) * H + h) * 128 + slab * NS) * (dt == kF32 ? 4 : 2);
+#pragma unroll
+                for (int j = 0; j < NS; j += 4) st4(dst, dt, j, make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]));
+            }
+        };
+        // gated, warps 0-1, while M U runs: this row's gate factors sigmoid(z) (1 + w) of chunk py_x
+        // -> GZ (row-private, fp32).  Waits for the z tile itself (its own acquire of bar_m).
+        auto gz_prep = [&]() {
+            if (!GATED || py_L <= 0) return;
+            const int bb = py_x & 1;
+            if (!tc::mbar_wait_bounded(bar_m + bb, (py_x >> 1) & 1, a.budget)) {
+                raise_error(kErrTimeout);
+                gated_ok = false;
+                return;
+            }
+            const uint8_t* zs = smem + Cf::OFF_ZS + bb * 64 * Cf::ROWB;
+            uint8_t* gz = smem + Cf::OFF_GZ;
+#pragma unroll
+            for (int cc = 0; cc < NS / 8; ++cc) {
+                const uint4 zr = *reinterpret_cast<const uint4*>(zs + tc::swz_off(tid, cc, Cf::ROWB));
+                const uint32_t zw[4] = {zr.x, zr.y, zr.z, zr.w};
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 z2 = a.z_dt == kBF16 ? unpack2<true>(zw[e]) : unpack2<false>(zw[e]);
+                    f[2 * e] = __fdividef(nw[8 * cc + 2 * e], 1.f + __expf(-z2.x));
+                    f[2 * e + 1] = __fdividef(nw[8 * cc + 2 * e + 1], 1.f + __expf(-z2.y));
+                }
+                *reinterpret_cast<float4*>(gz + tc::swz_off(tid, 2 * cc, 4 * NS)) = make_float4(f[0], f[1], f[2], f[3]);
+                *reinterpret_cast<float4*>(gz + tc::swz_off(tid, 2 * cc + 1, 4 * NS)) = make_float4(f[4], f[5], f[6], f[7]);
+            }
+        };
         auto y_epilogue = [&]() {
             if (warp < 2 && py_L > 0) {
                 float t[NS];
                 tc::tmem_ld32(trow + Cf::COL_MU, t);
 #pragma unroll
                 for (int j = 0; j < NS; ++j) t[j] = a.scale * (py_g * qs[j] + t[j]);
-                if (py_L == kChunk) {
-                    uint8_t* ys = smem + Cf::OFF_YS;
-                    if (a.y_dt == kF32) {
+                if constexpr (GATED) {
+                    float ss = 0.f;
 #pragma unroll
-                        for (int cc = 0; cc < NS / 4; ++cc)
-                            *reinterpret_cast<float4*>(ys + tc::swz_off(tid, cc, yrow)) =
-                                make_float4(t[4 * cc], t[4 * cc + 1], t[4 * cc + 2], t[4 * cc + 3]);
-                    } else if (a.y_dt == kBF16) {
-#pragma unroll
-                        for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, yrow), pack8<true>(t + 8 * cc));
-                    } else {
-#pragma unroll
-                        for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, yrow), pack8<false>(t + 8 * cc));
+                    for (int j = 0; j < NS; ++j) {
+                        ss += t[j] * t[j];
+                        yt[j] = t[j];
                     }
-                } else if (tid < py_L) {
-                    void* dst = reinterpret_cast<uint8_t*>(a.y) + (((size_t)(py_c0 + tid) * H + h) * 128 + slab * NS) * ybytes;
-#pragma unroll
-                    for (int j = 0; j < NS; j += 4) st4(dst, a.y_dt, j, make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]));
+                    send_sums(py_x, ss);
+                    yt_pending = true;
+                } else {
+                    stage_rows(t, a.y_dt);
                 }
             }
         };
-        auto y_store = [&]() {  // after a barrier that follows y_epilogue
+        auto gate_out = [&]() {  // warps 0-1, after y_epilogue; then M slot and z slot are free
+            if (!GATED || !yt_pending) return;
+            yt_pending = false;
+            const int bb = py_x & 1;
+            const uint32_t par = (py_x >> 1) & 1;
+            const bool w = tc::mbar_wait_bounded(bar_rs + bb, par, a.budget);
+            if (w) n_recv = py_x + 1;
+            if (!w) {
+                raise_error(kErrTimeout);
+                gated_ok = false;
+            } else {
+                const float* rs = reinterpret_cast<const float*>(smem + Cf::OFF_RS) + bb * 4 * 64;
+                float tot = 0.f;
+#pragma unroll
+                for (int p = 0; p < NSLAB; ++p) tot += rs[p * 64 + tid];
+                const float inv = rsqrtf(tot / (NS * NSLAB) + a.eps);
+                const uint8_t* gz = smem + Cf::OFF_GZ;
+#pragma unroll
+                for (int cc = 0; cc < NS / 4; ++cc) {
+                    const float4 f = *reinterpret_cast<const float4*>(gz + tc::swz_off(tid, cc, 4 * NS));
+                    yt[4 * cc] *= inv * f.x;
+                    yt[4 * cc + 1] *= inv * f.y;
+                    yt[4 * cc + 2] *= inv * f.z;
+                    yt[4 * cc + 3] *= inv * f.w;
+                }
+                stage_rows(yt, a.z_dt);
+            }
+            tc::bar_sync(4, 64);  // every read of the z slot (gz_prep) is done
+            if (tid == 0) tc::mbar_arrive(bar_mfree + bb);
+        };
+        auto y_store = [&]() {  // after a barrier that follows the staging
             if (tid == 0 && py_L == kChunk) {
                 tc::tma_store_3d(&maps.y, slab * NS, h, py_c0, smem + Cf::OFF_YS);
                 tc::bulk_commit();
@@ -683,13 +794,15 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             bool wm = true, wy = true;
             if (c > 0) {  // the previous chunk's M U, then its y while [Q;W] S runs
                 wm = issue_mu(c - 1);
+                if (warp < 2) gz_prep();
                 wy = wait_mu();
-                if (wy) y_epilogue();
+                if (wy || GATED) y_epilogue();  // gated: the cluster exchange keeps step
             }
             c1_pending = false;
             const bool w1 = wait_mma(bar_c1, ph_c1);
             c2_pending = false;
             const bool w2 = wait_mma(bar_c2, ph_c2);
+            if (warp < 2) gate_out();
 
             {
                 float d1[NS], d2[NS];
@@ -717,7 +830,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     for (int j = 0; j < NS; ++j) qs[j] = d1[j] + d2[j];
                 }
             }
-            if (!(ok = operands_ready(wm && wy && w1 && w2))) break;  // also orders the staged y rows
+            if (!(ok = operands_ready(wm && wy && w1 && w2 && gated_ok))) break;  // also orders the staged y rows
             y_store();
 
             // K^T U' -> state increment; its completion also releases slot b and K stage kst
@@ -744,14 +857,17 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             py_c0 = c0;
             py_L = L;
             py_g = gR;
+            py_x = c;
             if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next y_epilogue writes it
             if (!(ok = operands_ready(w3))) break;
         }
         if (ok && nchunks > 0) {  // the last chunk's M U and y
             const bool wm = issue_mu(nchunks - 1);
+            if (warp < 2) gz_prep();
             const bool wy = wait_mu();
-            if (wy) y_epilogue();
-            if ((ok = operands_ready(wm && wy))) y_store();
+            if (wy || GATED) y_epilogue();
+            if (warp < 2) gate_out();
+            if ((ok = operands_ready(wm && wy && gated_ok))) y_store();
         }
         // never free TMEM under an MMA in flight
         if (c1_pending) tc::mbar_wait_bounded(bar_c1, ph_c1, 4000000000ull);
@@ -759,6 +875,15 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (ds_pending) tc::mbar_wait_bounded(bar_ds, ph_ds, 4000000000ull);
         if (mu_pending) tc::mbar_wait_bounded(bar_y, ph_y, 4000000000ull);
         if (tid == 0) tc::bulk_wait0();
+        if (GATED && warp < 2) {
+            // the rest of the cluster protocol after an early exit: send the chunks not sent (zeros),
+            // then wait for every phase not yet seen -- one phase armed at a time, so each wait's
+            // parity is unambiguous, and bytes sent to this CTA all land before it exits
+            for (int x = n_recv; x < nchunks; ++x) {
+                if (x >= n_sent) send_sums(x, 0.f);
+                tc::mbar_wait_bounded(bar_rs + (x & 1), (x >> 1) & 1, 4000000000ull);
+            }
+        }
         if (ok && a.S_T) {
 #pragma unroll
             for (int j = 0; j < NS; j += 4)
@@ -807,8 +932,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         auto issue_m = [&](int ci) {  // M of chunk ci -> M slot ci & 1 (issuer thread only)
             const int bb = ci & 1;
             (bb ? m_last1 : m_last0) = ci;
-            tc::mbar_arrive_expect_tx(bar_m + bb, Cf::M_TX);
+            tc::mbar_arrive_expect_tx(bar_m + bb, GATED ? Cf::M_TX + Cf::Z_TX : Cf::M_TX);
             tc::bulk_g2s(smem + Cf::OFF_M + bb * 8192, rec_ptr(ci) + kRecM, 8192, bar_m + bb);
+            if constexpr (GATED)
+                tc::tma_load_3d(smem + Cf::OFF_ZS + bb * 64 * Cf::ROWB, &maps.z, slab * NS, h, t_begin + ci * kChunk,
+                                bar_m + bb);
         };
         auto issue_tt = [&](int ci) {  // T_w (twice) and T_u of chunk ci -> TT rows 0-127, 192-255
             tt_issued = ci;
@@ -832,6 +960,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::prefetch_tmap(&maps.k);
             tc::prefetch_tmap(&maps.q);
             tc::prefetch_tmap(&maps.v);
+            if constexpr (GATED) tc::prefetch_tmap(&maps.z);
         }
         if (nchunks > 0) {
             issue_kv(0);
@@ -970,6 +1099,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         (void)ok;
     }
 
+    if constexpr (GATED) tc::cluster_sync();  // no CTA leaves while a peer may still write to it
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -984,7 +1114,9 @@ inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, 
     using Ch = ChainCfg<NS>;
     cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel<BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, UtCfg::BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_chain_kernel<NS, BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
+    e = cudaFuncSetAttribute(chunk_chain_kernel<NS, BF, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_chain_kernel<NS, BF, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
     if (e != cudaSuccess) return e;
     const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
     if (nvc > 0) {
@@ -993,9 +1125,27 @@ inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, 
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    LaunchScope timed(st, "chunk_chain_kernel");
-    chunk_chain_kernel<NS, BF><<<(unsigned)(a.num_seqs * a.H * (128 / NS)), 256, Ch::BYTES, st>>>(a, maps);
-    return cudaGetLastError();
+    const unsigned grid = (unsigned)(a.num_seqs * a.H * (128 / NS));
+    if (a.out == nullptr) {
+        LaunchScope timed(st, "chunk_chain_kernel");
+        chunk_chain_kernel<NS, BF, false><<<grid, 256, Ch::BYTES, st>>>(a, maps);
+        return cudaGetLastError();
+    }
+    // gated: the 128 / NS slab CTAs of a (sequence, head) form one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = Ch::BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 128 / NS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope timed(st, "chunk_chain_gated_kernel");
+    return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<NS, BF, true>, a, maps);
 }
 
 // Both kernels of the chunked path on stream st.  *why is set (and nothing launched) when the
@@ -1007,13 +1157,17 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
         return cudaSuccess;
     }
     constexpr int NS = 32;
-    // y tiles are NS columns = 64 B (16-bit) or 128 B (fp32) per row, stored with the matching swizzle
-    const CUtensorMapSwizzle yswz = a.y_dt == kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    ChainMaps maps;
+    // y (or out) tiles are NS columns = 64 B (16-bit) or 128 B (fp32) per row, stored with the
+    // matching swizzle; the gated variant stores out and loads z slabs
+    const bool gated = a.out != nullptr;
+    const int st_dt = gated ? a.z_dt : a.y_dt;
+    const CUtensorMapSwizzle yswz = st_dt == kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    ChainMaps maps = {};  // the z map stays empty without the gate
     if (!encode_map_3d(&maps.k, a.k, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.q, a.q, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, 128, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, 128, NS, kChunk, yswz)) {
+        !encode_map_3d(&maps.y, gated ? a.out : a.y, st_dt, a.N, a.H, 128, NS, kChunk, yswz) ||
+        (gated && !encode_map_3d(&maps.z, a.z, a.z_dt, a.N, a.H, 128, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B))) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaSuccess;
     }

@@ -268,6 +268,35 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     return GDN_OK;
 }
 
+gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                                 const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
+                                 int dv, int chunk, float scale, gdn_dtype_t in_dtype, const void* z,
+                                 const float* norm_w, float eps, gdn_dtype_t io_dtype, void* out, float* S_T,
+                                 void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(io_dtype), "bad dtype");
+    REQUIRE(eps >= 0.f, "eps < 0");
+    REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
+    REQUIRE((long long)N * H * 128 < (1LL << 40), "problem too large");
+    if (chunk != 64 || dk != 128 || dv != 128 || in_dtype == GDN_F32 || io_dtype == GDN_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "the gated variant runs the tensor-core path only (chunk 64, dk=dv=128, "
+                                         "bf16/f16 inputs, bf16/f16 z and out)");
+    if (N == 0 && S_T == nullptr) return GDN_OK;
+    REQUIRE_PTR(g, "g"); REQUIRE_PTR(beta, "beta"); REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k");
+    REQUIRE_PTR(v, "v"); REQUIRE_PTR(z, "z"); REQUIRE_PTR(norm_w, "norm_w"); REQUIRE_PTR(out, "out");
+    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens"); OPT_PTR(workspace, "workspace");
+    const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+    REQUIRE(workspace_bytes >= need && (need == 0 || workspace != nullptr), "workspace of %zu bytes < %zu",
+            workspace_bytes, need);
+    gdn::ChunkArgs a{q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, chunk, scale, (int)in_dtype,
+                     (int)io_dtype, nullptr, S_T, workspace, wait_budget(), z, norm_w, eps, (int)io_dtype, out};
+    const char* why = nullptr;
+    cudaError_t e = gdn::chunk_tc_launch(a, reinterpret_cast<cudaStream_t>(stream), &why);
+    if (why) return fail(GDN_ERR_CUDA, "chunk_tc: %s", why);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "chunk_tc gated: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
 gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* g, const float* beta,
                                    const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
                                    int dv, int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t y_dtype, void* y,

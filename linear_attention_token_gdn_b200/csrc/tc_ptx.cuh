@@ -260,3 +260,38 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
 
 }  // namespace tc
 }  // namespace gdn
+
+namespace gdn {
+namespace tc {
+
+// ---------------------------------------------------------------- thread-block clusters
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address in CTA `rank`'s shared memory of the variable at local shared address `saddr`.
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Asynchronous 4-byte store into the shared memory of a CTA of the cluster (address from mapa);
+// its completion is counted, in bytes, on that CTA's mbarrier `cbar` (also from mapa): a thread
+// that sees the barrier's phase complete sees the value.  No fence is involved.
+__device__ __forceinline__ void st_async_f32(uint32_t caddr, float v, uint32_t cbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(caddr),
+                 "r"(__float_as_uint(v)), "r"(cbar)
+                 : "memory");
+}
+
+// Barrier over every thread of the cluster (all threads of the CTA must call it).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+}  // namespace tc
+}  // namespace gdn

@@ -33,6 +33,8 @@ SIGNATURES = {
     "gdn_chunk_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
     "gdn_chunk_fwd": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P,
                        _Z, _P], _I),
+    "gdn_chunk_fwd_gated": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _F, _I, _P,
+                             _P, _P, _Z, _P], _I),
     "gdn_chunk_fwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P], _I),
     "gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
@@ -176,6 +178,30 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=None, chunk=6
                                _ptr(S_T), _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                _stream(stream)))
     return y, S_T
+
+
+def chunk_fwd_gated(q, k, v, g, beta, z, norm_w, eps=1e-6, S0=None, cu_seqlens=None, num_seqs=None, scale=1.0,
+                    final_state=True, out=None, S_T=None, workspace=None, stream=None):
+    """gdn_chunk_fwd_gated: the chunk-64 prefill with eq. (11)'s output gate fused (y is not
+    written).  Returns (out [N, H, dv] in z's dtype, S_T or None)."""
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    elif num_seqs is None:
+        num_seqs = 1
+    if out is None:
+        out = torch.empty(N, H, dv, device=q.device, dtype=z.dtype)
+    if S_T is None and final_state:
+        S_T = torch.empty(num_seqs, H, dk, dv, device=q.device, dtype=torch.float32)
+    ws_bytes = workspace_size(N, num_seqs, H, dk, dv, 64)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    _check(lib().gdn_chunk_fwd_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                                     num_seqs, N, H, dk, dv, 64, float(scale), _dt(q), _ptr(z), _ptr(norm_w),
+                                     float(eps), _dt(z), _ptr(out), _ptr(S_T), _ptr(workspace),
+                                     0 if workspace is None else workspace.numel(), _stream(stream)))
+    return out, S_T
 
 
 def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=None, chunk=64, scale=1.0,

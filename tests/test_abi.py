@@ -69,6 +69,32 @@ def test_chunk_fwd_tensor_core_path_limits(L, over):
     assert chunk_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
 
 
+def gated_call(L, **over):
+    a = dict(q=A, k=A, v=A, g=A, beta=A, S0=None, cu=None, num_seqs=2, N=64, H=2, dk=128, dv=128, chunk=64,
+             scale=1.0, in_dt=gdn.BF16, z=A, w=A, eps=1e-6, io_dt=gdn.BF16, out=A, S_T=None, ws=A,
+             ws_bytes=1 << 30, stream=None)
+    a.update(over)
+    return L.gdn_chunk_fwd_gated(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["cu"], a["num_seqs"],
+                                 a["N"], a["H"], a["dk"], a["dv"], a["chunk"], a["scale"], a["in_dt"], a["z"],
+                                 a["w"], a["eps"], a["io_dt"], a["out"], a["S_T"], a["ws"], a["ws_bytes"],
+                                 a["stream"])
+
+
+@pytest.mark.parametrize("over", [
+    dict(z=None), dict(out=MIS), dict(w=None), dict(eps=-1.0), dict(io_dt=5), dict(N=-1), dict(N=63),
+    dict(ws_bytes=0, ws=None), dict(q=None),
+])
+def test_chunk_fwd_gated_rejects_bad_arguments(L, over):
+    assert gated_call(L, **over) == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.last_error_message() != ""
+
+
+@pytest.mark.parametrize("over", [dict(chunk=0), dict(chunk=32), dict(dk=64, dv=64), dict(in_dt=gdn.F32),
+                                  dict(io_dt=gdn.F32)])
+def test_chunk_fwd_gated_is_tensor_core_only(L, over):
+    assert gated_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
+
+
 def test_workspace_size_is_zero_without_records(L):
     assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0     # token recurrence
     assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 128) == 0   # not built

@@ -229,7 +229,7 @@ def out_gate_bound(ref_y, z, norm_w, tol):
 
 def test_full_mixer_workload_sampled_heads():
     """Packed variable-length sequences, H=16, d=128, bf16 throughout: prep -> chunked
-    recurrence -> out gate through the C ABI, against the fp64 oracle mixer on sampled heads.
+    recurrence -> out gate through the C ABI (and prep -> the chunked pass with the gate fused), against the fp64 oracle mixer on sampled heads.
     q, k, v are stored in bf16 between prep and the recurrence, and the oracle rounds them the
     same way.  y meets the chunked path's bound; out meets that bound propagated through the
     RMS normalisation of eq. (11), plus its own bf16 rounding."""
@@ -239,6 +239,7 @@ def test_full_mixer_workload_sampled_heads():
                                 out_dtype=torch.bfloat16)
     y, S_T = gdn.chunk_fwd(q, k, v, g, beta, None, m["cu_seqlens"], chunk=64, y_dtype=torch.float32)
     out = gdn.out_gate(y, m["z"], m["norm_w"], m["eps"])
+    out_f, S_f = gdn.chunk_fwd_gated(q, k, v, g, beta, m["z"], m["norm_w"], m["eps"], None, m["cu_seqlens"])
     d = m["d"]
     for h in (0, 9):
         hs = slice(h, h + 1)
@@ -253,9 +254,55 @@ def test_full_mixer_workload_sampled_heads():
         got = out[:, hs].double().cpu().numpy()
         bound = out_gate_bound(ref_y, m["z"][:, hs], m["norm_w"], TOL_16) + UNIT_ROUNDOFF[out.dtype] * np.abs(ref_out)
         worst = float(np.max(np.abs(got - ref_out) / bound))
-        print(f"mixer head {h}: y err {ey:.2e}, out within {worst:.2f} of its bound")
-        assert worst <= 1.0, (h, worst)
+        worst_f = float(np.max(np.abs(out_f[:, hs].double().cpu().numpy() - ref_out) / bound))
+        print(f"mixer head {h}: y err {ey:.2e}, out within {worst:.2f} of its bound, fused gate {worst_f:.2f}")
+        assert worst <= 1.0 and worst_f <= 1.0, (h, worst, worst_f)
     gdn.check_device_error()
+
+
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+def test_chunk_fwd_gated_small_ragged(dt):
+    """The fused out gate: ragged tails, an empty and a one-token sequence, S0 != 0.  out meets
+    the chunked path's bound propagated through eq. (11); S_T is the plain path's."""
+    lengths = [3 * 64 + 17, 64, 1, 0, 130]
+    x = inputs.make_prefill(2, "cuda", seed=24, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
+    gen = torch.Generator(device="cuda").manual_seed(25)
+    N, H, dv = x["v"].shape
+    z = torch.randn(N, H, dv, device="cuda", generator=gen).to(dt)
+    w = torch.randn(dv, device="cuda", generator=gen) * 0.5
+    out, S_T = gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], z, w, 1e-6, x["S0"],
+                                   x["cu_seqlens"])
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
+    ref_out = oracle.out_gate(y_ref, z, w, 1e-6)
+    bound = out_gate_bound(y_ref, z, w, TOL_16) + UNIT_ROUNDOFF[dt] * np.abs(ref_out)
+    worst = float(np.max(np.abs(out.double().cpu().numpy() - ref_out) / bound))
+    assert worst <= 1.0, worst
+    assert err(S_T, S_ref) < TOL_16
+    gdn.check_device_error()
+
+
+def test_chunk_fwd_gated_bounded_wait_reports_timeout():
+    """The gated variant's cluster exchange waits are bounded too: with a one-cycle budget the
+    call flags GDN_ERR_TIMEOUT and every CTA of every cluster still leaves; the next call is
+    correct."""
+    x = inputs.make_prefill(1, "cuda", seed=26, T=256, H=2)
+    N, H, dv = x["v"].shape
+    z = torch.ones(N, H, dv, device="cuda", dtype=x["q"].dtype)
+    w = torch.zeros(dv, device="cuda")
+    try:
+        gdn.set_wait_budget(1)
+        gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], z, w, 1e-6, None, x["cu_seqlens"])
+        with pytest.raises(gdn.GDNError) as e:
+            gdn.check_device_error()
+        assert e.value.status == gdn.GDN_ERR_TIMEOUT
+    finally:
+        gdn.set_wait_budget(0)
+    out, _ = gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], z, w, 1e-6, None, x["cu_seqlens"])
+    gdn.check_device_error()
+    y_ref, _ = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+    ref_out = oracle.out_gate(y_ref, z, w, 1e-6)
+    bound = out_gate_bound(y_ref, z, w, TOL_16) + UNIT_ROUNDOFF[out.dtype] * np.abs(ref_out)
+    assert float(np.max(np.abs(out.double().cpu().numpy() - ref_out) / bound)) <= 1.0
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
