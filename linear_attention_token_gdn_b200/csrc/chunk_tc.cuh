@@ -488,8 +488,8 @@ struct ChainCfg {
 //   chain -> producer   ds_done[b]   the state MMA of c completed: [Q;W] slot b, U~ columns b and
 //                                    K stage c % 3 are free (everything else of c was read before)
 //                       m_empty[b]   M U of c completed: M slot b and U slot b are free
-// The chain issues M U of chunk c at the start of chunk c + 1, right after that chunk's first
-// MMAs, and forms y of c while they run.
+// The chain issues M U of chunk c once chunk c + 1's [Q;W] S has completed (the MMA front end is
+// idle while warps 2-3 form U) and forms y of c meanwhile.
 template <int NS, bool BF, bool GATED>
 __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a,
                                                              const __grid_constant__ ChainMaps maps) {
@@ -791,18 +791,19 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 tc::mma_commit(hf ? bar_c2 : bar_c1);
             }
             c1_pending = c2_pending = true;
-            bool wm = true, wy = true;
-            if (c > 0) {  // the previous chunk's M U, then its y while [Q;W] S runs
-                wm = issue_mu(c - 1);
-                if (warp < 2) gz_prep();
-                wy = wait_mu();
-                if (wy || GATED) y_epilogue();  // gated: the cluster exchange keeps step
-            }
+            if (c > 0 && warp < 2) gz_prep();  // gated: gate factors of the previous chunk meanwhile
             c1_pending = false;
             const bool w1 = wait_mma(bar_c1, ph_c1);
             c2_pending = false;
             const bool w2 = wait_mma(bar_c2, ph_c2);
-            if (warp < 2) gate_out();
+            // The previous chunk's M U, then its y (warps 0-1), while warps 2-3 form U: the MMA front
+            // end is otherwise idle until the state MMA, so M U delays neither product of the chain.
+            bool wm = true, wy = true;
+            if (c > 0) {
+                wm = issue_mu(c - 1);
+                wy = wait_mu();
+                if (wy || GATED) y_epilogue();  // gated: the cluster exchange keeps step
+            }
 
             {
                 float d1[NS], d2[NS];
@@ -830,7 +831,8 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     for (int j = 0; j < NS; ++j) qs[j] = d1[j] + d2[j];
                 }
             }
-            if (!(ok = operands_ready(wm && wy && w1 && w2 && gated_ok))) break;  // also orders the staged y rows
+            if (warp < 2) gate_out();
+            if (!(ok = operands_ready(wm && wy && w1 && w2 && gated_ok))) break;  // also orders the staged rows
             y_store();
 
             // K^T U' -> state increment; its completion also releases slot b and K stage kst
@@ -858,12 +860,12 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             py_L = L;
             py_g = gR;
             py_x = c;
-            if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next y_epilogue writes it
+            if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next staging writes it
             if (!(ok = operands_ready(w3))) break;
         }
         if (ok && nchunks > 0) {  // the last chunk's M U and y
-            const bool wm = issue_mu(nchunks - 1);
             if (warp < 2) gz_prep();
+            const bool wm = issue_mu(nchunks - 1);
             const bool wy = wait_mu();
             if (wy || GATED) y_epilogue();
             if (warp < 2) gate_out();
