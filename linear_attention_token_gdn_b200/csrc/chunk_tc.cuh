@@ -773,7 +773,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 break;
             }
             tc::tc_fence_after();
-            const float* vb = vec(b);  // gamma[0:64] Gamma[64:128] f[128:192]
+            const float* vb = vec(b);  // gamma[0:64] Gamma[64:128] f[128:192] (g prefetch [192:256])
             const int c0 = meta[2 * b], L = meta[2 * b + 1];
             const float gC = vb[64 + 63];
             const float gR = tid < 64 ? vb[64 + tid] : 0.f;
@@ -948,10 +948,15 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::bulk_g2s(smem + Cf::OFF_TT + 8192, rec_ptr(ci) + kRecTw, 8192, bar_tt);
             tc::bulk_g2s(smem + Cf::OFF_TT + 24576, rec_ptr(ci) + kRecTu, 8192, bar_tt);
         };
-        float pg = 0.f;  // g of the next chunk (beta is already inside T_w, T_u)
+        // g of chunk ci (beta is already inside T_w, T_u) -> vec(ci & 1)[192:256] by cp.async, two
+        // chunks ahead, so no thread waits on the load; one cp.async group per chunk (warps 4-5)
         auto load_gates = [&](int ci) {
-            const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
-            if (it < 64) pg = it < L ? a.g[(size_t)(c0 + it) * H + h] : 0.f;
+            if (it < 64 && ci < nchunks) {
+                const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
+                const bool in = it < L;
+                tc::cp_async4(vec(ci & 1) + 192 + it, in ? a.g + (size_t)(c0 + it) * H + h : a.g, in ? 4u : 0u);
+            }
+            if (it < 64) tc::cp_async_commit();
         };
         // TT rows 128-191 stay zero: A = [0; T_u] leaves lanes 0-63 of the U~ accumulator at zero
 #pragma unroll
@@ -967,8 +972,9 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (nchunks > 0) {
             issue_kv(0);
             issue_tt(0);
-            load_gates(0);
         }
+        load_gates(0);
+        load_gates(1);
 
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1, kst = c % 3;
@@ -987,7 +993,8 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             //      f = exp(gamma_C - gamma) -----------------------------------------------------------
             if (it < 64) {
                 constexpr int BID_G = 3;
-                float gv = pg;
+                tc::cp_async_wait<1>();  // this chunk's group; the next chunk's may still be in flight
+                float gv = vb[192 + it];
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, gv, o);
@@ -1087,8 +1094,9 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 if (tc::mbar_wait_bounded(bar_mfree + b, ((c >> 1) & 1) ^ 1, a.budget)) issue_m(c);
                 else raise_error(kErrTimeout);
             }
-            if (c + 1 < nchunks) load_gates(c + 1);
+            load_gates(c + 2);
         }
+        if (it < 64) tc::cp_async_wait<0>();  // no copy into shared memory left in flight
         // never leave with copies into this CTA's shared memory in flight
         if (kv_issued > kv_landed) tc::mbar_wait_bounded(bar_kv + kv_issued % 3, (kv_issued / 3) & 1, 4000000000ull);
         if (kv_issued > kv_landed + 1)
