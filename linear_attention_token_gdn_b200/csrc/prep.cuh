@@ -111,39 +111,18 @@ __device__ __forceinline__ void lds_row(const uint8_t* p, float (&x)[PER]) {
     }
 }
 
-// One tensor (q, k or v) of one head over tokens [t0, t1): ShortConv -> SiLU (-> L2Norm), read
-// from the CTA's tile, whose row r holds token tt - (TAPS - 1) + r (rows before a sequence
-// start are masked, rows before token 0 or past N are zero-filled by the copy).  The tokens of
-// a batch are computed independently, so their reductions interleave.
-template <int D, int TAPS, bool NORM, int IDT>
-__device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, int tt, const float* __restrict__ w,
-                                            int W, void* __restrict__ out, int out_dt, float eps, int t0, int t1,
-                                            int H, int h, int lane, SeqWalk sw) {
+// The batches of one tensor over tokens [t0, t1).  CLEAN: the window [t0 - (TAPS - 1), t1) lies
+// in one sequence, so no tap is masked and no token needs its sequence start.
+template <int D, int TAPS, bool NORM, int IDT, bool CLEAN>
+__device__ __forceinline__ void prep_batches(const uint8_t* __restrict__ row0, const float (&wp)[TAPS][D >= 32 ? D / 32 : 1],
+                                             float (&xb)[TAPS - 1 + kPrepBatch][D >= 32 ? D / 32 : 1], void* __restrict__ out,
+                                             int out_dt, float eps, int t0, int t1, int H, int h, int c0, bool active,
+                                             SeqWalk& sw) {
     constexpr int PER = D >= 32 ? D / 32 : 1;
     constexpr int HIST = TAPS - 1;
     constexpr int B = kPrepBatch;
     constexpr int ESZ = IDT == kF32 ? 4 : 2;
-    const bool active = D >= 32 || lane < D;
-    const int c0 = (D >= 32 ? lane * PER : lane);
-    const uint8_t* row0 = tile + (t0 - tt) * D * ESZ + c0 * ESZ;  // row of token t0 - HIST + r at row0 + r * D * ESZ
-    float wp[TAPS][PER];  // wp[TAPS - W + j] = w[c][j]
-#pragma unroll
-    for (int i = 0; i < TAPS; ++i) {
-#pragma unroll
-        for (int u = 0; u < PER; ++u) {
-            const int j = i - (TAPS - W);
-            wp[i][u] = (active && j >= 0) ? w[((size_t)h * D + c0 + u) * W + j] : 0.f;
-        }
-    }
-    float xb[HIST + B][PER];  // [0, HIST): the rows before the batch; then the batch
-#pragma unroll
-    for (int i = 0; i < HIST; ++i) {
-        if (active) lds_row<PER, IDT>(row0 + i * D * ESZ, xb[i]);
-        else {
-#pragma unroll
-            for (int u = 0; u < PER; ++u) xb[i][u] = 0.f;
-        }
-    }
+#pragma unroll 1
     for (int tb = t0; tb < t1; tb += B) {
         const int rb = tb - t0 + HIST;  // tile row of token tb
 #pragma unroll
@@ -154,16 +133,18 @@ __device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, in
                 for (int u = 0; u < PER; ++u) xb[HIST + k][u] = 0.f;
             }
         }
-        int lim[B];  // previous tokens of the same sequence (-1: past t1)
+        int lim[B];  // previous tokens of the same sequence (unused when CLEAN)
+        if constexpr (!CLEAN) {
 #pragma unroll
-        for (int k = 0; k < B; ++k) lim[k] = tb + k < t1 ? tb + k - sw.start_of(tb + k) : -1;
+            for (int k = 0; k < B; ++k) lim[k] = tb + k < t1 ? tb + k - sw.start_of(tb + k) : -1;
+        }
         float y[B][PER];
 #pragma unroll
         for (int k = 0; k < B; ++k) {
 #pragma unroll
             for (int u = 0; u < PER; ++u) {
                 float acc = 0.f;
-                if (lim[k] >= HIST) {
+                if (CLEAN || lim[k] >= HIST) {
 #pragma unroll
                     for (int i = 0; i < TAPS; ++i) acc += wp[i][u] * xb[k + i][u];
                 } else {
@@ -205,6 +186,50 @@ __device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, in
             for (int u = 0; u < PER; ++u) xb[i][u] = xb[B + i][u];
         }
     }
+}
+
+// One tensor (q, k or v) of one head over tokens [t0, t1), at most kPrepRun / 2 of them:
+// ShortConv -> SiLU (-> L2Norm), read from the CTA's tile, whose row r holds token
+// tt - (TAPS - 1) + r (rows before a sequence start are masked, rows before token 0 or past N
+// are zero-filled by the copy).  The tokens of a batch are computed independently, so their
+// reductions interleave.
+template <int D, int TAPS, bool NORM, int IDT>
+__device__ __forceinline__ void prep_tensor(const uint8_t* __restrict__ tile, int tt, const float* __restrict__ w,
+                                            int W, void* __restrict__ out, int out_dt, float eps, int t0, int t1,
+                                            int H, int h, int lane, SeqWalk sw) {
+    constexpr int PER = D >= 32 ? D / 32 : 1;
+    constexpr int HIST = TAPS - 1;
+    constexpr int B = kPrepBatch;
+    constexpr int ESZ = IDT == kF32 ? 4 : 2;
+    const bool active = D >= 32 || lane < D;
+    const int c0 = (D >= 32 ? lane * PER : lane);
+    const uint8_t* row0 = tile + (t0 - tt) * D * ESZ + c0 * ESZ;  // row of token t0 - HIST + r at row0 + r * D * ESZ
+    float wp[TAPS][PER];  // wp[TAPS - W + j] = w[c][j]
+#pragma unroll
+    for (int i = 0; i < TAPS; ++i) {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int j = i - (TAPS - W);
+            wp[i][u] = (active && j >= 0) ? w[((size_t)h * D + c0 + u) * W + j] : 0.f;
+        }
+    }
+    float xb[HIST + B][PER];  // [0, HIST): the rows before the batch; then the batch
+#pragma unroll
+    for (int i = 0; i < HIST; ++i) {
+        if (active) lds_row<PER, IDT>(row0 + i * D * ESZ, xb[i]);
+        else {
+#pragma unroll
+            for (int u = 0; u < PER; ++u) xb[i][u] = 0.f;
+        }
+    }
+    if constexpr (TAPS <= 4) {  // (the wider conv has no registers for a second copy of the loop)
+        const int s0 = sw.start_of(t0);  // t0's sequence is [s0, sw.nxt)
+        if (t0 - s0 >= HIST && t1 <= sw.nxt) {
+            prep_batches<D, TAPS, NORM, IDT, true>(row0, wp, xb, out, out_dt, eps, t0, t1, H, h, c0, active, sw);
+            return;
+        }
+    }
+    prep_batches<D, TAPS, NORM, IDT, false>(row0, wp, xb, out, out_dt, eps, t0, t1, H, h, c0, active, sw);
 }
 
 // TMA descriptors of the three projection outputs, [N, H, d] each; box = d x 1 x (run + taps - 1).
