@@ -423,7 +423,7 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
     gbuf = torch.empty(N, H, device="cuda")
     bbuf = torch.empty(N, H, device="cuda")
-    ym = torch.empty(N, H, 128, device="cuda")
+    ym = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)  # y between the chunked pass and the gate
     out = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)
     nsq = m["num_seqs"]
     wsm = torch.empty(max(gdn.workspace_size(N, nsq, H, 128, 128, 64), 16), device="cuda", dtype=torch.uint8)

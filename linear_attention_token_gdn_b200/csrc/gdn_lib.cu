@@ -176,6 +176,34 @@ gdn_status_t noalloc_scratch(void** out) {
 
 }  // namespace
 
+namespace {
+
+template <int DV, int YT, int ZT>
+void launch_out_gate_t(const void* y, const void* z, const float* w, float eps, long long rows, void* out,
+                       cudaStream_t st) {
+    const long long per_block = (long long)gdn::kGateWarps * gdn::GateShape<DV, YT, ZT>::ROWS_PER_WARP;
+    const unsigned grid = (unsigned)((rows + per_block - 1) / per_block);
+    gdn::out_gate_kernel<DV, YT, ZT><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, w, eps, rows, out);
+}
+
+template <int DV, int YT>
+void launch_out_gate_y(const void* y, const void* z, const float* w, float eps, long long rows, int zt, void* out,
+                       cudaStream_t st) {
+    if (zt == gdn::kF32) launch_out_gate_t<DV, YT, gdn::kF32>(y, z, w, eps, rows, out, st);
+    else if (zt == gdn::kBF16) launch_out_gate_t<DV, YT, gdn::kBF16>(y, z, w, eps, rows, out, st);
+    else launch_out_gate_t<DV, YT, gdn::kF16>(y, z, w, eps, rows, out, st);
+}
+
+template <int DV>
+void launch_out_gate(const void* y, const void* z, const float* w, float eps, long long rows, int yt, int zt,
+                     void* out, cudaStream_t st) {
+    if (yt == gdn::kF32) launch_out_gate_y<DV, gdn::kF32>(y, z, w, eps, rows, zt, out, st);
+    else if (yt == gdn::kBF16) launch_out_gate_y<DV, gdn::kBF16>(y, z, w, eps, rows, zt, out, st);
+    else launch_out_gate_y<DV, gdn::kF16>(y, z, w, eps, rows, zt, out, st);
+}
+
+}  // namespace
+
 extern "C" {
 
 int gdn_version(void) { return 100; }
@@ -348,15 +376,13 @@ gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, flo
     if (N == 0) return GDN_OK;
     REQUIRE_PTR(y, "y"); REQUIRE_PTR(z, "z"); REQUIRE_PTR(norm_w, "norm_w"); REQUIRE_PTR(out, "out");
     const long long rows = (long long)N * H;
-    const long long per_block = (long long)gdn::kGateWarps * gdn::kGateRows;
-    const unsigned grid = (unsigned)((rows + per_block - 1) / per_block);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     gdn::LaunchScope timed(st, "out_gate_kernel");
     switch (dv) {
-        case 16: gdn::out_gate_kernel<16><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
-        case 32: gdn::out_gate_kernel<32><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
-        case 64: gdn::out_gate_kernel<64><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
-        default: gdn::out_gate_kernel<128><<<grid, 32 * gdn::kGateWarps, 0, st>>>(y, z, norm_w, eps, rows, y_dtype, io_dtype, out); break;
+        case 16: launch_out_gate<16>(y, z, norm_w, eps, rows, (int)y_dtype, (int)io_dtype, out, st); break;
+        case 32: launch_out_gate<32>(y, z, norm_w, eps, rows, (int)y_dtype, (int)io_dtype, out, st); break;
+        case 64: launch_out_gate<64>(y, z, norm_w, eps, rows, (int)y_dtype, (int)io_dtype, out, st); break;
+        default: launch_out_gate<128>(y, z, norm_w, eps, rows, (int)y_dtype, (int)io_dtype, out, st); break;
     }
     return launched("out_gate_kernel");
 }

@@ -298,8 +298,8 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ wq,
     void* out = ten == 0 ? q : ten == 1 ? k : v;
     const int ta = t0 + (warp & 1) * (kPrepRun / 2), tb = min(ta + kPrepRun / 2, t1);
     if (ta >= tb) return;
-    SeqWalk swh;
-    swh.init(cu, num_seqs, N, ta);
+    SeqWalk swh = sw;  // walks on from the run's first token: no second search
+    swh.start_of(ta);
     // eqs. (6), (7): q and k are normalised; eq. (8): v is not
 #define GDN_PREP_TENSOR(IDT)                                                                                     \
     if (ten < 2) prep_tensor<DK, TAPS, true, IDT>(tile, t0, w, W, out, out_dt, eps, ta, tb, H, h, lane, swh);   \

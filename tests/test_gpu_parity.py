@@ -148,13 +148,18 @@ def test_prep_matches_oracle(d, out_dt, case):
     gdn.check_device_error()
 
 
-@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
-def test_out_gate_matches_oracle(io):
-    gen = torch.Generator(device="cuda").manual_seed(3)
-    y = torch.randn(300, 4, 128, device="cuda", generator=gen) * 2
-    z = torch.randn(300, 4, 128, device="cuda", generator=gen).to(io)
-    w = torch.randn(128, device="cuda", generator=gen) * 0.02
+@pytest.mark.parametrize("dv", [128, 64, 32, 16])
+@pytest.mark.parametrize("y_dt,io", [(torch.float32, torch.float32), (torch.float32, torch.bfloat16),
+                                     (torch.bfloat16, torch.bfloat16), (torch.float16, torch.float16),
+                                     (torch.bfloat16, torch.float32)])
+def test_out_gate_matches_oracle(dv, y_dt, io):
+    """Every (y, z/out) storage pair and head size; 301 x 3 rows, so the last block is ragged."""
+    gen = torch.Generator(device="cuda").manual_seed(3 + dv)
+    y = (torch.randn(301, 3, dv, device="cuda", generator=gen) * 2).to(y_dt)
+    z = torch.randn(301, 3, dv, device="cuda", generator=gen).to(io)
+    w = torch.randn(dv, device="cuda", generator=gen) * 0.02
     out = gdn.out_gate(y, z, w, 1e-6)
+    assert out.dtype == io
     ref = oracle.out_gate(y, z, w, 1e-6)
     assert err(out, ref) < TOL_F32
 
@@ -227,7 +232,8 @@ def out_gate_bound(ref_y, z, norm_w, tol):
     return gain * 2.0 * np.sqrt(d) * dy2 / np.maximum(row, 1e-30)
 
 
-def test_full_mixer_workload_sampled_heads():
+@pytest.mark.parametrize("y_dt", [torch.float32, torch.bfloat16])
+def test_full_mixer_workload_sampled_heads(y_dt):
     """Packed variable-length sequences, H=16, d=128, bf16 throughout: prep -> chunked
     recurrence -> out gate through the C ABI (and prep -> the chunked pass with the gate fused), against the fp64 oracle mixer on sampled heads.
     q, k, v are stored in bf16 between prep and the recurrence, and the oracle rounds them the
@@ -237,7 +243,7 @@ def test_full_mixer_workload_sampled_heads():
     q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
                                 m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
                                 out_dtype=torch.bfloat16)
-    y, S_T = gdn.chunk_fwd(q, k, v, g, beta, None, m["cu_seqlens"], chunk=64, y_dtype=torch.float32)
+    y, S_T = gdn.chunk_fwd(q, k, v, g, beta, None, m["cu_seqlens"], chunk=64, y_dtype=y_dt)
     out = gdn.out_gate(y, m["z"], m["norm_w"], m["eps"])
     out_f, S_f = gdn.chunk_fwd_gated(q, k, v, g, beta, m["z"], m["norm_w"], m["eps"], None, m["cu_seqlens"])
     d = m["d"]
