@@ -4,20 +4,15 @@
 // HBM-bound elementwise work.  The storage types are template parameters, so every load is a
 // straight-line 16-byte vector access: a lane owns PER adjacent channels (4 when y, z and out
 // are all fp32, else 8), DV / PER lanes share a row, and a warp covers 32 / (DV / PER) rows per
-// pass and kGateRows passes; every row's y and z are loaded before the reductions, which
-// interleave.
+// pass and kGateRows passes (half as many with 8 channels); every row's y and z are loaded
+// before the reductions, which interleave.
 #pragma once
 #include "common.cuh"
 
 namespace gdn {
 
 constexpr int kGateWarps = 8;
-constexpr int kGateRows = 4;  // passes per warp
-
-template <int DT>
-__device__ __forceinline__ constexpr int dt_bytes() {
-    return DT == kF32 ? 4 : 2;
-}
+constexpr int kGateRows = 4;  // passes per warp with 4 channels per lane (2 with 8)
 
 // PER consecutive elements of storage type DT starting at element i (16-byte aligned).
 template <int DT, int PER>
@@ -72,7 +67,8 @@ struct GateShape {
     static constexpr int PER = PER0 < DV ? PER0 : DV;  // channels per lane
     static constexpr int LPR = DV / PER;                // lanes per row
     static constexpr int RPP = 32 / LPR;                // rows per warp pass
-    static constexpr int ROWS_PER_WARP = RPP * kGateRows;
+    static constexpr int PASSES = PER == 8 ? kGateRows / 2 : kGateRows;
+    static constexpr int ROWS_PER_WARP = RPP * PASSES;
 };
 
 template <int DV, int YT, int ZT>
@@ -80,7 +76,7 @@ __global__ void __launch_bounds__(32 * kGateWarps)
 out_gate_kernel(const void* __restrict__ y, const void* __restrict__ z, const float* __restrict__ w, float eps,
                 long long rows, void* __restrict__ out) {
     using S = GateShape<DV, YT, ZT>;
-    constexpr int PER = S::PER, LPR = S::LPR, R = kGateRows;
+    constexpr int PER = S::PER, LPR = S::LPR, R = S::PASSES;
     const int lane = threadIdx.x & 31;
     const int sub = lane / LPR, c0 = (lane % LPR) * PER;
     const long long r0 = ((long long)blockIdx.x * kGateWarps + (threadIdx.x >> 5)) * S::ROWS_PER_WARP + sub;
