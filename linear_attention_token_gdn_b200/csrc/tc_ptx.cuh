@@ -279,12 +279,6 @@ namespace tc {
 
 // ---------------------------------------------------------------- thread-block clusters
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
 // Address in CTA `rank`'s shared memory of the variable at local shared address `saddr`.
 __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     uint32_t r;
