@@ -141,7 +141,9 @@ gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const f
  *              into dense products; between chunks the state is carried in fp32.
  * workspace: device scratch of at least gdn_chunk_fwd_workspace_size(...) bytes
  * (may be NULL when that size is 0).  Tokens at index >= cu_seqlens[num_seqs] are
- * neither read nor written.
+ * neither read nor written.  N = 0 (every sequence empty): nothing is done without S_T;
+ * with S_T, it receives S0 (zeros when S0 is NULL), and q, k, v, g, beta, y and the
+ * workspace may be NULL.
  */
 size_t gdn_chunk_fwd_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk);
 

@@ -273,17 +273,21 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
     REQUIRE((long long)N * H * (dk > dv ? dk : dv) < (1LL << 40), "problem too large");
     if (N == 0 && S_T == nullptr) return GDN_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (chunk != 0 && chunk != 64)
+        return fail(GDN_ERR_UNSUPPORTED, "chunk=%d: the tensor-core path is built for chunk 64 (chunk 0 for the recurrence)", chunk);
+    if (chunk == 64 && (dk != 128 || dv != 128 || in_dtype == GDN_F32))
+        return fail(GDN_ERR_UNSUPPORTED, "chunked path needs dk=dv=128 and bf16/f16 inputs (use chunk=0)");
+    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens");
+    if (N == 0)  // every sequence is empty: S_T = S0 (or zero), by the recurrence, which reads no token
+        return dispatch_dims<RecurrentLaunch>(dk, dv, q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, scale,
+                                              (int)in_dtype, (int)y_dtype, y, S_T, st);
     REQUIRE_PTR(g, "g"); REQUIRE_PTR(beta, "beta"); REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k");
     REQUIRE_PTR(v, "v"); REQUIRE_PTR(y, "y");
-    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens"); OPT_PTR(workspace, "workspace");
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    OPT_PTR(workspace, "workspace");
     if (chunk == 0)
         return dispatch_dims<RecurrentLaunch>(dk, dv, q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, scale,
                                               (int)in_dtype, (int)y_dtype, y, S_T, st);
-    if (chunk != 64)
-        return fail(GDN_ERR_UNSUPPORTED, "chunk=%d: the tensor-core path is built for chunk 64 (chunk 0 for the recurrence)", chunk);
-    if (dk != 128 || dv != 128 || in_dtype == GDN_F32)
-        return fail(GDN_ERR_UNSUPPORTED, "chunked path needs dk=dv=128 and bf16/f16 inputs (use chunk=0)");
     const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
     REQUIRE(workspace_bytes >= need && (need == 0 || workspace != nullptr), "workspace of %zu bytes < %zu",
             workspace_bytes, need);
@@ -310,9 +314,14 @@ gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, co
         return fail(GDN_ERR_UNSUPPORTED, "the gated variant runs the tensor-core path only (chunk 64, dk=dv=128, "
                                          "bf16/f16 inputs, bf16/f16 z and out)");
     if (N == 0 && S_T == nullptr) return GDN_OK;
+    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens");
+    if (N == 0)  // every sequence is empty: S_T = S0 (or zero), by the recurrence, which reads no token
+        return dispatch_dims<RecurrentLaunch>(dk, dv, q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, scale,
+                                              (int)in_dtype, (int)io_dtype, nullptr, S_T,
+                                              reinterpret_cast<cudaStream_t>(stream));
     REQUIRE_PTR(g, "g"); REQUIRE_PTR(beta, "beta"); REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k");
     REQUIRE_PTR(v, "v"); REQUIRE_PTR(z, "z"); REQUIRE_PTR(norm_w, "norm_w"); REQUIRE_PTR(out, "out");
-    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens"); OPT_PTR(workspace, "workspace");
+    OPT_PTR(workspace, "workspace");
     const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
     REQUIRE(workspace_bytes >= need && (need == 0 || workspace != nullptr), "workspace of %zu bytes < %zu",
             workspace_bytes, need);

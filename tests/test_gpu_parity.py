@@ -180,6 +180,23 @@ def test_chunk_tc_small_ragged(dt, y_dt):
     gdn.check_device_error()
 
 
+@pytest.mark.parametrize("chunk", [64, 0, "gated"])
+def test_chunk_fwd_all_sequences_empty_carries_the_state(chunk):
+    """N = 0 with S_T requested: every sequence is empty, so S_T = S0 (zeros without S0)."""
+    x = inputs.make_prefill(2, "cuda", seed=27, lengths=[0, 0, 0], H=2, S0_std=0.2)
+    assert x["q"].shape[0] == 0
+    for S0 in (x["S0"], None):
+        if chunk == "gated":
+            z = torch.empty(0, 2, 128, device="cuda", dtype=x["q"].dtype)
+            w = torch.zeros(128, device="cuda")
+            _, S_T = gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], z, w, 1e-6, S0, x["cu_seqlens"])
+        else:
+            _, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], S0, x["cu_seqlens"], chunk=chunk)
+        want = torch.zeros_like(S_T) if S0 is None else S0
+        assert torch.equal(S_T, want)
+    gdn.check_device_error()
+
+
 def test_chunk_tc_matches_recurrent_path_no_initial_state():
     x = inputs.make_prefill(1, "cuda", seed=22, T=256, H=4)
     y1, S1 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
