@@ -197,6 +197,33 @@ def test_chunk_fwd_all_sequences_empty_carries_the_state(chunk):
     gdn.check_device_error()
 
 
+@pytest.mark.parametrize("case", ["beta0", "alpha1_beta1", "reset", "mixed"])
+def test_chunk_tc_degenerate_gates(case):
+    """The chunked tensor-core path at the method's degenerate points, against the oracle:
+    beta = 0 (pure decay of S0), alpha = beta = 1 (no decay, full overwrite), g = -60 on every
+    token (the state resets each token: decay factors underflow to zero inside the chunk
+    masks), and a mix of all three across heads.  Two sequences, ragged tail, S0 != 0."""
+    x = inputs.make_prefill(2, "cuda", seed=28, lengths=[150, 77], H=4, S0_std=0.2)
+    g, beta = x["g"].clone(), x["beta"].clone()
+    if case == "beta0":
+        beta.zero_()
+    elif case == "alpha1_beta1":
+        g.zero_()
+        beta.fill_(1.0)
+    elif case == "reset":
+        g.fill_(-60.0)
+    else:
+        beta[:, 0] = 0.0
+        g[:, 1] = 0.0
+        beta[:, 1] = 1.0
+        g[:, 2] = -60.0
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], g, beta, x["S0"], x["cu_seqlens"], chunk=64, y_dtype=torch.float32)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], g, beta, x["S0"], x["cu_seqlens"])
+    ey, es = err(y, y_ref), err(S_T, S_ref)
+    assert ey < TOL_16 and es < TOL_16, (case, ey, es)
+    gdn.check_device_error()
+
+
 def test_chunk_tc_matches_recurrent_path_no_initial_state():
     x = inputs.make_prefill(1, "cuda", seed=22, T=256, H=4)
     y1, S1 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
