@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // heads vary fastest across the grid, so CTAs resident together read whole token rows
     const int H = a.H, v = (int)(blockIdx.x / (unsigned)H), h = (int)(blockIdx.x % (unsigned)H);
+    tc::launch_dependents();  // the chain kernel may start its prologue once every CTA is resident
     if (warp == 0) {
         int n = 0, j = 0;
         const bool found = locate_chunk(a.cu, a.num_seqs, a.N, v, n, j);
@@ -895,6 +896,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         // =============================== producer group ================================
         constexpr int BID = 2;
         const int it = tid - 128;
+        tc::wait_prerequisites();  // the records of chunk_ut_kernel are complete and visible
         uint32_t ph_w = 0, ph_u = 0;
         bool ok = true;
         constexpr uint32_t id_v = idesc16<false>(128, NS, false, true);  // T_u V in fp16
@@ -1136,24 +1138,28 @@ inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, 
         if (e != cudaSuccess) return e;
     }
     const unsigned grid = (unsigned)(a.num_seqs * a.H * (128 / NS));
-    if (a.out == nullptr) {
-        LaunchScope timed(st, "chunk_chain_kernel");
-        chunk_chain_kernel<NS, BF, false><<<grid, 256, Ch::BYTES, st>>>(a, maps);
-        return cudaGetLastError();
-    }
-    // gated: the 128 / NS slab CTAs of a (sequence, head) form one cluster
+    // Programmatic dependent launch: the chain's prologue overlaps the tail of chunk_ut_kernel;
+    // its producer waits for that grid before reading a record.  Gated: the 128 / NS slab CTAs
+    // of a (sequence, head) form one cluster.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = Ch::BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 128 / NS;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 128 / NS;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    if (a.out == nullptr) {
+        cfg.numAttrs = 1;
+        LaunchScope timed(st, "chunk_chain_kernel");
+        return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<NS, BF, false>, a, maps);
+    }
+    cfg.numAttrs = 2;
     LaunchScope timed(st, "chunk_chain_gated_kernel");
     return cudaLaunchKernelEx(&cfg, chunk_chain_kernel<NS, BF, true>, a, maps);
 }

@@ -295,6 +295,16 @@ __device__ __forceinline__ void st_async_f32(uint32_t caddr, float v, uint32_t c
                  : "memory");
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Lets the grid launched after this one on the stream (with programmatic stream
+// serialization) start once every CTA of this grid has executed this or exited.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Waits until the grids this one depends on have completed and their memory is visible
+// (returns at once when the launch had no programmatic dependency).
+__device__ __forceinline__ void wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Barrier over every thread of the cluster (all threads of the CTA must call it).
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
