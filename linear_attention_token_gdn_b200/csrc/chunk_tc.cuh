@@ -29,10 +29,14 @@
 //                           [0; U~] + [Q; -W] S -> Q S and U = U~ - W S in one accumulator
 //                           K^T U'              -> S' = Gamma_C S + K^T U'
 //                       with U' = diag(Gamma_C / Gamma) U, while M U, for
-//                       Y = Gamma (Q S) + M U, is issued with the next chunk's first MMAs.
+//                       Y = Gamma (Q S) + M U, is issued once the next chunk's [Q; -W] S
+//                       has completed, when the MMA front end is otherwise idle.
 //                       Q/W/M slots are double-buffered, K/V stages triple-buffered, all
 //                       handed over with mbarriers; full chunks of y leave through swizzled
-//                       TMA stores.
+//                       TMA stores.  It is launched as a programmatic dependent of
+//                       chunk_ut_kernel.  The gated variant applies eq. (11)'s output gate
+//                       in the y epilogue, the four slab CTAs of a (sequence, head) forming
+//                       one cluster that exchanges row sums of squares.
 // Operands are 16-bit with fp32 accumulation in TMEM.  Each tcgen05.mma instruction costs
 // the SM's MMA front end about as much below N = 128 as at N = 128, so products are shaped
 // to use few instructions.  q and k enter exactly as stored (bf16 or fp16), so their partners
