@@ -28,8 +28,10 @@
  * Decay.    alpha is passed as g = log(alpha) (fp32): the chunked algorithm works
  *           with cumulative log-decays, and alpha itself can underflow in fp32.
  * Memory.   Every pointer is a DEVICE pointer owned by the caller, 16-byte
- *           aligned.  The library allocates nothing and keeps no per-call state;
- *           calls are re-entrant from several host threads.
+ *           aligned.  The compute calls allocate nothing and keep no per-call state
+ *           (gdn_chunk_fwd_noalloc's scratch is part of the library's device image;
+ *           only the timing calls create CUDA events); calls are re-entrant from
+ *           several host threads.
  * Streams.  `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *           only enqueues work on it and returns; nothing synchronises.
  * Errors.   Argument errors are detected on the host before anything is enqueued
