@@ -55,8 +55,10 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv") if os.path.isdir(
-            os.path.join(ROOT, "gpurun_out")) else f"/tmp/gdn_clocks_{os.getpid()}.csv"
+        # raw samples: $GDN_CLOCKS_DIR/clocks_rank<i>.csv when that directory is set, else /tmp
+        out_dir = os.environ.get("GDN_CLOCKS_DIR")
+        self.path = (os.path.join(out_dir, f"clocks_rank{gpu_index}.csv") if out_dir and os.path.isdir(out_dir)
+                     else f"/tmp/gdn_clocks_{os.getpid()}_{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -172,7 +174,7 @@ def cpu_model():
     return "unknown"
 
 
-def cpu_baseline(cfg_idx=1, target_s=12.0):
+def cpu_baseline(workload=None, target_s=12.0):
     """The fp64 oracle (unmodified) on the host cores, on a bounded sample of the prefill
     workload: the first `nh` heads of every sequence (all of them, repeated, when the whole
     workload takes less than target_s), sized to ~target_s of wall time.  Also reports the
@@ -180,8 +182,9 @@ def cpu_baseline(cfg_idx=1, target_s=12.0):
     import oracle
     from linear_attention_token_gdn_b200 import inputs
 
-    c = inputs.CONFIGS[cfg_idx]
-    x = inputs.make_prefill(cfg_idx, "cpu")
+    workload = inputs.PREFILL if workload is None else workload
+    c = inputs.WORKLOAD_SPECS[workload]
+    x = inputs.make_prefill(workload, "cpu")
     ncores = os.cpu_count() or 1
     # calibrate: one (sequence, head) unit single-threaded on a 512-token slice
     T = c["T"]
@@ -215,7 +218,7 @@ def run_reference(args):
     times = []
     work = 0
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(1, target_s=args.ref_step_s)
+        r = cpu_baseline(target_s=args.ref_step_s)
         if i >= args.warmup:
             times.append(1.0 / r["value"])
             cb = r
@@ -263,8 +266,8 @@ def run_ours(args):
         return 0
 
     # ---- headline: prefill workload, three rotating input sets --------------------------
-    c = inputs.CONFIGS[1]
-    sets = [inputs.make_prefill(1, "cuda", seed=rank_seed(inputs.SEED_BASE + 1, rank) + s) for s in range(3)]
+    c = inputs.WORKLOAD_SPECS[inputs.PREFILL]
+    sets = [inputs.make_prefill(inputs.PREFILL, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.PREFILL, rank) + s) for s in range(3)]
     N, H = sets[0]["N"], sets[0]["H"]
     nseq = sets[0]["num_seqs"]
     outs = [(torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16),
@@ -337,7 +340,7 @@ def run_ours(args):
         line["other_workloads"] = extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak)
     if rank == 0:
         if args.impl_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(1, target_s=args.cpu_s)
+            line["cpu_baseline"] = cpu_baseline(target_s=args.cpu_s)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -347,9 +350,9 @@ def run_ours(args):
 
 def wl_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     """decode: 256 x 32 heads, 100 in-place steps per "step"."""
-    c = inputs.CONFIGS[3]
-    state = inputs.make_decode_state(3, "cuda", seed=rank_seed(inputs.SEED_BASE + 3, rank))
-    steps_in = [inputs.make_decode_step(3, "cuda", step=s, seed=rank_seed(inputs.SEED_BASE + 3, rank))
+    c = inputs.WORKLOAD_SPECS[inputs.DECODE]
+    state = inputs.make_decode_state(inputs.DECODE, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.DECODE, rank))
+    steps_in = [inputs.make_decode_step(inputs.DECODE, "cuda", step=s, seed=rank_seed(inputs.SEED_BASE + inputs.DECODE, rank))
                 for s in range(c["steps"])]
     y = torch.empty(c["B"], c["H"], 128, device="cuda", dtype=torch.bfloat16)
 
@@ -389,7 +392,7 @@ def wl_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
 def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     """long prefill: B=1, H=32, T=32768, S0 != 0."""
-    x = inputs.make_prefill(2, "cuda", seed=rank_seed(inputs.SEED_BASE + 2, rank))
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.LONG_PREFILL, rank))
     N, H, nseq = x["N"], x["H"], x["num_seqs"]
     yb = torch.empty(N, H, 128, device="cuda", dtype=torch.bfloat16)
     ST = torch.empty(nseq, H, 128, 128, device="cuda")
@@ -406,7 +409,7 @@ def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     kl = kernel_table(gdn.timing_stop(), n_lp)
     op_s = sum(k["avg_us"] for k in kl) / 1e6
     bl = prefill_bytes(N, H, nseq, S0=True)
-    return {"workload": inputs.CONFIGS[2]["name"], "value": N * H * world / dt, "unit": UNIT,
+    return {"workload": inputs.WORKLOAD_SPECS[inputs.LONG_PREFILL]["name"], "value": N * H * world / dt, "unit": UNIT,
                 "ms_per_step": dt * 1e3,
                 "roofline": {"bound": "hbm", "achieved": bl / op_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                              "frac": bl / op_s / 1e9 / hbm_peak,
@@ -418,7 +421,7 @@ def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     """full mixer on 4 packed sequences: prep -> chunk -> out gate (the variant with the gate
     fused into the chunked pass is timed beside it)."""
-    m = inputs.make_mixer(4, "cuda", seed=rank_seed(inputs.SEED_BASE + 4, rank))
+    m = inputs.make_mixer(inputs.MIXER, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.MIXER, rank))
     N, H = m["N"], m["H"]
     bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
     gbuf = torch.empty(N, H, device="cuda")
@@ -448,7 +451,7 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
                         world) / n_m
     km = kernel_table(gdn.timing_stop(), n_m)
     fused_min = N * (H * 3 * 128 * 2 + H * 2 * 2 + H * 128 * 2 + H * 128 * 2)
-    return {"workload": inputs.CONFIGS[4]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
+    return {"workload": inputs.WORKLOAD_SPECS[inputs.MIXER]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
                 "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
                 "ms_per_step_gate_fused_into_chunk": dt_fused * 1e3,
                 "roofline": {"bound": "hbm", "achieved": fused_min / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",

@@ -31,16 +31,19 @@ import torch
 
 SEED_BASE = 20261202
 
-CONFIGS = {
-    0: dict(name="tiny_fp32_B1_H2_T64_d16", kind="prefill", B=1, H=2, T=64, d=16, dtype=torch.float32,
+# workload keys (each workload's seed is SEED_BASE + its key)
+TINY, PREFILL, LONG_PREFILL, DECODE, MIXER = 0, 1, 2, 3, 4
+
+WORKLOAD_SPECS = {
+    TINY: dict(name="tiny_fp32_B1_H2_T64_d16", kind="prefill", B=1, H=2, T=64, d=16, dtype=torch.float32,
             expA=(1.0, 16.0), S0_std=0.0, chunk=0),
-    1: dict(name="prefill_B2_H16_T4096_d128", kind="prefill", B=2, H=16, T=4096, d=128,
+    PREFILL: dict(name="prefill_B2_H16_T4096_d128", kind="prefill", B=2, H=16, T=4096, d=128,
             dtype=torch.bfloat16, expA=(1.0, 16.0), S0_std=0.0, chunk=64),
-    2: dict(name="prefill_B1_H32_T32768_d128", kind="prefill", B=1, H=32, T=32768, d=128,
+    LONG_PREFILL: dict(name="prefill_B1_H32_T32768_d128", kind="prefill", B=1, H=32, T=32768, d=128,
             dtype=torch.bfloat16, expA=(1.0, 64.0), S0_std=0.02, chunk=64),
-    3: dict(name="decode_B256_H32_d128_x100", kind="decode", B=256, H=32, d=128, dtype=torch.bfloat16,
+    DECODE: dict(name="decode_B256_H32_d128_x100", kind="decode", B=256, H=32, d=128, dtype=torch.bfloat16,
             expA=(1.0, 16.0), state_std=0.05, steps=100),
-    4: dict(name="mixer_4seq_H16_d128_N<=32768", kind="mixer", nseq=4, H=16, d=128, L=(1024, 8192),
+    MIXER: dict(name="mixer_4seq_H16_d128_N<=32768", kind="mixer", nseq=4, H=16, d=128, L=(1024, 8192),
             dtype=torch.bfloat16, W=4, conv_std=0.5, norm_std=0.02, expA=(1.0, 16.0), ba_std=0.5,
             eps=1e-6),
 }
@@ -70,10 +73,10 @@ def decay_and_write_gates(n, H, expA_range, gen, device):
     return g.to(torch.float32), beta.to(torch.float32)
 
 
-def make_prefill(cfg=1, device="cpu", seed=None, **over):
+def make_prefill(cfg=PREFILL, device="cpu", seed=None, **over):
     """Inputs of a prefill workload.  Keyword overrides: B, T, H, d (or dk/dv), dtype,
     S0_std, expA, lengths (packed variable lengths; overrides B and T)."""
-    c = dict(CONFIGS[cfg])
+    c = dict(WORKLOAD_SPECS[cfg])
     c.update(over)
     dk = c.get("dk", c["d"])
     dv = c.get("dv", c["d"])
@@ -99,8 +102,8 @@ def make_prefill(cfg=1, device="cpu", seed=None, **over):
                 chunk=c.get("chunk", 64))
 
 
-def make_decode_state(cfg=3, device="cpu", seed=None, **over):
-    c = dict(CONFIGS[cfg])
+def make_decode_state(cfg=DECODE, device="cpu", seed=None, **over):
+    c = dict(WORKLOAD_SPECS[cfg])
     c.update(over)
     dk = c.get("dk", c["d"])
     dv = c.get("dv", c["d"])
@@ -109,9 +112,9 @@ def make_decode_state(cfg=3, device="cpu", seed=None, **over):
     return torch.randn(slots, c["H"], dk, dv, generator=gen, device=device, dtype=torch.float32) * c["state_std"]
 
 
-def make_decode_step(cfg=3, device="cpu", step=0, seed=None, **over):
+def make_decode_step(cfg=DECODE, device="cpu", step=0, seed=None, **over):
     """Fresh one-token inputs for decode step ``step``."""
-    c = dict(CONFIGS[cfg])
+    c = dict(WORKLOAD_SPECS[cfg])
     c.update(over)
     dk = c.get("dk", c["d"])
     dv = c.get("dv", c["d"])
@@ -124,16 +127,16 @@ def make_decode_step(cfg=3, device="cpu", step=0, seed=None, **over):
     return dict(q=q, k=k, v=v, g=g, beta=beta)
 
 
-def mixer_lengths(cfg=4, seed=None, nseq=None, L=None):
-    c = CONFIGS[cfg]
+def mixer_lengths(cfg=MIXER, seed=None, nseq=None, L=None):
+    c = WORKLOAD_SPECS[cfg]
     rng = np.random.Generator(np.random.PCG64(SEED_BASE + cfg if seed is None else seed))
     lo, hi = c["L"] if L is None else L
     return [int(x) for x in rng.integers(lo, hi + 1, size=c["nseq"] if nseq is None else nseq)]
 
 
-def make_mixer(cfg=4, device="cpu", seed=None, lengths=None, **over):
+def make_mixer(cfg=MIXER, device="cpu", seed=None, lengths=None, **over):
     """Raw (post-projection) inputs of the full mixer workload."""
-    c = dict(CONFIGS[cfg])
+    c = dict(WORKLOAD_SPECS[cfg])
     c.update(over)
     H, d, W = c["H"], c["d"], c["W"]
     if lengths is None:

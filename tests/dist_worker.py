@@ -19,7 +19,7 @@ def run(rank, world, port, queue):
         t = gd.max_over_ranks(local_time, w, device="cpu")
         gd.barrier(w, cuda=False)
         seed = gd.rank_seed(inputs.SEED_BASE, r)
-        x = inputs.make_prefill(0, "cpu", seed=seed)      # this rank's own replica of the workload
+        x = inputs.make_prefill(inputs.TINY, "cpu", seed=seed)      # this rank's own replica of the workload
         y, _ = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
         queue.put({"rank": r, "world": w, "local": local, "t": t, "seed": seed, "y_sum": float(abs(y).sum()),
                    "value": gd.aggregate(64, w, t)})

@@ -39,7 +39,7 @@ def test_two_gloo_ranks():
     assert all(d["value"] == 64 * 2 / 1.0 for d in out)
     assert out[0]["seed"] != out[1]["seed"]
     for d in out:                                      # replica r == one process on rank r's seed
-        x = inputs.make_prefill(0, "cpu", seed=d["seed"])
+        x = inputs.make_prefill(inputs.TINY, "cpu", seed=d["seed"])
         y, _ = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
         assert np.isclose(float(np.abs(y).sum()), d["y_sum"], rtol=0, atol=0)
     assert out[0]["y_sum"] != out[1]["y_sum"]

@@ -47,7 +47,7 @@ def err(gpu, ref):
 
 def test_recurrent_tiny_fp32_workload():
     """The tiny workload: B=1, H=2, T=64, dk=dv=16, fp32, S0 = 0."""
-    x = inputs.make_prefill(0, "cuda")
+    x = inputs.make_prefill(inputs.TINY, "cuda")
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=0)
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
     assert err(y, y_ref) < TOL_F32
@@ -59,7 +59,7 @@ def test_recurrent_tiny_fp32_workload():
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16, torch.float16])
 def test_recurrent_varlen_shapes_dtypes(dk, dv, dt):
     lengths = [37, 1, 0, 70]
-    x = inputs.make_prefill(1, "cuda", seed=11 + dk + dv, lengths=lengths, H=3, dk=dk, dv=dv, dtype=dt,
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=11 + dk + dv, lengths=lengths, H=3, dk=dk, dv=dv, dtype=dt,
                             S0_std=0.3)
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=0,
                            y_dtype=torch.float32)
@@ -75,11 +75,11 @@ def test_recurrent_varlen_shapes_dtypes(dk, dv, dt):
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
 def test_decode_steps_with_slots(dk, dv, dt):
     B, H, slots = 5, 3, 9
-    state = inputs.make_decode_state(3, "cuda", seed=5, B=slots, H=H, dk=dk, dv=dv)
+    state = inputs.make_decode_state(inputs.DECODE, "cuda", seed=5, B=slots, H=H, dk=dk, dv=dv)
     slot = torch.tensor([7, 0, 3, 8, 1], dtype=torch.int32, device="cuda")
     ref_state = state.double().cpu().numpy()
     for step in range(3):
-        x = inputs.make_decode_step(3, "cuda", step=step, seed=5, B=B, H=H, dk=dk, dv=dv, dtype=dt)
+        x = inputs.make_decode_step(inputs.DECODE, "cuda", step=step, seed=5, B=B, H=H, dk=dk, dv=dv, dtype=dt)
         y = gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, slot, y_dtype=torch.float32)
         y_ref, ref_state = oracle.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], ref_state, slot)
         assert err(y, y_ref) < TOL_F32
@@ -90,12 +90,12 @@ def test_decode_steps_with_slots(dk, dv, dt):
 def test_decode_full_workload_sampled_heads():
     """256 x 32 heads, dk = dv = 128, 100 in-place steps (bf16 q/k/v, bf16 y): check sampled
     (row, head) pairs against the oracle run on those heads alone, every step."""
-    c = inputs.CONFIGS[3]
-    state = inputs.make_decode_state(3, "cuda")
+    c = inputs.WORKLOAD_SPECS[inputs.DECODE]
+    state = inputs.make_decode_state(inputs.DECODE, "cuda")
     picks = [(0, 0), (17, 5), (255, 31), (128, 16)]
     ref = {p: state[p[0], p[1]].double().cpu().numpy()[None, None] for p in picks}
     for step in range(c["steps"]):
-        x = inputs.make_decode_step(3, "cuda", step=step)
+        x = inputs.make_decode_step(inputs.DECODE, "cuda", step=step)
         y = gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state)
         if step % 11 == 0 or step == c["steps"] - 1:
             for (b, h) in picks:
@@ -115,7 +115,7 @@ def test_decode_full_workload_sampled_heads():
 
 def test_decode_rejects_out_of_range_slot_on_device():
     state = torch.zeros(2, 1, 16, 16, device="cuda")
-    x = inputs.make_decode_step(3, "cuda", B=1, H=1, dk=16, dv=16, dtype=torch.float32)
+    x = inputs.make_decode_step(inputs.DECODE, "cuda", B=1, H=1, dk=16, dv=16, dtype=torch.float32)
     gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state,
                     torch.tensor([5], dtype=torch.int32, device="cuda"))
     with pytest.raises(gdn.GDNError) as e:
@@ -133,9 +133,9 @@ def test_prep_matches_oracle(d, out_dt, case):
     """Sequences that start inside a 64-token run and runs that start inside a sequence; the
     edge case adds an empty and a one-token sequence, conv width 3 and a ragged last run."""
     if case == "three_seqs":
-        m = inputs.make_mixer(4, "cuda", lengths=[33, 5, 64], d=d, H=3)
+        m = inputs.make_mixer(inputs.MIXER, "cuda", lengths=[33, 5, 64], d=d, H=3)
     else:
-        m = inputs.make_mixer(4, "cuda", lengths=[70, 0, 1, 129], d=d, H=2, W=3, seed=77)
+        m = inputs.make_mixer(inputs.MIXER, "cuda", lengths=[70, 0, 1, 129], d=d, H=2, W=3, seed=77)
     q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
                                 m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
                                 out_dtype=out_dt)
@@ -171,7 +171,7 @@ def test_out_gate_matches_oracle(dv, y_dt, io):
 def test_chunk_tc_small_ragged(dt, y_dt):
     """Several chunks per sequence, ragged tails, an empty and a one-token sequence, S0 != 0."""
     lengths = [3 * 64 + 17, 64, 1, 0, 130]
-    x = inputs.make_prefill(2, "cuda", seed=21, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=21, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64,
                            y_dtype=y_dt)
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
@@ -183,7 +183,7 @@ def test_chunk_tc_small_ragged(dt, y_dt):
 @pytest.mark.parametrize("chunk", [64, 0, "gated"])
 def test_chunk_fwd_all_sequences_empty_carries_the_state(chunk):
     """N = 0 with S_T requested: every sequence is empty, so S_T = S0 (zeros without S0)."""
-    x = inputs.make_prefill(2, "cuda", seed=27, lengths=[0, 0, 0], H=2, S0_std=0.2)
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=27, lengths=[0, 0, 0], H=2, S0_std=0.2)
     assert x["q"].shape[0] == 0
     for S0 in (x["S0"], None):
         if chunk == "gated":
@@ -203,7 +203,7 @@ def test_chunk_tc_degenerate_gates(case):
     beta = 0 (pure decay of S0), alpha = beta = 1 (no decay, full overwrite), g = -60 on every
     token (the state resets each token: decay factors underflow to zero inside the chunk
     masks), and a mix of all three across heads.  Two sequences, ragged tail, S0 != 0."""
-    x = inputs.make_prefill(2, "cuda", seed=28, lengths=[150, 77], H=4, S0_std=0.2)
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=28, lengths=[150, 77], H=4, S0_std=0.2)
     g, beta = x["g"].clone(), x["beta"].clone()
     if case == "beta0":
         beta.zero_()
@@ -225,7 +225,7 @@ def test_chunk_tc_degenerate_gates(case):
 
 
 def test_chunk_tc_matches_recurrent_path_no_initial_state():
-    x = inputs.make_prefill(1, "cuda", seed=22, T=256, H=4)
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=22, T=256, H=4)
     y1, S1 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
                            y_dtype=torch.float32)
     y0, S0 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=0,
@@ -237,7 +237,7 @@ def test_chunk_tc_matches_recurrent_path_no_initial_state():
 
 def test_chunk_tc_prefill_workload_full():
     """B=2, H=16, T=4096, dk=dv=128, bf16, S0 = 0, chunk 64: every output checked."""
-    x = inputs.make_prefill(1, "cuda")
+    x = inputs.make_prefill(inputs.PREFILL, "cuda")
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
     ey, es = err(y, y_ref), err(S_T, S_ref)
@@ -249,7 +249,7 @@ def test_chunk_tc_prefill_workload_full():
 def test_chunk_tc_long_prefill_sampled_heads():
     """B=1, H=32, T=32768, S0 ~ N(0, 0.02), exp(A) up to 64: heads checked one by one
     (slowest- and fastest-decaying heads included)."""
-    x = inputs.make_prefill(2, "cuda")
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda")
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64)
     mean_g = x["g"].mean(0)
     heads = sorted({0, int(mean_g.argmin()), int(mean_g.argmax()), 19})
@@ -283,7 +283,7 @@ def test_full_mixer_workload_sampled_heads(y_dt):
     q, k, v are stored in bf16 between prep and the recurrence, and the oracle rounds them the
     same way.  y meets the chunked path's bound; out meets that bound propagated through the
     RMS normalisation of eq. (11), plus its own bf16 rounding."""
-    m = inputs.make_mixer(4, "cuda")
+    m = inputs.make_mixer(inputs.MIXER, "cuda")
     q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
                                 m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
                                 out_dtype=torch.bfloat16)
@@ -315,7 +315,7 @@ def test_chunk_fwd_gated_small_ragged(dt):
     """The fused out gate: ragged tails, an empty and a one-token sequence, S0 != 0.  out meets
     the chunked path's bound propagated through eq. (11); S_T is the plain path's."""
     lengths = [3 * 64 + 17, 64, 1, 0, 130]
-    x = inputs.make_prefill(2, "cuda", seed=24, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=24, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
     gen = torch.Generator(device="cuda").manual_seed(25)
     N, H, dv = x["v"].shape
     z = torch.randn(N, H, dv, device="cuda", generator=gen).to(dt)
@@ -335,7 +335,7 @@ def test_chunk_fwd_gated_bounded_wait_reports_timeout():
     """The gated variant's cluster exchange waits are bounded too: with a one-cycle budget the
     call flags GDN_ERR_TIMEOUT and every CTA of every cluster still leaves; the next call is
     correct."""
-    x = inputs.make_prefill(1, "cuda", seed=26, T=256, H=2)
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=26, T=256, H=2)
     N, H, dv = x["v"].shape
     z = torch.ones(N, H, dv, device="cuda", dtype=x["q"].dtype)
     w = torch.zeros(dv, device="cuda")
@@ -359,7 +359,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     """Failure detection without a GPU fault: with a one-cycle wait budget every mbarrier
     wait of the chunked kernel gives up, the kernel flags GDN_ERR_TIMEOUT, drains its MMAs,
     frees TMEM and returns; the next call with the default budget is correct again."""
-    x = inputs.make_prefill(1, "cuda", seed=23, T=256, H=2)
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=23, T=256, H=2)
     try:
         gdn.set_wait_budget(1)
         gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
@@ -377,12 +377,12 @@ def test_bounded_wait_reports_timeout_and_context_survives():
 
 def test_launch_timing_reports_each_kernel():
     """gdn_timing_start/stop bracket every library launch with events on its stream."""
-    x = inputs.make_prefill(1, "cuda", seed=31, T=512, H=2)
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=31, T=512, H=2)
     gdn.timing_start(16)
     for _ in range(2):
         gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64)
-    gdn.decode_step(*(inputs.make_decode_step(3, "cuda", B=2, H=2)[k] for k in ("q", "k", "v", "g", "beta")),
-                    inputs.make_decode_state(3, "cuda", B=2, H=2))
+    gdn.decode_step(*(inputs.make_decode_step(inputs.DECODE, "cuda", B=2, H=2)[k] for k in ("q", "k", "v", "g", "beta")),
+                    inputs.make_decode_state(inputs.DECODE, "cuda", B=2, H=2))
     t = gdn.timing_stop()
     assert list(t) == ["chunk_ut_kernel", "chunk_chain_kernel", "decode_step_kernel"]
     assert [c for c, _ in t.values()] == [2, 2, 1]

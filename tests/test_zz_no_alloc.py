@@ -39,7 +39,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(cuda_device):
     # two calls in a row with different inputs: the second finds the first one's records
     # in the shared scratch and must not depend on them
     for seed, lengths in ((41, [700, 64, 1, 333]), (42, [129, 1000])):
-        x = inputs.make_prefill(2, "cuda", seed=seed, lengths=lengths, H=4, S0_std=0.1)
+        x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=seed, lengths=lengths, H=4, S0_std=0.1)
         y_ref, S_ref = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"],
                                      chunk=64, y_dtype=torch.float32)
         y = torch.full_like(y_ref, float("nan"))
