@@ -15,7 +15,8 @@ Every function follows "On the design of Qwen3.8-Next architecture"
 * :func:`prep`        -- eqs. (6)-(10) ("GDN parameterisation").
 * :func:`out_gate`    -- eq. (11) without the output projection W_o.
 * :func:`mixer`       -- prep -> recurrence -> out_gate in fp64 (optionally with q, k, v
-  rounded once to a 16-bit storage format between prep and the recurrence).
+  rounded once to a 16-bit storage format between prep and the recurrence,
+  :func:`round_to_format`).
 
 The pins that tie these functions to the page (closed form eq. (5), pure decay,
 exact retrieval, brute-force products, textbook special cases, a hand-worked
@@ -172,6 +173,22 @@ def prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bia
     return q, k, v, g, beta
 
 
+# significant bits and smallest exponent step of the 16-bit storage formats
+_FORMATS = {"bf16": (8, -133), "fp16": (11, -24)}
+
+
+def round_to_format(x, fmt):
+    """x (float64) rounded once to the nearest value of a 16-bit storage format, ties to the
+    even significand (IEEE 754 round-to-nearest-even), returned as float64.  fmt: "bf16"
+    (8 significant bits, fp32's exponent range) or "fp16" (11 significant bits, subnormal
+    step 2^-24).  Values are assumed inside the format's finite range."""
+    bits, min_step = _FORMATS[fmt]
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                                    # |x| = m 2^e, 1/2 <= m < 1
+    step = np.ldexp(1.0, np.maximum(e - bits, min_step))  # spacing of the format at |x|
+    return np.round(x / step) * step                      # np.round: ties to even
+
+
 def out_gate(y, z, w, eps=1e-6):
     """Eq. (11) without W_o: sigmoid(z) * zero-centred RMSNorm(y), per (token, head) over dv."""
     y, z, w = _f64(y), _f64(z), _f64(w)
@@ -186,17 +203,18 @@ def mixer(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bi
           cu_seqlens=None, num_seqs=1, S0=None, eps_l2=1e-6, eps_rms=1e-6, nthreads=0, inter_dtype=None):
     """The full post-projection mixer in fp64: eqs. (6)-(10), (1)-(4), (11) without W_o.
 
-    inter_dtype (None, torch.bfloat16 or torch.float16): the storage format of q, k, v between
-    the input side (6)-(8) and the recurrence.  The pages leave it open; a mixer that keeps
-    them in 16-bit memory rounds each value once to the nearest representable number, which
-    this models with torch's round-to-nearest-even conversion.  None keeps fp64.
+    inter_dtype (None, "bf16", "fp16", or torch.bfloat16 / torch.float16): the storage format
+    of q, k, v between the input side (6)-(8) and the recurrence.  The pages leave it open;
+    a mixer that keeps them in 16-bit memory rounds each value once to the nearest
+    representable number (round_to_format).  None keeps fp64.
 
     Returns (out [N, H, dv], y [N, H, dv], S_T).
     """
     q, k, v, g, beta = prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log,
                             alpha_bias, cu_seqlens, num_seqs, eps_l2, nthreads)
     if inter_dtype is not None:
-        import torch  # its dtype conversion is the rounding step; no other torch arithmetic here
-        q, k, v = (torch.from_numpy(np.ascontiguousarray(t)).to(inter_dtype).double().numpy() for t in (q, k, v))
+        fmt = inter_dtype if isinstance(inter_dtype, str) else {"torch.bfloat16": "bf16",
+                                                                 "torch.float16": "fp16"}[str(inter_dtype)]
+        q, k, v = (round_to_format(t, fmt) for t in (q, k, v))
     y, S_T = recurrence(q, k, v, g, beta, S0, cu_seqlens, num_seqs, 1.0, nthreads)
     return out_gate(y, z, norm_w, eps_rms), y, S_T

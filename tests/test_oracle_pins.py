@@ -341,6 +341,51 @@ def test_mixer_composes_the_three_stages():
     assert np.array_equal(out, oracle.out_gate(y2, z, nw))
 
 
+# IEEE 754 binary16: p = 11, emin = -14; bfloat16: p = 8, emin = -126.  The subnormal spacing
+# is 2^(emin - p + 1).
+@pytest.mark.parametrize("fmt,bits,emin", [("bf16", 8, -126), ("fp16", 11, -14)])
+def test_round_to_format_is_single_round_to_nearest_even(fmt, bits, emin):
+    """The 16-bit storage rounding of the mixer (one IEEE round-to-nearest-even from fp64):
+    every result has at most `bits` significant bits, lies within half a spacing of x, is the
+    nearer neighbour, and exact midpoints go to the even significand.  Checked by integer
+    arithmetic on the significand, not by a library conversion."""
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal(200000) * np.exp(rng.uniform(-6, 6, 200000))
+    r = oracle.round_to_format(x, fmt)
+    m, e = np.frexp(x)
+    step = np.ldexp(1.0, np.maximum(e - bits, emin - bits + 1))  # spacing at |x| (subnormals too)
+    k = r / step                                        # r in units of the spacing at |x|
+    assert np.all(k == np.round(k))                     # representable: an integer multiple
+    assert np.all(np.abs(r - x) <= step / 2)            # nearest (within half a spacing)
+    # midpoints: x = (2j + 1) step / 2 for integer j goes to the even multiple of step
+    j = np.floor(x / step)
+    mid = (j + 0.5) * step
+    rm = oracle.round_to_format(mid, fmt)
+    # (j + 0.5) step may sit at a binade edge where the spacing differs; keep the interior ones
+    inside = ((np.frexp(mid)[1] == e) & (np.frexp(j * step)[1] == e) & (np.frexp((j + 1) * step)[1] == e)
+              & (e - bits >= emin - bits + 1))
+    want = np.where(j % 2 == 0, j * step, (j + 1) * step)
+    assert np.all(rm[inside] == want[inside]) and inside.sum() > 100000
+    # just above / below a midpoint: away from / towards j
+    up = oracle.round_to_format(mid + step * 2.0 ** -20, fmt)
+    dn = oracle.round_to_format(mid - step * 2.0 ** -20, fmt)
+    assert np.all(up[inside] == ((j + 1) * step)[inside]) and np.all(dn[inside] == (j * step)[inside])
+
+
+def test_mixer_inter_dtype_rounds_q_k_v_before_the_recurrence():
+    rng = np.random.default_rng(34)
+    c = _prep_case(rng, [6, 4], H=2, dk=4, dv=4)
+    N = int(c["cu_seqlens"][-1])
+    z = rng.standard_normal((N, 2, 4))
+    nw = rng.standard_normal(4) * 0.02
+    out, y, S_T = oracle.mixer(z=z, norm_w=nw, inter_dtype="bf16", **c)
+    q, k, v, g, beta = oracle.prep(**c)
+    q, k, v = (oracle.round_to_format(t, "bf16") for t in (q, k, v))
+    y2, S2 = oracle.recurrence(q, k, v, g, beta, None, c["cu_seqlens"])
+    assert np.array_equal(y, y2) and np.array_equal(S_T, S2)
+    assert np.array_equal(out, oracle.out_gate(y2, z, nw))
+
+
 def test_thread_count_does_not_change_results():
     rng = np.random.default_rng(32)
     q, k, v, g, beta, S0 = rand_inputs(rng, 40, 5, 8, 8, nseq=2)
