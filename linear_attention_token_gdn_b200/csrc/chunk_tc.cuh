@@ -93,8 +93,9 @@ constexpr int kRecTu = 8192;       // T_u = T diag(beta), fp16 (meets V converte
 constexpr int kRecM = 16384;       // M, fp16 (meets U, another computed operand)
 constexpr int kRecBytes = 24576;
 
-// Upper bound of the number of 64-token chunks over all sequences.
-inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
+// Upper bound of the number of 64-token chunks over all sequences (the records the workspace
+// holds); it holds for every valid cu_seqlens.
+__host__ __device__ inline long long chunk_count_bound(int N, int num_seqs, bool varlen) {
     if (!varlen) {
         const long long L = N / num_seqs;
         return (long long)num_seqs * ((L + kChunk - 1) / kChunk);
@@ -529,7 +530,6 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     const int H = a.H;
     int t_begin, t_end;
     seq_bounds(a.cu, n, a.num_seqs, a.N, t_begin, t_end);
-    const int nchunks = (t_end - t_begin + kChunk - 1) / kChunk;
 
     if (warp == 0) {
         const int base = chunks_before(a.cu, a.num_seqs, a.N, n);
@@ -546,6 +546,14 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int rec_base = *s_base;
+    // malformed cu_seqlens (flagged by seq_bounds) can describe more chunks than the workspace
+    // holds: never index past its last record
+    const long long rec_end = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
+    int nchunks = (t_end - t_begin + kChunk - 1) / kChunk;
+    if (rec_base + (long long)nchunks > rec_end) {
+        if (tid == 0) raise_error(kErrSeqlens);
+        nchunks = (int)max(0LL, rec_end - rec_base);
+    }
     const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     auto vec = [&](int b) { return reinterpret_cast<float*>(smem + Cf::OFF_VEC + b * 1024); };
     auto QWoff = [&](int b) { return Cf::OFF_QW + b * 2 * Cf::QW_HALF; };

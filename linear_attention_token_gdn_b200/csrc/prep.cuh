@@ -262,6 +262,13 @@ prep_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ wq,
     SeqWalk sw;
     sw.init(cu, num_seqs, N, t0);
     const int t1 = min(t0 + kPrepRun, sw.stop);  // tokens past the last sequence stay untouched
+    if (warp == 6 && blockIdx.x == 0 && cu != nullptr) {
+        // the walk only meets the sequences this CTA covers: one warp checks them all
+        // (cu[0] >= 0, non-decreasing, cu[num_seqs] <= N) and flags a malformed array
+        bool bad = false;
+        for (int m = lane; m < num_seqs; m += 32) bad |= cu[m] < 0 || cu[m + 1] < cu[m] || cu[m + 1] > N;
+        if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(kErrSeqlens);
+    }
     if (t0 >= t1) return;  // uniform over the CTA
     const int esz = in_dt == kF32 ? 4 : 2;
     const int tqk = prep_tile_bytes(DK, TAPS, esz), tv = prep_tile_bytes(DV, TAPS, esz);

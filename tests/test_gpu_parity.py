@@ -224,6 +224,55 @@ def test_chunk_tc_degenerate_gates(case):
     gdn.check_device_error()
 
 
+@pytest.mark.parametrize("path", ["chunk64", "gated", "chunk0", "prep"])
+def test_malformed_cu_seqlens_is_reported(path):
+    """cu_seqlens = [0, 640, 0, 640] over N = 640 tokens: the middle sequence runs backwards
+    and the third overlaps the first, describing 20 chunks where the workspace holds 13
+    records.  Every path clamps the bounds (the chunked pass also its chunk count to the
+    workspace), flags GDN_ERR_INVALID_ARG in the device error word and leaves the context
+    usable."""
+    N, H, d = 640, 2, 128
+    gen = torch.Generator(device="cuda").manual_seed(29)
+    cu = torch.tensor([0, 640, 0, 640], dtype=torch.int32, device="cuda")
+    bf = lambda *shape: torch.randn(*shape, device="cuda", generator=gen).to(torch.bfloat16)
+    if path == "prep":
+        w = lambda: torch.randn(H * d, 4, device="cuda", generator=gen) * 0.5
+        gdn.prep(bf(N, H, d), bf(N, H, d), bf(N, H, d), w(), w(), w(), bf(N, H), bf(N, H),
+                 torch.zeros(H, device="cuda"), torch.zeros(H, device="cuda"), cu)
+    else:
+        x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=29, B=1, T=N, H=H)
+        if path == "gated":
+            gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], bf(N, H, d),
+                                torch.zeros(d, device="cuda"), 1e-6, None, cu)
+        else:
+            gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, cu, chunk=64 if path == "chunk64" else 0)
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.check_device_error()
+    assert e.value.status == gdn.GDN_ERR_INVALID_ARG
+    gdn.check_device_error()  # the word was cleared
+    # a well-formed call right after is correct
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=30, lengths=[100, 28], H=2)
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
+                           y_dtype=torch.float32)
+    gdn.check_device_error()
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
+    assert err(y, y_ref) < TOL_16 and err(S_T, S_ref) < TOL_16
+
+
+@pytest.mark.parametrize("d", [128, 32])
+def test_prep_wide_conv(d):
+    """Conv widths 5-8 take the wider (8-tap) kernel instantiation: width 6 against the oracle."""
+    m = inputs.make_mixer(inputs.MIXER, "cuda", lengths=[40, 3, 70], d=d, H=2, W=6, seed=78)
+    q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
+                                m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
+                                out_dtype=torch.float32)
+    ref = oracle.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
+                      m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"])
+    for got, want in zip((q, k, v), ref[:3]):
+        assert err(got, want) < TOL_F32
+    gdn.check_device_error()
+
+
 def test_chunk_tc_matches_recurrent_path_no_initial_state():
     x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=22, T=256, H=4)
     y1, S1 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
