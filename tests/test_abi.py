@@ -109,6 +109,7 @@ def test_workspace_size_covers_every_chunk(L):
 
 def test_zero_tokens_is_a_no_op(L):
     assert chunk_call(L, N=0, q=None, y=None) == gdn.GDN_OK
+    assert gated_call(L, N=0, q=None, z=None, out=None, w=None) == gdn.GDN_OK
     assert L.gdn_decode_step(None, None, None, None, None, None, None, 0, 0, 4, 128, 128, 1.0, 1, 1, None,
                              None) == gdn.GDN_OK
     assert L.gdn_out_gate(None, None, None, 1e-6, 0, 4, 128, 1, 1, None, None) == gdn.GDN_OK
