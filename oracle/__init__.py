@@ -66,7 +66,7 @@ def _load():
             lib.oracle_out_gate.argtypes = [_D, _D, _D, ctypes.c_double, ctypes.c_long, ctypes.c_int,
                                             ctypes.c_int, _D]
             lib.oracle_decode_step.argtypes = [_D, _D, _D, _D, _D, _D, _I64, ctypes.c_int, ctypes.c_int,
-                                               ctypes.c_int, ctypes.c_int, ctypes.c_double, _D]
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, ctypes.c_int]
             lib.oracle_threads_used.argtypes = [ctypes.c_int, ctypes.c_long]
             lib.oracle_threads_used.restype = ctypes.c_int
             _lib = lib
@@ -128,13 +128,19 @@ def recurrence(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=1, scale=1.0
     return y, S_T
 
 
-def decode_step(q, k, v, g, beta, state, state_slot=None, scale=1.0):
+def decode_step(q, k, v, g, beta, state, state_slot=None, scale=1.0, nthreads=0, inplace=False):
     """One token per row: eqs. (1)-(4) against ``state`` [slots, H, dk, dv].
 
-    Returns (y [B, H, dv], new_state) in float64; the input state is not modified.
+    Returns (y [B, H, dv], new_state) in float64.  The input state is not modified, unless
+    ``inplace`` is set and ``state`` is already a C-contiguous float64 array, which is then
+    updated and returned (long multi-step checks avoid copying the whole state every step).
     """
     q, k, v, g, beta = (_f64(t) for t in (q, k, v, g, beta))
-    st = _f64(state).copy()
+    if inplace:
+        assert isinstance(state, np.ndarray) and state.dtype == np.float64 and state.flags.c_contiguous
+        st = state
+    else:
+        st = _f64(state).copy()
     B, H, dk = q.shape
     dv = v.shape[2]
     slot = None
@@ -148,7 +154,7 @@ def decode_step(q, k, v, g, beta, state, state_slot=None, scale=1.0):
     y = np.zeros((B, H, dv))
     _load().oracle_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(st),
                                None if slot is None else slot.ctypes.data_as(_I64),
-                               B, H, dk, dv, float(scale), _ptr(y))
+                               B, H, dk, dv, float(scale), _ptr(y), int(nthreads))
     return y, st
 
 

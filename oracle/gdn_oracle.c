@@ -260,17 +260,34 @@ void oracle_out_gate(const double* y, const double* z, const double* w, double e
  * q, k: [B, H, dk]; v, y: [B, H, dv]; g, beta: [B, H];
  * state: [num_slots, H, dk, dv], updated in place; slot: [B] or NULL (row i -> slot i).
  */
+typedef struct {
+    const double *q, *k, *v, *g, *beta;
+    double* state;
+    const int64_t* slot;
+    int H, dk, dv;
+    double scale;
+    double* y;
+} dec_ctx;
+
+/* One (row, head) unit of a decode step: the same token_update as the prefill oracle. */
+static void dec_unit(void* vctx, long unit) {
+    dec_ctx* c = (dec_ctx*)vctx;
+    const int H = c->H, dk = c->dk, dv = c->dv;
+    const long b = unit / H;
+    const int h = (int)(unit % H);
+    const int64_t s = c->slot ? c->slot[b] : b;
+    const size_t bh = (size_t)b * H + h;
+    double* e = (double*)malloc(sizeof(double) * dv);
+    token_update(c->state + ((size_t)s * H + h) * dk * dv, c->q + bh * dk, c->k + bh * dk, c->v + bh * dv,
+                 exp(c->g[bh]), c->beta[bh], dk, dv, c->scale, c->y + bh * dv, e);
+    free(e);
+}
+
+/* Rows name distinct slots, so the (row, head) units are independent; they run on nthreads
+ * threads (0: every hardware thread). */
 void oracle_decode_step(const double* q, const double* k, const double* v, const double* g,
                         const double* beta, double* state, const int64_t* slot, int B, int H,
-                        int dk, int dv, double scale, double* y) {
-    double* e = (double*)malloc(sizeof(double) * dv);
-    for (int b = 0; b < B; ++b) {
-        const int64_t s = slot ? slot[b] : b;
-        for (int h = 0; h < H; ++h) {
-            const size_t bh = (size_t)b * H + h;
-            token_update(state + ((size_t)s * H + h) * dk * dv, q + bh * dk, k + bh * dk, v + bh * dv,
-                         exp(g[bh]), beta[bh], dk, dv, scale, y + bh * dv, e);
-        }
-    }
-    free(e);
+                        int dk, int dv, double scale, double* y, int nthreads) {
+    dec_ctx c = {q, k, v, g, beta, state, slot, H, dk, dv, scale, y};
+    run_units(dec_unit, &c, (long)B * H, nthreads);
 }

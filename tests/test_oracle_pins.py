@@ -253,6 +253,72 @@ def test_prep_conv_is_causal_fir_filter_then_silu():
                 assert rel(v[a:b, h, ch], pre * scipy.special.expit(pre)) < RTOL
 
 
+def _l2norm_reference(x, eps):
+    """x / sqrt(sum_i x_i^2 + eps) over the last axis (the head dimension)."""
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+@pytest.mark.parametrize("eps", [1e-6, 1e-3])
+def test_prep_q_k_are_conv_silu_then_l2norm(eps):
+    """Eqs. (6)-(7) on the q and k branches: each channel of x_q (x_k) through its own causal
+    FIR filter with w_q (w_k) (scipy.signal.lfilter, taps reversed, zero history at every
+    sequence start), SiLU = x logistic(x) (scipy.special.expit), then divided by
+    sqrt(sum over the head of x^2 + eps).  x_q, x_k and w_q, w_k are all distinct, so
+    convolving q with w_k or building q from x_k fails; one sequence of head 0 has inputs
+    scaled by 1e-3, where sum x^2 is comparable to eps, so eps outside the square root
+    (x / (|x| + eps)) or a missing eps fails too."""
+    rng = np.random.default_rng(24)
+    lengths = [7, 2, 11]
+    c = _prep_case(rng, lengths, H=2, dk=6)
+    cu = c["cu_seqlens"]
+    a0, b0 = cu[2], cu[3]
+    for key in ("x_q", "x_k"):
+        c[key][a0:b0, 0, :] *= 1e-3
+    q, k, _, _, _ = oracle.prep(**c, eps=eps)
+    H, dk = c["x_q"].shape[1:]
+    for out, x, w in ((q, c["x_q"], c["w_q"]), (k, c["x_k"], c["w_k"])):
+        want = np.zeros_like(out)
+        for n in range(len(lengths)):
+            a, b = cu[n], cu[n + 1]
+            for h in range(H):
+                for ch in range(dk):
+                    pre = scipy.signal.lfilter(w[h * dk + ch][::-1], [1.0], x[a:b, h, ch])
+                    want[a:b, h, ch] = pre * scipy.special.expit(pre)
+        want = _l2norm_reference(want, eps)
+        assert rel(out, want) < RTOL
+        # the small-input rows really are in the regime where eps matters
+        assert np.min(np.linalg.norm(out[a0:b0, 0], axis=-1)) < 0.999
+
+
+def test_prep_q_k_pins_reject_planted_mistakes():
+    """The q/k pin distinguishes the plausible slips: q convolved with w_k, q built from x_k,
+    and eps moved outside the square root.  Each slip is planted in a copy of the pinned
+    arithmetic on the CPU; the oracle's q must match the correct form and none of the slips."""
+    rng = np.random.default_rng(25)
+    lengths = [5, 9]
+    c = _prep_case(rng, lengths, H=1, dk=4)
+    c["x_q"][:, 0, :] *= np.where(np.arange(c["x_q"].shape[0]) < 5, 1e-3, 1.0)[:, None]
+    eps = 1e-6
+    q, _, _, _, _ = oracle.prep(**c, eps=eps)
+    cu = c["cu_seqlens"]
+
+    def branch(x, w, norm):
+        o = np.zeros_like(x)
+        for n in range(len(lengths)):
+            a, b = cu[n], cu[n + 1]
+            for ch in range(x.shape[2]):
+                pre = scipy.signal.lfilter(w[ch][::-1], [1.0], x[a:b, 0, ch])
+                o[a:b, 0, ch] = pre * scipy.special.expit(pre)
+        return norm(o)
+
+    good = lambda o: _l2norm_reference(o, eps)
+    eps_outside = lambda o: o / (np.linalg.norm(o, axis=-1, keepdims=True) + eps)
+    assert rel(q, branch(c["x_q"], c["w_q"], good)) < RTOL
+    for wrong in (branch(c["x_q"], c["w_k"], good), branch(c["x_k"], c["w_q"], good),
+                  branch(c["x_q"], c["w_q"], eps_outside)):
+        assert rel(q, wrong) > 1e-3
+
+
 def test_prep_one_hot_taps_identity_and_shift():
     rng = np.random.default_rng(21)
     lengths = [4, 6]
