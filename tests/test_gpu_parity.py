@@ -18,6 +18,7 @@ import torch
 import oracle
 from linear_attention_token_gdn_b200 import build as gbuild
 from linear_attention_token_gdn_b200 import gdn, inputs
+from parity_metric import excess_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -35,12 +36,8 @@ UNIT_ROUNDOFF = {torch.float32: 0.0, torch.float16: 2.0 ** -11, torch.bfloat16: 
 
 
 def err(gpu, ref):
-    u = UNIT_ROUNDOFF[gpu.dtype]
-    g = gpu.detach().double().cpu().numpy()
-    ref = np.asarray(ref)
-    assert np.all(np.isfinite(g))
-    excess = np.maximum(np.abs(g - ref) - u * np.abs(ref), 0.0)
-    return float(np.max(excess) / max(np.max(np.abs(ref)), 1e-30))
+    """The parity metric (tests/parity_metric.py) of a GPU tensor against the oracle."""
+    return excess_rel_err(gpu.detach().double().cpu().numpy(), ref, UNIT_ROUNDOFF[gpu.dtype])
 
 
 # --------------------------------------------------------------- recurrent (chunk=0)
@@ -87,29 +84,24 @@ def test_decode_steps_with_slots(dk, dv, dt):
     gdn.check_device_error()
 
 
-def test_decode_full_workload_sampled_heads():
-    """256 x 32 heads, dk = dv = 128, 100 in-place steps (bf16 q/k/v, bf16 y): check sampled
-    (row, head) pairs against the oracle run on those heads alone, every step."""
+def test_decode_full_workload_every_head():
+    """256 x 32 heads, dk = dv = 128, 100 in-place steps (bf16 q/k/v, bf16 y): the oracle steps
+    every (row, head) pair alongside (fp64, in place); y of every pair is checked on four of
+    the steps and the whole state after the last one."""
     c = inputs.WORKLOAD_SPECS[inputs.DECODE]
     state = inputs.make_decode_state(inputs.DECODE, "cuda")
-    picks = [(0, 0), (17, 5), (255, 31), (128, 16)]
-    ref = {p: state[p[0], p[1]].double().cpu().numpy()[None, None] for p in picks}
+    ref = state.double().cpu().numpy()
+    checked = {0, 37, 71, c["steps"] - 1}
     for step in range(c["steps"]):
         x = inputs.make_decode_step(inputs.DECODE, "cuda", step=step)
         y = gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state)
-        if step % 11 == 0 or step == c["steps"] - 1:
-            for (b, h) in picks:
-                sl = lambda t: t[b:b + 1, h:h + 1]
-                y_ref, ref[(b, h)] = oracle.decode_step(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
-                                                        sl(x["beta"]), ref[(b, h)])
-                assert err(y[b, h], y_ref[0, 0]) < TOL_F32
-        else:
-            for (b, h) in picks:
-                sl = lambda t: t[b:b + 1, h:h + 1]
-                _, ref[(b, h)] = oracle.decode_step(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
-                                                    sl(x["beta"]), ref[(b, h)])
-    for (b, h) in picks:
-        assert err(state[b, h], ref[(b, h)][0, 0]) < TOL_F32
+        y_ref, ref = oracle.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], ref, inplace=True)
+        if step in checked:
+            ey = err(y, y_ref)
+            assert ey < TOL_F32, (step, ey)
+    es = err(state, ref)
+    print(f"decode workload: state err {es:.2e} after {c['steps']} steps")
+    assert es < TOL_F32
     gdn.check_device_error()
 
 
@@ -127,7 +119,7 @@ def test_decode_rejects_out_of_range_slot_on_device():
 # ------------------------------------------------------------- prep / out gate
 
 @pytest.mark.parametrize("d", [128, 64, 32, 16])
-@pytest.mark.parametrize("out_dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("out_dt", [torch.float32, torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("case", ["three_seqs", "edge"])
 def test_prep_matches_oracle(d, out_dt, case):
     """Sequences that start inside a 64-token run and runs that start inside a sequence; the
@@ -295,74 +287,84 @@ def test_chunk_tc_prefill_workload_full():
     gdn.check_device_error()
 
 
-def test_chunk_tc_long_prefill_sampled_heads():
-    """B=1, H=32, T=32768, S0 ~ N(0, 0.02), exp(A) up to 64: heads checked one by one
-    (slowest- and fastest-decaying heads included)."""
+def test_chunk_tc_long_prefill_every_head():
+    """B=1, H=32, T=32768, S0 ~ N(0, 0.02), exp(A) up to 64: every head and every output."""
     x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda")
     y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64)
-    mean_g = x["g"].mean(0)
-    heads = sorted({0, int(mean_g.argmin()), int(mean_g.argmax()), 19})
-    for h in heads:
-        sl = slice(h, h + 1)
-        y_ref, S_ref = oracle.recurrence(x["q"][:, sl], x["k"][:, sl], x["v"][:, sl], x["g"][:, sl],
-                                         x["beta"][:, sl], x["S0"][:, sl], x["cu_seqlens"])
-        assert err(y[:, sl], y_ref) < TOL_16, h
-        assert err(S_T[:, sl], S_ref) < TOL_16, h
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
+    ey, es = err(y, y_ref), err(S_T, S_ref)
+    print(f"long prefill workload: y err {ey:.2e}, S_T err {es:.2e}")
+    assert ey < TOL_16 and es < TOL_16
+    # per head as well: a head whose outputs are small must not hide behind the global max
+    for h in range(x["H"]):
+        assert err(y[:, h], y_ref[:, h]) < TOL_16, h
+        assert err(S_T[:, h], S_ref[:, h]) < TOL_16, h
     gdn.check_device_error()
 
 
-def out_gate_bound(ref_y, z, norm_w, tol):
-    """Per-element bound on |out - out_ref| implied by |y - y_ref| <= tol max|y_ref| (the
-    chunked path's own bound), propagated through eq. (11): out = sigmoid(z) (1 + w) u with
-    u = sqrt(d) y / |y|_2 per row, and |du|_2 <= sqrt(d) |dy|_2 / |y|_2 to first order (the
-    factor 2 covers the second-order term).  Rows whose y is small are ill-conditioned and
-    get a correspondingly wide bound."""
-    ref_y = np.asarray(ref_y)
-    d = ref_y.shape[-1]
-    gain = np.abs(1.0 / (1.0 + np.exp(-z.double().cpu().numpy())) * (1.0 + norm_w.double().cpu().numpy()))
-    dy2 = np.sqrt(d) * tol * np.max(np.abs(ref_y))               # |dy|_2 per row
-    row = np.sqrt(np.sum(ref_y ** 2, axis=-1, keepdims=True))    # |y_ref|_2 per row
-    return gain * 2.0 * np.sqrt(d) * dy2 / np.maximum(row, 1e-30)
-
-
-@pytest.mark.parametrize("y_dt", [torch.float32, torch.bfloat16])
-def test_full_mixer_workload_sampled_heads(y_dt):
-    """Packed variable-length sequences, H=16, d=128, bf16 throughout: prep -> chunked
-    recurrence -> out gate through the C ABI (and prep -> the chunked pass with the gate fused), against the fp64 oracle mixer on sampled heads.
-    q, k, v are stored in bf16 between prep and the recurrence, and the oracle rounds them the
-    same way.  y meets the chunked path's bound; out meets that bound propagated through the
-    RMS normalisation of eq. (11), plus its own bf16 rounding."""
-    m = inputs.make_mixer(inputs.MIXER, "cuda")
+def _mixer_call(m, inter):
+    """prep with q, k, v stored in `inter` (bf16 or fp16), then the unfused chunked pass
+    (fp32 and bf16 y) with the out gate, and the pass with the gate fused, on the same q, k, v."""
     q, k, v, g, beta = gdn.prep(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"], m["beta_logit"],
                                 m["alpha_logit"], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"],
-                                out_dtype=torch.bfloat16)
-    y, S_T = gdn.chunk_fwd(q, k, v, g, beta, None, m["cu_seqlens"], chunk=64, y_dtype=y_dt)
-    out = gdn.out_gate(y, m["z"], m["norm_w"], m["eps"])
-    out_f, S_f = gdn.chunk_fwd_gated(q, k, v, g, beta, m["z"], m["norm_w"], m["eps"], None, m["cu_seqlens"])
-    d = m["d"]
-    for h in (0, 9):
-        hs = slice(h, h + 1)
-        cs = slice(h * d, (h + 1) * d)
-        ref_out, ref_y, _ = oracle.mixer(m["x_q"][:, hs], m["x_k"][:, hs], m["x_v"][:, hs], m["w_q"][cs],
-                                         m["w_k"][cs], m["w_v"][cs], m["beta_logit"][:, hs],
-                                         m["alpha_logit"][:, hs], m["A_log"][hs], m["alpha_bias"][hs],
-                                         m["z"][:, hs], m["norm_w"], m["cu_seqlens"], eps_l2=m["eps"],
-                                         eps_rms=m["eps"], inter_dtype=torch.bfloat16)
-        ey = err(y[:, hs], ref_y)
-        assert ey < TOL_16, (h, ey)
-        got = out[:, hs].double().cpu().numpy()
-        bound = out_gate_bound(ref_y, m["z"][:, hs], m["norm_w"], TOL_16) + UNIT_ROUNDOFF[out.dtype] * np.abs(ref_out)
-        worst = float(np.max(np.abs(got - ref_out) / bound))
-        worst_f = float(np.max(np.abs(out_f[:, hs].double().cpu().numpy() - ref_out) / bound))
-        print(f"mixer head {h}: y err {ey:.2e}, out within {worst:.2f} of its bound, fused gate {worst_f:.2f}")
-        assert worst <= 1.0 and worst_f <= 1.0, (h, worst, worst_f)
+                                out_dtype=inter)
+    res = {}
+    for y_dt in (torch.float32, torch.bfloat16):
+        y, S_T = gdn.chunk_fwd(q, k, v, g, beta, None, m["cu_seqlens"], chunk=64, y_dtype=y_dt)
+        res[y_dt] = (y, S_T, gdn.out_gate(y, m["z"], m["norm_w"], m["eps"]))
+    res["fused"] = gdn.chunk_fwd_gated(q, k, v, g, beta, m["z"], m["norm_w"], m["eps"], None, m["cu_seqlens"])
     gdn.check_device_error()
+    return res
+
+
+@pytest.mark.parametrize("inter", [torch.float16, torch.bfloat16])
+def test_full_mixer_workload_every_head(inter):
+    """Packed variable-length sequences, H=16, d=128: prep -> chunked recurrence -> out gate
+    through the C ABI, and prep -> the chunked pass with the gate fused, against the fp64
+    oracle mixer on every head.  q, k, v are stored in `inter` between prep and the
+    recurrence, and the oracle rounds them to the same format at the same point.  y and S_T
+    meet the tensor-core bound (3e-3, beyond the output's own rounding) in both formats.
+
+    The gated output meets the same bound with fp16 storage, the mixer's configuration.  With
+    bf16 storage it is not compared: the GPU's fp32 prep and the oracle's fp64 prep round about
+    one stored element in 10^5 to neighbouring bf16 values, and eq. (11)'s per-row RMS
+    normalisation amplifies such a one-ulp (0.4 %) input difference past 3e-3 on rows whose y
+    is small -- a property of comparing two roundings of different approximations, shown on the
+    CPU by tests/test_precision_model.py::test_bf16_storage_double_rounding_alone_exceeds_the_out_bound.
+    The fused epilogue is checked on its own in both formats: eq. (11) applied by the oracle to
+    the fp32 y of the same chunked pass, within the fp32 bound."""
+    m = inputs.make_mixer(inputs.MIXER, "cuda")
+    res = _mixer_call(m, inter)
+    ref_out, ref_y, ref_S = oracle.mixer(m["x_q"], m["x_k"], m["x_v"], m["w_q"], m["w_k"], m["w_v"],
+                                         m["beta_logit"], m["alpha_logit"], m["A_log"], m["alpha_bias"], m["z"],
+                                         m["norm_w"], m["cu_seqlens"], eps_l2=m["eps"], eps_rms=m["eps"],
+                                         inter_dtype=inter)
+    for y_dt in (torch.float32, torch.bfloat16):
+        y, S_T, out = res[y_dt]
+        ey, es, eo = err(y, ref_y), err(S_T, ref_S), err(out, ref_out)
+        print(f"mixer ({inter}, y {y_dt}): y err {ey:.2e}, S_T err {es:.2e}, out err {eo:.2e}")
+        assert ey < TOL_16 and es < TOL_16, (y_dt, ey, es)
+        if inter == torch.float16:
+            assert eo < TOL_16, (y_dt, eo)
+            for h in range(m["H"]):
+                assert err(out[:, h], ref_out[:, h]) < TOL_16, (y_dt, h)
+    out_f, S_f = res["fused"]
+    y32 = res[torch.float32][0]
+    ef_epi = err(out_f, oracle.out_gate(y32, m["z"], m["norm_w"], m["eps"]))
+    ef = err(out_f, ref_out)
+    print(f"mixer ({inter}), gate fused: epilogue err {ef_epi:.2e}, out err {ef:.2e}")
+    assert ef_epi < TOL_F32
+    if inter == torch.float16:
+        assert ef < TOL_16
+    assert torch.equal(S_f, res[torch.float32][1])
 
 
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 def test_chunk_fwd_gated_small_ragged(dt):
-    """The fused out gate: ragged tails, an empty and a one-token sequence, S0 != 0.  out meets
-    the chunked path's bound propagated through eq. (11); S_T is the plain path's."""
+    """The fused out gate: ragged tails, an empty and a one-token sequence, S0 != 0.  Its
+    epilogue against eq. (11) applied by the oracle to the fp32 y of the unfused pass (fp32
+    bound), its output against the oracle's (tensor-core bound), S_T equal to the unfused
+    pass's."""
     lengths = [3 * 64 + 17, 64, 1, 0, 130]
     x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=24, lengths=lengths, H=3, dtype=dt, S0_std=0.2)
     gen = torch.Generator(device="cuda").manual_seed(25)
@@ -371,12 +373,13 @@ def test_chunk_fwd_gated_small_ragged(dt):
     w = torch.randn(dv, device="cuda", generator=gen) * 0.5
     out, S_T = gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], z, w, 1e-6, x["S0"],
                                    x["cu_seqlens"])
+    y32, S32 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"], chunk=64,
+                             y_dtype=torch.float32)
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
-    ref_out = oracle.out_gate(y_ref, z, w, 1e-6)
-    bound = out_gate_bound(y_ref, z, w, TOL_16) + UNIT_ROUNDOFF[dt] * np.abs(ref_out)
-    worst = float(np.max(np.abs(out.double().cpu().numpy() - ref_out) / bound))
-    assert worst <= 1.0, worst
+    assert err(out, oracle.out_gate(y32, z, w, 1e-6)) < TOL_F32
+    assert err(out, oracle.out_gate(y_ref, z, w, 1e-6)) < TOL_16
     assert err(S_T, S_ref) < TOL_16
+    assert torch.equal(S_T, S32)
     gdn.check_device_error()
 
 
@@ -398,10 +401,11 @@ def test_chunk_fwd_gated_bounded_wait_reports_timeout():
         gdn.set_wait_budget(0)
     out, _ = gdn.chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], z, w, 1e-6, None, x["cu_seqlens"])
     gdn.check_device_error()
+    y32, _ = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"], chunk=64,
+                           y_dtype=torch.float32)
     y_ref, _ = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], None, x["cu_seqlens"])
-    ref_out = oracle.out_gate(y_ref, z, w, 1e-6)
-    bound = out_gate_bound(y_ref, z, w, TOL_16) + UNIT_ROUNDOFF[out.dtype] * np.abs(ref_out)
-    assert float(np.max(np.abs(out.double().cpu().numpy() - ref_out) / bound)) <= 1.0
+    assert err(out, oracle.out_gate(y32, z, w, 1e-6)) < TOL_F32
+    assert err(out, oracle.out_gate(y_ref, z, w, 1e-6)) < TOL_16
 
 
 def test_bounded_wait_reports_timeout_and_context_survives():
