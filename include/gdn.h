@@ -188,9 +188,13 @@ gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, co
  *   - A call whose scratch need, gdn_chunk_fwd_workspace_size(N, num_seqs, H, dk, dv,
  *     chunk), exceeds GDN_NOALLOC_SCRATCH_BYTES returns GDN_ERR_INVALID_ARG with the
  *     two sizes in gdn_last_error_message().  (chunk = 0 needs no scratch.)
- *   - The first call on a device looks up that device's address of the array
- *     (cudaGetSymbolAddress) with the device current; make that first call before any
- *     stream capture.  Later calls reuse the address.
+ *   - The first call in a CUDA context (the device's primary context, or whichever
+ *     context is current on the calling thread) looks up that context's address of the
+ *     array (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     Later calls in the same context reuse the address; after the context is destroyed
+ *     (e.g. cudaDeviceReset) the next call looks it up again.
+ *   - Arguments the tensor-core path does not accept (other chunk sizes, head sizes or an
+ *     fp32 input) need no scratch and get gdn_chunk_fwd's own answer.
  *   - All calls share the one array, which keeps the last call's contents; every
  *     record a call reads was written earlier in the same call, so nothing needs
  *     clearing.  Calls that overlap on the GPU (different streams, or devices sharing

@@ -5,6 +5,7 @@
 // argument is wrong; it never synchronises and never allocates.
 #include <atomic>
 #include <mutex>
+#include <vector>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -105,7 +106,7 @@ struct RecurrentLaunch {
                             const float* S0, const int32_t* cu, int num_seqs, int N, int H, float scale,
                             int in_dt, int y_dt, void* y, float* S_T, cudaStream_t st) {
         using Sh = gdn::RecShape<DK, DV>;
-        const unsigned grid = (unsigned)(num_seqs * H * (DV / Sh::SLAB));
+        const unsigned grid = (unsigned)((long long)num_seqs * H * (DV / Sh::SLAB));  // <= 2^31 (host check)
         gdn::LaunchScope timed(st, "recurrent_fwd_kernel");
         gdn::recurrent_fwd_kernel<DK, DV><<<grid, Sh::THREADS, 0, st>>>(
             q, k, v, g, beta, S0, cu, num_seqs, N, H, scale, in_dt, y_dt, y, S_T);
@@ -153,24 +154,58 @@ struct PrepLaunch {
 // Scratch of gdn_chunk_fwd_noalloc: part of the device image, one copy per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
 
+// The array's device address belongs to the CUDA context that loaded the library's module:
+// a reset of the device's primary context unloads the module, and the next context may load
+// it elsewhere.  So the address is cached per context, keyed by the context's unique id.
+struct NoallocEntry {
+    unsigned long long ctx_id;
+    void* addr;
+};
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[256] = {};  // device address of g_noalloc_scratch, per device ordinal
+std::vector<NoallocEntry> g_noalloc_cache;
 
-// Device address of the scratch array on the current device; looked up once per device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<F>(p);
+}
+
+// Device address of the scratch array in the calling thread's current context; looked up
+// (cudaGetSymbolAddress) the first time a context is seen.
 gdn_status_t noalloc_scratch(void** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= 256) return fail(GDN_ERR_UNSUPPORTED, "device ordinal %d", dev);
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    if (!get_current || !get_id) return fail(GDN_ERR_CUDA, "driver entry points cuCtxGetCurrent / cuCtxGetId");
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return fail(GDN_ERR_CUDA, "cuCtxGetCurrent failed");
+    void* p = nullptr;
+    if (ctx == nullptr) {  // no context bound to this thread yet: the runtime binds the device's own
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || p == nullptr)
             return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
-        g_noalloc_addr[dev] = p;
+        if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return fail(GDN_ERR_CUDA, "no current CUDA context");
     }
-    *out = g_noalloc_addr[dev];
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return fail(GDN_ERR_CUDA, "cuCtxGetId failed");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (const NoallocEntry& en : g_noalloc_cache)
+        if (en.ctx_id == id) {
+            *out = en.addr;
+            return GDN_OK;
+        }
+    if (p == nullptr) {
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    }
+    g_noalloc_cache.push_back({id, p});
+    *out = p;
     return GDN_OK;
 }
 
@@ -272,6 +307,7 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     REQUIRE(chunk >= 0, "chunk=%d < 0", chunk);
     REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
     REQUIRE((long long)N * H * (dk > dv ? dk : dv) < (1LL << 40), "problem too large");
+    REQUIRE((long long)num_seqs * H * 128 <= 0x7fffffffLL, "num_seqs*H too large (%d x %d)", num_seqs, H);
     if (N == 0 && S_T == nullptr) return GDN_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (chunk != 0 && chunk != 64)
@@ -310,6 +346,7 @@ gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, co
     REQUIRE(eps >= 0.f, "eps < 0");
     REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
     REQUIRE((long long)N * H * 128 < (1LL << 40), "problem too large");
+    REQUIRE((long long)num_seqs * H * 128 <= 0x7fffffffLL, "num_seqs*H too large (%d x %d)", num_seqs, H);
     if (chunk != 64 || dk != 128 || dv != 128 || in_dtype == GDN_F32 || io_dtype == GDN_F32)
         return fail(GDN_ERR_UNSUPPORTED, "the gated variant runs the tensor-core path only (chunk 64, dk=dv=128, "
                                          "bf16/f16 inputs, bf16/f16 z and out)");
@@ -338,7 +375,10 @@ gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
                                    const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
                                    int dv, int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t y_dtype, void* y,
                                    float* S_T, gdn_stream_t stream) {
-    const size_t need = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+    // only a call the tensor-core path accepts needs scratch; anything else goes straight to
+    // gdn_chunk_fwd's own checks, so both entry points answer a bad call the same way
+    const bool tc = chunk == 64 && dk == 128 && dv == 128 && in_dtype != GDN_F32;
+    const size_t need = tc ? gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk) : 0;
     if (need > GDN_NOALLOC_SCRATCH_BYTES)
         return fail(GDN_ERR_INVALID_ARG, "needs %zu bytes of scratch; the no-allocation entry point holds %llu",
                     need, (unsigned long long)GDN_NOALLOC_SCRATCH_BYTES);
