@@ -429,6 +429,8 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     fused into the chunked pass is timed beside it)."""
     m = inputs.make_mixer(inputs.MIXER, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.MIXER, rank))
     N, H = m["N"], m["H"]
+    # q, k, v between prep and the chunked pass in fp16 (11 significant bits; the storage the
+    # mixer parity test checks on every head)
     bufs = [torch.empty(N, H, 128, device="cuda", dtype=torch.float16) for _ in range(3)]
     gbuf = torch.empty(N, H, device="cuda")
     bbuf = torch.empty(N, H, device="cuda")
@@ -491,12 +493,56 @@ def main():
     ap.add_argument("--cpu-s", type=float, default=12.0, help="target seconds of the CPU-baseline sample")
     ap.add_argument("--ref-step-s", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", dest="impl_cpu_baseline", action="store_false")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="rendezvous, barrier and max-over-ranks only (gloo, no GPU work); rank 0 prints n_gpus")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus)
+    _, world, _ = env_rank()
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        return 2
+    if args.launch_check:
+        return launch_check(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
+
+
+def launch_ranks(n):
+    """`bench.py --gpus N` started as one process: start N ranks of this same command line
+    under torch.distributed.run (one node, rendezvous on 127.0.0.1) and return its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def launch_check(args):
+    """The launch plumbing alone: every rank joins a gloo group, passes the barrier and takes
+    part in the max-over-ranks reduction; rank 0 prints the world size it saw."""
+    from datetime import timedelta
+
+    import torch.distributed as dist
+    rank, world, local = env_rank()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    try:
+        gdist.barrier(world, cuda=False)
+        slowest = gdist.max_over_ranks(float(rank + 1), world, device="cpu")
+        if rank == 0:
+            print(json.dumps({"launch_check": True, "n_gpus": world, "max_over_ranks": slowest}), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":

@@ -61,3 +61,26 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
     args = bench.argparse.Namespace(steps=1, warmup=3, ref_step_s=1.0)
     assert bench.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_bench_gpus_flag_starts_the_ranks_itself():
+    """`python bench.py --gpus 2` from a plain shell (no launcher environment) starts two ranks
+    itself; the ranks rendezvous, reduce over each other and rank 0 reports n_gpus = 2."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                              "MASTER_PORT")}
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--launch-check"],
+                         capture_output=True, text=True, timeout=300, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [json.loads(l) for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["max_over_ranks"] == 2.0
+
+
+def test_bench_rejects_a_world_size_that_differs_from_gpus():
+    import subprocess
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--launch-check"],
+                         capture_output=True, text=True, timeout=120, env=env)
+    assert res.returncode == 2 and "WORLD_SIZE=1" in res.stderr
