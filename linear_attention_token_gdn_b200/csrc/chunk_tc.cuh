@@ -14,36 +14,41 @@
 // factors <= 1, so a row needs 4 + 16 exponentials instead of 64.
 //
 // Two kernels:
-//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, four CTAs per SM.
-//                       [K;Q] K^T on tcgen05 (the 16-bit inputs used directly as
-//                       operands), the decay masks, and the unit-lower-triangular inverse
-//                       T in fp32 on the CUDA cores.  Writes a 24 KB record per
-//                       (chunk, head): T_w = T diag(beta Gamma), T_u = T diag(beta) and M,
-//                       already in the 128B-swizzled operand layout.
+//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, two CTAs per SM.
+//                       [K;Q] K^T on tcgen05 (the 16-bit inputs used directly as operands),
+//                       the decay masks, and the unit-lower-triangular inverse T in fp32 on the
+//                       CUDA cores; then one N = 256 product [T_w; T_u] [K | V] with
+//                       T_w = T diag(beta Gamma) and T_u = T diag(beta) gives W = T_w K and
+//                       U~ = T_u V.  Writes a 40 KB record per (chunk, head): -W and M in the
+//                       128B-swizzled operand layout and U~ as four 32-column slabs, all fp16.
 //   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
-//                       the chunks.  A producer warpgroup brings each chunk's K, Q and V
-//                       tiles in with TMA, straight into operand slots, and computes
-//                       W = T_w K and [0; U~] = [0; T_u] V on the tensor cores; a chain
-//                       warpgroup carries the fp32 state (one row per thread) through two
-//                       dependent tensor-core round trips per chunk:
-//                           [0; U~] + [Q; -W] S -> Q S and U = U~ - W S in one accumulator
-//                           K^T U'              -> S' = Gamma_C S + K^T U'
+//                       the chunks.  A producer warpgroup only copies: each chunk's K and Q by
+//                       TMA, -W, U~ and M from the record by bulk copies, straight into operand
+//                       slots (bf16 K and Q converted to fp16 in place).  A chain warpgroup
+//                       carries the fp32 state (one row per thread) through two dependent
+//                       tensor-core round trips per chunk:
+//                           [Q; -W] S        -> Q S and -W S, so U = U~ - W S
+//                           K^T U'           -> S' = Gamma_C S + K^T U'
 //                       with U' = diag(Gamma_C / Gamma) U, while M U, for
 //                       Y = Gamma (Q S) + M U, is issued once the next chunk's [Q; -W] S
-//                       has completed, when the MMA front end is otherwise idle.
-//                       Q/W/M slots are double-buffered, K/V stages triple-buffered, all
+//                       has completed, when the MMA front end is otherwise idle.  Sixteen MMA
+//                       instructions per chunk, none of them in the producer.
+//                       Q/W/M/U~ slots are double-buffered, K stages triple-buffered, all
 //                       handed over with mbarriers; full chunks of y leave through swizzled
 //                       TMA stores.  It is launched as a programmatic dependent of
 //                       chunk_ut_kernel.  The gated variant applies eq. (11)'s output gate
 //                       in the y epilogue, the four slab CTAs of a (sequence, head) forming
 //                       one cluster that exchanges row sums of squares.
-// Operands are 16-bit with fp32 accumulation in TMEM.  Each tcgen05.mma instruction costs
-// the SM's MMA front end about as much below N = 128 as at N = 128, so products are shaped
-// to use few instructions.  q and k enter exactly as stored (bf16 or fp16), so their partners
-// (T_w, W, S, U') take the same format; U' enters as a rounded high half plus its remainder,
-// side by side in one N = 64 operand, because its rounding would show in the state.  Products
-// between values we compute -- T_u V (V converted to fp16 in place) and M U -- run in fp16
-// (11 significant bits).
+// Operands are 16-bit with fp32 accumulation in TMEM.  A tcgen05.mma instruction with
+// M = 128 costs the SM's MMA pipe about 95 cycles for any N up to 64 (N = 128: about 147,
+// N = 256: about 173, measured), so products are shaped to use few instructions, and the
+// per-(chunk, head) products are formed once in chunk_ut_kernel rather than once per slab.
+// bf16 inputs must lie inside the fp16 range (|x| < 65504), as unit-norm keys and queries do.  [K;Q] K^T reads q and k exactly as stored.  Every product of the
+// chain runs on fp16 operands (11 significant bits): bf16 q, k and v are converted to fp16 in
+// shared memory when they land (exact for |x| >= 2^-14), and their partners T_w, W, S and U'
+// are formed in fp16.  bf16 partners (8 bits) would let the error of a row whose y is small
+// exceed the bound once eq. (11) normalises that row.  U' enters as a rounded high half plus
+// its remainder, side by side in one N = 64 operand.
 // Operand tiles use the 128B / 64B swizzled canonical layouts, so one tile serves as K-major
 // or MN-major operand.  Every wait is bounded (ChunkArgs::budget clock cycles); a wait that
 // runs out sets the device error word, lets in-flight MMAs and copies drain, and the CTA
@@ -55,6 +60,7 @@
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "tmap.cuh"
+#include "warp_mma.cuh"
 
 namespace gdn {
 
@@ -78,20 +84,21 @@ struct ChunkArgs {
     void* out;
 };
 
-// TMA descriptors of the chain kernel: [N, H, 128] views of k, q (64-column halves, 128B
-// swizzle), v and z (NS-column slab, 64B swizzle) and y -- or out, when the gate is fused --
+// TMA descriptors of both kernels: [N, H, 128] views of k, q and v (64-column halves, 128B
+// swizzle), z (NS-column slab, 64B swizzle) and y -- or out, when the gate is fused --
 // (NS-column slab stores, swizzled to the row width).
 struct ChainMaps {
     CUtensorMap k, q, v, y, z;
 };
 
 constexpr int kChunk = 64;
-// Record of one (chunk, head), written by chunk_ut_kernel: three [64 rows x 128 B] operand tiles
-// in the 128B-swizzled K-major layout.
-constexpr int kRecTw = 0;          // T_w = T diag(beta Gamma), 16-bit in the input's format (meets K)
-constexpr int kRecTu = 8192;       // T_u = T diag(beta), fp16 (meets V converted to fp16)
-constexpr int kRecM = 16384;       // M, fp16 (meets U, another computed operand)
-constexpr int kRecBytes = 24576;
+// Record of one (chunk, head), written by chunk_ut_kernel, all fp16:
+constexpr int kRecW = 0;           // -W: two dk halves, each [64 rows x 128 B] 128B-swizzled K-major,
+                                   // ready to be rows 64-127 of the chain's [Q; -W] operand
+constexpr int kRecM = 16384;       // M: [64 rows x 128 B] 128B-swizzled K-major
+constexpr int kRecU = 24576;       // U~: four 32-column dv slabs, each [64 rows x 64 B] row-major
+constexpr int kRecUSlab = 4096;
+constexpr int kRecBytes = 40960;
 
 // Upper bound of the number of 64-token chunks over all sequences (the records the workspace
 // holds); it holds for every valid cu_seqlens.
@@ -195,42 +202,82 @@ __host__ __device__ constexpr uint32_t idesc16(int M, int N, bool a_mn, bool b_m
 
 __device__ __forceinline__ void st16(uint8_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
+// bytes (a multiple of 16 * NT) of bf16 values at p rewritten as fp16, 16 bytes per thread per
+// pass over NT threads (it = the thread's index among them).
+template <int NT = 128>
+__device__ __forceinline__ void to_f16_inplace(uint8_t* p, int bytes, int it) {
+    for (int off = it * 16; off < bytes; off += NT * 16) {
+        uint4* p16 = reinterpret_cast<uint4*>(p + off);
+        const uint4 u = *p16;
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack2<true>(w4[e]);
+            o4[e] = pack2<false>(f.x, f.y);
+        }
+        *p16 = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+}
+
 // =====================================================================================
 // chunk_ut_kernel: per (chunk, head) -- masks and the UT transform
 // =====================================================================================
 
 struct UtCfg {
+    static constexpr int THREADS = 256;
     static constexpr int LD = 68;                           // fp32 row stride of A and T
-    static constexpr int OFF_KQ = 0;                        // [K;Q] as stored: 2 x [128 x 128 B]
-    static constexpr int OFF_A = 0;                         // fp32 A [64][LD], over [K;Q] once read
-    static constexpr int OFF_Z = OFF_A + 64 * LD * 4;       // fp32 Z [3][16][20], likewise
-    static constexpr int OFF_T = 32768;                     // fp32 T [64][LD]
-    static constexpr int OFF_VEC = OFF_T + 64 * LD * 4;     // gamma, Gamma, beta, colf: 4 x 64
+    // [K h0 | Q h0 | K h1 | Q h1 | V h0 | (gap) | V h1], 8 KB tiles [64 rows x 128 B], 128B
+    // swizzle.  [K_h; Q_h] is the A operand of half h of [K;Q] K^T; K h0, K h1, V h0, V h1 sit
+    // 16 KB apart, the column-block stride of the MN-major B operand [K | V] (N = 256).
+    static constexpr int OFF_K = 0, OFF_Q = 8192, OFF_V = 32768, KV_LBO = 16384;
+    // fp32 scratch of the block inverse over Q h0 once [K;Q] K^T has read it: the level-one
+    // products [2 blocks][16][LDX1] and the level-two product [32][LDX2]
+    static constexpr int OFF_X1 = 8192, LDX1 = 20, OFF_X2 = OFF_X1 + 2 * 16 * LDX1 * 4, LDX2 = 36;
+    static constexpr int OFF_VEC = 40960;                   // gamma, Gamma, beta, colf: 4 x 64 (gap)
     static constexpr int OFF_META = OFF_VEC + 1024;
     static constexpr int OFF_BAR = OFF_META + 32;
-    static constexpr int BYTES = OFF_BAR + 32 + 1024;
-    static_assert(OFF_Z + 3 * 16 * 20 * 4 <= OFF_T, "A and Z fit in the [K;Q] tiles");
-    static constexpr uint32_t TMEM_COLS = 64;
+    static constexpr int OFF_A = 57344;                     // fp32 A [64][LD]; later [T_w; T_u]
+    static constexpr int OFF_TOP = OFF_A;                   //   fp16 [128 rows x 128 B], 128B swizzle
+    static constexpr int OFF_T = OFF_A + 64 * LD * 4;       // fp32 T [64][LD]
+    static constexpr int BYTES = OFF_T + 64 * LD * 4 + 1024;
+    static_assert(OFF_BAR + 64 <= OFF_V + 16384, "vectors and barriers fit in the gap");
+    static_assert(OFF_X2 + 32 * LDX2 * 4 <= 16384, "inverse scratch fits in Q h0");
+    static_assert(64 * LD * 4 >= 16384 && OFF_A % 1024 == 0, "[T_w; T_u] fits over A");
+    static constexpr uint32_t TMEM_COLS = 256;              // [K;Q] K^T (cols 0-63), then [T_w;T_u][K|V]
 };
 
+// One CTA (eight warps) per (chunk, head): the UT transform of the chunk and the products that
+// depend on it alone.  [K;Q] K^T gives A and M; T = (I + A)^-1 in fp32 (16x16 diagonal blocks by
+// forward substitution on the CUDA cores, the off-diagonal blocks by recursive doubling,
+//     T21 = -T22 A21 T11   for 16x16 blocks, then the same for the 32x32 halves,
+// as warp-level mma.sync products of fp32 values split into fp16 pairs); then one N = 256
+// product
+//     [T_w; T_u] [K | V]  ->  lanes 0-63: W = T_w K (columns 0-127),
+//                             lanes 64-127: U~ = T_u V (columns 128-255)
+// (the other two blocks are not used), with T_w = T diag(beta Gamma), T_u = T diag(beta), K and
+// V converted to fp16 once [K;Q] K^T has read them.  -W, M and U~ go to the record in fp16.
 template <bool BF>
-__global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
-                                                          const __grid_constant__ ChainMaps maps) {
+__global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
+                                                                     const __grid_constant__ ChainMaps maps) {
     using Cf = UtCfg;
-    constexpr int LD = Cf::LD;
+    constexpr int LD = Cf::LD, NT = Cf::THREADS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(smem);
     float* fA = reinterpret_cast<float*>(smem + Cf::OFF_A);
     float* fT = reinterpret_cast<float*>(smem + Cf::OFF_T);
-    float* fZ = reinterpret_cast<float*>(smem + Cf::OFF_Z);
+    float* fX1 = reinterpret_cast<float*>(smem + Cf::OFF_X1);
+    float* fX2 = reinterpret_cast<float*>(smem + Cf::OFF_X2);
     float* vb = reinterpret_cast<float*>(smem + Cf::OFF_VEC);  // gamma[0:64] Gamma[64:128] beta[128:192] colf[192:256]
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);       // MMA done
-    uint64_t* bar_ld = bar + 1;                                            // K, Q tiles landed
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);       // MMA done (two phases)
+    uint64_t* bar_ld = bar + 1;                                            // K, Q, V tiles landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 16);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // TMEM lane quadrant and column half of this warp in the epilogues (two warps per quadrant)
+    const int quad = warp & 3, chalf = warp >> 2;
     // heads vary fastest across the grid, so CTAs resident together read whole token rows
     const int H = a.H, v = (int)(blockIdx.x / (unsigned)H), h = (int)(blockIdx.x % (unsigned)H);
     tc::launch_dependents();  // the chain kernel may start its prologue once every CTA is resident
@@ -250,18 +297,19 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
     const int t0 = t_begin + meta[2] * kChunk, L = min(kChunk, t_end - t0);
     uint8_t* rec = reinterpret_cast<uint8_t*>(a.workspace) + ((size_t)v * H + h) * kRecBytes;
 
-    // ---- K (rows 0-63) and Q (rows 64-127) as they are stored (bf16 or fp16), by TMA into the
-    //      128B-swizzled operand layout.  Rows past the sequence end hold other tokens; they
-    //      only meet beta = 0 or the strictly-upper mask, so nothing needs clearing. ----------------
+    // ---- K, Q, V as they are stored (bf16 or fp16), by TMA into the 128B-swizzled operand
+    //      layout.  Rows past the sequence end hold other tokens (or the fill of a load past N);
+    //      they only meet beta = 0 or the strictly-upper mask, so nothing needs clearing. ---------
     if (tid == 0) {
         tc::mbar_init(bar, 1);
         tc::mbar_init(bar_ld, 1);
         tc::fence_mbar_init();
-        tc::mbar_arrive_expect_tx(bar_ld, 4 * 8192);
+        tc::mbar_arrive_expect_tx(bar_ld, 6 * 8192);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tc::tma_load_3d(smem + Cf::OFF_KQ + hf * 16384, &maps.k, 64 * hf, h, t0, bar_ld);
-            tc::tma_load_3d(smem + Cf::OFF_KQ + hf * 16384 + 8192, &maps.q, 64 * hf, h, t0, bar_ld);
+            tc::tma_load_3d(smem + Cf::OFF_K + hf * 16384, &maps.k, 64 * hf, h, t0, bar_ld);
+            tc::tma_load_3d(smem + Cf::OFF_Q + hf * 16384, &maps.q, 64 * hf, h, t0, bar_ld);
+            tc::tma_load_3d(smem + Cf::OFF_V + hf * Cf::KV_LBO, &maps.v, 64 * hf, h, t0, bar_ld);
         }
     }
     if (tid < 64) {
@@ -292,10 +340,10 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
         tc::mbar_wait_bounded(bar_ld, 0, 4000000000ull);
     }
 
-    // ---- [K;Q] K^T ---------------------------------------------------------------------------
+    // ---- [K;Q] K^T (the inputs' own format) -------------------------------------------------------
     if (tid == 0 && landed) {
         constexpr uint32_t id = idesc16<BF>(128, 64, false, false);
-        const uint64_t d0 = tc::smem_desc(sbase + Cf::OFF_KQ, 16, 1024, tc::kSw128);
+        const uint64_t d0 = tc::smem_desc(sbase + Cf::OFF_K, 16, 1024, tc::kSw128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
             const uint64_t d = desc_add(d0, (kk >> 2) * 16384 + (kk & 3) * 32);
@@ -313,44 +361,53 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
     }
     tc::tc_fence_after();
 
+    bool done2 = false;
     if (landed && done) {
-        // ---- masks: A (fp32, over the consumed [K;Q] tiles) for the solve; M (fp16) straight
-        //      into the record ---------------------------------------------------------------------
+        // ---- masks: A (fp32) for the solve; M (fp16) straight into the record.  TMEM lane
+        //      32 quad + lane is row r of [K;Q] K^T, this warp takes columns 32 chalf .. +31 -----------
         {
-            float x[64];
-            const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-            tc::tmem_ld32(trow, x);
-            tc::tmem_ld32(trow + 32, x + 32);
-            const int r = tid & 63, R = r >> 4, rl = r & 15;
+            float x[32];
+            tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + 32 * chalf, x);
+            const int r = (32 * quad + lane) & 63, R = r >> 4, rl = r & 15;
             const float gr = vb[r];
-            const bool isA = tid < 64;
-            float rowf[4], dg[16];
-#pragma unroll
-            for (int S = 0; S < 4; ++S) rowf[S] = S < R ? __expf(gr - vb[16 * S + 15]) : 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) dg[jj] = (isA ? jj < rl : jj <= rl) ? __expf(gr - vb[16 * R + jj]) : 0.f;
+            const bool isA = quad < 2;
             const float sc = isA ? vb[128 + r] : 1.f;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                float m[8];
+            for (int blk = 0; blk < 2; ++blk) {
+                const int S = 2 * chalf + blk;
+                // blocks before the row's own: exp(gamma_r - gamma_e) exp(gamma_e - gamma_s), both <= 1
+                const float rowf = S < R ? __expf(gr - vb[16 * S + 15]) : 0.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s = 8 * cc + e, S = s >> 4;
-                    const float f = S < R ? rowf[S] * vb[192 + s] : (S == R ? dg[s & 15] : 0.f);
-                    m[e] = sc * f * x[s];
-                }
-                if (isA) {
-                    sts4(fA + r * LD + 8 * cc, make_float4(m[0], m[1], m[2], m[3]));
-                    sts4(fA + r * LD + 8 * cc + 4, make_float4(m[4], m[5], m[6], m[7]));
-                } else {
-                    st16(rec + kRecM + tc::swz_off(r, cc, 128), pack8<false>(m));
+                for (int e = 0; e < 16; ++e) {
+                    const int s = 16 * S + e;
+                    float f = rowf * vb[192 + s];
+                    if (S == R) f = (isA ? e < rl : e <= rl) ? __expf(gr - vb[s]) : 0.f;
+                    x[16 * blk + e] *= sc * f;
                 }
             }
+            if (isA) {
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4)
+                    sts4(fA + r * LD + 32 * chalf + 4 * c4, make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]));
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) st16(rec + kRecM + tc::swz_off(r, 4 * chalf + cc, 128), pack8<false>(x + 8 * cc));
+            }
         }
+        // K and V to fp16 in place for the second product (exact for |x| >= 2^-14); [K;Q] K^T
+        // has completed, so nothing reads them meanwhile
+        if constexpr (BF) {
+            to_f16_inplace<NT>(smem + Cf::OFF_K, 8192, tid);
+            to_f16_inplace<NT>(smem + Cf::OFF_K + 16384, 8192, tid);
+            to_f16_inplace<NT>(smem + Cf::OFF_V, 8192, tid);
+            to_f16_inplace<NT>(smem + Cf::OFF_V + Cf::KV_LBO, 8192, tid);
+        }
+        tc::tc_fence_before();
         __syncthreads();
 
-        // ---- T = (I + A)^-1: 16x16 diagonal blocks by forward substitution (lane = column) -----
-        if (lane < 16) {
+        // ---- T = (I + A)^-1.  16x16 diagonal blocks by forward substitution (warps 0-3, lane =
+        //      column); the zeros above each diagonal are written too ---------------------------
+        if (warp < 4 && lane < 16) {
             const int b0 = warp * 16, jc = lane;
             float xs[16];
 #pragma unroll
@@ -370,51 +427,57 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
             for (int r = 0; r < 16; ++r) fT[(b0 + r) * LD + b0 + jc] = xs[r];
         }
         __syncthreads();
-        // off-diagonal blocks, d = i - j = 1, 2, 3:  T_ij = -T_ii sum_{m=j}^{i-1} A_im T_mj
-        // work item = (block, row rr, 4-column group cg)
-        for (int d = 1; d < 4; ++d) {
-            const int items = (4 - d) * 64;
-            for (int o = tid; o < items; o += 128) {
-                const int blk = o >> 6, i = d + blk, jb = i - d, rr = (o >> 2) & 15, cg = o & 3;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int m = jb; m < i; ++m) {
-#pragma unroll
-                    for (int s4 = 0; s4 < 4; ++s4) {
-                        const float4 av = lds4(fA + (16 * i + rr) * LD + 16 * m + 4 * s4);
-                        const float a4[4] = {av.x, av.y, av.z, av.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float4 t = lds4(fT + (16 * m + 4 * s4 + e) * LD + 16 * jb + 4 * cg);
-                            acc.x += a4[e] * t.x; acc.y += a4[e] * t.y; acc.z += a4[e] * t.z; acc.w += a4[e] * t.w;
-                        }
-                    }
-                }
-                sts4(fZ + (blk * 16 + rr) * 20 + 4 * cg, acc);
-            }
-            __syncthreads();
-            for (int o = tid; o < items; o += 128) {
-                const int blk = o >> 6, i = d + blk, jb = i - d, rr = (o >> 2) & 15, cg = o & 3;
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int s4 = 0; s4 < 4; ++s4) {
-                    const float4 tv = lds4(fT + (16 * i + rr) * LD + 16 * i + 4 * s4);
-                    const float t4[4] = {tv.x, tv.y, tv.z, tv.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s = 4 * s4 + e;
-                        const float tt = s <= rr ? t4[e] : 0.f;
-                        const float4 z = lds4(fZ + (blk * 16 + s) * 20 + 4 * cg);
-                        acc.x -= tt * z.x; acc.y -= tt * z.y; acc.z -= tt * z.z; acc.w -= tt * z.w;
-                    }
-                }
-                sts4(fT + (16 * i + rr) * LD + 16 * jb + 4 * cg, acc);
-            }
-            __syncthreads();
+        // level one (warps 0-3): T_i,i-1 = -T_ii (A_i,i-1 T_i-1,i-1) for i = 1, 3, one 8-column
+        // tile per warp
+        if (warp < 4) {
+            const int bi = warp >> 1, nt = warp & 1, i = 2 * bi + 1, j = i - 1;
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            wm::load_a(fA, LD, 16 * i, 16 * j, 1.f, ah, al);
+            wm::load_b(fT, LD, 16 * j, 16 * j + 8 * nt, bh, bl);
+            wm::mma_split(d, ah, al, bh, bl);
+            float* x1 = fX1 + bi * 16 * Cf::LDX1;
+            wm::store_c(x1, Cf::LDX1, 0, 8 * nt, d);
+            __syncwarp();
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
+            wm::load_a(fT, LD, 16 * i, 16 * i, -1.f, ah, al);
+            wm::load_b(x1, Cf::LDX1, 0, 8 * nt, bh, bl);
+            wm::mma_split(e, ah, al, bh, bl);
+            wm::store_c(fT, LD, 16 * i, 16 * j + 8 * nt, e);
         }
-        // ---- T_w = T diag(beta Gamma) (input's format), T_u = T diag(beta) (fp16) -> record ------
+        __syncthreads();
+        // level two (all warps): X = A[32:64, 0:32] T[0:32, 0:32], then T[32:64, 0:32] = -T[32:64,
+        // 32:64] X; one 16x8 tile per warp, skipping the zero upper-right 16x16 blocks
+        {
+            const int mt = warp >> 2, nt = warp & 3;
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int idx = tid + 128 * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
+            for (int kt = 0; kt < 2; ++kt) {
+                if (kt == 0 && nt >= 2) continue;  // T[0:16, 16:32] = 0
+                wm::load_a(fA, LD, 32 + 16 * mt, 16 * kt, 1.f, ah, al);
+                wm::load_b(fT, LD, 16 * kt, 8 * nt, bh, bl);
+                wm::mma_split(d, ah, al, bh, bl);
+            }
+            wm::store_c(fX2, Cf::LDX2, 16 * mt, 8 * nt, d);
+            __syncthreads();
+            float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kt = 0; kt < 2; ++kt) {
+                if (mt == 0 && kt == 1) continue;  // T[32:48, 48:64] = 0
+                wm::load_a(fT, LD, 32 + 16 * mt, 32 + 16 * kt, -1.f, ah, al);
+                wm::load_b(fX2, Cf::LDX2, 16 * kt, 8 * nt, bh, bl);
+                wm::mma_split(e, ah, al, bh, bl);
+            }
+            wm::store_c(fT, LD, 32 + 16 * mt, 8 * nt, e);
+        }
+        __syncthreads();
+        // ---- [T_w; T_u] (fp16) over A: T_w = T diag(beta Gamma) in rows 0-63, T_u = T diag(beta)
+        //      in rows 64-127, K-major with K = the chunk position s --------------------------------
+        uint8_t* top = smem + Cf::OFF_TOP;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx = tid + NT * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
             const float4 t0v = lds4(fT + r * LD + 8 * cc), t1v = lds4(fT + r * LD + 8 * cc + 4);
             const float4 b0v = lds4(vb + 128 + 8 * cc), b1v = lds4(vb + 128 + 8 * cc + 4);
             float t8[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
@@ -426,8 +489,49 @@ __global__ void __launch_bounds__(128, 4) chunk_ut_kernel(const __grid_constant_
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) t8[e] = (8 * cc + e <= r) ? t8[e] * s8[e] : 0.f;
-            if (which == 0) st16(rec + kRecTw + tc::swz_off(r, cc, 128), pack8<BF>(t8));
-            else st16(rec + kRecTu + tc::swz_off(r, cc, 128), pack8<false>(t8));
+            st16(top + tc::swz_off(64 * which + r, cc, 128), pack8<false>(t8));
+        }
+        tc::fence_async_smem();
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+
+        // ---- [T_w; T_u] [K | V] -> TMEM columns 0-255 (fp16, N = 256, four k-steps) ------------
+        if (tid == 0) {
+            constexpr uint32_t id = idesc16<false>(128, 256, false, true);
+            const uint64_t da = tc::smem_desc(sbase + Cf::OFF_TOP, 16, 1024, tc::kSw128);
+            const uint64_t db = tc::smem_desc(sbase + Cf::OFF_K, Cf::KV_LBO, 1024, tc::kSw128);  // MN-major
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) tc::mma_f16(tmem, desc_add(da, kk * 32), desc_add(db, kk * 2048), id, kk > 0);
+            tc::mma_commit(bar);
+        }
+        done2 = tc::mbar_wait_bounded(bar, 1, a.budget);
+        if (!done2) {
+            raise_error(kErrTimeout);
+            tc::mbar_wait_bounded(bar, 1, 4000000000ull);
+        }
+        tc::tc_fence_after();
+        if (done2) {
+            // quadrants 0-1: -W row r, columns 64 chalf .. +63 -> dk half chalf of the record;
+            // quadrants 2-3: U~ row r, columns 128 + 64 chalf .. +63 -> dv slabs 2 chalf, 2 chalf + 1
+            const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+            const int r = (32 * quad + lane) & 63;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float x[32];
+                tc::tmem_ld32(trow + (quad < 2 ? 0 : 128) + 64 * chalf + 32 * q, x);
+                if (quad < 2) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = -x[e];
+                    uint8_t* dst = rec + kRecW + chalf * 8192;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) st16(dst + tc::swz_off(r, 4 * q + cc, 128), pack8<false>(x + 8 * cc));
+                } else {
+                    uint8_t* dst = rec + kRecU + (2 * chalf + q) * kRecUSlab + r * 64;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) st16(dst + 16 * cc, pack8<false>(x + 8 * cc));
+                }
+            }
         }
     }
     tc::tc_fence_before();
@@ -449,12 +553,11 @@ struct ChainCfg {
     static constexpr uint32_t SWZ = NS == 32 ? tc::kSw64 : tc::kSw128;
     static constexpr int QW_HALF = 128 * 128;                  // one 64-column half of [Q;W]
     static constexpr int K_HALF = 64 * 128;                    // one 64-column half of K
-    static constexpr int OFF_QW = 0;                           // [2 slots] [Q;W]: 2 halves x [128 x 128 B]
-    static constexpr int OFF_M = OFF_QW + 2 * 2 * QW_HALF;     // [2 slots] M fp16: [64 x 128 B]
+    static constexpr int OFF_QW = 0;                           // [3 stages] [Q;-W]: 2 halves x [128 x 128 B]
+    static constexpr int OFF_M = OFF_QW + 3 * 2 * QW_HALF;     // [2 slots] M fp16: [64 x 128 B]
     static constexpr int OFF_KS = OFF_M + 2 * 8192;            // [3 stages] K: 2 halves x [64 x 128 B]
-    static constexpr int OFF_TT = OFF_KS + 3 * 2 * K_HALF;     // [T_w; T_w; 0; T_u]: [256 x 128 B]
-    static constexpr int OFF_VS = OFF_TT + 32768;              // [3 stages] V slab [64 x ROWB]
-    static constexpr int OFF_SS = OFF_VS + 3 * 64 * ROWB;      // S [128 x ROWB]
+    static constexpr int OFF_UT = OFF_KS + 3 * 2 * K_HALF;     // [3 stages] U~ slab fp16 [64 x ROWB], row-major
+    static constexpr int OFF_SS = OFF_UT + 3 * 64 * ROWB;      // S [128 x ROWB]
     static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // [2 slots] U fp16: [64 x ROWB]
     static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // [U' hi | U' lo]: [64 x UROWB]
     static constexpr int OFF_YS = OFF_SU2 + 64 * UROWB;        // y rows for the TMA store [64 x NS x 4 B]
@@ -467,34 +570,36 @@ struct ChainCfg {
     static constexpr int OFF_BAR = OFF_NW + NS * 4;
     static constexpr int NBARS = 22;
     static constexpr int BYTES = OFF_BAR + 256 + 1024;
-    static constexpr uint32_t KV_TX = 2 * K_HALF + 64 * ROWB;  // K and the V slab of one chunk
-    static constexpr uint32_t Q_TX = 2 * 8192;                 // Q of one chunk
+    static constexpr uint32_t K_TX = 2 * K_HALF;               // K of one chunk
+    static constexpr uint32_t OP_TX = 2 * 8192 + 2 * 8192 + 64 * ROWB;  // Q, -W and the U~ slab of one chunk
     static constexpr uint32_t M_TX = 8192;                     // M of one chunk
     static constexpr uint32_t Z_TX = 64 * ROWB;                // z slab of one chunk (gated)
-    // TMEM columns
-    static constexpr uint32_t COL_U = 0;                       // [2 slots] x NS: [0; U~] + [Q; -W] S over dk 0-63
-    static constexpr uint32_t COL_W = 2 * NS;                  // 128: W (both lane halves)
-    static constexpr uint32_t COL_1B = COL_W + 128;            // NS: [Q; -W] S over dk 64-127
-    static constexpr uint32_t COL_MU = COL_1B + NS;            // NS: M U (lanes 0-63)
-    static constexpr uint32_t COL_DS = COL_MU + NS;            // 2 NS: [K^T U' hi | K^T U' lo]
-    static constexpr uint32_t TMEM_COLS = 512;
+    // TMEM columns; the products of chunk c that y of c needs stay until chunk c + 1 reads them
+    static constexpr uint32_t COL_U = 0;                       // [2 slots] x NS: [Q; -W] S over dk 0-63
+    static constexpr uint32_t COL_1B = COL_U + 2 * NS;         // [2 slots] x NS: [Q; -W] S over dk 64-127
+    static constexpr uint32_t COL_MU = COL_1B + 2 * NS;        // [2 slots] x NS: M U (lanes 0-63)
+    static constexpr uint32_t COL_DS = COL_MU + 2 * NS;        // 2 NS: [K^T U' hi | K^T U' lo]
+    static constexpr uint32_t TMEM_COLS = 256;
     static_assert(COL_DS + 2 * NS <= TMEM_COLS, "TMEM budget");
     static_assert(NS == 32, "[hi | lo] operand rows are one 128-byte swizzle atom");
     static_assert(NBARS * 8 <= 192, "barrier area");
     static_assert(BYTES <= 232448, "shared memory budget");
-    static_assert(OFF_M % 1024 == 0 && OFF_KS % 1024 == 0 && OFF_TT % 1024 == 0 && OFF_YS % 1024 == 0 &&
-                      OFF_VS % 1024 == 0 && OFF_SS % 1024 == 0 && OFF_SU % 1024 == 0 && OFF_SU2 % 1024 == 0 && OFF_ZS % 1024 == 0 &&
+    static_assert(OFF_M % 1024 == 0 && OFF_KS % 1024 == 0 && OFF_YS % 1024 == 0 && OFF_UT % 1024 == 0 &&
+                      OFF_SS % 1024 == 0 && OFF_SU % 1024 == 0 && OFF_SU2 % 1024 == 0 && OFF_ZS % 1024 == 0 &&
                       OFF_GZ % 1024 == 0,
                   "swizzle atoms");
 };
 
-// Synchronisation of one chunk c in slot b = c & 1 (stage c % 3 for K and V):
-//   producer -> chain   full[b]      W(c) in [Q;W] slot b, U~(c) in TMEM, gates and bounds of c
-//                       q[b], m[b]   Q(c), M(c) landed (TMA / bulk copy bytes)
-//   chain -> producer   ds_done[b]   the state MMA of c completed: [Q;W] slot b, U~ columns b and
-//                                    K stage c % 3 are free (everything else of c was read before)
+// Synchronisation of one chunk c, in stage s = c % 3 for Q, -W, U~ and K, and slot b = c & 1 for M
+// and the hand-over:
+//   producer -> chain   full[b]      Q(c) and -W(c) in [Q;-W] stage s, U~(c) in U~ stage s, K(c) in
+//                                    K stage s (all fp16), gates and bounds of c
+//                       m[b]         M(c) landed (bulk copy bytes)
+//   chain -> producer   ds_done[s]   the state MMA of c completed: the [Q;-W], U~ and K stages s are
+//                                    free (everything else of c was read before); the producer
+//                                    refills them with chunk c + 3, two chain periods ahead of use
 //                       m_empty[b]   M U of c completed: M slot b and U slot b are free
-// The chain issues M U of chunk c once chunk c + 1's [Q;W] S has completed (the MMA front end is
+// The chain issues M U of chunk c once chunk c + 1's [Q;-W] S has completed (the MMA front end is
 // idle while warps 2-3 form U) and forms y of c meanwhile.
 template <int NS, bool BF, bool GATED>
 __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_constant__ ChunkArgs a,
@@ -506,20 +611,18 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     const uint32_t sbase = tc::smem_u32(smem);
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
-    uint64_t* bar_p = bars + 0;        // producer: W = T_w K complete
-    uint64_t* bar_p2 = bars + 1;       // producer: U~ = T_u V complete
-    uint64_t* bar_c1 = bars + 2;       // chain: [Q;W] S over dk 0-63 complete
-    uint64_t* bar_c2 = bars + 3;       // chain: [Q;W] S over dk 64-127 complete
-    uint64_t* bar_ds = bars + 4;       // chain: K^T U' complete
-    uint64_t* bar_y = bars + 5;        // chain: M U complete
-    uint64_t* bar_tt = bars + 6;       // T_w, T_u of the next chunk landed in TT
-    uint64_t* bar_full = bars + 7;     // [2 slots]
-    uint64_t* bar_dsd = bars + 9;      // [2 slots] ds_done
-    uint64_t* bar_mfree = bars + 11;   // [2 slots] m_empty
-    uint64_t* bar_q = bars + 13;       // [2 slots]
-    uint64_t* bar_m = bars + 15;       // [2 slots]
-    uint64_t* bar_kv = bars + 17;      // [3 stages] K and V landed (bytes)
-    uint64_t* bar_rs = bars + 20;      // [2] the 4 slab CTAs' y^2 sums of a chunk landed (gated, bytes)
+    uint64_t* bar_c1 = bars + 0;       // chain: [Q;-W] S over dk 0-63 complete
+    uint64_t* bar_c2 = bars + 1;       // chain: [Q;-W] S over dk 64-127 complete
+    uint64_t* bar_ds = bars + 2;       // chain: K^T U' complete
+    uint64_t* bar_y = bars + 3;        // chain: M U complete
+    uint64_t* bar_full = bars + 4;     // [2 slots]
+    uint64_t* bar_dsd = bars + 6;      // [3 stages] ds_done
+    uint64_t* bar_mfree = bars + 9;    // [2 slots] m_empty
+    uint64_t* bar_q = bars + 11;       // [3 stages] Q, -W and U~ of a chunk landed (bytes)
+    uint64_t* bar_m = bars + 14;       // [2 slots]
+    uint64_t* bar_kv = bars + 16;      // [3 stages] K landed (bytes)
+    uint64_t* bar_rs = bars + 19;      // [2] the 4 slab CTAs' y^2 sums of a chunk landed (gated, bytes)
+    uint64_t* bar_drain = bars + 21;   // every MMA of the three issuing threads completed (exit)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 192);
     int* s_base = reinterpret_cast<int*>(smem + Cf::OFF_BAR + 200);
 
@@ -536,7 +639,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         if (lane == 0) *s_base = base;
     }
     if (tid == 0) {
-        for (int i = 0; i < Cf::NBARS; ++i) tc::mbar_init(bars + i, 1);
+        for (int i = 0; i < Cf::NBARS; ++i) tc::mbar_init(bars + i, i == 21 ? 3 : 1);
         tc::fence_mbar_init();
     }
     if (warp == 1) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
@@ -558,13 +661,22 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     auto vec = [&](int b) { return reinterpret_cast<float*>(smem + Cf::OFF_VEC + b * 1024); };
     auto QWoff = [&](int b) { return Cf::OFF_QW + b * 2 * Cf::QW_HALF; };
     auto Koff = [&](int s) { return Cf::OFF_KS + s * 2 * Cf::K_HALF; };
-    auto Voff = [&](int s) { return Cf::OFF_VS + s * 64 * Cf::ROWB; };
 
     if (warp < 4) {
         // =============================== chain group ===================================
-        constexpr int BID = 1;
+        // Per chunk c (slot b = c & 1, stage kst = c % 3):
+        //   thread 0 / 32   [Q; -W] S(c) over the two dk halves -> COL_U[b], COL_1B[b]; thread 0 then
+        //                   issues M U(c - 1) -> COL_MU[(c - 1) & 1] behind it
+        //   warps 2-3       U = U~ - W S (lanes 64-127) -> U (fp16) and U' = f U (hi + lo); thread 64
+        //                   issues K^T U'(c) as soon as these two warps have written U'
+        //   warps 0-1       meanwhile y of chunk c - 1 = scale (Gamma (Q S) + M U), all three
+        //                   products read from TMEM, staged and stored
+        //   all             S = Gamma_C S + K^T U' (one dk row per thread) -> fp16 S operand
+        // so the state's critical path holds two MMA round trips and the U epilogue, and the y
+        // work of warps 0-1 overlaps it.
+        constexpr int BID = 1, BID_U = 5, BID_Y = 4;
         uint32_t ph_c1 = 0, ph_c2 = 0, ph_ds = 0, ph_y = 0;
-        bool ok = true, c1_pending = false, c2_pending = false, ds_pending = false, mu_pending = false;
+        bool ok = true;
         // each thread waits for a tcgen05.commit on its own; a timeout flags the error, lets the
         // MMAs drain, and is combined over the group at the next barrier
         auto wait_mma = [&](uint64_t* bar, uint32_t& ph) -> bool {
@@ -586,8 +698,8 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::tc_fence_after();
             return all;
         };
-        constexpr uint32_t id_slab = idesc16<BF>(128, NS, false, true);    // [Q;W] S
-        constexpr uint32_t id_ds = idesc16<BF>(128, 2 * NS, true, true);   // K^T [U' hi | U' lo]
+        constexpr uint32_t id_slab = idesc16<false>(128, NS, false, true);    // [Q;W] S
+        constexpr uint32_t id_ds = idesc16<false>(128, 2 * NS, true, true);   // K^T [U' hi | U' lo]
         constexpr uint32_t id_mu = idesc16<false>(128, NS, false, true);   // M U, both fp16
         // operand descriptors at k-step 0 of slot / stage 0; k-steps and slots are byte offsets
         const uint64_t dQW0 = tc::smem_desc(sbase + Cf::OFF_QW, 16, 1024, tc::kSw128);      // K-major [Q;W]
@@ -605,52 +717,46 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
         }
 #pragma unroll
-        for (int c = 0; c < NS / 8; ++c) st16(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB), pack8<BF>(S + 8 * c));
+        for (int c = 0; c < NS / 8; ++c) st16(smem + Cf::OFF_SS + tc::swz_off(tid, c, Cf::ROWB), pack8<false>(S + 8 * c));
         float* nw = reinterpret_cast<float*>(smem + Cf::OFF_NW);
         if (GATED && tid < NS) nw[tid] = 1.f + a.norm_w[slab * NS + tid];
         operands_ready(true);
 
-        // M U of chunk ci (slot bb) -> COL_MU; by thread 0 once M(ci) has landed.  A wait that runs
+        // M U of chunk ci (slot bb) -> COL_MU[bb]; by thread 0 once M(ci) has landed.  A wait that runs
         // out is flagged and then completed (the copy always lands), so the MMA is always issued
         // and every commit below arrives.
-        auto issue_mu = [&](int ci) -> bool {
-            bool w = true;
-            if (tid == 0) {
-                const int bb = ci & 1;
-                w = tc::mbar_wait_bounded(bar_m + bb, (ci >> 1) & 1, a.budget);
-                if (!w) {
-                    raise_error(kErrTimeout);
-                    tc::mbar_wait_bounded(bar_m + bb, (ci >> 1) & 1, 4000000000ull);
-                }
-                const uint64_t am0 = desc_add(dM0, bb * 8192), bu0 = desc_add(dSU0, bb * 64 * Cf::ROWB);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // rows 0-63: M U (rows 64-127 read the next tile: unused)
-                    tc::mma_f16(tmem + Cf::COL_MU, desc_add(am0, kk * 32), desc_add(bu0, kk * 16 * Cf::ROWB), id_mu,
-                                kk > 0);
-                tc::mma_commit(bar_y);
-                if constexpr (!GATED) tc::mma_commit(bar_mfree + bb);  // gated: gate_out frees it
+        auto issue_mu = [&](int ci) -> bool {  // thread 0
+            const int bb = ci & 1;
+            bool w = tc::mbar_wait_bounded(bar_m + bb, (ci >> 1) & 1, a.budget);
+            if (!w) {
+                raise_error(kErrTimeout);
+                tc::mbar_wait_bounded(bar_m + bb, (ci >> 1) & 1, 4000000000ull);
             }
-            mu_pending = true;
+            const uint64_t am0 = desc_add(dM0, bb * 8192), bu0 = desc_add(dSU0, bb * 64 * Cf::ROWB);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // rows 0-63: M U (rows 64-127 read the next tile: unused)
+                tc::mma_f16(tmem + Cf::COL_MU + bb * NS, desc_add(am0, kk * 32), desc_add(bu0, kk * 16 * Cf::ROWB),
+                            id_mu, kk > 0);
+            tc::mma_commit(bar_y);
+            if constexpr (!GATED) tc::mma_commit(bar_mfree + bb);  // gated: gate_out frees it
             return w;
         };
 
-        // y of chunk py (warps 0-1): y = scale (Gamma_r (Q S) + M U); a full chunk is staged in
+        // y of chunk py_x (warps 0-1): y = scale (Gamma_r (Q S) + M U); a full chunk is staged in
         // swizzled rows for one TMA store, a sequence's last partial chunk goes out with plain stores.
         int py_c0 = 0, py_L = 0;
         float py_g = 0.f;         // its Gamma_r (rows 0-63)
-        float qs[NS];             // its (Q S) row (rows 0-63)
-        int py_x = -1;            // its index in the sequence (gated: selects buffers and phases)
+        int py_x = -1;            // its index in the sequence (selects TMEM slots, gated buffers, phases)
         bool gated_ok = true;
         // Gated: out = sigmoid(z) y / sqrt(mean_dv(y^2) + eps) (1 + w).  The four slab CTAs of the
         // cluster each hold 32 of the 128 columns of y.  For every chunk each CTA stores every row's
         // partial sum of squares into all four CTAs' shared memory with st.async, whose bytes
         // complete on the receiver's own bar_rs phase (armed by the receiver: 4 x 64 x 4 bytes).
-        // y_epilogue sends and keeps y in yt; gate_out, after the next MMA wait, waits for the phase,
-        // forms the full mean and gates yt with the z tile the producer loaded beside M.  Every CTA
-        // sends and receives exactly nchunks times, also after an error (see the drain below), so
-        // no store is still in flight towards a CTA when it exits.
+        // y_prev sends and keeps y in yt; gate_out waits for the phase, forms the full mean and gates
+        // yt with the z tile the producer loaded beside M.  Every CTA sends and receives exactly
+        // nchunks times, also after an error (see the drain below), so no store is still in flight
+        // towards a CTA when it exits.
         float yt[NS];
-        bool yt_pending = false;
         int n_sent = 0, n_recv = 0;  // chunks sent to the cluster / phases of bar_rs waited for
         constexpr uint32_t RS_TX = NSLAB * 64 * 4;
         auto send_sums = [&](int x, float ss) {  // warps 0-1
@@ -684,10 +790,9 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 for (int j = 0; j < NS; j += 4) st4(dst, dt, j, make_float4(t[j], t[j + 1], t[j + 2], t[j + 3]));
             }
         };
-        // gated, warps 0-1, while M U runs: this row's gate factors sigmoid(z) (1 + w) of chunk py_x
-        // -> GZ (row-private, fp32).  Waits for the z tile itself (its own acquire of bar_m).
+        // gated: this row's gate factors sigmoid(z) (1 + w) of chunk py_x -> GZ (row-private, fp32).
+        // Waits for the z tile itself (its own acquire of bar_m).
         auto gz_prep = [&]() {
-            if (!GATED || py_L <= 0) return;
             const int bb = py_x & 1;
             if (!tc::mbar_wait_bounded(bar_m + bb, (py_x >> 1) & 1, a.budget)) {
                 raise_error(kErrTimeout);
@@ -711,29 +816,9 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 *reinterpret_cast<float4*>(gz + tc::swz_off(tid, 2 * cc + 1, 4 * NS)) = make_float4(f[4], f[5], f[6], f[7]);
             }
         };
-        auto y_epilogue = [&]() {
-            if (warp < 2 && py_L > 0) {
-                float t[NS];
-                tc::tmem_ld32(trow + Cf::COL_MU, t);
-#pragma unroll
-                for (int j = 0; j < NS; ++j) t[j] = a.scale * (py_g * qs[j] + t[j]);
-                if constexpr (GATED) {
-                    float ss = 0.f;
-#pragma unroll
-                    for (int j = 0; j < NS; ++j) {
-                        ss += t[j] * t[j];
-                        yt[j] = t[j];
-                    }
-                    send_sums(py_x, ss);
-                    yt_pending = true;
-                } else {
-                    stage_rows(t, a.y_dt);
-                }
-            }
-        };
-        auto gate_out = [&]() {  // warps 0-1, after y_epilogue; then M slot and z slot are free
-            if (!GATED || !yt_pending) return;
-            yt_pending = false;
+        // gated, after send_sums: wait for the cluster's sums of chunk py_x, gate yt, stage it; then the
+        // M / z slot is free
+        auto gate_out = [&]() {
             const int bb = py_x & 1;
             const uint32_t par = (py_x >> 1) & 1;
             const bool w = tc::mbar_wait_bounded(bar_rs + bb, par, a.budget);
@@ -758,29 +843,50 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 }
                 stage_rows(yt, a.z_dt);
             }
-            tc::bar_sync(4, 64);  // every read of the z slot (gz_prep) is done
+            tc::bar_sync(BID_Y, 64);  // every read of the z slot (gz_prep) is done
             if (tid == 0) tc::mbar_arrive(bar_mfree + bb);
         };
-        auto y_store = [&]() {  // after a barrier that follows the staging
-            if (tid == 0 && py_L == kChunk) {
-                tc::tma_store_3d(&maps.y, slab * NS, h, py_c0, smem + Cf::OFF_YS);
-                tc::bulk_commit();
+        // y of chunk py_x by warps 0-1, once its M U (issued by thread 0) has completed
+        auto y_prev = [&]() -> bool {
+            const bool wy = wait_mma(bar_y, ph_y);
+            if (tid == 0) tc::bulk_wait_read0();  // YS is free again
+            tc::bar_sync(BID_Y, 64);
+            if (py_L > 0) {
+                const int pb = py_x & 1;
+                float t[NS], q1[NS];
+                tc::tmem_ld32(trow + Cf::COL_MU + pb * NS, t);
+                tc::tmem_ld32(trow + Cf::COL_U + pb * NS, q1);
+#pragma unroll
+                for (int j = 0; j < NS; ++j) t[j] += py_g * q1[j];
+                tc::tmem_ld32(trow + Cf::COL_1B + pb * NS, q1);
+#pragma unroll
+                for (int j = 0; j < NS; ++j) t[j] = a.scale * (t[j] + py_g * q1[j]);
+                if constexpr (GATED) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int j = 0; j < NS; ++j) {
+                        ss += t[j] * t[j];
+                        yt[j] = t[j];
+                    }
+                    send_sums(py_x, ss);
+                    gz_prep();
+                    gate_out();
+                } else {
+                    stage_rows(t, a.y_dt);
+                }
+                tc::fence_async_smem();
+                tc::bar_sync(BID_Y, 64);
+                if (tid == 0 && py_L == kChunk) {
+                    tc::tma_store_3d(&maps.y, slab * NS, h, py_c0, smem + Cf::OFF_YS);
+                    tc::bulk_commit();
+                }
             }
-            py_L = 0;
-        };
-        // wait for M U of the previous chunk (warps 0-1 need it; all threads keep the phase)
-        auto wait_mu = [&]() -> bool {
-            bool w = true;
-            if (warp < 2) w = wait_mma(bar_y, ph_y);
-            else ph_y ^= 1u;
-            mu_pending = false;
-            return w;
+            return wy && gated_ok;
         };
 
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1, kst = c % 3;
-            bool w = tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget);
-            w = w && tc::mbar_wait_bounded(bar_q + b, (c >> 1) & 1, a.budget);
+            const bool w = tc::mbar_wait_bounded(bar_full + b, (c >> 1) & 1, a.budget);
             if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (tid == 0) raise_error(kErrTimeout);
                 break;
@@ -792,74 +898,72 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const float gR = tid < 64 ? vb[64 + tid] : 0.f;
             const float fR = tid >= 64 ? vb[128 + tid - 64] : 0.f;
 
-            // [Q; -W] S over dk 0-63 (thread 0) is added onto [0; U~] already in COL_U[b]; dk 64-127
-            // (thread 32) goes to COL_1B.  Their sum: Q S in lanes 0-63, U = U~ - W S in lanes 64-127.
+            // [Q; -W] S over dk 0-63 (thread 0) into COL_U[b] and over dk 64-127 (thread 32) into
+            // COL_1B[b].  Their sum: Q S in lanes 0-63, -W S in lanes 64-127.  Then thread 0 queues
+            // the previous chunk's M U behind it.
+            bool wm = true;
             if (tid == 0 || tid == 32) {
                 const int hf = tid >> 5;
-                const uint64_t a0 = desc_add(dQW0, QWoff(b) + hf * Cf::QW_HALF);
+                const uint64_t a0 = desc_add(dQW0, QWoff(kst) + hf * Cf::QW_HALF);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(tmem + (hf ? Cf::COL_1B : Cf::COL_U + b * NS), desc_add(a0, kk * 32),
-                                desc_add(dSS0, (hf * 4 + kk) * 16 * Cf::ROWB), id_slab, hf == 0 || kk > 0);
+                    tc::mma_f16(tmem + (hf ? Cf::COL_1B : Cf::COL_U) + b * NS, desc_add(a0, kk * 32),
+                                desc_add(dSS0, (hf * 4 + kk) * 16 * Cf::ROWB), id_slab, kk > 0);
                 tc::mma_commit(hf ? bar_c2 : bar_c1);
+                if (tid == 0 && c > 0) wm = issue_mu(c - 1);
             }
-            c1_pending = c2_pending = true;
-            if (c > 0 && warp < 2) gz_prep();  // gated: gate factors of the previous chunk meanwhile
-            c1_pending = false;
-            const bool w1 = wait_mma(bar_c1, ph_c1);
-            c2_pending = false;
-            const bool w2 = wait_mma(bar_c2, ph_c2);
-            // The previous chunk's M U, then its y (warps 0-1), while warps 2-3 form U: the MMA front
-            // end is otherwise idle until the state MMA, so M U delays neither product of the chain.
-            bool wm = true, wy = true;
-            if (c > 0) {
-                wm = issue_mu(c - 1);
-                wy = wait_mu();
-                if (wy || GATED) y_epilogue();  // gated: the cluster exchange keeps step
-            }
-
-            {
+            bool w1 = true, w2 = true, wy = true;
+            if (warp >= 2) {
+                // U = U~ - W S (fp16, for M U), U' = f U (hi + lo, for K^T U'), then K^T U' at once
+                w1 = wait_mma(bar_c1, ph_c1);
+                w2 = wait_mma(bar_c2, ph_c2);
                 float d1[NS], d2[NS];
                 tc::tmem_ld32(trow + Cf::COL_U + b * NS, d1);
-                tc::tmem_ld32(trow + Cf::COL_1B, d2);
-                if (warp >= 2) {  // U (fp16, for M U), U' = f U (hi + lo, for K^T U')
-                    const int r = tid - 64;
-                    float ut[NS];
+                tc::tmem_ld32(trow + Cf::COL_1B + b * NS, d2);
+                const int r = tid - 64;
+                float ut[NS];
+                const uint8_t* urow = smem + Cf::OFF_UT + kst * 64 * Cf::ROWB + r * Cf::ROWB;
 #pragma unroll
-                    for (int j = 0; j < NS; ++j) ut[j] = d1[j] + d2[j];
-                    uint8_t* su = smem + Cf::OFF_SU + b * 64 * Cf::ROWB;
+                for (int cc = 0; cc < NS / 8; ++cc) {
+                    const uint4 u4 = *reinterpret_cast<const uint4*>(urow + 16 * cc);
+                    const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
-                    for (int cc = 0; cc < NS / 8; ++cc) {
-                        uint4 hi, lo;
-                        st16(su + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(ut + 8 * cc));
-                        float u2[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
-                        split8<BF>(u2, hi, lo);
-                        st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::UROWB), hi);
-                        st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc + NS / 8, Cf::UROWB), lo);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = unpack2<false>(uw[e]);
+                        ut[8 * cc + 2 * e] = f.x + d1[8 * cc + 2 * e] + d2[8 * cc + 2 * e];
+                        ut[8 * cc + 2 * e + 1] = f.y + d1[8 * cc + 2 * e + 1] + d2[8 * cc + 2 * e + 1];
                     }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < NS; ++j) qs[j] = d1[j] + d2[j];
                 }
-            }
-            if (warp < 2) gate_out();
-            if (!(ok = operands_ready(wm && wy && w1 && w2 && gated_ok))) break;  // also orders the staged rows
-            y_store();
-
-            // K^T U' -> state increment; its completion also releases slot b and K stage kst
-            if (tid == 0) {
-                const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
+                uint8_t* su = smem + Cf::OFF_SU + b * 64 * Cf::ROWB;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::UROWB), id_ds, kk > 0);
-                tc::mma_commit(bar_ds);
-                tc::mma_commit(bar_dsd + b);
+                for (int cc = 0; cc < NS / 8; ++cc) {
+                    uint4 hi, lo;
+                    st16(su + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(ut + 8 * cc));
+                    float u2[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
+                    split8<false>(u2, hi, lo);
+                    st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::UROWB), hi);
+                    st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc + NS / 8, Cf::UROWB), lo);
+                }
+                tc::fence_async_smem();
+                tc::tc_fence_before();
+                tc::bar_sync(BID_U, 64);
+                // K^T U' -> state increment; its completion also releases stage kst
+                if (tid == 64) {
+                    tc::tc_fence_after();
+                    const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::UROWB),
+                                    id_ds, kk > 0);
+                    tc::mma_commit(bar_ds);
+                    tc::mma_commit(bar_dsd + kst);
+                }
+            } else if (c > 0) {
+                wy = y_prev();  // warps 0-1: y of chunk c - 1 meanwhile
             }
-            ds_pending = false;
             const bool w3 = wait_mma(bar_ds, ph_ds);
-
             {
                 float t[NS], t2[NS];
                 tc::tmem_ld32(trow + Cf::COL_DS, t);
@@ -867,28 +971,24 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
 #pragma unroll
                 for (int j = 0; j < NS; ++j) S[j] = gC * S[j] + (t[j] + t2[j]);
 #pragma unroll
-                for (int cc = 0; cc < NS / 8; ++cc) st16(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB), pack8<BF>(S + 8 * cc));
+                for (int cc = 0; cc < NS / 8; ++cc) st16(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB), pack8<false>(S + 8 * cc));
             }
             py_c0 = c0;
             py_L = L;
             py_g = gR;
             py_x = c;
-            if (tid == 0) tc::bulk_wait_read0();  // YS is free before the next staging writes it
-            if (!(ok = operands_ready(w3))) break;
+            if (!(ok = operands_ready(wm && w1 && w2 && wy && w3))) break;
         }
         if (ok && nchunks > 0) {  // the last chunk's M U and y
-            if (warp < 2) gz_prep();
-            const bool wm = issue_mu(nchunks - 1);
-            const bool wy = wait_mu();
-            if (wy || GATED) y_epilogue();
-            if (warp < 2) gate_out();
-            if ((ok = operands_ready(wm && wy && gated_ok))) y_store();
+            bool wm = true;
+            if (tid == 0) wm = issue_mu(nchunks - 1);
+            bool wy = true;
+            if (warp < 2) wy = y_prev();
+            ok = tc::bar_and(BID, 128, wm && wy);
         }
-        // never free TMEM under an MMA in flight
-        if (c1_pending) tc::mbar_wait_bounded(bar_c1, ph_c1, 4000000000ull);
-        if (c2_pending) tc::mbar_wait_bounded(bar_c2, ph_c2, 4000000000ull);
-        if (ds_pending) tc::mbar_wait_bounded(bar_ds, ph_ds, 4000000000ull);
-        if (mu_pending) tc::mbar_wait_bounded(bar_y, ph_y, 4000000000ull);
+        // every MMA of the three issuing threads has completed before TMEM is freed
+        if (tid == 0 || tid == 32 || tid == 64) tc::mma_commit(bar_drain);
+        tc::mbar_wait_bounded(bar_drain, 0, 4000000000ull);
         if (tid == 0) tc::bulk_wait0();
         if (GATED && warp < 2) {
             // the rest of the cluster protocol after an early exit: send the chunks not sent (zeros),
@@ -906,44 +1006,40 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         }
     } else {
         // =============================== producer group ================================
+        // Copies and conversions only: every product of the chunk that does not involve the state
+        // (-W, U~, M) comes from chunk_ut_kernel's record.
         constexpr int BID = 2;
         const int it = tid - 128;
         tc::wait_prerequisites();  // the records of chunk_ut_kernel are complete and visible
-        uint32_t ph_w = 0, ph_u = 0;
         bool ok = true;
-        constexpr uint32_t id_v = idesc16<false>(128, NS, false, true);  // T_u V in fp16
-        constexpr uint32_t id_w = idesc16<BF>(128, 128, false, true);
-        const uint64_t dTT0 = tc::smem_desc(sbase + Cf::OFF_TT, 16, 1024, tc::kSw128);
-        const uint64_t dV0 = tc::smem_desc(sbase + Cf::OFF_VS, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-        const uint64_t dK0 = tc::smem_desc(sbase + Cf::OFF_KS, Cf::K_HALF, 1024, tc::kSw128);  // MN-major K
 
         // copies are issued by one thread of warp 6, which has no part in the gate arithmetic
         constexpr int kIssuer = 64;
         // copies in flight into this CTA's shared memory, for the exit drain
-        int kv_issued = -1, kv_landed = -1, tt_issued = -1, tt_landed = -1;
-        int q_last0 = -1, q_last1 = -1, m_last0 = -1, m_last1 = -1;
+        int k_issued = -1, k_landed = -1, op_issued = -1, op_landed = -1;
+        int m_last0 = -1, m_last1 = -1;
         auto rec_ptr = [&](int ci) {
             return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
         };
-        auto issue_kv = [&](int ci) {  // K and the V slab of chunk ci -> stage ci % 3
-            kv_issued = ci;
+        // K of chunk ci -> stage ci % 3; Q of ci -> rows 0-63 of [Q;-W] stage ci % 3, -W of ci (record)
+        // -> rows 64-127, this slab's U~ (record) -> U~ stage ci % 3
+        auto issue_stage = [&](int ci) {
+            k_issued = op_issued = ci;
             if (it != kIssuer) return;
             const int c0 = t_begin + ci * kChunk, s = ci % 3;
             uint64_t* bk = bar_kv + s;
-            tc::mbar_arrive_expect_tx(bk, Cf::KV_TX);
+            tc::mbar_arrive_expect_tx(bk, Cf::K_TX);
             tc::tma_load_3d(smem + Koff(s), &maps.k, 0, h, c0, bk);
             tc::tma_load_3d(smem + Koff(s) + Cf::K_HALF, &maps.k, 64, h, c0, bk);
-            tc::tma_load_3d(smem + Voff(s), &maps.v, slab * NS, h, c0, bk);
-        };
-        auto issue_q = [&](int ci) {  // Q of chunk ci -> rows 0-63 of [Q;W] slot ci & 1
-            const int bb = ci & 1;
-            (bb ? q_last1 : q_last0) = ci;
-            if (it != kIssuer) return;
-            const int c0 = t_begin + ci * kChunk;
-            uint8_t* qw = smem + QWoff(bb);
-            tc::mbar_arrive_expect_tx(bar_q + bb, Cf::Q_TX);
-            tc::tma_load_3d(qw, &maps.q, 0, h, c0, bar_q + bb);
-            tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bar_q + bb);
+            uint8_t* qw = smem + QWoff(s);
+            const uint8_t* rp = rec_ptr(ci);
+            tc::mbar_arrive_expect_tx(bar_q + s, Cf::OP_TX);
+            tc::tma_load_3d(qw, &maps.q, 0, h, c0, bar_q + s);
+            tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bar_q + s);
+            tc::bulk_g2s(qw + 64 * 128, rp + kRecW, 8192, bar_q + s);
+            tc::bulk_g2s(qw + Cf::QW_HALF + 64 * 128, rp + kRecW + 8192, 8192, bar_q + s);
+            tc::bulk_g2s(smem + Cf::OFF_UT + s * 64 * Cf::ROWB, rp + kRecU + slab * kRecUSlab, 64 * Cf::ROWB,
+                         bar_q + s);
         };
         auto issue_m = [&](int ci) {  // M of chunk ci -> M slot ci & 1 (issuer thread only)
             const int bb = ci & 1;
@@ -954,15 +1050,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 tc::tma_load_3d(smem + Cf::OFF_ZS + bb * 64 * Cf::ROWB, &maps.z, slab * NS, h, t_begin + ci * kChunk,
                                 bar_m + bb);
         };
-        auto issue_tt = [&](int ci) {  // T_w (twice) and T_u of chunk ci -> TT rows 0-127, 192-255
-            tt_issued = ci;
-            if (it != kIssuer) return;
-            tc::mbar_arrive_expect_tx(bar_tt, 3 * 8192);
-            tc::bulk_g2s(smem + Cf::OFF_TT, rec_ptr(ci) + kRecTw, 8192, bar_tt);
-            tc::bulk_g2s(smem + Cf::OFF_TT + 8192, rec_ptr(ci) + kRecTw, 8192, bar_tt);
-            tc::bulk_g2s(smem + Cf::OFF_TT + 24576, rec_ptr(ci) + kRecTu, 8192, bar_tt);
-        };
-        // g of chunk ci (beta is already inside T_w, T_u) -> vec(ci & 1)[192:256] by cp.async, two
+        // g of chunk ci (beta is already inside -W, U~ and M) -> vec(ci & 1)[192:256] by cp.async, two
         // chunks ahead, so no thread waits on the load; one cp.async group per chunk (warps 4-5)
         auto load_gates = [&](int ci) {
             if (it < 64 && ci < nchunks) {
@@ -972,21 +1060,12 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             if (it < 64) tc::cp_async_commit();
         };
-        // TT rows 128-191 stay zero: A = [0; T_u] leaves lanes 0-63 of the U~ accumulator at zero
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            st16(smem + Cf::OFF_TT + 16384 + (it + 128 * i) * 16, make_uint4(0, 0, 0, 0));
-        tc::fence_async_smem();
         if (it == kIssuer) {
             tc::prefetch_tmap(&maps.k);
             tc::prefetch_tmap(&maps.q);
-            tc::prefetch_tmap(&maps.v);
             if constexpr (GATED) tc::prefetch_tmap(&maps.z);
         }
-        if (nchunks > 0) {
-            issue_kv(0);
-            issue_tt(0);
-        }
+        if (nchunks > 0) issue_stage(0);
         load_gates(0);
         load_gates(1);
 
@@ -994,14 +1073,17 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             const int b = c & 1, kst = c % 3;
             const int c0 = t_begin + c * kChunk, L = min(kChunk, t_end - c0);
             float* vb = vec(b);
-            // slot b, U~ columns b and K stage (c + 1) % 3 are free once the state MMA of c - 2 is done
-            bool w = tc::mbar_wait_bounded(bar_dsd + b, ((c >> 1) & 1) ^ 1, a.budget);
-            if (!(ok = tc::bar_and(BID, 128, w))) {
-                if (it == 0) raise_error(kErrTimeout);
-                break;
+            // the copies of chunk c + 1 go into stage (c + 1) % 3 once chunk c - 2's state MMA, the
+            // last reader of that stage, is done: two chain periods of lead
+            if (c + 1 < nchunks) {
+                bool w = true;
+                if (c >= 2) w = tc::mbar_wait_bounded(bar_dsd + (c - 2) % 3, ((c - 2) / 3) & 1, a.budget);
+                if (!(ok = tc::bar_and(BID, 128, w))) {
+                    if (it == 0) raise_error(kErrTimeout);
+                    break;
+                }
+                issue_stage(c + 1);
             }
-            issue_q(c);
-            if (c + 1 < nchunks) issue_kv(c + 1);
 
             // ---- gates of chunk c (warps 4-5): gamma (inclusive prefix sum), Gamma,
             //      f = exp(gamma_C - gamma) -----------------------------------------------------------
@@ -1026,77 +1108,20 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 vb[128 + it] = __expf(vb[63] - vb[it]);
             }
 
-            // ---- W = T_w K (thread 0; both lane halves) and U~ = T_u V (thread 32; lanes 64-127),
-            //      two issuers with their own commits ---------------------------------------------------
-            w = tc::mbar_wait_bounded(bar_kv + kst, (c / 3) & 1, a.budget);
-            w = w && tc::mbar_wait_bounded(bar_tt, c & 1, a.budget);
+            // ---- K(c), Q(c), -W(c), U~(c) landed; bf16 K and Q -> fp16 in place ---------------------
+            bool w = tc::mbar_wait_bounded(bar_kv + kst, (c / 3) & 1, a.budget);
+            w = w && tc::mbar_wait_bounded(bar_q + kst, (c / 3) & 1, a.budget);
             if (!(ok = tc::bar_and(BID, 128, w))) {
                 if (it == 0) raise_error(kErrTimeout);
                 break;
             }
-            kv_landed = c;
-            tt_landed = c;
-            if constexpr (BF) {  // V slab bf16 -> fp16 in place (exact for every normal value)
-                uint8_t* vs = smem + Voff(kst);
-#pragma unroll
-                for (int i = 0; i < (64 * Cf::ROWB) / (16 * 128); ++i) {
-                    uint4* p16 = reinterpret_cast<uint4*>(vs + (it + 128 * i) * 16);
-                    const uint4 u = *p16;
-                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-                    uint32_t o4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = unpack2<true>(w4[e]);
-                        o4[e] = pack2<false>(f.x, f.y);
-                    }
-                    *p16 = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-                }
-                tc::fence_async_smem();
-                tc::bar_sync(BID, 128);
-            }
-            tc::tc_fence_after();
-            if (it == 0) {
-                const uint64_t bk0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(tmem + Cf::COL_W, desc_add(dTT0, kk * 32), desc_add(bk0, kk * 2048), id_w, kk > 0);
-                tc::mma_commit(bar_p);
-            } else if (it == 32) {  // [0; T_u] V (fp16): lanes 0-63 zero, lanes 64-127 U~
-                const uint64_t bv0 = desc_add(dV0, Voff(kst) - Cf::OFF_VS);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc::mma_f16(tmem + Cf::COL_U + b * NS, desc_add(dTT0, 16384 + kk * 32),
-                                desc_add(bv0, kk * 16 * Cf::ROWB), id_v, kk > 0);
-                tc::mma_commit(bar_p2);
-            }
-            bool ww = tc::mbar_wait_bounded(bar_p, ph_w, a.budget);
-            if (!ww) {
-                raise_error(kErrTimeout);
-                tc::mbar_wait_bounded(bar_p, ph_w, 4000000000ull);
-            }
-            ph_w ^= 1u;
-            bool wu = tc::mbar_wait_bounded(bar_p2, ph_u, a.budget);
-            if (!wu) {
-                raise_error(kErrTimeout);
-                tc::mbar_wait_bounded(bar_p2, ph_u, 4000000000ull);
-            }
-            ph_u ^= 1u;
-            tc::tc_fence_after();
-            if (!(ok = tc::bar_and(BID, 128, ww && wu))) break;
-            if (c + 1 < nchunks) issue_tt(c + 1);  // the MMAs have read TT
-
-            // ---- -W -> rows 64-127 of [Q; -W] in slot b: lanes 0-63 write columns 0-63, lanes 64-127
-            //      columns 64-127 (each lane half of the accumulator holds all of W) ------------------
-            {
-                const int r = it & 63, hf = it >> 6;
-                float wv[64];
-                tc::tmem_ld32(trow + Cf::COL_W + 64 * hf, wv);
-                tc::tmem_ld32(trow + Cf::COL_W + 64 * hf + 32, wv + 32);
-#pragma unroll
-                for (int j = 0; j < 64; ++j) wv[j] = -wv[j];
-                uint8_t* qw = smem + QWoff(b) + hf * Cf::QW_HALF;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) st16(qw + tc::swz_off(64 + r, cc, 128), pack8<BF>(wv + 8 * cc));
+            k_landed = op_landed = c;
+            if constexpr (BF) {
+                // bf16 -> fp16 is exact for |x| >= 2^-14; the smaller entries of a unit-norm key or
+                // query lose at most 2^-25 absolute
+                to_f16_inplace(smem + Koff(kst), 2 * Cf::K_HALF, it);
+                to_f16_inplace(smem + QWoff(kst), 64 * 128, it);               // Q rows of half 0
+                to_f16_inplace(smem + QWoff(kst) + Cf::QW_HALF, 64 * 128, it);  // Q rows of half 1
             }
             tc::fence_async_smem();
             tc::tc_fence_before();
@@ -1112,12 +1137,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         }
         if (it < 64) tc::cp_async_wait<0>();  // no copy into shared memory left in flight
         // never leave with copies into this CTA's shared memory in flight
-        if (kv_issued > kv_landed) tc::mbar_wait_bounded(bar_kv + kv_issued % 3, (kv_issued / 3) & 1, 4000000000ull);
-        if (kv_issued > kv_landed + 1)
-            tc::mbar_wait_bounded(bar_kv + (kv_issued - 1) % 3, ((kv_issued - 1) / 3) & 1, 4000000000ull);
-        if (tt_issued > tt_landed) tc::mbar_wait_bounded(bar_tt, tt_issued & 1, 4000000000ull);
-        if (q_last0 >= 0) tc::mbar_wait_bounded(bar_q + 0, (q_last0 >> 1) & 1, 4000000000ull);
-        if (q_last1 >= 0) tc::mbar_wait_bounded(bar_q + 1, (q_last1 >> 1) & 1, 4000000000ull);
+        for (int ci = max(k_landed + 1, 0); ci <= k_issued; ++ci)  // at most two outstanding
+            tc::mbar_wait_bounded(bar_kv + ci % 3, (ci / 3) & 1, 4000000000ull);
+        for (int ci = max(op_landed + 1, 0); ci <= op_issued; ++ci)
+            tc::mbar_wait_bounded(bar_q + ci % 3, (ci / 3) & 1, 4000000000ull);
         if (m_last0 >= 0) tc::mbar_wait_bounded(bar_m + 0, (m_last0 >> 1) & 1, 4000000000ull);
         if (m_last1 >= 0) tc::mbar_wait_bounded(bar_m + 1, (m_last1 >> 1) & 1, 4000000000ull);
         (void)ok;
@@ -1145,11 +1168,11 @@ inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, 
     const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
     if (nvc > 0) {
         LaunchScope timed(st, "chunk_ut_kernel");
-        chunk_ut_kernel<BF><<<(unsigned)(nvc * a.H), 128, UtCfg::BYTES, st>>>(a, maps);
+        chunk_ut_kernel<BF><<<(unsigned)(nvc * a.H), UtCfg::THREADS, UtCfg::BYTES, st>>>(a, maps);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    const unsigned grid = (unsigned)(a.num_seqs * a.H * (128 / NS));
+    const unsigned grid = (unsigned)((long long)a.num_seqs * a.H * (128 / NS));  // <= 2^31 (host check)
     // Programmatic dependent launch: the chain's prologue overlaps the tail of chunk_ut_kernel;
     // its producer waits for that grid before reading a record.  Gated: the 128 / NS slab CTAs
     // of a (sequence, head) form one cluster.
@@ -1193,7 +1216,7 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
     ChainMaps maps = {};  // the z map stays empty without the gate
     if (!encode_map_3d(&maps.k, a.k, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.q, a.q, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, 128, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_map_3d(&maps.v, a.v, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.y, gated ? a.out : a.y, st_dt, a.N, a.H, 128, NS, kChunk, yswz) ||
         (gated && !encode_map_3d(&maps.z, a.z, a.z_dt, a.N, a.H, 128, NS, kChunk, CU_TENSOR_MAP_SWIZZLE_64B))) {
         *why = "cuTensorMapEncodeTiled failed";

@@ -101,9 +101,9 @@ def test_workspace_size_is_zero_without_records(L):
 
 
 def test_workspace_size_covers_every_chunk(L):
-    # one 24 KB record per (64-token chunk, head); packed sequences add one partial chunk each
-    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 24576
-    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 24576
+    # one 40 KB record per (64-token chunk, head); packed sequences add one partial chunk each
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 40960
+    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 40960
     assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0
 
 
@@ -153,3 +153,20 @@ def test_timing_rejects_bad_use(L):
     assert L.gdn_timing_start(1 << 21) == gdn.GDN_ERR_INVALID_ARG
     # stopping while timing is off is an argument error, with or without a device
     assert L.gdn_timing_stop(0, None, None, None, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(W=0), dict(W=9), dict(x_q=None), dict(dk=48), dict(conv=None),
+                                  dict(l2=-1.0), dict(num_slots=1), dict(out=MIS)])
+def test_mixer_decode_rejects_bad_arguments(L, over):
+    a = dict(W=4, x_q=A, dk=128, conv=A, l2=1e-6, num_slots=4, out=A)
+    a.update(over)
+    st = L.gdn_mixer_decode_step(a["x_q"], A, A, A, A, A, a["W"], A, A, A, A, A, A, a["l2"], 1e-6, a["conv"], A,
+                                 None, a["num_slots"], 4, 2, a["dk"], 128, 1.0, 1, 1, a["out"], None)
+    assert st == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_mixer_decode_without_history_needs_no_conv_state(L):
+    """conv width 1 keeps no history: a NULL conv_state passes validation (nothing launched
+    for zero rows)."""
+    assert L.gdn_mixer_decode_step(A, A, A, A, A, A, 1, A, A, A, A, A, A, 1e-6, 1e-6, None, A, None, 4, 0, 2, 128,
+                                   128, 1.0, 1, 1, A, None) == gdn.GDN_OK
