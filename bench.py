@@ -470,7 +470,60 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
                 "gpu_launches": sum(k["launches"] for k in km)}
 
 
-WORKLOADS = {"decode": wl_decode, "long": wl_long, "mixer": wl_mixer}
+def wl_mixer_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    """full-mixer decode: 256 sequences x H=32, d=128, conv width 4, 100 steps of
+    gdn_mixer_decode_step (conv history, prep, recurrence and out gate in one kernel), the fp32
+    state and the conv history updated in place."""
+    c = inputs.WORKLOAD_SPECS[inputs.DECODE]
+    B, H, d, W = c["B"], c["H"], 128, 4
+    seed = rank_seed(inputs.SEED_BASE + inputs.DECODE, rank)
+    state = inputs.make_decode_state(inputs.DECODE, "cuda", seed=seed)
+    m = inputs.make_mixer(inputs.MIXER, "cuda", seed=seed, lengths=[B], H=H)  # weights and one token of inputs
+    gen = torch.Generator(device="cuda").manual_seed(seed + 5)
+    conv = (torch.randn(B, W - 1, H, 3 * d, device="cuda", generator=gen)).to(torch.bfloat16)
+    steps_in = []
+    for s in range(c["steps"]):
+        x = inputs.make_mixer(inputs.MIXER, "cuda", seed=seed * 1000 + s, lengths=[B], H=H)
+        steps_in.append({k: x[k] for k in ("x_q", "x_k", "x_v", "beta_logit", "alpha_logit", "z")})
+    out = torch.empty(B, H, d, device="cuda", dtype=torch.bfloat16)
+
+    def dec(i):
+        for x in steps_in:
+            gdn.mixer_decode_step(x["x_q"], x["x_k"], x["x_v"], m["w_q"], m["w_k"], m["w_v"], x["beta_logit"],
+                                  x["alpha_logit"], m["A_log"], m["alpha_bias"], x["z"], m["norm_w"], conv, state,
+                                  l2_eps=m["eps"], rms_eps=m["eps"], out=out)
+
+    barrier(torch, dist, world)
+    dt_eager = max_over_ranks(torch, dist, timed(torch, dec, 3, 1, stream, on_start=lambda: gdn.timing_start(4096)),
+                              world)
+    kd = kernel_table(gdn.timing_stop(), 3)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        dec(0)
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(graph):
+        dec(0)
+    barrier(torch, dist, world)
+    dt = max_over_ranks(torch, dist, timed(torch, lambda i: graph.replay(), 3, 1, stream), world)
+    del graph
+    per_launch = dt / (3 * c["steps"])
+    upd = B * H
+    # per (row, head): fp32 state read + write, conv history read + write, the token's q/k/v
+    # projections, two logits, z, out (all bf16)
+    bytes_l = upd * (2 * d * d * 4 + 2 * (W - 1) * 3 * d * 2 + 3 * d * 2 + 2 * 2 + d * 2 + d * 2)
+    return {"workload": f"mixer_decode_B{B}_H{H}_d{d}_W{W}_x100", "value": upd * world / per_launch,
+            "unit": "state-updates/s", "us_per_step": per_launch * 1e6, "launch": "CUDA graph of the 100 steps",
+            "eager_us_per_step": dt_eager / (3 * c["steps"]) * 1e6,
+            "roofline": {"bound": "hbm", "achieved": bytes_l / per_launch / 1e9, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": bytes_l / per_launch / 1e9 / hbm_peak,
+                         "kernel": "mixer_decode_kernel", "alg_bytes_per_launch": bytes_l,
+                         "kernel_avg_us": kd[0]["avg_us"] if kd else None},
+            "gpu_launches": 3 * c["steps"]}
+
+
+WORKLOADS = {"decode": wl_decode, "long": wl_long, "mixer": wl_mixer, "mixer_decode": wl_mixer_decode}
 
 
 def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
@@ -488,7 +541,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true")
-    ap.add_argument("--only", choices=["decode", "long", "mixer"], default=None,
+    ap.add_argument("--only", choices=["decode", "long", "mixer", "mixer_decode"], default=None,
                     help="run one secondary workload alone and print its line (profiling aid)")
     ap.add_argument("--cpu-s", type=float, default=12.0, help="target seconds of the CPU-baseline sample")
     ap.add_argument("--ref-step-s", type=float, default=8.0)

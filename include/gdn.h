@@ -225,6 +225,31 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const 
                              gdn_dtype_t y_dtype, void* y, gdn_stream_t stream);
 
 /*
+ * gdn_mixer_decode_step -- one token per row through the whole mixer of section 2.1.1, one
+ * kernel: eqs. (6)-(10) on the token's projection outputs and the row's causal conv history,
+ * eqs. (1)-(4) against the resident state, and eq. (11)'s output gate (without W_o).  q, k, v
+ * stay in fp32 inside the kernel (never stored).
+ *   x_q, x_k [B,H,dk], x_v [B,H,dv], beta_logit, alpha_logit [B,H], z [B,H,dv]: in_dtype.
+ *   conv_w_q, conv_w_k [H*dk, W], conv_w_v [H*dv, W] fp32 (W = conv_width in [1, 8]; tap W-1
+ *     meets the current token, as in gdn_prep); A_log, alpha_bias [H] fp32; norm_w [dv] fp32.
+ *   conv_state [num_slots, W-1, H, 2*dk + dv] in_dtype: for each slot the W-1 previous raw
+ *     inputs, oldest first, each one head's q channels, then k, then v.  Read and shifted in
+ *     place: afterwards it holds the W-1 newest inputs, the current one last.  A new sequence
+ *     starts from zeros (the zero history of a sequence start).  May be NULL when W = 1.
+ *   state [num_slots,H,dk,dv] fp32, in place; state_slot as in gdn_decode_step (row b uses slot
+ *     state_slot[b] of both state and conv_state).
+ *   out [B,H,dv]: out_dtype.  l2_eps inside the L2Norm square root, rms_eps inside the RMSNorm
+ *   one; scale multiplies the readout as in gdn_chunk_fwd.
+ */
+gdn_status_t gdn_mixer_decode_step(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
+                                   const float* conv_w_k, const float* conv_w_v, int conv_width,
+                                   const void* beta_logit, const void* alpha_logit, const float* A_log,
+                                   const float* alpha_bias, const void* z, const float* norm_w, float l2_eps,
+                                   float rms_eps, void* conv_state, float* state, const int32_t* state_slot,
+                                   int num_slots, int B, int H, int dk, int dv, float scale, gdn_dtype_t in_dtype,
+                                   gdn_dtype_t out_dtype, void* out, gdn_stream_t stream);
+
+/*
  * gdn_out_gate -- eq. (11) without the output projection W_o:
  *   out = sigmoid(z) * y / sqrt(mean_dv(y^2) + eps) * (1 + norm_w)
  * per (token, head) over dv; norm_w [dv] fp32 is shared by all heads (the

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "launch_timer.cuh"
 #include "decode.cuh"
+#include "mixer_decode.cuh"
 #include "out_gate.cuh"
 #include "prep.cuh"
 #include "recurrent.cuh"
@@ -97,6 +98,16 @@ struct DecodeLaunch {
         gdn::decode_step_kernel<DK, DV><<<(unsigned)(B * H), Sh::THREADS, 0, st>>>(
             q, k, v, g, beta, state, slot, num_slots, H, scale, in_dt, y_dt, y);
         return launched("decode_step_kernel");
+    }
+};
+
+template <int DK, int DV>
+struct MixerDecodeLaunch {
+    static gdn_status_t run(const gdn::MixerDecodeArgs& args, int B, cudaStream_t st) {
+        using Sh = gdn::DecodeShape<DK, DV>;
+        gdn::LaunchScope timed(st, "mixer_decode_kernel");
+        gdn::mixer_decode_kernel<DK, DV><<<(unsigned)(B * args.H), Sh::THREADS, 0, st>>>(args);
+        return launched("mixer_decode_kernel");
     }
 };
 
@@ -291,6 +302,34 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, const 
     REQUIRE_PTR(beta, "beta"); REQUIRE_PTR(state, "state"); REQUIRE_PTR(y, "y"); OPT_PTR(state_slot, "state_slot");
     return dispatch_dims<DecodeLaunch>(dk, dv, q, k, v, g, beta, state, state_slot, num_slots, B, H, scale,
                                        (int)in_dtype, (int)y_dtype, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status_t gdn_mixer_decode_step(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
+                                   const float* conv_w_k, const float* conv_w_v, int conv_width,
+                                   const void* beta_logit, const void* alpha_logit, const float* A_log,
+                                   const float* alpha_bias, const void* z, const float* norm_w, float l2_eps,
+                                   float rms_eps, void* conv_state, float* state, const int32_t* state_slot,
+                                   int num_slots, int B, int H, int dk, int dv, float scale, gdn_dtype_t in_dtype,
+                                   gdn_dtype_t out_dtype, void* out, gdn_stream_t stream) {
+    REQUIRE(B >= 0 && H >= 1 && num_slots >= 0, "bad sizes B=%d H=%d num_slots=%d", B, H, num_slots);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(out_dtype), "bad dtype");
+    REQUIRE(conv_width >= 1 && conv_width <= 8, "conv_width=%d not in [1, 8]", conv_width);
+    REQUIRE(l2_eps >= 0.f && rms_eps >= 0.f, "eps < 0");
+    REQUIRE(state_slot != nullptr || num_slots >= B, "num_slots=%d < B=%d without state_slot", num_slots, B);
+    REQUIRE((long long)B * H <= 0x7fffffffLL, "B*H too large");
+    if (B == 0) return GDN_OK;
+    REQUIRE_PTR(x_q, "x_q"); REQUIRE_PTR(x_k, "x_k"); REQUIRE_PTR(x_v, "x_v");
+    REQUIRE_PTR(conv_w_q, "conv_w_q"); REQUIRE_PTR(conv_w_k, "conv_w_k"); REQUIRE_PTR(conv_w_v, "conv_w_v");
+    REQUIRE_PTR(beta_logit, "beta_logit"); REQUIRE_PTR(alpha_logit, "alpha_logit");
+    REQUIRE_PTR(A_log, "A_log"); REQUIRE_PTR(alpha_bias, "alpha_bias"); REQUIRE_PTR(z, "z");
+    REQUIRE_PTR(norm_w, "norm_w"); REQUIRE_PTR(state, "state"); REQUIRE_PTR(out, "out");
+    if (conv_width > 1) REQUIRE_PTR(conv_state, "conv_state");
+    OPT_PTR(state_slot, "state_slot");
+    const gdn::MixerDecodeArgs args{x_q, x_k, x_v, conv_w_q, conv_w_k, conv_w_v, conv_width, beta_logit,
+                                    alpha_logit, A_log, alpha_bias, z, norm_w, l2_eps, rms_eps, conv_state,
+                                    state, state_slot, num_slots, H, scale, (int)in_dtype, (int)out_dtype, out};
+    return dispatch_dims<MixerDecodeLaunch>(dk, dv, args, B, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t gdn_chunk_fwd_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk) {

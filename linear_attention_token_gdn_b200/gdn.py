@@ -37,6 +37,8 @@ SIGNATURES = {
                              _P, _P, _Z, _P], _I),
     "gdn_chunk_fwd_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P], _I),
     "gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P], _I),
+    "gdn_mixer_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _F, _F, _P, _P, _P, _I, _I,
+                               _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
     "gdn_timing_start": ([_I], _I),
     "gdn_timing_stop": ([_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double),
@@ -235,6 +237,24 @@ def decode_step(q, k, v, g, beta, state, state_slot=None, scale=1.0, y_dtype=Non
                                  state.shape[0], B, H, dk, dv, float(scale), _dt(q), _DT[y.dtype], _ptr(y),
                                  _stream(stream)))
     return y
+
+
+def mixer_decode_step(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bias, z, norm_w,
+                      conv_state, state, state_slot=None, l2_eps=1e-6, rms_eps=1e-6, scale=1.0, out_dtype=None,
+                      out=None, stream=None):
+    """gdn_mixer_decode_step: one token per row through the whole mixer; ``conv_state``
+    [slots, W-1, H, 2 dk + dv] and ``state`` are updated in place.  Returns out [B, H, dv]."""
+    B, H, dk = x_q.shape
+    dv = x_v.shape[2]
+    W = w_q.shape[1]
+    if out is None:
+        out = torch.empty(B, H, dv, device=x_q.device, dtype=x_q.dtype if out_dtype is None else out_dtype)
+    _check(lib().gdn_mixer_decode_step(_ptr(x_q), _ptr(x_k), _ptr(x_v), _ptr(w_q), _ptr(w_k), _ptr(w_v), W,
+                                       _ptr(beta_logit), _ptr(alpha_logit), _ptr(A_log), _ptr(alpha_bias), _ptr(z),
+                                       _ptr(norm_w), float(l2_eps), float(rms_eps), _ptr(conv_state), _ptr(state),
+                                       _ptr(state_slot), state.shape[0], B, H, dk, dv, float(scale), _dt(x_q),
+                                       _DT[out.dtype], _ptr(out), _stream(stream)))
+    return out
 
 
 def out_gate(y, z, norm_w, eps=1e-6, out=None, stream=None):
