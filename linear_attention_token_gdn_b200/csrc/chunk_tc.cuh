@@ -19,12 +19,14 @@
 //                       the decay masks, and the unit-lower-triangular inverse T in fp32 on the
 //                       CUDA cores; then one N = 256 product [T_w; T_u] [K | V] with
 //                       T_w = T diag(beta Gamma) and T_u = T diag(beta) gives W = T_w K and
-//                       U~ = T_u V.  Writes a 40 KB record per (chunk, head): -W and M in the
-//                       128B-swizzled operand layout and U~ as four 32-column slabs, all fp16.
+//                       U~ = T_u V.  Writes a 40.5 KB record per (chunk, head): -W and M in the
+//                       128B-swizzled operand layout and U~ as four 32-column slabs, all fp16,
+//                       and the chunk's gates Gamma_r and Gamma_C / Gamma_r in fp32.
 //   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
 //                       the chunks.  A producer warpgroup only copies: each chunk's K and Q by
-//                       TMA, -W, U~ and M from the record by bulk copies, straight into operand
-//                       slots (bf16 K and Q converted to fp16 in place).  A chain warpgroup
+//                       TMA, -W, U~, M and the gates from the record by bulk copies, straight into
+//                       operand slots (bf16 K and Q converted to fp16 in place), one chunk ahead
+//                       of the chain.  A chain warpgroup
 //                       carries the fp32 state (one row per thread) through two dependent
 //                       tensor-core round trips per chunk:
 //                           [Q; -W] S        -> Q S and -W S, so U = U~ - W S
@@ -47,8 +49,8 @@
 // chain runs on fp16 operands (11 significant bits): bf16 q, k and v are converted to fp16 in
 // shared memory when they land (exact for |x| >= 2^-14), and their partners T_w, W, S and U'
 // are formed in fp16.  bf16 partners (8 bits) would let the error of a row whose y is small
-// exceed the bound once eq. (11) normalises that row.  U' enters as a rounded high half plus
-// its remainder, side by side in one N = 64 operand.
+// exceed the bound once eq. (11) normalises that row.  U' = f U enters as one fp16 value (the
+// state's error stays near 5e-4 of its scale, well inside the bound).
 // Operand tiles use the 128B / 64B swizzled canonical layouts, so one tile serves as K-major
 // or MN-major operand.  Every wait is bounded (ChunkArgs::budget clock cycles); a wait that
 // runs out sets the device error word, lets in-flight MMAs and copies drain, and the CTA
@@ -98,7 +100,8 @@ constexpr int kRecW = 0;           // -W: two dk halves, each [64 rows x 128 B] 
 constexpr int kRecM = 16384;       // M: [64 rows x 128 B] 128B-swizzled K-major
 constexpr int kRecU = 24576;       // U~: four 32-column dv slabs, each [64 rows x 64 B] row-major
 constexpr int kRecUSlab = 4096;
-constexpr int kRecBytes = 40960;
+constexpr int kRecG = 40960;       // Gamma_r = exp(gamma_r) [64] then f_r = exp(gamma_C - gamma_r) [64], fp32
+constexpr int kRecBytes = 41472;
 
 // Upper bound of the number of 64-token chunks over all sequences (the records the workspace
 // holds); it holds for every valid cu_seqlens.
@@ -181,20 +184,6 @@ __device__ __forceinline__ uint4 pack8(const float* x) {
     return make_uint4(pack2<BF>(x[0], x[1]), pack2<BF>(x[2], x[3]), pack2<BF>(x[4], x[5]), pack2<BF>(x[6], x[7]));
 }
 
-// x = hi + lo + O(2^-16 |x|) for bf16 (2^-22 for fp16): hi = round(x), lo = round(x - hi).
-template <bool BF>
-__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
-    uint32_t h[4], l[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        h[i] = pack2<BF>(x[2 * i], x[2 * i + 1]);
-        const float2 f = unpack2<BF>(h[i]);
-        l[i] = pack2<BF>(x[2 * i] - f.x, x[2 * i + 1] - f.y);
-    }
-    hi = make_uint4(h[0], h[1], h[2], h[3]);
-    lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
 template <bool BF>
 __host__ __device__ constexpr uint32_t idesc16(int M, int N, bool a_mn, bool b_mn) {
     return BF ? tc::idesc_bf16(M, N, a_mn, b_mn) : tc::idesc_f16(M, N, a_mn, b_mn);
@@ -202,21 +191,26 @@ __host__ __device__ constexpr uint32_t idesc16(int M, int N, bool a_mn, bool b_m
 
 __device__ __forceinline__ void st16(uint8_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
 
-// bytes (a multiple of 16 * NT) of bf16 values at p rewritten as fp16, 16 bytes per thread per
-// pass over NT threads (it = the thread's index among them).
-template <int NT = 128>
-__device__ __forceinline__ void to_f16_inplace(uint8_t* p, int bytes, int it) {
-    for (int off = it * 16; off < bytes; off += NT * 16) {
-        uint4* p16 = reinterpret_cast<uint4*>(p + off);
-        const uint4 u = *p16;
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+// BYTES (a multiple of 16 * NT) of bf16 values at p rewritten as fp16, 16 bytes per thread per
+// pass over NT threads (it = the thread's index among them), every load issued before the first
+// conversion.
+template <int NT, int BYTES>
+__device__ __forceinline__ void to_f16_block(uint8_t* p, int it) {
+    static_assert(BYTES % (16 * NT) == 0, "whole passes");
+    constexpr int ITER = BYTES / (16 * NT);
+    uint4 u[ITER];
+#pragma unroll
+    for (int k = 0; k < ITER; ++k) u[k] = *reinterpret_cast<const uint4*>(p + (it + k * NT) * 16);
+#pragma unroll
+    for (int k = 0; k < ITER; ++k) {
+        const uint32_t w4[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
         uint32_t o4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const float2 f = unpack2<true>(w4[e]);
             o4[e] = pack2<false>(f.x, f.y);
         }
-        *p16 = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        *reinterpret_cast<uint4*>(p + (it + k * NT) * 16) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
 }
 
@@ -329,6 +323,11 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __gri
     if (tid < 64) {
         vb[64 + tid] = __expf(vb[tid]);
         vb[192 + tid] = __expf(vb[tid | 15] - vb[tid]);  // exp(gamma_e - gamma_s), e = end of s's block
+        // the chain's gates of this chunk: Gamma_r and f_r = exp(gamma_C - gamma_r) (positions past
+        // the sequence end carry g = 0, so gamma_C = gamma of the last token)
+        float* rg = reinterpret_cast<float*>(rec + kRecG);
+        rg[tid] = vb[64 + tid];
+        rg[64 + tid] = __expf(vb[63] - vb[tid]);
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -397,10 +396,10 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __gri
         // K and V to fp16 in place for the second product (exact for |x| >= 2^-14); [K;Q] K^T
         // has completed, so nothing reads them meanwhile
         if constexpr (BF) {
-            to_f16_inplace<NT>(smem + Cf::OFF_K, 8192, tid);
-            to_f16_inplace<NT>(smem + Cf::OFF_K + 16384, 8192, tid);
-            to_f16_inplace<NT>(smem + Cf::OFF_V, 8192, tid);
-            to_f16_inplace<NT>(smem + Cf::OFF_V + Cf::KV_LBO, 8192, tid);
+            to_f16_block<NT, 8192>(smem + Cf::OFF_K, tid);
+            to_f16_block<NT, 8192>(smem + Cf::OFF_K + 16384, tid);
+            to_f16_block<NT, 8192>(smem + Cf::OFF_V, tid);
+            to_f16_block<NT, 8192>(smem + Cf::OFF_V + Cf::KV_LBO, tid);
         }
         tc::tc_fence_before();
         __syncthreads();
@@ -549,7 +548,6 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __gri
 template <int NS>
 struct ChainCfg {
     static constexpr int ROWB = NS * 2;                        // bytes per row of a 16-bit slab tile
-    static constexpr int UROWB = 2 * ROWB;                     // [hi | lo] rows of U': 128 B
     static constexpr uint32_t SWZ = NS == 32 ? tc::kSw64 : tc::kSw128;
     static constexpr int QW_HALF = 128 * 128;                  // one 64-column half of [Q;W]
     static constexpr int K_HALF = 64 * 128;                    // one 64-column half of K
@@ -559,29 +557,28 @@ struct ChainCfg {
     static constexpr int OFF_UT = OFF_KS + 3 * 2 * K_HALF;     // [3 stages] U~ slab fp16 [64 x ROWB], row-major
     static constexpr int OFF_SS = OFF_UT + 3 * 64 * ROWB;      // S [128 x ROWB]
     static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // [2 slots] U fp16: [64 x ROWB]
-    static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // [U' hi | U' lo]: [64 x UROWB]
-    static constexpr int OFF_YS = OFF_SU2 + 64 * UROWB;        // y rows for the TMA store [64 x NS x 4 B]
+    static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // U' = f U fp16: [64 x ROWB]
+    static constexpr int OFF_YS = OFF_SU2 + 64 * ROWB;         // y rows for the TMA store [64 x NS x 4 B]
     static constexpr int OFF_ZS = OFF_YS + 64 * NS * 4;        // [2 slots] z slab [64 x ROWB] (gated)
     static constexpr int OFF_GZ = OFF_ZS + 2 * 64 * ROWB;      // sigmoid(z) (1 + w) rows, fp32 [64 x NS] (gated)
-    static constexpr int OFF_VEC = OFF_GZ + 64 * NS * 4;       // [2 slots] gamma, Gamma, f: 3 x 64 floats
-    static constexpr int OFF_META = OFF_VEC + 2 * 1024;        // [2 slots] {c0, L}
-    static constexpr int OFF_RS = OFF_META + 64;               // [2] [4 slabs] [64 rows] y^2 sums (gated)
+    static constexpr int OFF_GT = OFF_GZ + 64 * NS * 4;        // [3 stages] Gamma [64], f [64] fp32 (record)
+    static constexpr int OFF_RS = OFF_GT + 3 * 512;            // [2] [4 slabs] [64 rows] y^2 sums (gated)
     static constexpr int OFF_NW = OFF_RS + 2 * 4 * 64 * 4;     // 1 + norm_w of this slab (gated)
     static constexpr int OFF_BAR = OFF_NW + NS * 4;
     static constexpr int NBARS = 22;
     static constexpr int BYTES = OFF_BAR + 256 + 1024;
     static constexpr uint32_t K_TX = 2 * K_HALF;               // K of one chunk
-    static constexpr uint32_t OP_TX = 2 * 8192 + 2 * 8192 + 64 * ROWB;  // Q, -W and the U~ slab of one chunk
+    static constexpr uint32_t OP_TX = 2 * 8192 + 2 * 8192 + 64 * ROWB + 512;  // Q, -W, the U~ slab, gates
     static constexpr uint32_t M_TX = 8192;                     // M of one chunk
     static constexpr uint32_t Z_TX = 64 * ROWB;                // z slab of one chunk (gated)
     // TMEM columns; the products of chunk c that y of c needs stay until chunk c + 1 reads them
     static constexpr uint32_t COL_U = 0;                       // [2 slots] x NS: [Q; -W] S over dk 0-63
     static constexpr uint32_t COL_1B = COL_U + 2 * NS;         // [2 slots] x NS: [Q; -W] S over dk 64-127
     static constexpr uint32_t COL_MU = COL_1B + 2 * NS;        // [2 slots] x NS: M U (lanes 0-63)
-    static constexpr uint32_t COL_DS = COL_MU + 2 * NS;        // 2 NS: [K^T U' hi | K^T U' lo]
+    static constexpr uint32_t COL_DS = COL_MU + 2 * NS;        // NS: K^T U' 
     static constexpr uint32_t TMEM_COLS = 256;
     static_assert(COL_DS + 2 * NS <= TMEM_COLS, "TMEM budget");
-    static_assert(NS == 32, "[hi | lo] operand rows are one 128-byte swizzle atom");
+    static_assert(NS == 32, "slab operand rows are one 64-byte swizzle atom");
     static_assert(NBARS * 8 <= 192, "barrier area");
     static_assert(BYTES <= 232448, "shared memory budget");
     static_assert(OFF_M % 1024 == 0 && OFF_KS % 1024 == 0 && OFF_YS % 1024 == 0 && OFF_UT % 1024 == 0 &&
@@ -609,7 +606,6 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(smem);
-    int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);
     uint64_t* bar_c1 = bars + 0;       // chain: [Q;-W] S over dk 0-63 complete
     uint64_t* bar_c2 = bars + 1;       // chain: [Q;-W] S over dk 64-127 complete
@@ -658,7 +654,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         nchunks = (int)max(0LL, rec_end - rec_base);
     }
     const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    auto vec = [&](int b) { return reinterpret_cast<float*>(smem + Cf::OFF_VEC + b * 1024); };
+    auto gates = [&](int s) { return reinterpret_cast<const float*>(smem + Cf::OFF_GT + s * 512); };
     auto QWoff = [&](int b) { return Cf::OFF_QW + b * 2 * Cf::QW_HALF; };
     auto Koff = [&](int s) { return Cf::OFF_KS + s * 2 * Cf::K_HALF; };
 
@@ -667,7 +663,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         // Per chunk c (slot b = c & 1, stage kst = c % 3):
         //   thread 0 / 32   [Q; -W] S(c) over the two dk halves -> COL_U[b], COL_1B[b]; thread 0 then
         //                   issues M U(c - 1) -> COL_MU[(c - 1) & 1] behind it
-        //   warps 2-3       U = U~ - W S (lanes 64-127) -> U (fp16) and U' = f U (hi + lo); thread 64
+        //   warps 2-3       U = U~ - W S (lanes 64-127) -> U (fp16) and U' = f U (fp16); thread 64
         //                   issues K^T U'(c) as soon as these two warps have written U'
         //   warps 0-1       meanwhile y of chunk c - 1 = scale (Gamma (Q S) + M U), all three
         //                   products read from TMEM, staged and stored
@@ -699,7 +695,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             return all;
         };
         constexpr uint32_t id_slab = idesc16<false>(128, NS, false, true);    // [Q;W] S
-        constexpr uint32_t id_ds = idesc16<false>(128, 2 * NS, true, true);   // K^T [U' hi | U' lo]
+        constexpr uint32_t id_ds = idesc16<false>(128, NS, true, true);       // K^T U' 
         constexpr uint32_t id_mu = idesc16<false>(128, NS, false, true);   // M U, both fp16
         // operand descriptors at k-step 0 of slot / stage 0; k-steps and slots are byte offsets
         const uint64_t dQW0 = tc::smem_desc(sbase + Cf::OFF_QW, 16, 1024, tc::kSw128);      // K-major [Q;W]
@@ -707,7 +703,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         const uint64_t dM0 = tc::smem_desc(sbase + Cf::OFF_M, 16, 1024, tc::kSw128);
         const uint64_t dSS0 = tc::smem_desc(sbase + Cf::OFF_SS, 128 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
         const uint64_t dSU0 = tc::smem_desc(sbase + Cf::OFF_SU, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
-        const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::UROWB, 8 * Cf::UROWB, tc::kSw128);
+        const uint64_t dSU20 = tc::smem_desc(sbase + Cf::OFF_SU2, 64 * Cf::ROWB, 8 * Cf::ROWB, Cf::SWZ);
 
         const size_t st_base = ((size_t)n * H + h) * 128 * 128 + (size_t)tid * 128 + slab * NS;
         float S[NS];
@@ -892,11 +888,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 break;
             }
             tc::tc_fence_after();
-            const float* vb = vec(b);  // gamma[0:64] Gamma[64:128] f[128:192] (g prefetch [192:256])
-            const int c0 = meta[2 * b], L = meta[2 * b + 1];
-            const float gC = vb[64 + 63];
-            const float gR = tid < 64 ? vb[64 + tid] : 0.f;
-            const float fR = tid >= 64 ? vb[128 + tid - 64] : 0.f;
+            const float* gt = gates(kst);  // Gamma[0:64], f[64:128] of chunk c
+            const int c0 = t_begin + c * kChunk, L = min(kChunk, t_end - c0);
+            const float gC = gt[63];
+            const float gR = tid < 64 ? gt[tid] : 0.f;
+            const float fR = tid >= 64 ? gt[tid] : 0.f;
 
             // [Q; -W] S over dk 0-63 (thread 0) into COL_U[b] and over dk 64-127 (thread 32) into
             // COL_1B[b].  Their sum: Q S in lanes 0-63, -W S in lanes 64-127.  Then thread 0 queues
@@ -914,7 +910,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             bool w1 = true, w2 = true, wy = true;
             if (warp >= 2) {
-                // U = U~ - W S (fp16, for M U), U' = f U (hi + lo, for K^T U'), then K^T U' at once
+                // U = U~ - W S (fp16, for M U), U' = f U (fp16, for K^T U'), then K^T U' at once
                 w1 = wait_mma(bar_c1, ph_c1);
                 w2 = wait_mma(bar_c2, ph_c2);
                 float d1[NS], d2[NS];
@@ -937,14 +933,11 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 uint8_t* su = smem + Cf::OFF_SU + b * 64 * Cf::ROWB;
 #pragma unroll
                 for (int cc = 0; cc < NS / 8; ++cc) {
-                    uint4 hi, lo;
                     st16(su + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(ut + 8 * cc));
                     float u2[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) u2[e] = fR * ut[8 * cc + e];
-                    split8<false>(u2, hi, lo);
-                    st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::UROWB), hi);
-                    st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc + NS / 8, Cf::UROWB), lo);
+                    st16(smem + Cf::OFF_SU2 + tc::swz_off(r, cc, Cf::ROWB), pack8<false>(u2));
                 }
                 tc::fence_async_smem();
                 tc::tc_fence_before();
@@ -955,7 +948,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                     const uint64_t ak0 = desc_add(dK0, Koff(kst) - Cf::OFF_KS);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::UROWB),
+                        tc::mma_f16(tmem + Cf::COL_DS, desc_add(ak0, kk * 2048), desc_add(dSU20, kk * 16 * Cf::ROWB),
                                     id_ds, kk > 0);
                     tc::mma_commit(bar_ds);
                     tc::mma_commit(bar_dsd + kst);
@@ -965,11 +958,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             }
             const bool w3 = wait_mma(bar_ds, ph_ds);
             {
-                float t[NS], t2[NS];
+                float t[NS];
                 tc::tmem_ld32(trow + Cf::COL_DS, t);
-                tc::tmem_ld32(trow + Cf::COL_DS + NS, t2);
 #pragma unroll
-                for (int j = 0; j < NS; ++j) S[j] = gC * S[j] + (t[j] + t2[j]);
+                for (int j = 0; j < NS; ++j) S[j] = gC * S[j] + t[j];
 #pragma unroll
                 for (int cc = 0; cc < NS / 8; ++cc) st16(smem + Cf::OFF_SS + tc::swz_off(tid, cc, Cf::ROWB), pack8<false>(S + 8 * cc));
             }
@@ -1007,24 +999,26 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     } else {
         // =============================== producer group ================================
         // Copies and conversions only: every product of the chunk that does not involve the state
-        // (-W, U~, M) comes from chunk_ut_kernel's record.
+        // (-W, U~, M) and its gates come from chunk_ut_kernel's record.  Software-pipelined one
+        // chunk ahead of the chain: while the chain works on chunk c, the producer issues the
+        // copies of chunk c + 2 into the stage chunk c - 1 has released, and finishes chunk c + 1
+        // (waits for its copies, converts bf16 K and Q to fp16, hands it over).
         constexpr int BID = 2;
         const int it = tid - 128;
         tc::wait_prerequisites();  // the records of chunk_ut_kernel are complete and visible
         bool ok = true;
 
-        // copies are issued by one thread of warp 6, which has no part in the gate arithmetic
+        // copies are issued by one thread of warp 6
         constexpr int kIssuer = 64;
         // copies in flight into this CTA's shared memory, for the exit drain
-        int k_issued = -1, k_landed = -1, op_issued = -1, op_landed = -1;
-        int m_last0 = -1, m_last1 = -1;
+        int st_issued = -1, st_landed = -1, m_last0 = -1, m_last1 = -1;
         auto rec_ptr = [&](int ci) {
             return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
         };
-        // K of chunk ci -> stage ci % 3; Q of ci -> rows 0-63 of [Q;-W] stage ci % 3, -W of ci (record)
-        // -> rows 64-127, this slab's U~ (record) -> U~ stage ci % 3
+        // K of chunk ci -> stage ci % 3; Q of ci -> rows 0-63 of [Q;-W] stage ci % 3; from the record:
+        // -W -> rows 64-127, this slab's U~ -> U~ stage, the gates -> gate stage
         auto issue_stage = [&](int ci) {
-            k_issued = op_issued = ci;
+            st_issued = ci;
             if (it != kIssuer) return;
             const int c0 = t_begin + ci * kChunk, s = ci % 3;
             uint64_t* bk = bar_kv + s;
@@ -1040,6 +1034,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             tc::bulk_g2s(qw + Cf::QW_HALF + 64 * 128, rp + kRecW + 8192, 8192, bar_q + s);
             tc::bulk_g2s(smem + Cf::OFF_UT + s * 64 * Cf::ROWB, rp + kRecU + slab * kRecUSlab, 64 * Cf::ROWB,
                          bar_q + s);
+            tc::bulk_g2s(smem + Cf::OFF_GT + s * 512, rp + kRecG, 512, bar_q + s);
         };
         auto issue_m = [&](int ci) {  // M of chunk ci -> M slot ci & 1 (issuer thread only)
             const int bb = ci & 1;
@@ -1050,15 +1045,28 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 tc::tma_load_3d(smem + Cf::OFF_ZS + bb * 64 * Cf::ROWB, &maps.z, slab * NS, h, t_begin + ci * kChunk,
                                 bar_m + bb);
         };
-        // g of chunk ci (beta is already inside -W, U~ and M) -> vec(ci & 1)[192:256] by cp.async, two
-        // chunks ahead, so no thread waits on the load; one cp.async group per chunk (warps 4-5)
-        auto load_gates = [&](int ci) {
-            if (it < 64 && ci < nchunks) {
-                const int c0 = t_begin + ci * kChunk, L = min(kChunk, t_end - c0);
-                const bool in = it < L;
-                tc::cp_async4(vec(ci & 1) + 192 + it, in ? a.g + (size_t)(c0 + it) * H + h : a.g, in ? 4u : 0u);
+        // chunk ci landed -> bf16 K and Q to fp16 in place -> handed to the chain (full[ci & 1])
+        auto finish = [&](int ci) -> bool {
+            const int s = ci % 3;
+            bool w = tc::mbar_wait_bounded(bar_kv + s, (ci / 3) & 1, a.budget);
+            w = w && tc::mbar_wait_bounded(bar_q + s, (ci / 3) & 1, a.budget);
+            if (!tc::bar_and(BID, 128, w)) {
+                if (it == 0) raise_error(kErrTimeout);
+                return false;
             }
-            if (it < 64) tc::cp_async_commit();
+            st_landed = ci;
+            if constexpr (BF) {
+                // bf16 -> fp16 is exact for |x| >= 2^-14; the smaller entries of a unit-norm key or
+                // query lose at most 2^-25 absolute
+                to_f16_block<128, 2 * Cf::K_HALF>(smem + Koff(s), it);
+                to_f16_block<128, 64 * 128>(smem + QWoff(s), it);               // Q rows of half 0
+                to_f16_block<128, 64 * 128>(smem + QWoff(s) + Cf::QW_HALF, it);  // Q rows of half 1
+            }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            tc::bar_sync(BID, 128);
+            if (it == 0) tc::mbar_arrive(bar_full + (ci & 1));
+            return true;
         };
         if (it == kIssuer) {
             tc::prefetch_tmap(&maps.k);
@@ -1066,81 +1074,33 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
             if constexpr (GATED) tc::prefetch_tmap(&maps.z);
         }
         if (nchunks > 0) issue_stage(0);
-        load_gates(0);
-        load_gates(1);
+        if (nchunks > 1) issue_stage(1);
+        if (nchunks > 0) ok = finish(0);
 
-        for (int c = 0; c < nchunks; ++c) {
-            const int b = c & 1, kst = c % 3;
-            const int c0 = t_begin + c * kChunk, L = min(kChunk, t_end - c0);
-            float* vb = vec(b);
-            // the copies of chunk c + 1 go into stage (c + 1) % 3 once chunk c - 2's state MMA, the
-            // last reader of that stage, is done: two chain periods of lead
-            if (c + 1 < nchunks) {
-                bool w = true;
-                if (c >= 2) w = tc::mbar_wait_bounded(bar_dsd + (c - 2) % 3, ((c - 2) / 3) & 1, a.budget);
+        for (int c = 0; ok && c < nchunks; ++c) {
+            // chunk c - 1's state MMA done: stage (c + 2) % 3, which it last read, is free, and the
+            // chain has taken chunk c - 1 from full[(c + 1) & 1], so handing over chunk c + 1 there
+            // cannot overtake it
+            if (c >= 1) {
+                const bool w = tc::mbar_wait_bounded(bar_dsd + (c - 1) % 3, ((c - 1) / 3) & 1, a.budget);
                 if (!(ok = tc::bar_and(BID, 128, w))) {
                     if (it == 0) raise_error(kErrTimeout);
                     break;
                 }
-                issue_stage(c + 1);
             }
-
-            // ---- gates of chunk c (warps 4-5): gamma (inclusive prefix sum), Gamma,
-            //      f = exp(gamma_C - gamma) -----------------------------------------------------------
-            if (it < 64) {
-                constexpr int BID_G = 3;
-                tc::cp_async_wait<1>();  // this chunk's group; the next chunk's may still be in flight
-                float gv = vb[192 + it];
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, gv, o);
-                    if (lane >= o) gv += y;
-                }
-                vb[it] = gv;
-                if (it == 0) {
-                    meta[2 * b] = c0;
-                    meta[2 * b + 1] = L;
-                }
-                tc::bar_sync(BID_G, 64);
-                if (it >= 32) vb[it] += vb[31];
-                tc::bar_sync(BID_G, 64);
-                vb[64 + it] = __expf(vb[it]);
-                vb[128 + it] = __expf(vb[63] - vb[it]);
-            }
-
-            // ---- K(c), Q(c), -W(c), U~(c) landed; bf16 K and Q -> fp16 in place ---------------------
-            bool w = tc::mbar_wait_bounded(bar_kv + kst, (c / 3) & 1, a.budget);
-            w = w && tc::mbar_wait_bounded(bar_q + kst, (c / 3) & 1, a.budget);
-            if (!(ok = tc::bar_and(BID, 128, w))) {
-                if (it == 0) raise_error(kErrTimeout);
-                break;
-            }
-            k_landed = op_landed = c;
-            if constexpr (BF) {
-                // bf16 -> fp16 is exact for |x| >= 2^-14; the smaller entries of a unit-norm key or
-                // query lose at most 2^-25 absolute
-                to_f16_inplace(smem + Koff(kst), 2 * Cf::K_HALF, it);
-                to_f16_inplace(smem + QWoff(kst), 64 * 128, it);               // Q rows of half 0
-                to_f16_inplace(smem + QWoff(kst) + Cf::QW_HALF, 64 * 128, it);  // Q rows of half 1
-            }
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            tc::bar_sync(BID, 128);
-            if (it == 0) tc::mbar_arrive(bar_full + b);  // hand chunk c to the chain group
-
-            // ---- M of chunk c, once M U of c - 2 has read the slot ---------------------------------
+            if (c + 2 < nchunks) issue_stage(c + 2);
+            if (c + 1 < nchunks && !(ok = finish(c + 1))) break;
+            // M of chunk c, once M U of c - 2 has read the slot (M U of c is issued during chunk c + 1)
             if (it == kIssuer) {
-                if (tc::mbar_wait_bounded(bar_mfree + b, ((c >> 1) & 1) ^ 1, a.budget)) issue_m(c);
+                if (tc::mbar_wait_bounded(bar_mfree + (c & 1), ((c >> 1) & 1) ^ 1, a.budget)) issue_m(c);
                 else raise_error(kErrTimeout);
             }
-            load_gates(c + 2);
         }
-        if (it < 64) tc::cp_async_wait<0>();  // no copy into shared memory left in flight
         // never leave with copies into this CTA's shared memory in flight
-        for (int ci = max(k_landed + 1, 0); ci <= k_issued; ++ci)  // at most two outstanding
+        for (int ci = max(st_landed + 1, 0); ci <= st_issued; ++ci) {  // at most two outstanding
             tc::mbar_wait_bounded(bar_kv + ci % 3, (ci / 3) & 1, 4000000000ull);
-        for (int ci = max(op_landed + 1, 0); ci <= op_issued; ++ci)
             tc::mbar_wait_bounded(bar_q + ci % 3, (ci / 3) & 1, 4000000000ull);
+        }
         if (m_last0 >= 0) tc::mbar_wait_bounded(bar_m + 0, (m_last0 >> 1) & 1, 4000000000ull);
         if (m_last1 >= 0) tc::mbar_wait_bounded(bar_m + 1, (m_last1 >> 1) & 1, 4000000000ull);
         (void)ok;

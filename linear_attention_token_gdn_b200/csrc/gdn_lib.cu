@@ -106,7 +106,8 @@ struct MixerDecodeLaunch {
     static gdn_status_t run(const gdn::MixerDecodeArgs& args, int B, cudaStream_t st) {
         using Sh = gdn::DecodeShape<DK, DV>;
         gdn::LaunchScope timed(st, "mixer_decode_kernel");
-        gdn::mixer_decode_kernel<DK, DV><<<(unsigned)(B * args.H), Sh::THREADS, 0, st>>>(args);
+        if (args.W <= 4) gdn::mixer_decode_kernel<DK, DV, 4><<<(unsigned)(B * args.H), Sh::THREADS, 0, st>>>(args);
+        else gdn::mixer_decode_kernel<DK, DV, 8><<<(unsigned)(B * args.H), Sh::THREADS, 0, st>>>(args);
         return launched("mixer_decode_kernel");
     }
 };

@@ -36,8 +36,11 @@ struct MixerDecodeArgs {
     void* out;
 };
 
-template <int DK, int DV>
-__global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS) mixer_decode_kernel(const MixerDecodeArgs a) {
+// TAPS: the largest conv width the instantiation takes (4 or 8), so that the window lives in
+// registers with static indices.
+template <int DK, int DV, int TAPS>
+__global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 1)
+    mixer_decode_kernel(const MixerDecodeArgs a) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int NT = Sh::THREADS, CH = 2 * DK + DV;  // channels of one head's conv input
     const int bh = blockIdx.x;                         // row * H + head
@@ -67,31 +70,67 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS) mixer_decode_ker
     }
 
     // ---- eqs. (6)-(8): ShortConv over [history, current] then SiLU, one channel per thread; the
-    //      history is shifted in place (entry j <- entry j + 1, the current input last) ----------
+    //      history is shifted in place (entry j <- entry j + 1, the current input last).  Every
+    //      global load of this phase is issued before any arithmetic or store, so their latencies
+    //      overlap each other and the state loads. ----------------------------------------------
+    constexpr int CPT = (CH + NT - 1) / NT;     // channels per thread
+    constexpr int HMAX = TAPS - 1;              // history entries at most
     const int W = a.W, HW = W - 1;
     const size_t hist_stride = (size_t)H * CH;  // elements between history entries of a slot
     const size_t hist0 = (size_t)s * HW * hist_stride + (size_t)h * CH;
-    for (int c = tid; c < CH; c += NT) {
-        const bool isq = c < DK, isk = !isq && c < 2 * DK;
-        const int i = isq ? c : (isk ? c - DK : c - 2 * DK);
-        const void* xp = isq ? a.x_q : (isk ? a.x_k : a.x_v);
-        const float* wp = (isq ? a.w_q : (isk ? a.w_k : a.w_v)) + ((size_t)h * (isq || isk ? DK : DV) + i) * W;
-        const float xc = ld1(xp, a.in_dt, (size_t)bh * (isq || isk ? DK : DV) + i);
-        float acc = wp[W - 1] * xc;  // tap W-1 meets the current token
-        float prev = xc;
-        for (int j = HW - 1; j >= 0; --j) {  // entry j is token t - (W - 1) + j
-            const size_t at = hist0 + (size_t)j * hist_stride + c;
-            const float xj = ld1(a.conv_state, a.in_dt, at);
-            acc += wp[j] * xj;
-            st1(a.conv_state, a.in_dt, at, prev);  // entry j takes entry j + 1 (the newest: xc)
-            prev = xj;
+    float xw[CPT][HMAX], taps[CPT][HMAX];       // history oldest first, and its taps
+    float xcur[CPT], tcur[CPT];                 // the current input and tap W-1
+    float bl = 0.f, al = 0.f, Ah = 0.f, bh_ = 0.f;
+    if (tid == 0) {
+        bl = ld1(a.beta_logit, a.in_dt, bh);
+        al = ld1(a.alpha_logit, a.in_dt, bh);
+        Ah = a.A_log[h];
+        bh_ = a.alpha_bias[h];
+    }
+#pragma unroll
+    for (int u = 0; u < CPT; ++u) {
+        const int c = tid + u * NT;
+        if (c < CH) {
+            const bool isq = c < DK, isk = !isq && c < 2 * DK;
+            const int i = isq ? c : (isk ? c - DK : c - 2 * DK);
+            const int d = isq || isk ? DK : DV;
+            const void* xp = isq ? a.x_q : (isk ? a.x_k : a.x_v);
+            const float* wp = (isq ? a.w_q : (isk ? a.w_k : a.w_v)) + ((size_t)h * d + i) * W;
+#pragma unroll
+            for (int j = 0; j < HMAX; ++j) {
+                if (j < HW) {
+                    taps[u][j] = wp[j];
+                    xw[u][j] = ld1(a.conv_state, a.in_dt, hist0 + (size_t)j * hist_stride + c);
+                }
+            }
+            tcur[u] = wp[W - 1];
+            xcur[u] = ld1(xp, a.in_dt, (size_t)bh * d + i);
         }
-        s_x[c] = acc / (1.f + __expf(-acc));  // SiLU
+    }
+#pragma unroll
+    for (int u = 0; u < CPT; ++u) {
+        const int c = tid + u * NT;
+        if (c < CH) {
+            float acc = tcur[u] * xcur[u];  // tap W-1 meets the current token
+#pragma unroll
+            for (int j = 0; j < HMAX; ++j)
+                if (j < HW) acc += taps[u][j] * xw[u][j];
+            s_x[c] = acc / (1.f + __expf(-acc));  // SiLU
+#pragma unroll
+            for (int j = 0; j < HMAX; ++j) {  // entry j takes entry j + 1; the last the current input
+                if (j < HW) {
+                    float nx = xcur[u];
+#pragma unroll
+                    for (int jj = 0; jj < HMAX; ++jj)
+                        if (jj == j + 1 && jj < HW) nx = xw[u][jj];
+                    st1(a.conv_state, a.in_dt, hist0 + (size_t)j * hist_stride + c, nx);
+                }
+            }
+        }
     }
     if (tid == 0) {  // eqs. (9)-(10)
-        const float bl = ld1(a.beta_logit, a.in_dt, bh), al = ld1(a.alpha_logit, a.in_dt, bh);
         s_gate[1] = sigmoidf_(bl);
-        s_gate[0] = expf(-expf(a.A_log[h]) * softplusf_(al + a.alpha_bias[h]));
+        s_gate[0] = expf(-expf(Ah) * softplusf_(al + bh_));
     }
     __syncthreads();
     // L2Norm of q (warp 0) and k (warp 1), and k.q (warp 2) once both are normalised

@@ -101,9 +101,9 @@ def test_workspace_size_is_zero_without_records(L):
 
 
 def test_workspace_size_covers_every_chunk(L):
-    # one 40 KB record per (64-token chunk, head); packed sequences add one partial chunk each
-    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 40960
-    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 40960
+    # one 40.5 KB record per (64-token chunk, head); packed sequences add one partial chunk each
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 41472
+    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 41472
     assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0
 
 
