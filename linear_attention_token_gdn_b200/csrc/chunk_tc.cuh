@@ -14,12 +14,12 @@
 // factors <= 1, so a row needs 4 + 16 exponentials instead of 64.
 //
 // Two kernels:
-//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, two CTAs per SM.
-//                       [K;Q] K^T on tcgen05 (the 16-bit inputs used directly as operands),
-//                       the decay masks, and the unit-lower-triangular inverse T in fp32 on the
-//                       CUDA cores; then one N = 256 product [T_w; T_u] [K | V] with
-//                       T_w = T diag(beta Gamma) and T_u = T diag(beta) gives W = T_w K and
-//                       U~ = T_u V.  Writes a 40.5 KB record per (chunk, head): -W and M in the
+//   chunk_ut_kernel     one CTA per (chunk, head), fully parallel, three CTAs per SM, on
+//                       warp-level tensor-core products (mma.sync): [K;Q] K^T on the 16-bit
+//                       inputs as stored, the decay masks on the accumulators, the
+//                       unit-lower-triangular inverse T in fp32, then W = T_w K and U~ = T_u V
+//                       with T_w = T diag(beta Gamma) and T_u = T diag(beta) in fp16.  Writes a
+//                       40.5 KB record per (chunk, head) by bulk copies: -W and M in the
 //                       128B-swizzled operand layout and U~ as four 32-column slabs, all fp16,
 //                       and the chunk's gates Gamma_r and Gamma_C / Gamma_r in fp32.
 //   chunk_chain_kernel  one CTA per (sequence, head, 32-column dv slab), sequential over
@@ -41,20 +41,20 @@
 //                       chunk_ut_kernel.  The gated variant applies eq. (11)'s output gate
 //                       in the y epilogue, the four slab CTAs of a (sequence, head) forming
 //                       one cluster that exchanges row sums of squares.
-// Operands are 16-bit with fp32 accumulation in TMEM.  A tcgen05.mma instruction with
-// M = 128 costs the SM's MMA pipe about 95 cycles for any N up to 64 (N = 128: about 147,
-// N = 256: about 173, measured), so products are shaped to use few instructions, and the
+// The chain's operands are 16-bit with fp32 accumulation in TMEM.  A tcgen05.mma instruction
+// with M = 128 costs the SM's MMA pipe about 95 cycles for any N up to 64 (N = 128: about 147,
+// N = 256: about 173, measured), so its products are shaped to use few instructions, and the
 // per-(chunk, head) products are formed once in chunk_ut_kernel rather than once per slab.
 // bf16 inputs must lie inside the fp16 range (|x| < 65504), as unit-norm keys and queries do.  [K;Q] K^T reads q and k exactly as stored.  Every product of the
-// chain runs on fp16 operands (11 significant bits): bf16 q, k and v are converted to fp16 in
-// shared memory when they land (exact for |x| >= 2^-14), and their partners T_w, W, S and U'
+// chain runs on fp16 operands (11 significant bits): bf16 q, k and v are converted to fp16 (exact
+// for |x| >= 2^-14; in registers in chunk_ut_kernel, in shared memory when they land in the chain), and their partners T_w, W, S and U'
 // are formed in fp16.  bf16 partners (8 bits) would let the error of a row whose y is small
 // exceed the bound once eq. (11) normalises that row.  U' = f U enters as one fp16 value (the
 // state's error stays near 5e-4 of its scale, well inside the bound).
 // Operand tiles use the 128B / 64B swizzled canonical layouts, so one tile serves as K-major
 // or MN-major operand.  Every wait is bounded (ChunkArgs::budget clock cycles); a wait that
 // runs out sets the device error word, lets in-flight MMAs and copies drain, and the CTA
-// returns after freeing TMEM.
+// returns (after freeing TMEM, in the chain).
 #pragma once
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -98,7 +98,8 @@ constexpr int kChunk = 64;
 constexpr int kRecW = 0;           // -W: two dk halves, each [64 rows x 128 B] 128B-swizzled K-major,
                                    // ready to be rows 64-127 of the chain's [Q; -W] operand
 constexpr int kRecM = 16384;       // M: [64 rows x 128 B] 128B-swizzled K-major
-constexpr int kRecU = 24576;       // U~: four 32-column dv slabs, each [64 rows x 64 B] row-major
+constexpr int kRecU = 24576;       // U~: four 32-column dv slabs, each [64 rows x 64 B] 64B-swizzled
+                                   // (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3))
 constexpr int kRecUSlab = 4096;
 constexpr int kRecG = 40960;       // Gamma_r = exp(gamma_r) [64] then f_r = exp(gamma_C - gamma_r) [64], fp32
 constexpr int kRecBytes = 41472;
@@ -124,32 +125,6 @@ __device__ __forceinline__ int seq_chunks(const int32_t* cu, int m, int num_seqs
     int a, b;
     seq_bounds(cu, m, num_seqs, N, a, b);
     return (b - a + kChunk - 1) / kChunk;
-}
-
-// Virtual chunk v -> (sequence n, chunk j of n).  Warp-collective; false if v is past the end.
-__device__ bool locate_chunk(const int32_t* cu, int num_seqs, int N, int v, int& n, int& j) {
-    const int lane = threadIdx.x & 31;
-    int base = 0;
-    for (int m0 = 0; m0 < num_seqs; m0 += 32) {
-        const int m = m0 + lane;
-        const int cnt = m < num_seqs ? seq_chunks(cu, m, num_seqs, N) : 0;
-        int inc = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += t;
-        }
-        const int total = __shfl_sync(0xffffffffu, inc, 31);
-        if (v < base + total) {
-            const unsigned hit = __ballot_sync(0xffffffffu, base + inc > v);
-            const int l = __ffs(hit) - 1;
-            n = m0 + l;
-            j = v - (base + __shfl_sync(0xffffffffu, inc, l) - __shfl_sync(0xffffffffu, cnt, l));
-            return true;
-        }
-        base += total;
-    }
-    return false;
 }
 
 // Number of chunks of sequences 0 .. n-1 (warp-collective).
@@ -220,39 +195,82 @@ __device__ __forceinline__ void to_f16_block(uint8_t* p, int it) {
 
 struct UtCfg {
     static constexpr int THREADS = 256;
-    static constexpr int LD = 68;                           // fp32 row stride of A and T
-    // [K h0 | Q h0 | K h1 | Q h1 | V h0 | (gap) | V h1], 8 KB tiles [64 rows x 128 B], 128B
-    // swizzle.  [K_h; Q_h] is the A operand of half h of [K;Q] K^T; K h0, K h1, V h0, V h1 sit
-    // 16 KB apart, the column-block stride of the MN-major B operand [K | V] (N = 256).
-    static constexpr int OFF_K = 0, OFF_Q = 8192, OFF_V = 32768, KV_LBO = 16384;
-    // fp32 scratch of the block inverse over Q h0 once [K;Q] K^T has read it: the level-one
-    // products [2 blocks][16][LDX1] and the level-two product [32][LDX2]
-    static constexpr int OFF_X1 = 8192, LDX1 = 20, OFF_X2 = OFF_X1 + 2 * 16 * LDX1 * 4, LDX2 = 36;
-    static constexpr int OFF_VEC = 40960;                   // gamma, Gamma, beta, colf: 4 x 64 (gap)
-    static constexpr int OFF_META = OFF_VEC + 1024;
-    static constexpr int OFF_BAR = OFF_META + 32;
-    static constexpr int OFF_A = 57344;                     // fp32 A [64][LD]; later [T_w; T_u]
-    static constexpr int OFF_TOP = OFF_A;                   //   fp16 [128 rows x 128 B], 128B swizzle
-    static constexpr int OFF_T = OFF_A + 64 * LD * 4;       // fp32 T [64][LD]
-    static constexpr int BYTES = OFF_T + 64 * LD * 4 + 1024;
-    static_assert(OFF_BAR + 64 <= OFF_V + 16384, "vectors and barriers fit in the gap");
-    static_assert(OFF_X2 + 32 * LDX2 * 4 <= 16384, "inverse scratch fits in Q h0");
-    static_assert(64 * LD * 4 >= 16384 && OFF_A % 1024 == 0, "[T_w; T_u] fits over A");
-    static constexpr uint32_t TMEM_COLS = 256;              // [K;Q] K^T (cols 0-63), then [T_w;T_u][K|V]
+    // K, Q, V as stored (bf16 or fp16), each two 8 KB dk (dv) halves [64 rows x 128 B] in the
+    // 128B-swizzled layout TMA writes.  After [K;Q] K^T the Q tile stages M (the record's layout)
+    // until it has been stored, then holds [T_w; T_u] (fp16, [128 rows x 128 B], same swizzle);
+    // -W overwrites K in place (the record's layout) once W has been formed.
+    static constexpr int OFF_K = 0, OFF_Q = 16384, OFF_V = 32768;
+    // fp32 A, turned into T in place [64][LD]; its upper triangle is scratch of the block inverse;
+    // once [T_w; T_u] has been formed, it stages U~ (the record's four slabs)
+    static constexpr int LD = 68, OFF_A = 49152;
+    // per-position vectors (fp32): gamma, beta, beta Gamma, colf [64] each, then rowf [64][4]
+    static constexpr int OFF_VEC = OFF_A + 64 * LD * 4;
+    static constexpr int V_GAMMA = 0, V_BETA = 64, V_BG = 128, V_COLF = 192, V_ROWF = 256;
+    static constexpr int OFF_META = OFF_VEC + 4 * (V_ROWF + 256);
+    static constexpr int OFF_BAR = OFF_META + 32;           // K and Q landed, V landed
+    static constexpr int BYTES = OFF_BAR + 16 + 1024;       // + the 1024-byte alignment slack
+    static_assert(64 * LD * 4 >= 16384 && OFF_A % 1024 == 0, "U~ staging fits over A");
 };
 
-// One CTA (eight warps) per (chunk, head): the UT transform of the chunk and the products that
-// depend on it alone.  [K;Q] K^T gives A and M; T = (I + A)^-1 in fp32 (16x16 diagonal blocks by
-// forward substitution on the CUDA cores, the off-diagonal blocks by recursive doubling,
-//     T21 = -T22 A21 T11   for 16x16 blocks, then the same for the 32x32 halves,
-// as warp-level mma.sync products of fp32 values split into fp16 pairs); then one N = 256
-// product
-//     [T_w; T_u] [K | V]  ->  lanes 0-63: W = T_w K (columns 0-127),
-//                             lanes 64-127: U~ = T_u V (columns 128-255)
-// (the other two blocks are not used), with T_w = T diag(beta Gamma), T_u = T diag(beta), K and
-// V converted to fp16 once [K;Q] K^T has read them.  -W, M and U~ go to the record in fp16.
+// Shared-memory byte offset of 16-byte chunk c of row r in a [rows x 128 B] 128B-swizzled tile.
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ void sts32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
+
+// Virtual chunk v -> (sequence n, chunk j of n) and the bounds [tb, te) of sequence n, from one
+// pass over cu_seqlens.  Warp-collective; false if v is past the end.
+__device__ bool locate_chunk(const int32_t* cu, int num_seqs, int N, int v, int& n, int& j, int& tb, int& te) {
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    for (int m0 = 0; m0 < num_seqs; m0 += 32) {
+        const int m = m0 + lane;
+        int sa = 0, sb = 0;
+        if (m < num_seqs) seq_bounds(cu, m, num_seqs, N, sa, sb);
+        const int cnt = (sb - sa + kChunk - 1) / kChunk;
+        int inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += t;
+        }
+        const int total = __shfl_sync(0xffffffffu, inc, 31);
+        if (v < base + total) {
+            const unsigned hit = __ballot_sync(0xffffffffu, base + inc > v);
+            const int l = __ffs(hit) - 1;
+            n = m0 + l;
+            j = v - (base + __shfl_sync(0xffffffffu, inc, l) - __shfl_sync(0xffffffffu, cnt, l));
+            tb = __shfl_sync(0xffffffffu, sa, l);
+            te = __shfl_sync(0xffffffffu, sb, l);
+            return true;
+        }
+        base += total;
+    }
+    return false;
+}
+
+// Lower 16x8 tile idx (0..19, row-major over 16-row tiles R and 8-column strips j <= 2R + 1).
+__device__ __forceinline__ void lower_tile(int idx, int& R, int& j) {
+    R = idx < 2 ? 0 : idx < 6 ? 1 : idx < 12 ? 2 : 3;
+    j = idx - (R == 0 ? 0 : R == 1 ? 2 : R == 2 ? 6 : 12);
+}
+
+// One CTA (eight warps) per (chunk, head), three CTAs per SM, on warp-level tensor-core products
+// (mma.sync): each product here is small and triangular, so a tcgen05 round trip (issue, commit,
+// TMEM load) would cost more than the arithmetic.
+//   1. [K;Q] K^T on the inputs as stored (bf16 or fp16), lower 16x8 tiles only: warp w takes
+//      the rows of K (w < 4) or Q (w >= 4) against column strips w % 4 and 7 - w % 4, five tiles.
+//   2. The decay masks on the accumulators: A = beta_r exp(gamma_r - gamma_s) (s < r) to fp32
+//      shared memory, M = exp(gamma_r - gamma_s) (s <= r) to fp16 and out to the record.
+//   3. T = (I + A)^-1 in fp32, in place: 16x16 diagonal blocks by forward substitution, then
+//          T21 = -T22 (A21 T11)   for 16x16 blocks, then the same for the 32x32 halves,
+//      as mma.sync products of fp32 values split into fp16 pairs (about fp32 accuracy).
+//   4. [T_w; T_u] = [T diag(beta Gamma); T diag(beta)] in fp16, then W = T_w K (warps 0-3) and
+//      U~ = T_u V (warps 4-7) with K and V converted to fp16 in registers (exact for
+//      |x| >= 2^-14), lower blocks only.
+//   5. -W, U~ and M leave as bulk copies of tiles staged in the record's layout; the gates
+//      Gamma_r and Gamma_C / Gamma_r go to the record directly.
 template <bool BF>
-__global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
+__global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
                                                                      const __grid_constant__ ChainMaps maps) {
     using Cf = UtCfg;
     constexpr int LD = Cf::LD, NT = Cf::THREADS;
@@ -260,153 +278,196 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __gri
     uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(smem);
     float* fA = reinterpret_cast<float*>(smem + Cf::OFF_A);
-    float* fT = reinterpret_cast<float*>(smem + Cf::OFF_T);
-    float* fX1 = reinterpret_cast<float*>(smem + Cf::OFF_X1);
-    float* fX2 = reinterpret_cast<float*>(smem + Cf::OFF_X2);
-    float* vb = reinterpret_cast<float*>(smem + Cf::OFF_VEC);  // gamma[0:64] Gamma[64:128] beta[128:192] colf[192:256]
+    float* vb = reinterpret_cast<float*>(smem + Cf::OFF_VEC);
     int* meta = reinterpret_cast<int*>(smem + Cf::OFF_META);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);       // MMA done (two phases)
-    uint64_t* bar_ld = bar + 1;                                            // K, Q, V tiles landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cf::OFF_BAR + 16);
+    uint64_t* bar_kq = reinterpret_cast<uint64_t*>(smem + Cf::OFF_BAR);  // K and Q landed
+    uint64_t* bar_v = bar_kq + 1;                                        // V landed
+    uint8_t* Kt = smem + Cf::OFF_K;
+    uint8_t* Qt = smem + Cf::OFF_Q;
+    const uint32_t kb = sbase + Cf::OFF_K, qb = sbase + Cf::OFF_Q;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // TMEM lane quadrant and column half of this warp in the epilogues (two warps per quadrant)
-    const int quad = warp & 3, chalf = warp >> 2;
+    const int g8 = lane >> 2, t4 = lane & 3;   // fragment row and column pair of this lane
+    const int mi = lane >> 3, rr = lane & 7;   // ldmatrix: the matrix and row this lane addresses
     // heads vary fastest across the grid, so CTAs resident together read whole token rows
     const int H = a.H, v = (int)(blockIdx.x / (unsigned)H), h = (int)(blockIdx.x % (unsigned)H);
     tc::launch_dependents();  // the chain kernel may start its prologue once every CTA is resident
+
+    // ---- locate the chunk; K and Q, then V, as they are stored, by TMA.  Rows past the sequence end
+    //      hold other tokens (or the fill of a load past N); they only meet beta = 0 or the
+    //      strictly-upper mask, so nothing needs clearing. -------------------------------------------
     if (warp == 0) {
-        int n = 0, j = 0;
-        const bool found = locate_chunk(a.cu, a.num_seqs, a.N, v, n, j);
+        int n = 0, j = 0, tb = 0, te = 0;
+        const bool found = locate_chunk(a.cu, a.num_seqs, a.N, v, n, j, tb, te);
         if (lane == 0) {
+            const int t0 = tb + j * kChunk;
             meta[0] = found;
-            meta[1] = n;
-            meta[2] = j;
+            meta[1] = t0;
+            meta[2] = min(kChunk, te - t0);
+            if (found) {
+                tc::mbar_init(bar_kq, 1);
+                tc::mbar_init(bar_v, 1);
+                tc::fence_mbar_init();
+                tc::mbar_arrive_expect_tx(bar_kq, 4 * 8192);
+                tc::mbar_arrive_expect_tx(bar_v, 2 * 8192);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    tc::tma_load_3d(Kt + hf * 8192, &maps.k, 64 * hf, h, t0, bar_kq);
+                    tc::tma_load_3d(Qt + hf * 8192, &maps.q, 64 * hf, h, t0, bar_kq);
+                }
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) tc::tma_load_3d(smem + Cf::OFF_V + hf * 8192, &maps.v, 64 * hf, h, t0, bar_v);
+            }
         }
     }
     __syncthreads();
-    if (!meta[0]) return;
-    int t_begin, t_end;
-    seq_bounds(a.cu, meta[1], a.num_seqs, a.N, t_begin, t_end);
-    const int t0 = t_begin + meta[2] * kChunk, L = min(kChunk, t_end - t0);
+    if (!meta[0]) return;  // uniform
+    const int t0 = meta[1], L = meta[2];
     uint8_t* rec = reinterpret_cast<uint8_t*>(a.workspace) + ((size_t)v * H + h) * kRecBytes;
-
-    // ---- K, Q, V as they are stored (bf16 or fp16), by TMA into the 128B-swizzled operand
-    //      layout.  Rows past the sequence end hold other tokens (or the fill of a load past N);
-    //      they only meet beta = 0 or the strictly-upper mask, so nothing needs clearing. ---------
-    if (tid == 0) {
-        tc::mbar_init(bar, 1);
-        tc::mbar_init(bar_ld, 1);
-        tc::fence_mbar_init();
-        tc::mbar_arrive_expect_tx(bar_ld, 6 * 8192);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            tc::tma_load_3d(smem + Cf::OFF_K + hf * 16384, &maps.k, 64 * hf, h, t0, bar_ld);
-            tc::tma_load_3d(smem + Cf::OFF_Q + hf * 16384, &maps.q, 64 * hf, h, t0, bar_ld);
-            tc::tma_load_3d(smem + Cf::OFF_V + hf * Cf::KV_LBO, &maps.v, 64 * hf, h, t0, bar_ld);
+    auto drain = [&]() {  // a copy did not land in time: flag it and let every copy finish
+        if (tid == 0) {
+            raise_error(kErrTimeout);
+            tc::mbar_wait_bounded(bar_kq, 0, 4000000000ull);
+            tc::mbar_wait_bounded(bar_v, 0, 4000000000ull);
         }
-    }
-    if (tid < 64) {
-        float gv = tid < L ? a.g[(size_t)(t0 + tid) * H + h] : 0.f;
-        vb[128 + tid] = tid < L ? a.beta[(size_t)(t0 + tid) * H + h] : 0.f;
+    };
+
+    // ---- gates (warp 1, two positions per lane): gamma = inclusive prefix sum of g inside the
+    //      chunk (positions past the sequence end carry g = 0, beta = 0), Gamma = exp(gamma); the
+    //      record gets Gamma_r and f_r = exp(gamma_C - gamma_r).  The decay exp(gamma_r - gamma_s)
+    //      of a pair in different 16-blocks is split at the end e of s's block into
+    //      rowf[r][blk s] = exp(gamma_r - gamma_e) and colf[s] = exp(gamma_e - gamma_s), both <= 1.
+    if (warp == 1) {
+        const int r0 = 2 * lane;
+        const size_t i0 = (size_t)(t0 + r0) * H + h;
+        const float g0 = r0 < L ? a.g[i0] : 0.f, g1 = r0 + 1 < L ? a.g[i0 + H] : 0.f;
+        const float b0 = r0 < L ? a.beta[i0] : 0.f, b1 = r0 + 1 < L ? a.beta[i0 + H] : 0.f;
+        float s = g0 + g1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, gv, o);
-            if (lane >= o) gv += y;
+            const float y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
         }
-        vb[tid] = gv;
-    }
-    if (warp == 0) tc::tmem_alloc(tmem_slot, Cf::TMEM_COLS);
-    __syncthreads();
-    if (tid >= 32 && tid < 64) vb[tid] += vb[31];
-    __syncthreads();
-    if (tid < 64) {
-        vb[64 + tid] = __expf(vb[tid]);
-        vb[192 + tid] = __expf(vb[tid | 15] - vb[tid]);  // exp(gamma_e - gamma_s), e = end of s's block
-        // the chain's gates of this chunk: Gamma_r and f_r = exp(gamma_C - gamma_r) (positions past
-        // the sequence end carry g = 0, so gamma_C = gamma of the last token)
+        float ex = __shfl_up_sync(0xffffffffu, s, 1);
+        if (lane == 0) ex = 0.f;
+        const float gm0 = ex + g0, gm1 = gm0 + g1;
+        const float gC = __shfl_sync(0xffffffffu, gm1, 31);
+        const float ge = __shfl_sync(0xffffffffu, gm1, lane | 7);  // gamma at the end of this 16-block
+        const float G0 = __expf(gm0), G1 = __expf(gm1);
+        *reinterpret_cast<float2*>(vb + Cf::V_GAMMA + r0) = make_float2(gm0, gm1);
+        *reinterpret_cast<float2*>(vb + Cf::V_BETA + r0) = make_float2(b0, b1);
+        *reinterpret_cast<float2*>(vb + Cf::V_BG + r0) = make_float2(b0 * G0, b1 * G1);
+        *reinterpret_cast<float2*>(vb + Cf::V_COLF + r0) = make_float2(__expf(ge - gm0), __expf(ge - gm1));
+        float rf0[4], rf1[4];
+#pragma unroll
+        for (int B = 0; B < 4; ++B) {
+            const float gb = __shfl_sync(0xffffffffu, gm1, 8 * B + 7);  // gamma at the end of block B
+            rf0[B] = B < (r0 >> 4) ? __expf(gm0 - gb) : 0.f;
+            rf1[B] = B < (r0 >> 4) ? __expf(gm1 - gb) : 0.f;
+        }
+        *reinterpret_cast<float4*>(vb + Cf::V_ROWF + 4 * r0) = make_float4(rf0[0], rf0[1], rf0[2], rf0[3]);
+        *reinterpret_cast<float4*>(vb + Cf::V_ROWF + 4 * r0 + 4) = make_float4(rf1[0], rf1[1], rf1[2], rf1[3]);
         float* rg = reinterpret_cast<float*>(rec + kRecG);
-        rg[tid] = vb[64 + tid];
-        rg[64 + tid] = __expf(vb[63] - vb[tid]);
+        *reinterpret_cast<float2*>(rg + r0) = make_float2(G0, G1);
+        *reinterpret_cast<float2*>(rg + 64 + r0) = make_float2(__expf(gC - gm0), __expf(gC - gm1));
     }
-    tc::tc_fence_before();
-    __syncthreads();
-    tc::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const bool landed = __syncthreads_and(tc::mbar_wait_bounded(bar_ld, 0, a.budget)) != 0;
-    if (!landed) {
-        if (tid == 0) raise_error(kErrTimeout);
-        tc::mbar_wait_bounded(bar_ld, 0, 4000000000ull);
+    if (!__syncthreads_and(tc::mbar_wait_bounded(bar_kq, 0, a.budget))) {
+        drain();
+        return;
     }
 
-    // ---- [K;Q] K^T (the inputs' own format) -------------------------------------------------------
-    if (tid == 0 && landed) {
-        constexpr uint32_t id = idesc16<BF>(128, 64, false, false);
-        const uint64_t d0 = tc::smem_desc(sbase + Cf::OFF_K, 16, 1024, tc::kSw128);
+    // ---- 1-2. [K;Q] K^T and the masks --------------------------------------------------------------
+    {
+        const int mat = warp >> 2, jj = warp & 3;             // mat 0: A from K rows, 1: M from Q rows
+        const int strip[2] = {jj, 7 - jj};                     // 8-column strips of this warp
+        const int rmin0 = jj >> 1, rmin1 = (7 - jj) >> 1;      // first 16-row tile at or below the diagonal
+        const uint32_t aop = mat ? qb : kb;
+        const int brow = 8 * (mi < 2 ? strip[0] : strip[1]) + rr;
+        float acc[4][2][4];
+#pragma unroll
+        for (int R = 0; R < 4; ++R)
+#pragma unroll
+            for (int si = 0; si < 2; ++si)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[R][si][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t d = desc_add(d0, (kk >> 2) * 16384 + (kk & 3) * 32);
-            tc::mma_f16(tmem, d, d, id, kk > 0);
-        }
-        tc::mma_commit(bar);
-    }
-    bool done = false;
-    if (landed) {  // uniform
-        done = __syncthreads_and(tc::mbar_wait_bounded(bar, 0, a.budget)) != 0;
-        if (!done) {
-            if (tid == 0) raise_error(kErrTimeout);
-            tc::mbar_wait_bounded(bar, 0, 4000000000ull);
-        }
-    }
-    tc::tc_fence_after();
-
-    bool done2 = false;
-    if (landed && done) {
-        // ---- masks: A (fp32) for the solve; M (fp16) straight into the record.  TMEM lane
-        //      32 quad + lane is row r of [K;Q] K^T, this warp takes columns 32 chalf .. +31 -----------
-        {
-            float x[32];
-            tc::tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + 32 * chalf, x);
-            const int r = (32 * quad + lane) & 63, R = r >> 4, rl = r & 15;
-            const float gr = vb[r];
-            const bool isA = quad < 2;
-            const float sc = isA ? vb[128 + r] : 1.f;
+            const uint32_t hoff = (kk >> 2) * 8192;
+            const int c = 2 * (kk & 3);
+            uint32_t bq[4];
+            wm::ldsm_x4(kb + hoff + sw128(brow, c + (mi & 1)), bq);
 #pragma unroll
-            for (int blk = 0; blk < 2; ++blk) {
-                const int S = 2 * chalf + blk;
-                // blocks before the row's own: exp(gamma_r - gamma_e) exp(gamma_e - gamma_s), both <= 1
-                const float rowf = S < R ? __expf(gr - vb[16 * S + 15]) : 0.f;
+            for (int R = 0; R < 4; ++R) {
+                if (R < rmin0) continue;  // warp-uniform; rmin0 <= rmin1
+                uint32_t af[4];
+                wm::ldsm_x4(aop + hoff + sw128(16 * R + rr + 8 * (mi & 1), c + (mi >> 1)), af);
+                wm::mma16816x<BF>(acc[R][0], af, bq[0], bq[1]);
+                if (R >= rmin1) wm::mma16816x<BF>(acc[R][1], af, bq[2], bq[3]);
+            }
+        }
+        // masks on the accumulators: element e of tile (R, si) is row 16R + g8 + 8 (e >> 1),
+        // column 8 strip + 2 t4 + (e & 1); its column block is strip / 2
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int s = 16 * S + e;
-                    float f = rowf * vb[192 + s];
-                    if (S == R) f = (isA ? e < rl : e <= rl) ? __expf(gr - vb[s]) : 0.f;
-                    x[16 * blk + e] *= sc * f;
+        for (int si = 0; si < 2; ++si) {
+            const int s0 = 8 * strip[si] + 2 * t4, rmin = si ? rmin1 : rmin0, sb = strip[si] >> 1;
+            const float2 gs = *reinterpret_cast<const float2*>(vb + Cf::V_GAMMA + s0);
+            const float2 cf = *reinterpret_cast<const float2*>(vb + Cf::V_COLF + s0);
+#pragma unroll
+            for (int R = 0; R < 4; ++R) {
+                if (R < rmin) continue;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int r = 16 * R + g8 + 8 * hh;
+                    const float sc = mat ? 1.f : vb[Cf::V_BETA + r];
+                    float f0, f1;
+                    if (sb < R) {  // an earlier block: the split factors (warp-uniform branch)
+                        const float rf = vb[Cf::V_ROWF + 4 * r + sb] * sc;
+                        f0 = rf * cf.x;
+                        f1 = rf * cf.y;
+                    } else {       // the row's own block
+                        const float gr = vb[Cf::V_GAMMA + r];
+                        f0 = (mat ? s0 <= r : s0 < r) ? sc * __expf(gr - gs.x) : 0.f;
+                        f1 = (mat ? s0 + 1 <= r : s0 + 1 < r) ? sc * __expf(gr - gs.y) : 0.f;
+                    }
+                    acc[R][si][2 * hh] *= f0;
+                    acc[R][si][2 * hh + 1] *= f1;
                 }
             }
-            if (isA) {
+        }
+        if (mat == 0) {
 #pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4)
-                    sts4(fA + r * LD + 32 * chalf + 4 * c4, make_float4(x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]));
-            } else {
+            for (int R = 0; R < 4; ++R)
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) st16(rec + kRecM + tc::swz_off(r, 4 * chalf + cc, 128), pack8<false>(x + 8 * cc));
+                for (int si = 0; si < 2; ++si)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        *reinterpret_cast<float2*>(fA + (16 * R + g8 + 8 * hh) * LD + 8 * strip[si] + 2 * t4) =
+                            make_float2(acc[R][si][2 * hh], acc[R][si][2 * hh + 1]);
+        } else {
+            tc::bar_sync(1, 128);  // every Q-row warp has finished reading Q
+#pragma unroll
+            for (int R = 0; R < 4; ++R)
+#pragma unroll
+                for (int si = 0; si < 2; ++si)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = 16 * R + g8 + 8 * hh;
+                        sts32(Qt + sw128(r, strip[si]) + 4 * t4, pack2<false>(acc[R][si][2 * hh], acc[R][si][2 * hh + 1]));
+                    }
+            tc::fence_async_smem();
+            tc::bar_sync(1, 128);
+            if (tid == 128) {
+                tc::bulk_s2g(rec + kRecM, Qt, 8192);
+                tc::bulk_commit();
             }
         }
-        // K and V to fp16 in place for the second product (exact for |x| >= 2^-14); [K;Q] K^T
-        // has completed, so nothing reads them meanwhile
-        if constexpr (BF) {
-            to_f16_block<NT, 8192>(smem + Cf::OFF_K, tid);
-            to_f16_block<NT, 8192>(smem + Cf::OFF_K + 16384, tid);
-            to_f16_block<NT, 8192>(smem + Cf::OFF_V, tid);
-            to_f16_block<NT, 8192>(smem + Cf::OFF_V + Cf::KV_LBO, tid);
-        }
-        tc::tc_fence_before();
-        __syncthreads();
+    }
+    __syncthreads();
 
-        // ---- T = (I + A)^-1.  16x16 diagonal blocks by forward substitution (warps 0-3, lane =
-        //      column); the zeros above each diagonal are written too ---------------------------
-        if (warp < 4 && lane < 16) {
+    // ---- 3. T = (I + A)^-1.  The diagonal blocks (warps 0-3, lane = column), in place once the warp
+    //      has read its block ----------------------------------------------------------------------
+    if (warp < 4) {
+        if (lane < 16) {
             const int b0 = warp * 16, jc = lane;
             float xs[16];
 #pragma unroll
@@ -417,128 +478,158 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 2) chunk_ut_kernel(const __gri
                     const float4 t = lds4(fA + (b0 + r) * LD + b0 + 4 * q4);
                     arow[4 * q4] = t.x; arow[4 * q4 + 1] = t.y; arow[4 * q4 + 2] = t.z; arow[4 * q4 + 3] = t.w;
                 }
-                float acc = (r == jc) ? 1.f : 0.f;
+                float s0 = 0.f, s1 = 0.f;  // two partial sums shorten the dependent chain
 #pragma unroll
-                for (int s = 0; s < r; ++s) acc -= arow[s] * xs[s];
-                xs[r] = acc;
+                for (int s = 0; s < r; ++s) {
+                    if (s & 1) s1 -= arow[s] * xs[s];
+                    else s0 -= arow[s] * xs[s];
+                }
+                xs[r] = ((r == jc) ? 1.f : 0.f) + (s0 + s1);
             }
+            __syncwarp(0x0000ffffu);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) fT[(b0 + r) * LD + b0 + jc] = xs[r];
+            for (int r = 0; r < 16; ++r) fA[(b0 + r) * LD + b0 + jc] = xs[r];
         }
-        __syncthreads();
-        // level one (warps 0-3): T_i,i-1 = -T_ii (A_i,i-1 T_i-1,i-1) for i = 1, 3, one 8-column
-        // tile per warp
-        if (warp < 4) {
-            const int bi = warp >> 1, nt = warp & 1, i = 2 * bi + 1, j = i - 1;
-            uint32_t ah[4], al[4], bh[2], bl[2];
+    }
+    __syncthreads();
+    // T_i,i-1 = -T_ii (A_i,i-1 T_i-1,i-1) for i = 1, 3 (warps 0, 1), over A_i,i-1; the product in
+    // brackets goes to the (unused) upper block at rows 0-15, columns 32 + 16 warp
+    if (warp < 2) {
+        const int bi = 2 * warp + 1, bj = bi - 1;
+        float* x1 = fA + 32 + 16 * warp;
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        wm::load_a(fA, LD, 16 * bi, 16 * bj, 1.f, ah, al);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
             float d[4] = {0.f, 0.f, 0.f, 0.f};
-            wm::load_a(fA, LD, 16 * i, 16 * j, 1.f, ah, al);
-            wm::load_b(fT, LD, 16 * j, 16 * j + 8 * nt, bh, bl);
+            wm::load_b(fA, LD, 16 * bj, 16 * bj + 8 * nt, bh, bl);
             wm::mma_split(d, ah, al, bh, bl);
-            float* x1 = fX1 + bi * 16 * Cf::LDX1;
-            wm::store_c(x1, Cf::LDX1, 0, 8 * nt, d);
-            __syncwarp();
+            wm::store_c(x1, LD, 0, 8 * nt, d);
+        }
+        __syncwarp();
+        wm::load_a(fA, LD, 16 * bi, 16 * bi, -1.f, ah, al);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
             float e[4] = {0.f, 0.f, 0.f, 0.f};
-            wm::load_a(fT, LD, 16 * i, 16 * i, -1.f, ah, al);
-            wm::load_b(x1, Cf::LDX1, 0, 8 * nt, bh, bl);
+            wm::load_b(x1, LD, 0, 8 * nt, bh, bl);
             wm::mma_split(e, ah, al, bh, bl);
-            wm::store_c(fT, LD, 16 * i, 16 * j + 8 * nt, e);
+            wm::store_c(fA, LD, 16 * bi, 16 * bj + 8 * nt, e);
         }
-        __syncthreads();
-        // level two (all warps): X = A[32:64, 0:32] T[0:32, 0:32], then T[32:64, 0:32] = -T[32:64,
-        // 32:64] X; one 16x8 tile per warp, skipping the zero upper-right 16x16 blocks
-        {
-            const int mt = warp >> 2, nt = warp & 3;
-            uint32_t ah[4], al[4], bh[2], bl[2];
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+    }
+    __syncthreads();
+    // X = A[32:64, 0:32] T[0:32, 0:32] into the upper block rows 0-31, columns 32-63; then
+    // T[32:64, 0:32] = -T[32:64, 32:64] X over A, one 16x8 tile per warp, skipping the zero
+    // upper-right 16x16 blocks
+    {
+        const int mt = warp >> 2, nt = warp & 3;
+        float* x2 = fA + 32;
+        uint32_t ah[4], al[4], bh[2], bl[2];
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int kt = 0; kt < 2; ++kt) {
-                if (kt == 0 && nt >= 2) continue;  // T[0:16, 16:32] = 0
-                wm::load_a(fA, LD, 32 + 16 * mt, 16 * kt, 1.f, ah, al);
-                wm::load_b(fT, LD, 16 * kt, 8 * nt, bh, bl);
-                wm::mma_split(d, ah, al, bh, bl);
-            }
-            wm::store_c(fX2, Cf::LDX2, 16 * mt, 8 * nt, d);
-            __syncthreads();
-            float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int kt = 0; kt < 2; ++kt) {
-                if (mt == 0 && kt == 1) continue;  // T[32:48, 48:64] = 0
-                wm::load_a(fT, LD, 32 + 16 * mt, 32 + 16 * kt, -1.f, ah, al);
-                wm::load_b(fX2, Cf::LDX2, 16 * kt, 8 * nt, bh, bl);
-                wm::mma_split(e, ah, al, bh, bl);
-            }
-            wm::store_c(fT, LD, 32 + 16 * mt, 8 * nt, e);
+        for (int kt = 0; kt < 2; ++kt) {
+            if (kt == 0 && nt >= 2) continue;  // T[0:16, 16:32] = 0
+            wm::load_a(fA, LD, 32 + 16 * mt, 16 * kt, 1.f, ah, al);
+            wm::load_b(fA, LD, 16 * kt, 8 * nt, bh, bl);
+            wm::mma_split(d, ah, al, bh, bl);
         }
+        wm::store_c(x2, LD, 16 * mt, 8 * nt, d);
+        if (tid == 128) tc::bulk_wait_read0();  // M has left the Q tile, which [T_w; T_u] overwrites
         __syncthreads();
-        // ---- [T_w; T_u] (fp16) over A: T_w = T diag(beta Gamma) in rows 0-63, T_u = T diag(beta)
-        //      in rows 64-127, K-major with K = the chunk position s --------------------------------
-        uint8_t* top = smem + Cf::OFF_TOP;
+        float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int idx = tid + NT * u, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
-            const float4 t0v = lds4(fT + r * LD + 8 * cc), t1v = lds4(fT + r * LD + 8 * cc + 4);
-            const float4 b0v = lds4(vb + 128 + 8 * cc), b1v = lds4(vb + 128 + 8 * cc + 4);
-            float t8[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-            float s8[8] = {b0v.x, b0v.y, b0v.z, b0v.w, b1v.x, b1v.y, b1v.z, b1v.w};
-            if (which == 0) {
-                const float4 g0v = lds4(vb + 64 + 8 * cc), g1v = lds4(vb + 64 + 8 * cc + 4);
-                s8[0] *= g0v.x; s8[1] *= g0v.y; s8[2] *= g0v.z; s8[3] *= g0v.w;
-                s8[4] *= g1v.x; s8[5] *= g1v.y; s8[6] *= g1v.z; s8[7] *= g1v.w;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) t8[e] = (8 * cc + e <= r) ? t8[e] * s8[e] : 0.f;
-            st16(top + tc::swz_off(64 * which + r, cc, 128), pack8<false>(t8));
+        for (int kt = 0; kt < 2; ++kt) {
+            if (mt == 0 && kt == 1) continue;  // T[32:48, 48:64] = 0
+            wm::load_a(fA, LD, 32 + 16 * mt, 32 + 16 * kt, -1.f, ah, al);
+            wm::load_b(x2, LD, 16 * kt, 8 * nt, bh, bl);
+            wm::mma_split(e, ah, al, bh, bl);
         }
-        tc::fence_async_smem();
-        tc::tc_fence_before();
-        __syncthreads();
-        tc::tc_fence_after();
+        wm::store_c(fA, LD, 32 + 16 * mt, 8 * nt, e);
+    }
+    __syncthreads();
 
-        // ---- [T_w; T_u] [K | V] -> TMEM columns 0-255 (fp16, N = 256, four k-steps) ------------
-        if (tid == 0) {
-            constexpr uint32_t id = idesc16<false>(128, 256, false, true);
-            const uint64_t da = tc::smem_desc(sbase + Cf::OFF_TOP, 16, 1024, tc::kSw128);
-            const uint64_t db = tc::smem_desc(sbase + Cf::OFF_K, Cf::KV_LBO, 1024, tc::kSw128);  // MN-major
+    // ---- 4. [T_w; T_u] (fp16, rows 0-63 and 64-127 of the Q tile), lower triangle incl. diagonal --
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) tc::mma_f16(tmem, desc_add(da, kk * 32), desc_add(db, kk * 2048), id, kk > 0);
-            tc::mma_commit(bar);
-        }
-        done2 = tc::mbar_wait_bounded(bar, 1, a.budget);
-        if (!done2) {
-            raise_error(kErrTimeout);
-            tc::mbar_wait_bounded(bar, 1, 4000000000ull);
-        }
-        tc::tc_fence_after();
-        if (done2) {
-            // quadrants 0-1: -W row r, columns 64 chalf .. +63 -> dk half chalf of the record;
-            // quadrants 2-3: U~ row r, columns 128 + 64 chalf .. +63 -> dv slabs 2 chalf, 2 chalf + 1
-            const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-            const int r = (32 * quad + lane) & 63;
+    for (int q = 0; q < 4; ++q) {
+        const int idx = tid + NT * q, which = idx >> 9, r = (idx >> 3) & 63, cc = idx & 7;
+        const float4 t0v = lds4(fA + r * LD + 8 * cc), t1v = lds4(fA + r * LD + 8 * cc + 4);
+        const float* sv = vb + (which ? Cf::V_BETA : Cf::V_BG) + 8 * cc;  // column scales beta Gamma, beta
+        const float4 b0v = lds4(sv), b1v = lds4(sv + 4);
+        float t8[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+        const float s8[8] = {b0v.x, b0v.y, b0v.z, b0v.w, b1v.x, b1v.y, b1v.z, b1v.w};
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                float x[32];
-                tc::tmem_ld32(trow + (quad < 2 ? 0 : 128) + 64 * chalf + 32 * q, x);
-                if (quad < 2) {
+        for (int e = 0; e < 8; ++e) t8[e] = (8 * cc + e <= r) ? t8[e] * s8[e] : 0.f;
+        st16(Qt + sw128(64 * which + r, cc), pack8<false>(t8));
+    }
+    const bool isU = warp >= 4;
+    if (!__syncthreads_and(isU ? tc::mbar_wait_bounded(bar_v, 0, a.budget) : true)) {
+        if (tid == 128) tc::bulk_wait0();
+        drain();
+        return;
+    }
+
+    // W = T_w K (warps 0-3) and U~ = T_u V (warps 4-7), 32 output columns per warp in two passes
+    // of 16; row tile R of the triangular T needs k-steps 0..R only.  -W overwrites the K columns
+    // this warp alone has read (the record's dk-half layout); U~ goes over A, which nothing reads
+    // any more (the record's 64B-swizzled 32-column slabs).
+    {
+        const uint32_t bopnd = isU ? sbase + Cf::OFF_V : kb;
+        const uint32_t aopnd = qb + (isU ? 64 * 128 : 0);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = -x[e];
-                    uint8_t* dst = rec + kRecW + chalf * 8192;
+        for (int p = 0; p < 2; ++p) {
+            const int n0 = 32 * (warp & 3) + 16 * p, hf = n0 >> 6, cb = (n0 & 63) >> 3;
+            float acc[4][2][4];
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) st16(dst + tc::swz_off(r, 4 * q + cc, 128), pack8<false>(x + 8 * cc));
-                } else {
-                    uint8_t* dst = rec + kRecU + (2 * chalf + q) * kRecUSlab + r * 64;
+            for (int R = 0; R < 4; ++R)
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) st16(dst + 16 * cc, pack8<false>(x + 8 * cc));
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[R][nt][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t bv[4];
+                wm::ldsm_x4_t(bopnd + hf * 8192 + sw128(16 * kk + rr + 8 * (mi & 1), cb + (mi >> 1)), bv);
+                if constexpr (BF) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) bv[e] = wm::bf2_to_h2(bv[e]);
+                }
+#pragma unroll
+                for (int R = kk; R < 4; ++R) {
+                    uint32_t af[4];
+                    wm::ldsm_x4(aopnd + sw128(16 * R + rr + 8 * (mi & 1), 2 * kk + (mi >> 1)), af);
+                    wm::mma16816x<false>(acc[R][0], af, bv[0], bv[1]);
+                    wm::mma16816x<false>(acc[R][1], af, bv[2], bv[3]);
                 }
             }
+            if (!isU) __syncwarp();  // every lane has read these K columns
+#pragma unroll
+            for (int R = 0; R < 4; ++R)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int r = 16 * R + g8 + 8 * hh;
+                        const float x0 = acc[R][nt][2 * hh], x1 = acc[R][nt][2 * hh + 1];
+                        if (!isU) {
+                            sts32(Kt + hf * 8192 + sw128(r, cb + nt) + 4 * t4, pack2<false>(-x0, -x1));
+                        } else {
+                            const int n = n0 + 8 * nt + 2 * t4;
+                            sts32(smem + Cf::OFF_A + (n >> 5) * kRecUSlab + tc::swz_off(r, (n & 31) >> 3, 64) +
+                                      (n & 7) * 2,
+                                  pack2<false>(x0, x1));
+                        }
+                    }
         }
     }
-    tc::tc_fence_before();
+    tc::fence_async_smem();
     __syncthreads();
-    if (warp == 0) {
-        tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, Cf::TMEM_COLS);
+    if (tid == 0) {
+        tc::bulk_s2g(rec + kRecW, Kt, 16384);
+        tc::bulk_s2g(rec + kRecU, smem + Cf::OFF_A, 16384);
+        tc::bulk_commit();
     }
+    // the CTA may leave once its staged tiles have been read; the writes complete before any later
+    // grid (or programmatic dependent waiting on this one) reads them
+    if (tid == 0 || tid == 128) tc::bulk_wait_read0();
 }
 
 // =====================================================================================
@@ -554,7 +645,7 @@ struct ChainCfg {
     static constexpr int OFF_QW = 0;                           // [3 stages] [Q;-W]: 2 halves x [128 x 128 B]
     static constexpr int OFF_M = OFF_QW + 3 * 2 * QW_HALF;     // [2 slots] M fp16: [64 x 128 B]
     static constexpr int OFF_KS = OFF_M + 2 * 8192;            // [3 stages] K: 2 halves x [64 x 128 B]
-    static constexpr int OFF_UT = OFF_KS + 3 * 2 * K_HALF;     // [3 stages] U~ slab fp16 [64 x ROWB], row-major
+    static constexpr int OFF_UT = OFF_KS + 3 * 2 * K_HALF;     // [3 stages] U~ slab fp16 [64 x ROWB], 64B-swizzled
     static constexpr int OFF_SS = OFF_UT + 3 * 64 * ROWB;      // S [128 x ROWB]
     static constexpr int OFF_SU = OFF_SS + 128 * ROWB;         // [2 slots] U fp16: [64 x ROWB]
     static constexpr int OFF_SU2 = OFF_SU + 2 * 64 * ROWB;     // U' = f U fp16: [64 x ROWB]
@@ -918,10 +1009,10 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 tc::tmem_ld32(trow + Cf::COL_1B + b * NS, d2);
                 const int r = tid - 64;
                 float ut[NS];
-                const uint8_t* urow = smem + Cf::OFF_UT + kst * 64 * Cf::ROWB + r * Cf::ROWB;
+                const uint8_t* ust = smem + Cf::OFF_UT + kst * 64 * Cf::ROWB;
 #pragma unroll
                 for (int cc = 0; cc < NS / 8; ++cc) {
-                    const uint4 u4 = *reinterpret_cast<const uint4*>(urow + 16 * cc);
+                    const uint4 u4 = *reinterpret_cast<const uint4*>(ust + tc::swz_off(r, cc, 64));
                     const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
