@@ -138,7 +138,7 @@ def traffic_per_call():
     if not os.path.exists(path):
         return None
     src = b"".join(open(os.path.join(ROOT, "linear_attention_token_gdn_b200", "csrc", f), "rb").read()
-                   for f in ("chunk_tc.cuh", "tc_ptx.cuh", "common.cuh"))
+                   for f in ("chunk_tc.cuh", "tc_ptx.cuh", "common.cuh", "warp_mma.cuh"))
     digest = hashlib.sha256(src).hexdigest()[:16]
     fields = {}
     for line in open(path):
