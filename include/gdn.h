@@ -259,6 +259,19 @@ gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, flo
                           int dv, gdn_dtype_t y_dtype, gdn_dtype_t io_dtype, void* out,
                           gdn_stream_t stream);
 
+/*
+ * gdn_state_map_apply -- S_out = M S_in + B for each of `rows` states: a sequence segment's
+ * affine map applied to a state, the step that gives a rank of a context-parallel prefill its
+ * initial state.  Eq. (5) (S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T) is
+ * affine in S_{t-1}, so a segment maps S_start to M S_start + B, where M [dk,dk] is the
+ * segment's state after starting from S = I with v = 0 and B [dk,dv] its state after starting
+ * from S = 0 (both are S_T outputs of gdn_chunk_fwd).
+ *   M [rows,dk,dk], B [rows,dk,dv] (NULL: zero), S_in, S_out [rows,dk,dv]: fp32, row-major.
+ *   S_out must not overlap M, B or S_in.  dk, dv in {16,32,64,128}.  fp32 accumulation.
+ */
+gdn_status_t gdn_state_map_apply(const float* M, const float* B, const float* S_in, float* S_out, int rows,
+                                 int dk, int dv, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,6 +18,7 @@
 #include "out_gate.cuh"
 #include "prep.cuh"
 #include "recurrent.cuh"
+#include "state_map.cuh"
 #include "chunk_tc.cuh"
 
 namespace {
@@ -474,6 +475,27 @@ gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, flo
         default: launch_out_gate<128>(y, z, norm_w, eps, rows, (int)y_dtype, (int)io_dtype, out, st); break;
     }
     return launched("out_gate_kernel");
+}
+
+gdn_status_t gdn_state_map_apply(const float* M, const float* B, const float* S_in, float* S_out, int rows, int dk,
+                                 int dv, gdn_stream_t stream) {
+    REQUIRE(rows >= 0, "rows=%d < 0", rows);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    if (rows == 0) return GDN_OK;
+    REQUIRE_PTR(M, "M"); REQUIRE_PTR(S_in, "S_in"); REQUIRE_PTR(S_out, "S_out"); OPT_PTR(B, "B");
+    const size_t nm = (size_t)rows * dk * dk * 4, ns = (size_t)rows * dk * dv * 4;
+    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
+        const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+        return x < y + nb && y < x + na;
+    };
+    REQUIRE(!overlap(S_out, ns, S_in, ns) && !overlap(S_out, ns, M, nm) && (B == nullptr || !overlap(S_out, ns, B, ns)),
+            "S_out overlaps an input");
+    const long long grid = (long long)rows * (dk / 16) * (dv / 16);
+    REQUIRE(grid <= 0x7fffffffLL, "rows=%d too large", rows);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    gdn::LaunchScope timed(st, "state_map_kernel");
+    gdn::state_map_kernel<<<(unsigned)grid, 256, 0, st>>>(M, B, S_in, S_out, dk, dv);
+    return launched("state_map_kernel");
 }
 
 gdn_status_t gdn_timing_start(int max_launches) {

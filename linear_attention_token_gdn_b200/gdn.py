@@ -40,6 +40,7 @@ SIGNATURES = {
     "gdn_mixer_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _F, _F, _P, _P, _P, _I, _I,
                                _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
+    "gdn_state_map_apply": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
     "gdn_timing_start": ([_I], _I),
     "gdn_timing_stop": ([_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double),
                          ctypes.POINTER(_I)], _I),
@@ -255,6 +256,18 @@ def mixer_decode_step(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_l
                                        _ptr(state_slot), state.shape[0], B, H, dk, dv, float(scale), _dt(x_q),
                                        _DT[out.dtype], _ptr(out), _stream(stream)))
     return out
+
+
+def state_map_apply(M, B, S_in, S_out=None, stream=None):
+    """gdn_state_map_apply: S_out = M S_in + B per state row (B may be None: zero).  M is
+    [..., dk, dk], B, S_in and S_out [..., dk, dv], fp32.  Returns S_out."""
+    dk, dv = S_in.shape[-2], S_in.shape[-1]
+    rows = S_in.numel() // (dk * dv)
+    if S_out is None:
+        S_out = torch.empty_like(S_in)
+    _check(lib().gdn_state_map_apply(_ptr(M), _ptr(B) if B is not None else None, _ptr(S_in), _ptr(S_out), rows, dk,
+                                     dv, _stream(stream)))
+    return S_out
 
 
 def out_gate(y, z, norm_w, eps=1e-6, out=None, stream=None):

@@ -170,3 +170,17 @@ def test_mixer_decode_without_history_needs_no_conv_state(L):
     for zero rows)."""
     assert L.gdn_mixer_decode_step(A, A, A, A, A, A, 1, A, A, A, A, A, A, 1e-6, 1e-6, None, A, None, 4, 0, 2, 128,
                                    128, 1.0, 1, 1, A, None) == gdn.GDN_OK
+
+
+def test_state_map_apply_validation(L):
+    """gdn_state_map_apply: nothing to do for zero rows; bad sizes, misaligned pointers and an
+    output overlapping an input are refused before any launch."""
+    assert L.gdn_state_map_apply(None, None, None, None, 0, 128, 128, None) == gdn.GDN_OK
+    assert L.gdn_state_map_apply(A, None, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x40000), 2, 48, 128,
+                                 None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_state_map_apply(A, MIS, ctypes.c_void_p(0x20000), ctypes.c_void_p(0x40000), 2, 128, 128,
+                                 None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_state_map_apply(A, None, A, A, 2, 128, 128, None) == gdn.GDN_ERR_INVALID_ARG    # S_out is S_in
+    assert L.gdn_state_map_apply(ctypes.c_void_p(0x100000), None, A, ctypes.c_void_p(0x108000), 1, 128, 128,
+                                 None) == gdn.GDN_ERR_INVALID_ARG                                   # S_out over M
+    assert gdn.last_error_message() != ""

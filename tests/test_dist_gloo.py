@@ -84,3 +84,31 @@ def test_bench_rejects_a_world_size_that_differs_from_gpus():
     res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--launch-check"],
                          capture_output=True, text=True, timeout=120, env=env)
     assert res.returncode == 2 and "WORLD_SIZE=1" in res.stderr
+
+
+def test_context_parallel_gather_and_fold_on_three_gloo_ranks():
+    """Context-parallel prefill's exchange and fold, on CPU: three gloo ranks each hold a
+    segment of two sequences (one segment ragged), form their affine maps with the oracle,
+    exchange them through the product's gather, fold the earlier ranks' maps onto S0 and run
+    their segment from the folded state.  Concatenated, the segments must give the oracle's
+    single pass over the whole sequences (eq. 5 makes each segment affine in its start state)."""
+    segs = [64, 40, 88]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=dist_worker.run_cp, args=(r, 3, port, q, segs)) for r in range(3)]
+    for p in procs:
+        p.start()
+    out = sorted((q.get(timeout=120) for _ in procs), key=lambda d: d["rank"])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    x = inputs.make_prefill(inputs.TINY, "cpu", B=2, T=sum(segs), H=2, d=16, S0_std=0.05)
+    y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], x["cu_seqlens"])
+    T = sum(segs)
+    for d in out:
+        a, b = sum(segs[:d["rank"]]), sum(segs[:d["rank"] + 1])
+        n = b - a
+        assert np.allclose(d["y"][:n], y_ref[a:b], rtol=1e-9, atol=1e-12)
+        assert np.allclose(d["y"][n:], y_ref[T + a:T + b], rtol=1e-9, atol=1e-12)
+    assert np.allclose(out[-1]["S_T"], S_ref, rtol=1e-9, atol=1e-12)
