@@ -209,6 +209,30 @@ gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
                                    void* y, float* S_T, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_fwd_prep -- gdn_prep (eqs. (6)-(10)) fused into gdn_chunk_fwd's chunked pass: the
+ * projection outputs x_q, x_k, x_v go through ShortConv -> SiLU (-> L2Norm) inside the chunk
+ * kernel, and q, k, v, g, beta never reach HBM (q and k are kept in the workspace for the
+ * sequential pass).  Arguments as gdn_prep and gdn_chunk_fwd:
+ *   x_q, x_k, x_v [N,H,128], beta_logit, alpha_logit [N,H]: in_dtype (BF16 or F16).
+ *   conv_w_* [H*128, conv_width] fp32, conv_width in [1, 8]; A_log, alpha_bias [H] fp32.
+ *   qkv_dtype (BF16 or F16): the format q, k, v are rounded to before eqs. (1)-(4), as
+ *   gdn_prep's out_dtype would store them; the products then run on it.
+ *   S0, cu_seqlens, y, S_T, scale as in gdn_chunk_fwd.
+ * Only chunk = 64 and dk = dv = 128 are built (others: GDN_ERR_UNSUPPORTED).
+ * workspace: at least gdn_chunk_fwd_prep_workspace_size(...) bytes.
+ */
+size_t gdn_chunk_fwd_prep_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk);
+
+gdn_status_t gdn_chunk_fwd_prep(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
+                                const float* conv_w_k, const float* conv_w_v, int conv_width,
+                                const void* beta_logit, const void* alpha_logit, const float* A_log,
+                                const float* alpha_bias, float l2_eps, const float* S0,
+                                const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk, int dv,
+                                int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t qkv_dtype,
+                                gdn_dtype_t y_dtype, void* y, float* S_T, void* workspace,
+                                size_t workspace_bytes, gdn_stream_t stream);
+
+/*
  * gdn_decode_step -- one token per row against a resident state, eqs. (1)-(4):
  *   S <- alpha S + beta k e^T with e = v - alpha S^T k, y = scale * S^T q (new S).
  *   q, k [B,H,dk], v [B,H,dv]: in_dtype.  g, beta [B,H] fp32.

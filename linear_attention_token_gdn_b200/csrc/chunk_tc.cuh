@@ -193,29 +193,111 @@ __device__ __forceinline__ void to_f16_block(uint8_t* p, int it) {
 // chunk_ut_kernel: per (chunk, head) -- masks and the UT transform
 // =====================================================================================
 
-struct UtCfg {
+// PREP: the kernel also runs eqs. (6)-(10) (prep fused into the chunked pass): it loads the raw
+// projection outputs with the conv history before the chunk, so each tile half holds 72 rows.
+template <bool PREP>
+struct UtCfgT {
     static constexpr int THREADS = 256;
-    // K, Q, V as stored (bf16 or fp16), each two 8 KB dk (dv) halves [64 rows x 128 B] in the
-    // 128B-swizzled layout TMA writes.  After [K;Q] K^T the Q tile stages M (the record's layout)
-    // until it has been stored, then holds [T_w; T_u] (fp16, [128 rows x 128 B], same swizzle);
-    // -W overwrites K in place (the record's layout) once W has been formed.
-    static constexpr int OFF_K = 0, OFF_Q = 16384, OFF_V = 32768;
+    // K, Q, V, each two dk (dv) halves of 128-byte rows.  Without PREP: [64 rows x 128 B] as stored
+    // (bf16 or fp16), in the 128B-swizzled layout TMA writes.  With PREP: the raw rows of tokens
+    // t0 - (W-1) .. t0 + 63, unswizzled, overwritten in place by q, k, v (row r = token t0 + r, the
+    // operand format, 128B-swizzled relative to the half's base).  After [K;Q] K^T the Q tile stages
+    // M (the record's layout) until it has been stored, then holds [T_w; T_u] (fp16, [128 rows x 128
+    // B], same swizzle); -W overwrites K in place in the record's layout (halves 8 KB apart: with
+    // 9 KB halves, -W row r of half 1 lands on K row r - 8 of the same columns).
+    static constexpr int HS = PREP ? 9216 : 8192;           // bytes per tile half
+    static constexpr int OFF_K = 0, OFF_Q = 2 * HS, OFF_V = 4 * HS;
     // fp32 A, turned into T in place [64][LD]; its upper triangle is scratch of the block inverse;
     // once [T_w; T_u] has been formed, it stages U~ (the record's four slabs)
-    static constexpr int LD = 68, OFF_A = 49152;
+    static constexpr int LD = 68, OFF_A = 6 * HS;
     // per-position vectors (fp32): gamma, beta, beta Gamma, colf [64] each, then rowf [64][4]
     static constexpr int OFF_VEC = OFF_A + 64 * LD * 4;
     static constexpr int V_GAMMA = 0, V_BETA = 64, V_BG = 128, V_COLF = 192, V_ROWF = 256;
-    static constexpr int OFF_META = OFF_VEC + 4 * (V_ROWF + 256);
+    static constexpr int OFF_PSS = OFF_VEC + 4 * (V_ROWF + 256);  // PREP: row sums of squares [q, k][half][64]
+    static constexpr int OFF_META = OFF_PSS + (PREP ? 4 * 256 : 0);
     static constexpr int OFF_BAR = OFF_META + 32;           // K and Q landed, V landed
-    static constexpr int BYTES = OFF_BAR + 16 + 1024;       // + the 1024-byte alignment slack
+    // the base is aligned to the 1024-byte swizzle atom for TMA's 128B swizzle; the unswizzled raw
+    // tiles need 128 bytes (and three CTAs of this size just fit an SM)
+    static constexpr int ALIGN = PREP ? 128 : 1024;
+    static constexpr int BYTES = OFF_BAR + 16 + ALIGN;
     static_assert(64 * LD * 4 >= 16384 && OFF_A % 1024 == 0, "U~ staging fits over A");
+    static_assert(2 * HS >= 16384, "[T_w; T_u] fits in the Q tile");
+    static_assert(3 * (BYTES + 1024) <= 228 * 1024, "three CTAs per SM");
+};
+using UtCfg = UtCfgT<false>;
+
+// Inputs of the fused prep (eqs. (6)-(10)); unused without PREP.
+struct PrepIn {
+    const float *w_q, *w_k, *w_v;        // conv taps [H*d, W] fp32
+    int W;                               // conv width, 1..8
+    const void *beta_logit, *alpha_logit;  // [N, H], raw_dt
+    const float *A_log, *alpha_bias;     // [H]
+    float l2_eps;
+    int raw_dt;                          // x_q, x_k, x_v and the logits: bf16 or fp16
+    void *q_out, *k_out;                 // [N, H, 128] q and k in the operand format (for the chain)
 };
 
 // Shared-memory byte offset of 16-byte chunk c of row r in a [rows x 128 B] 128B-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
 __device__ __forceinline__ void sts32(uint8_t* p, uint32_t v) { *reinterpret_cast<uint32_t*>(p) = v; }
+
+// This lane's two channels (2 lane, 2 lane + 1) of raw row `row` of a 128-byte-row tile half.
+__device__ __forceinline__ float2 raw_pair(const uint8_t* half, int row, int lane, int raw_dt) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(half + row * 128 + 4 * lane);
+    return raw_dt == kBF16 ? unpack2<true>(w) : unpack2<false>(w);
+}
+
+// Eqs. (6)-(8) before the norm: ShortConv -> SiLU of this lane's two channels for the 64 output rows
+// of a tile half whose raw row i holds token t0 - (W-1) + i, so output row r (token t0 + r) reads
+// raw rows r .. r + W-1, tap j meeting row r + j (the order gdn_prep adds the taps in).  The window
+// is right-aligned in eight registers, the taps zero-padded in front, so every index is static.
+// first: the chunk starts its sequence, so the W-1 rows before it are the zero history.
+// f(r, y0, y1) receives each output row in order; raw row r is not read after output row r.
+template <typename F>
+__device__ __forceinline__ void conv_silu_half(const uint8_t* half, int W, const float (&wl)[8][2], bool first,
+                                               int lane, int raw_dt, F&& f) {
+    float2 xw[8];  // at output row r: xw[i] = raw row r + W - 8 + i
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        const int row = W - 8 + i - 1;  // raw row of xw[i] before the first shift
+        xw[i] = (row < 0 || (first && row < W - 1)) ? make_float2(0.f, 0.f) : raw_pair(half, row, lane, raw_dt);
+    }
+#pragma unroll 1
+    for (int r0 = 0; r0 < 64; r0 += 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = r0 + k;
+#pragma unroll
+            for (int i = 0; i < 7; ++i) xw[i] = xw[i + 1];
+            xw[7] = raw_pair(half, r + W - 1, lane, raw_dt);
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                a0 += wl[i][0] * xw[i].x;
+                a1 += wl[i][1] * xw[i].y;
+            }
+            f(r, __fdividef(a0, 1.0f + __expf(-a0)), __fdividef(a1, 1.0f + __expf(-a1)));
+        }
+    }
+}
+
+// This lane's taps (channels 64 hf + 2 lane, +1 of head h), right-aligned: wl[8 - W + j] = w[c][j].
+__device__ __forceinline__ void prep_taps(const float* w, int W, int h, int hf, int lane, float (&wl)[8][2]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int j = i - (8 - W);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) wl[i][u] = j >= 0 ? w[((size_t)h * 128 + 64 * hf + 2 * lane + u) * W + j] : 0.f;
+    }
+}
+
+// Output row r of a tile half, in the operand format, over raw row r (its 16-byte chunks swizzled
+// relative to the half's base), once every lane of the warp is past reading raw row r.
+__device__ __forceinline__ void put_row(uint8_t* half, int r, int lane, uint32_t packed) {
+    __syncwarp();
+    sts32(half + sw128(r, lane >> 2) + ((lane & 3) << 2), packed);
+}
 
 // Virtual chunk v -> (sequence n, chunk j of n) and the bounds [tb, te) of sequence n, from one
 // pass over cu_seqlens.  Warp-collective; false if v is past the end.
@@ -269,13 +351,14 @@ __device__ __forceinline__ void lower_tile(int idx, int& R, int& j) {
 //      |x| >= 2^-14), lower blocks only.
 //   5. -W, U~ and M leave as bulk copies of tiles staged in the record's layout; the gates
 //      Gamma_r and Gamma_C / Gamma_r go to the record directly.
-template <bool BF>
+template <bool BF, bool PREP>
 __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __grid_constant__ ChunkArgs a,
-                                                                     const __grid_constant__ ChainMaps maps) {
-    using Cf = UtCfg;
+                                                                     const __grid_constant__ ChainMaps maps,
+                                                                     const __grid_constant__ PrepIn p) {
+    using Cf = UtCfgT<PREP>;
     constexpr int LD = Cf::LD, NT = Cf::THREADS;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align_smem_1024(smem_raw);
+    uint8_t* smem = PREP ? smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u) : align_smem_1024(smem_raw);
     const uint32_t sbase = tc::smem_u32(smem);
     float* fA = reinterpret_cast<float*>(smem + Cf::OFF_A);
     float* vb = reinterpret_cast<float*>(smem + Cf::OFF_VEC);
@@ -304,19 +387,27 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
             meta[0] = found;
             meta[1] = t0;
             meta[2] = min(kChunk, te - t0);
+            meta[3] = j == 0;
+            // the end of the last sequence: tokens from there to N belong to no sequence
+            meta[4] = a.cu ? min(max(a.cu[a.num_seqs], 0), a.N) : a.N;
             if (found) {
+                // with PREP the maps cover the raw projection outputs, 64 + W - 1 rows from the conv
+                // history on (a load before token 0 reads zeros)
+                const int row0 = PREP ? t0 - (p.W - 1) : t0;
+                const uint32_t half_bytes = PREP ? (64 + p.W - 1) * 128 : 8192;
                 tc::mbar_init(bar_kq, 1);
                 tc::mbar_init(bar_v, 1);
                 tc::fence_mbar_init();
-                tc::mbar_arrive_expect_tx(bar_kq, 4 * 8192);
-                tc::mbar_arrive_expect_tx(bar_v, 2 * 8192);
+                tc::mbar_arrive_expect_tx(bar_kq, 4 * half_bytes);
+                tc::mbar_arrive_expect_tx(bar_v, 2 * half_bytes);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    tc::tma_load_3d(Kt + hf * 8192, &maps.k, 64 * hf, h, t0, bar_kq);
-                    tc::tma_load_3d(Qt + hf * 8192, &maps.q, 64 * hf, h, t0, bar_kq);
+                    tc::tma_load_3d(Kt + hf * Cf::HS, &maps.k, 64 * hf, h, row0, bar_kq);
+                    tc::tma_load_3d(Qt + hf * Cf::HS, &maps.q, 64 * hf, h, row0, bar_kq);
                 }
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) tc::tma_load_3d(smem + Cf::OFF_V + hf * 8192, &maps.v, 64 * hf, h, t0, bar_v);
+                for (int hf = 0; hf < 2; ++hf)
+                    tc::tma_load_3d(smem + Cf::OFF_V + hf * Cf::HS, &maps.v, 64 * hf, h, row0, bar_v);
             }
         }
     }
@@ -324,6 +415,8 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
     if (!meta[0]) return;  // uniform
     const int t0 = meta[1], L = meta[2];
     uint8_t* rec = reinterpret_cast<uint8_t*>(a.workspace) + ((size_t)v * H + h) * kRecBytes;
+    const bool first = meta[3] != 0;  // the chunk starts its sequence (PREP: a zero conv history)
+    const int stop = meta[4];
     auto drain = [&]() {  // a copy did not land in time: flag it and let every copy finish
         if (tid == 0) {
             raise_error(kErrTimeout);
@@ -337,11 +430,26 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
     //      record gets Gamma_r and f_r = exp(gamma_C - gamma_r).  The decay exp(gamma_r - gamma_s)
     //      of a pair in different 16-blocks is split at the end e of s's block into
     //      rowf[r][blk s] = exp(gamma_r - gamma_e) and colf[s] = exp(gamma_e - gamma_s), both <= 1.
-    if (warp == 1) {
+    if (warp == (PREP ? 6 : 1)) {
         const int r0 = 2 * lane;
         const size_t i0 = (size_t)(t0 + r0) * H + h;
-        const float g0 = r0 < L ? a.g[i0] : 0.f, g1 = r0 + 1 < L ? a.g[i0 + H] : 0.f;
-        const float b0 = r0 < L ? a.beta[i0] : 0.f, b1 = r0 + 1 < L ? a.beta[i0 + H] : 0.f;
+        float g0 = 0.f, g1 = 0.f, b0 = 0.f, b1 = 0.f;
+        if constexpr (PREP) {  // eqs. (9), (10) as gdn_prep forms them
+            const float ea = expf(p.A_log[h]), bias = p.alpha_bias[h];
+            if (r0 < L) {
+                b0 = 1.0f / (1.0f + expf(-ld1(p.beta_logit, p.raw_dt, i0)));
+                g0 = -ea * softplusf_(ld1(p.alpha_logit, p.raw_dt, i0) + bias);
+            }
+            if (r0 + 1 < L) {
+                b1 = 1.0f / (1.0f + expf(-ld1(p.beta_logit, p.raw_dt, i0 + H)));
+                g1 = -ea * softplusf_(ld1(p.alpha_logit, p.raw_dt, i0 + H) + bias);
+            }
+        } else {
+            g0 = r0 < L ? a.g[i0] : 0.f;
+            g1 = r0 + 1 < L ? a.g[i0 + H] : 0.f;
+            b0 = r0 < L ? a.beta[i0] : 0.f;
+            b1 = r0 + 1 < L ? a.beta[i0 + H] : 0.f;
+        }
         float s = g0 + g1;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -375,6 +483,51 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
         drain();
         return;
     }
+    if constexpr (PREP) {
+        // ---- eqs. (6)-(8): q, k, v from the raw rows, in place.  Warps 0-5: tensor w >> 1 (q, k, v),
+        //      half w & 1, all 64 rows.  For q and k pass one sums each row's squares over this half
+        //      (the L2Norm needs both halves, exchanged through shared memory between the two warps
+        //      of the tensor); pass two recomputes the conv, normalises, rounds to the operand format
+        //      and writes each row over its raw row, and to q_out / k_out for the chain.  v: one
+        //      pass, no norm. --------------------------------------------------------------------
+        bool okv = true;
+        if (warp < 6) {
+            const int ten = warp >> 1, hf = warp & 1;
+            uint8_t* half = (ten == 0 ? Qt : ten == 1 ? Kt : smem + Cf::OFF_V) + hf * Cf::HS;
+            float wl[8][2];
+            prep_taps(ten == 0 ? p.w_q : ten == 1 ? p.w_k : p.w_v, p.W, h, hf, lane, wl);
+            if (ten < 2) {
+                float* pss = reinterpret_cast<float*>(smem + Cf::OFF_PSS) + ten * 128;
+                conv_silu_half(half, p.W, wl, first, lane, p.raw_dt, [&](int r, float y0, float y1) {
+                    const float ss = warp_sum(y0 * y0 + y1 * y1);
+                    if (lane == 0) pss[hf * 64 + r] = ss;
+                });
+                tc::bar_sync(2 + ten, 64);
+                uint16_t* gout = reinterpret_cast<uint16_t*>(ten ? p.k_out : p.q_out);
+                conv_silu_half(half, p.W, wl, first, lane, p.raw_dt, [&](int r, float y0, float y1) {
+                    const float inv = rsqrtf(pss[r] + pss[64 + r] + p.l2_eps);
+                    const uint32_t o = pack2<BF>(y0 * inv, y1 * inv);
+                    put_row(half, r, lane, o);
+                    // rows of this sequence; zeros for tokens of no sequence (the chain reads them in
+                    // its last chunk, against zero coefficients); rows of the next sequence are its
+                    // own CTA's
+                    uint32_t* gp =
+                        reinterpret_cast<uint32_t*>(gout + ((size_t)(t0 + r) * H + h) * 128 + 64 * hf + 2 * lane);
+                    if (r < L) *gp = o;
+                    else if (t0 + r >= stop && t0 + r < a.N) *gp = 0u;
+                });
+            } else {
+                okv = tc::mbar_wait_bounded(bar_v, 0, a.budget);
+                if (okv)
+                    conv_silu_half(half, p.W, wl, first, lane, p.raw_dt,
+                                   [&](int r, float y0, float y1) { put_row(half, r, lane, pack2<BF>(y0, y1)); });
+            }
+        }
+        if (!__syncthreads_and(okv)) {
+            drain();
+            return;
+        }
+    }
 
     // ---- 1-2. [K;Q] K^T and the masks --------------------------------------------------------------
     {
@@ -392,7 +545,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
                 for (int e = 0; e < 4; ++e) acc[R][si][e] = 0.f;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t hoff = (kk >> 2) * 8192;
+            const uint32_t hoff = (kk >> 2) * Cf::HS;
             const int c = 2 * (kk & 3);
             uint32_t bq[4];
             wm::ldsm_x4(kb + hoff + sw128(brow, c + (mi & 1)), bq);
@@ -561,7 +714,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
         st16(Qt + sw128(64 * which + r, cc), pack8<false>(t8));
     }
     const bool isU = warp >= 4;
-    if (!__syncthreads_and(isU ? tc::mbar_wait_bounded(bar_v, 0, a.budget) : true)) {
+    if (!__syncthreads_and(isU && !PREP ? tc::mbar_wait_bounded(bar_v, 0, a.budget) : true)) {
         if (tid == 128) tc::bulk_wait0();
         drain();
         return;
@@ -587,7 +740,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t bv[4];
-                wm::ldsm_x4_t(bopnd + hf * 8192 + sw128(16 * kk + rr + 8 * (mi & 1), cb + (mi >> 1)), bv);
+                wm::ldsm_x4_t(bopnd + hf * Cf::HS + sw128(16 * kk + rr + 8 * (mi & 1), cb + (mi >> 1)), bv);
                 if constexpr (BF) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) bv[e] = wm::bf2_to_h2(bv[e]);
@@ -1206,11 +1359,15 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
     }
 }
 
-template <bool BF>
-inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, cudaStream_t st) {
+// ut_maps: the tiles chunk_ut_kernel loads (q, k, v, or with PREP the raw projection outputs);
+// maps: the chain's (k and q as the chain reads them, y or out, z).
+template <bool BF, bool PREP>
+inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& ut_maps, const ChainMaps& maps, const PrepIn& p,
+                                     cudaStream_t st) {
     constexpr int NS = 32;
     using Ch = ChainCfg<NS>;
-    cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel<BF>, cudaFuncAttributeMaxDynamicSharedMemorySize, UtCfg::BYTES);
+    using Ut = UtCfgT<PREP>;
+    cudaError_t e = cudaFuncSetAttribute(chunk_ut_kernel<BF, PREP>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ut::BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chunk_chain_kernel<NS, BF, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, Ch::BYTES);
     if (e != cudaSuccess) return e;
@@ -1218,8 +1375,8 @@ inline cudaError_t chunk_tc_launch_t(const ChunkArgs& a, const ChainMaps& maps, 
     if (e != cudaSuccess) return e;
     const long long nvc = chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr);
     if (nvc > 0) {
-        LaunchScope timed(st, "chunk_ut_kernel");
-        chunk_ut_kernel<BF><<<(unsigned)(nvc * a.H), UtCfg::THREADS, UtCfg::BYTES, st>>>(a, maps);
+        LaunchScope timed(st, PREP ? "chunk_ut_prep_kernel" : "chunk_ut_kernel");
+        chunk_ut_kernel<BF, PREP><<<(unsigned)(nvc * a.H), Ut::THREADS, Ut::BYTES, st>>>(a, ut_maps, p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1273,7 +1430,36 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
         *why = "cuTensorMapEncodeTiled failed";
         return cudaSuccess;
     }
-    return a.in_dt == kBF16 ? chunk_tc_launch_t<true>(a, maps, st) : chunk_tc_launch_t<false>(a, maps, st);
+    const PrepIn none = {};
+    return a.in_dt == kBF16 ? chunk_tc_launch_t<true, false>(a, maps, maps, none, st)
+                            : chunk_tc_launch_t<false, false>(a, maps, maps, none, st);
+}
+
+// The chunked path with eqs. (6)-(10) fused into chunk_ut_kernel: x_q, x_k, x_v (p.raw_dt) are
+// the projection outputs; a.in_dt is the operand format q, k, v are rounded to (bf16 or fp16), in
+// which p.q_out / p.k_out receive q and k for the chain.  a.q, a.k, a.v, a.g, a.beta are unused.
+inline cudaError_t chunk_tc_prep_launch(const ChunkArgs& a, const PrepIn& p, const void* x_q, const void* x_k,
+                                        const void* x_v, cudaStream_t st, const char** why) {
+    *why = nullptr;
+    if (a.chunk != kChunk) {
+        *why = "only chunk = 64 is built";
+        return cudaSuccess;
+    }
+    constexpr int NS = 32;
+    const CUtensorMapSwizzle yswz = a.y_dt == kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    ChainMaps raw = {}, maps = {};
+    const uint32_t rows = 64 + p.W - 1;
+    if (!encode_map_3d(&raw.k, x_k, p.raw_dt, a.N, a.H, 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_map_3d(&raw.q, x_q, p.raw_dt, a.N, a.H, 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_map_3d(&raw.v, x_v, p.raw_dt, a.N, a.H, 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_map_3d(&maps.k, p.k_out, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_3d(&maps.q, p.q_out, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, 128, NS, kChunk, yswz)) {
+        *why = "cuTensorMapEncodeTiled failed";
+        return cudaSuccess;
+    }
+    return a.in_dt == kBF16 ? chunk_tc_launch_t<true, true>(a, raw, maps, p, st)
+                            : chunk_tc_launch_t<false, true>(a, raw, maps, p, st);
 }
 
 }  // namespace gdn

@@ -377,6 +377,55 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
     return GDN_OK;
 }
 
+size_t gdn_chunk_fwd_prep_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk) {
+    const size_t rec = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+    return rec == 0 ? 0 : rec + 2 * (size_t)N * H * dk * 2;  // + q and k in the operand format
+}
+
+gdn_status_t gdn_chunk_fwd_prep(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
+                                const float* conv_w_k, const float* conv_w_v, int conv_width, const void* beta_logit,
+                                const void* alpha_logit, const float* A_log, const float* alpha_bias, float l2_eps,
+                                const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
+                                int dv, int chunk, float scale, gdn_dtype_t in_dtype, gdn_dtype_t qkv_dtype,
+                                gdn_dtype_t y_dtype, void* y, float* S_T, void* workspace, size_t workspace_bytes,
+                                gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(qkv_dtype) && dtype_ok(y_dtype), "bad dtype");
+    REQUIRE(conv_width >= 1 && conv_width <= 8, "conv_width=%d not in [1, 8]", conv_width);
+    REQUIRE(l2_eps >= 0.f, "l2_eps < 0");
+    REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
+    REQUIRE((long long)N * H * 128 < (1LL << 40), "problem too large");
+    REQUIRE((long long)num_seqs * H * 128 <= 0x7fffffffLL, "num_seqs*H too large (%d x %d)", num_seqs, H);
+    if (chunk != 64 || dk != 128 || dv != 128 || in_dtype == GDN_F32 || qkv_dtype == GDN_F32)
+        return fail(GDN_ERR_UNSUPPORTED, "the fused prep runs the tensor-core path only (chunk 64, dk=dv=128, "
+                                         "16-bit inputs and q/k/v format)");
+    if (N == 0)  // every sequence is empty: S_T = S0 (or zero)
+        return gdn_chunk_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, S0, cu_seqlens, num_seqs, 0, H, dk, dv, 0,
+                             scale, qkv_dtype, y_dtype, y, S_T, nullptr, 0, stream);
+    REQUIRE_PTR(x_q, "x_q"); REQUIRE_PTR(x_k, "x_k"); REQUIRE_PTR(x_v, "x_v");
+    REQUIRE_PTR(conv_w_q, "conv_w_q"); REQUIRE_PTR(conv_w_k, "conv_w_k"); REQUIRE_PTR(conv_w_v, "conv_w_v");
+    REQUIRE_PTR(beta_logit, "beta_logit"); REQUIRE_PTR(alpha_logit, "alpha_logit");
+    REQUIRE_PTR(A_log, "A_log"); REQUIRE_PTR(alpha_bias, "alpha_bias"); REQUIRE_PTR(y, "y");
+    OPT_PTR(S0, "S0"); OPT_PTR(S_T, "S_T"); OPT_PTR(cu_seqlens, "cu_seqlens");
+    const size_t need = gdn_chunk_fwd_prep_workspace_size(N, num_seqs, H, dk, dv, chunk);
+    REQUIRE_PTR(workspace, "workspace");
+    REQUIRE(workspace_bytes >= need, "workspace of %zu bytes < %zu", workspace_bytes, need);
+    const size_t rec = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
+    uint8_t* q_out = reinterpret_cast<uint8_t*>(workspace) + rec;
+    uint8_t* k_out = q_out + (size_t)N * H * dk * 2;
+    gdn::PrepIn p{conv_w_q, conv_w_k, conv_w_v, conv_width, beta_logit, alpha_logit, A_log, alpha_bias, l2_eps,
+                  (int)in_dtype, q_out, k_out};
+    gdn::ChunkArgs a{nullptr, nullptr, nullptr, nullptr, nullptr, S0, cu_seqlens, num_seqs, N, H, chunk, scale,
+                     (int)qkv_dtype, (int)y_dtype, y, S_T, workspace, wait_budget()};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const char* why = nullptr;
+    cudaError_t e = gdn::chunk_tc_prep_launch(a, p, x_q, x_k, x_v, st, &why);
+    if (why) return fail(GDN_ERR_CUDA, "chunk_tc: %s", why);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "chunk_tc: %s", cudaGetErrorString(e));
+    return GDN_OK;
+}
+
 gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* g, const float* beta,
                                  const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
                                  int dv, int chunk, float scale, gdn_dtype_t in_dtype, const void* z,

@@ -41,6 +41,9 @@ SIGNATURES = {
                                _I, _I, _I, _F, _I, _I, _P, _P], _I),
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
     "gdn_state_map_apply": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
+    "gdn_chunk_fwd_prep_workspace_size": ([_I, _I, _I, _I, _I, _I], ctypes.c_size_t),
+    "gdn_chunk_fwd_prep": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _F, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                            _I, _P, _P, _P, ctypes.c_size_t, _P], _I),
     "gdn_timing_start": ([_I], _I),
     "gdn_timing_stop": ([_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(_I), ctypes.POINTER(ctypes.c_double),
                          ctypes.POINTER(_I)], _I),
@@ -256,6 +259,35 @@ def mixer_decode_step(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_l
                                        _ptr(state_slot), state.shape[0], B, H, dk, dv, float(scale), _dt(x_q),
                                        _DT[out.dtype], _ptr(out), _stream(stream)))
     return out
+
+
+def chunk_fwd_prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bias, S0=None,
+                   cu_seqlens=None, num_seqs=None, l2_eps=1e-6, scale=1.0, qkv_dtype=None, y_dtype=None, y=None,
+                   S_T=None, final_state=True, workspace=None, stream=None):
+    """gdn_chunk_fwd_prep: prep (eqs. (6)-(10)) fused into the chunked pass.  q, k, v are rounded
+    to qkv_dtype (default: the inputs' format) before the recurrence.  Returns (y, S_T or None)."""
+    N, H, dk = x_q.shape
+    dv = x_v.shape[2]
+    W = w_q.shape[-1]
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    elif num_seqs is None:
+        num_seqs = 1
+    qkv_dtype = x_q.dtype if qkv_dtype is None else qkv_dtype
+    y_dtype = qkv_dtype if y_dtype is None else y_dtype
+    if y is None:
+        y = torch.empty(N, H, dv, device=x_q.device, dtype=y_dtype)
+    if S_T is None and final_state:
+        S_T = torch.empty(num_seqs, H, dk, dv, device=x_q.device)
+    if workspace is None:
+        nbytes = lib().gdn_chunk_fwd_prep_workspace_size(N, num_seqs, H, dk, dv, 64)
+        workspace = torch.empty(max(nbytes, 16), device=x_q.device, dtype=torch.uint8)
+    _check(lib().gdn_chunk_fwd_prep(_ptr(x_q), _ptr(x_k), _ptr(x_v), _ptr(w_q), _ptr(w_k), _ptr(w_v), W,
+                                    _ptr(beta_logit), _ptr(alpha_logit), _ptr(A_log), _ptr(alpha_bias), float(l2_eps),
+                                    _ptr(S0), _ptr(cu_seqlens), num_seqs, N, H, dk, dv, 64, float(scale), _dt(x_q),
+                                    _DT[qkv_dtype], _DT[y_dtype], _ptr(y), _ptr(S_T), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y, S_T
 
 
 def state_map_apply(M, B, S_in, S_out=None, stream=None):

@@ -184,3 +184,29 @@ def test_state_map_apply_validation(L):
     assert L.gdn_state_map_apply(ctypes.c_void_p(0x100000), None, A, ctypes.c_void_p(0x108000), 1, 128, 128,
                                  None) == gdn.GDN_ERR_INVALID_ARG                                   # S_out over M
     assert gdn.last_error_message() != ""
+
+
+def prep_call(L, **over):
+    a = dict(xq=A, W=4, eps=1e-6, N=64, H=2, dk=128, dv=128, chunk=64, in_dt=gdn.BF16, qkv=gdn.F16, y_dt=gdn.BF16,
+             ws=A, ws_bytes=1 << 30)
+    a.update(over)
+    return L.gdn_chunk_fwd_prep(a["xq"], A, A, A, A, A, a["W"], A, A, A, A, a["eps"], None, None, 1, a["N"], a["H"],
+                                a["dk"], a["dv"], a["chunk"], 1.0, a["in_dt"], a["qkv"], a["y_dt"], A, None, a["ws"],
+                                a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over", [dict(W=0), dict(W=9), dict(eps=-1.0), dict(xq=None), dict(ws=None),
+                                  dict(ws_bytes=16), dict(in_dt=9), dict(dk=48)])
+def test_chunk_fwd_prep_rejects_bad_arguments(L, over):
+    assert prep_call(L, **over) == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.last_error_message() != ""
+
+
+@pytest.mark.parametrize("over", [dict(chunk=0), dict(dk=64, dv=64), dict(in_dt=gdn.F32), dict(qkv=gdn.F32)])
+def test_chunk_fwd_prep_is_tensor_core_only(L, over):
+    assert prep_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_chunk_fwd_prep_workspace_holds_records_and_q_k(L):
+    rec = L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64)
+    assert L.gdn_chunk_fwd_prep_workspace_size(8192, 2, 16, 128, 128, 64) == rec + 2 * 8192 * 16 * 128 * 2
