@@ -67,6 +67,9 @@ def _load():
                                             ctypes.c_int, _D]
             lib.oracle_decode_step.argtypes = [_D, _D, _D, _D, _D, _D, _I64, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_double, _D, ctypes.c_int]
+            lib.oracle_backward.argtypes = [_D, _D, _D, _D, _D, _D, _I64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, _D, _D, _D, _D, _D, _D, _D, _D,
+                                            ctypes.c_int]
             lib.oracle_threads_used.argtypes = [ctypes.c_int, ctypes.c_long]
             lib.oracle_threads_used.restype = ctypes.c_int
             _lib = lib
@@ -126,6 +129,25 @@ def recurrence(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=1, scale=1.0
                               cu.ctypes.data_as(_I64), num_seqs, H, dk, dv, float(scale),
                               _ptr(y), _ptr(S_T), int(nthreads))
     return y, S_T
+
+
+def backward(q, k, v, g, beta, dy, S0=None, dS_T=None, cu_seqlens=None, num_seqs=1, scale=1.0, nthreads=0):
+    """Reverse-mode gradients through eqs. (1)-(4): for a loss L with dL/dy = dy and
+    dL/dS_T = dS_T (None: zero), returns dict(dq, dk, dv, dg, dbeta, dS0) in float64 (dg is
+    the gradient with respect to g = log alpha)."""
+    q, k, v, g, beta, S0, dy, dS_T = (_f64(t) for t in (q, k, v, g, beta, S0, dy, dS_T))
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        num_seqs = len(cu_seqlens) - 1
+    cu = _cu(cu_seqlens, N, num_seqs)
+    out = dict(dq=np.zeros((N, H, dk)), dk=np.zeros((N, H, dk)), dv=np.zeros((N, H, dv)), dg=np.zeros((N, H)),
+               dbeta=np.zeros((N, H)), dS0=np.zeros((num_seqs, H, dk, dv)))
+    _load().oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), cu.ctypes.data_as(_I64),
+                            num_seqs, H, dk, dv, float(scale), _ptr(dy), _ptr(dS_T), _ptr(out["dq"]),
+                            _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]),
+                            int(nthreads))
+    return out
 
 
 def decode_step(q, k, v, g, beta, state, state_slot=None, scale=1.0, nthreads=0, inplace=False):

@@ -162,6 +162,132 @@ void oracle_recurrence(const double* q, const double* k, const double* v, const 
 }
 
 /* ------------------------------------------------------------------------- */
+/* Reverse-mode derivative of eqs. (1)-(4)                                     */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * For a loss L with dL/dy_t = dy_t and dL/dS_T = dS_T, the token step of eqs. (1)-(4),
+ *   S~ = alpha S,  e = v - S~^T k,  S_t = S~ + beta k e^T,  y = scale S_t^T q,
+ * (S = S_{t-1}, alpha = exp(g)) is walked backwards with D = dL/dS_t:
+ *   D  += scale q dy^T               dq = scale S_t dy
+ *   de  = beta D^T k                 dbeta = k^T D e          dk = beta D e - S~ de
+ *   dv  = de                         D~ = D - k de^T          (= dL/dS~)
+ *   dg  = alpha sum_ij D~_ij S_ij    D <- alpha D~            (= dL/dS_{t-1})
+ * and dS0 is D after the first token.  The states S_{t-1} come from a forward pass that
+ * keeps the state at the start of every 64 tokens and recomputes each such block's states
+ * before walking it backwards.
+ */
+typedef struct {
+    const double *q, *k, *v, *g, *beta, *S0, *dy, *dS_T;
+    const int64_t* cu;
+    int H, dk, dv;
+    double scale;
+    double *dq, *dk_, *dv_, *dg, *dbeta, *dS0;
+} bwd_ctx;
+
+enum { BWD_BLOCK = 64 };
+
+static void bwd_unit(void* vctx, long unit) {
+    bwd_ctx* c = (bwd_ctx*)vctx;
+    const int H = c->H, dk = c->dk, dv = c->dv;
+    const long n = unit / H;
+    const int h = (int)(unit % H);
+    const size_t SZ = (size_t)dk * dv;
+    const int64_t t0 = c->cu[n], t1 = c->cu[n + 1];
+    const long nb = (long)((t1 - t0 + BWD_BLOCK - 1) / BWD_BLOCK);
+    double* ck = (double*)malloc(sizeof(double) * SZ * (nb > 0 ? nb : 1));      /* state at each block start */
+    double* st = (double*)malloc(sizeof(double) * SZ * (BWD_BLOCK + 1));        /* one block's states */
+    double* S = (double*)calloc(SZ, sizeof(double));
+    double* D = (double*)calloc(SZ, sizeof(double));
+    double* e = (double*)malloc(sizeof(double) * dv);
+    double* de = (double*)malloc(sizeof(double) * dv);
+    double* ytmp = (double*)malloc(sizeof(double) * dv);
+    if (c->S0) memcpy(S, c->S0 + ((size_t)n * H + h) * SZ, sizeof(double) * SZ);
+    for (int64_t t = t0; t < t1; ++t) {
+        if ((t - t0) % BWD_BLOCK == 0) memcpy(ck + (size_t)((t - t0) / BWD_BLOCK) * SZ, S, sizeof(double) * SZ);
+        const size_t th = (size_t)t * H + h;
+        token_update(S, c->q + th * dk, c->k + th * dk, c->v + th * dv, exp(c->g[th]), c->beta[th], dk, dv, c->scale,
+                     ytmp, e);
+    }
+    if (c->dS_T) memcpy(D, c->dS_T + ((size_t)n * H + h) * SZ, sizeof(double) * SZ);
+    for (long b = nb - 1; b >= 0; --b) {
+        const int64_t tb = t0 + (int64_t)b * BWD_BLOCK, te = tb + BWD_BLOCK < t1 ? tb + BWD_BLOCK : t1;
+        memcpy(st, ck + (size_t)b * SZ, sizeof(double) * SZ);
+        for (int64_t t = tb; t < te; ++t) {  /* st[i] = S_{tb + i - 1}, the state before token tb + i */
+            const size_t th = (size_t)t * H + h;
+            double* nxt = st + (size_t)(t - tb + 1) * SZ;
+            memcpy(nxt, st + (size_t)(t - tb) * SZ, sizeof(double) * SZ);
+            token_update(nxt, c->q + th * dk, c->k + th * dk, c->v + th * dv, exp(c->g[th]), c->beta[th], dk, dv,
+                         c->scale, ytmp, e);
+        }
+        for (int64_t t = te - 1; t >= tb; --t) {
+            const size_t th = (size_t)t * H + h;
+            const double* q = c->q + th * dk;
+            const double* k = c->k + th * dk;
+            const double* v = c->v + th * dv;
+            const double* dyt = c->dy + th * dv;
+            const double alpha = exp(c->g[th]), beta = c->beta[th];
+            const double* Sp = st + (size_t)(t - tb) * SZ;      /* S_{t-1} */
+            const double* St = st + (size_t)(t - tb + 1) * SZ;  /* S_t */
+            for (int j = 0; j < dv; ++j) {                       /* e = v - alpha S_{t-1}^T k */
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += Sp[(size_t)i * dv + j] * k[i];
+                e[j] = v[j] - alpha * acc;
+            }
+            for (int i = 0; i < dk; ++i) {                       /* readout */
+                double acc = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    D[(size_t)i * dv + j] += c->scale * q[i] * dyt[j];
+                    acc += St[(size_t)i * dv + j] * dyt[j];
+                }
+                c->dq[th * dk + i] = c->scale * acc;
+            }
+            double db = 0.0;
+            for (int j = 0; j < dv; ++j) {                       /* de = beta D^T k */
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += D[(size_t)i * dv + j] * k[i];
+                de[j] = beta * acc;
+                db += acc * e[j];                                /* k^T D e */
+            }
+            c->dbeta[th] = db;
+            for (int i = 0; i < dk; ++i) {                       /* dk = beta D e - S~ de */
+                double a = 0.0, b2 = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    a += D[(size_t)i * dv + j] * e[j];
+                    b2 += alpha * Sp[(size_t)i * dv + j] * de[j];
+                }
+                c->dk_[th * dk + i] = beta * a - b2;
+            }
+            for (int j = 0; j < dv; ++j) c->dv_[th * dv + j] = de[j];
+            double da = 0.0;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j) {
+                    const size_t ij = (size_t)i * dv + j;
+                    D[ij] -= k[i] * de[j];                       /* D~ */
+                    da += D[ij] * Sp[ij];
+                    D[ij] *= alpha;                              /* dL/dS_{t-1} */
+                }
+            c->dg[th] = alpha * da;
+        }
+    }
+    memcpy(c->dS0 + ((size_t)n * H + h) * SZ, D, sizeof(double) * SZ);
+    free(ytmp); free(de); free(e); free(D); free(S); free(st); free(ck);
+}
+
+/*
+ * Gradients of L through eqs. (1)-(4) for packed sequences.  q, k, dq, dk: [N, H, dk];
+ * v, dy, dv: [N, H, dv]; g, beta, dg, dbeta: [N, H]; S0, dS_T, dS0: [num_seqs, H, dk, dv]
+ * (S0 and dS_T may be NULL = zeros).  Tokens outside every sequence are not written.
+ */
+void oracle_backward(const double* q, const double* k, const double* v, const double* g, const double* beta,
+                     const double* S0, const int64_t* cu_seqlens, int num_seqs, int H, int dk, int dv, double scale,
+                     const double* dy, const double* dS_T, double* dq, double* dk_, double* dv_, double* dg,
+                     double* dbeta, double* dS0, int nthreads) {
+    bwd_ctx c = {q, k, v, g, beta, S0, dy, dS_T, cu_seqlens, H, dk, dv, scale, dq, dk_, dv_, dg, dbeta, dS0};
+    run_units(bwd_unit, &c, (long)num_seqs * H, nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
 /* Input parameterisation, eqs. (6)-(10)                                       */
 /* ------------------------------------------------------------------------- */
 

@@ -458,3 +458,70 @@ def test_thread_count_does_not_change_results():
     a = oracle.recurrence(q, k, v, g, beta, S0, num_seqs=2, nthreads=1)
     b = oracle.recurrence(q, k, v, g, beta, S0, num_seqs=2, nthreads=7)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ----------------------------------------------------------------------------------------------
+# Reverse-mode derivative of eqs. (1)-(4): pinned by central finite differences of the forward
+# oracle, which fix every partial derivative independently of how the backward is written.
+# ----------------------------------------------------------------------------------------------
+
+def _fd_case(lengths, H, dk, dv, seed):
+    rng = np.random.default_rng(seed)
+    N = sum(lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    x = dict(q=rng.standard_normal((N, H, dk)) * 0.5, k=rng.standard_normal((N, H, dk)) * 0.5,
+             v=rng.standard_normal((N, H, dv)), g=-rng.uniform(0.05, 0.6, (N, H)), beta=rng.uniform(0.1, 0.9, (N, H)),
+             S0=rng.standard_normal((len(lengths), H, dk, dv)) * 0.3)
+    w = dict(y=rng.standard_normal((N, H, dv)), S=rng.standard_normal((len(lengths), H, dk, dv)))
+    return x, w, cu
+
+
+def _loss(x, w, cu, scale):
+    y, S_T = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], cu, scale=scale)
+    return float((w["y"] * y).sum() + (w["S"] * S_T).sum())
+
+
+@pytest.mark.parametrize("lengths,scale", [([5, 3], 1.0), ([70], 0.7), ([0, 4], 1.0)])
+def test_backward_matches_central_differences(lengths, scale):
+    """Every input (q, k, v, g, beta, S0): the oracle's gradient of L = <w_y, y> + <w_S, S_T>
+    against (L(x + h) - L(x - h)) / 2h, element by element.  The 70-token sequence crosses the
+    backward's 64-token recomputation block; the empty sequence contributes only dS0 = w_S."""
+    H, dk, dv = 2, 3, 2
+    x, w, cu = _fd_case(lengths, H, dk, dv, seed=91 + len(lengths))
+    grad = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], w["y"], S0=x["S0"], dS_T=w["S"],
+                           cu_seqlens=cu, scale=scale)
+    names = dict(q="dq", k="dk", v="dv", g="dg", beta="dbeta", S0="dS0")
+    h = 1e-6
+    for name, gname in names.items():
+        arr = x[name]
+        fd = np.zeros_like(arr)
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = arr[idx]
+            arr[idx] = old + h
+            lp = _loss(x, w, cu, scale)
+            arr[idx] = old - h
+            lm = _loss(x, w, cu, scale)
+            arr[idx] = old
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.abs(grad[gname] - fd).max() / max(np.abs(fd).max(), 1e-12)
+        assert err < 1e-6, (name, err)
+
+
+def test_backward_of_pure_decay_is_closed_form():
+    """beta = 0: S_t = alpha_t S_{t-1}, y_t = scale (prod alpha) S0^T q_t.  With one token,
+    dq = scale alpha S0 dy, dS0 = alpha (scale q dy^T + dS_T), dg = alpha <scale q dy^T + dS_T, S0>,
+    and v, k receive nothing."""
+    rng = np.random.default_rng(93)
+    dk, dv, scale = 3, 4, 0.8
+    q, k, v = rng.standard_normal((1, 1, dk)), rng.standard_normal((1, 1, dk)), rng.standard_normal((1, 1, dv))
+    g, beta = np.array([[-0.4]]), np.zeros((1, 1))
+    S0, dy, dST = rng.standard_normal((1, 1, dk, dv)), rng.standard_normal((1, 1, dv)), rng.standard_normal((1, 1, dk, dv))
+    grad = oracle.backward(q, k, v, g, beta, dy, S0=S0, dS_T=dST, scale=scale)
+    a = np.exp(-0.4)
+    G = scale * np.outer(q[0, 0], dy[0, 0]) + dST[0, 0]
+    assert np.allclose(grad["dq"][0, 0], scale * a * S0[0, 0] @ dy[0, 0])
+    assert np.allclose(grad["dS0"][0, 0], a * G)
+    assert np.isclose(grad["dg"][0, 0], a * (G * S0[0, 0]).sum())
+    assert np.allclose(grad["dv"], 0) and np.allclose(grad["dk"], 0)
