@@ -580,7 +580,39 @@ def wl_mixer_decode(torch, dist, gdn, inputs, args, rank, world, stream, hbm_pea
             "gpu_launches": 3 * c["steps"]}
 
 
-WORKLOADS = {"decode": wl_decode, "long": wl_long, "mixer": wl_mixer, "mixer_decode": wl_mixer_decode}
+def wl_backward(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    """backward of the prefill workload (B=2, H=16, T=4096, bf16 q/k/v and dy): gdn_chunk_bwd,
+    the token-sequential reverse pass with its checkpointing forward pass."""
+    x = inputs.make_prefill(inputs.PREFILL, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.PREFILL + 50, rank))
+    N, H, nseq = x["N"], x["H"], x["num_seqs"]
+    gen = torch.Generator(device="cuda").manual_seed(rank_seed(7, rank))
+    dy = torch.randn(N, H, 128, device="cuda", generator=gen).to(torch.bfloat16)
+    dS_T = torch.randn(nseq, H, 128, 128, device="cuda", generator=gen) * 0.01
+    ws = torch.empty(gdn.lib().gdn_chunk_bwd_workspace_size(N, nseq, H, 128, 128), device="cuda", dtype=torch.uint8)
+    out = dict(dq=torch.empty(N, H, 128, device="cuda"), dk=torch.empty(N, H, 128, device="cuda"),
+               dv=torch.empty(N, H, 128, device="cuda"), dg=torch.empty(N, H, device="cuda"),
+               dbeta=torch.empty(N, H, device="cuda"), dS0=torch.empty(nseq, H, 128, 128, device="cuda"))
+
+    def bwd(i):
+        gdn.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], dy, None, dS_T, x["cu_seqlens"], out=out, workspace=ws)
+
+    barrier(torch, dist, world)
+    n_b = 3
+    dt = max_over_ranks(torch, dist, timed(torch, bwd, n_b, 1, stream, on_start=lambda: gdn.timing_start(64)),
+                        world) / n_b
+    kb = kernel_table(gdn.timing_stop(), n_b)
+    # read q, k, v, dy (bf16), g, beta; write dq, dk, dv (fp32), dg, dbeta; dS_T in, dS0 out
+    alg = N * H * (3 * 128 * 2 + 128 * 2 + 8 + 3 * 128 * 4 + 8) + 2 * nseq * H * 128 * 128 * 4
+    return {"workload": "backward_prefill_B2_H16_T4096_d128", "value": N * H * world / dt, "unit": UNIT,
+            "ms_per_step": dt * 1e3,
+            "roofline": {"bound": "latency (token-sequential)", "achieved": alg / dt / 1e9, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": alg / dt / 1e9 / hbm_peak, "alg_bytes_per_step": alg,
+                         "kernels": kb},
+            "gpu_launches": sum(k["launches"] for k in kb)}
+
+
+WORKLOADS = {"decode": wl_decode, "long": wl_long, "mixer": wl_mixer, "mixer_decode": wl_mixer_decode,
+             "backward": wl_backward}
 
 
 def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
@@ -598,7 +630,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true")
-    ap.add_argument("--only", choices=["decode", "long", "mixer", "mixer_decode"], default=None,
+    ap.add_argument("--only", choices=["decode", "long", "mixer", "mixer_decode", "backward"], default=None,
                     help="run one secondary workload alone and print its line (profiling aid)")
     ap.add_argument("--cpu-s", type=float, default=12.0, help="target seconds of the CPU-baseline sample")
     ap.add_argument("--ref-step-s", type=float, default=8.0)

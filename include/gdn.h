@@ -233,6 +233,31 @@ gdn_status_t gdn_chunk_fwd_prep(const void* x_q, const void* x_k, const void* x_
                                 size_t workspace_bytes, gdn_stream_t stream);
 
 /*
+ * gdn_chunk_bwd -- gradients through eqs. (1)-(4) for packed sequences (the backward of
+ * gdn_chunk_fwd): for a loss L with dL/dy = dy and dL/dS_T = dS_T (NULL: zero), returns dL/dq,
+ * dL/dk, dL/dv, dL/dg (g = log alpha), dL/dbeta and dL/dS0.  Each token step
+ *   S~ = alpha S, e = v - S~^T k, S_t = S~ + beta k e^T, y = scale S_t^T q
+ * is walked backwards with D = dL/dS_t:
+ *   D += scale q dy^T; dq = scale S_t dy; de = beta D^T k; dbeta = k^T D e;
+ *   dk = beta D e - S~ de; dv = de; D~ = D - k de^T; dg = alpha <D~, S>; D <- alpha D~.
+ * The states come from a forward pass that checkpoints every 8 tokens into the workspace.
+ *   q, k, v, g, beta, S0, cu_seqlens, scale, in_dtype as given to gdn_chunk_fwd; dy [N,H,dv]
+ *   in dy_dtype; dS_T [num_seqs,H,dk,dv] fp32 or NULL.  Outputs, fp32: dq, dk [N,H,dk],
+ *   dv [N,H,dv], dg, dbeta [N,H], dS0 [num_seqs,H,dk,dv].  dq, dk, dg, dbeta are zeroed for
+ *   all N tokens and accumulated over 32-column slabs of the state with atomic adds, so their
+ *   last bits depend on the order of those adds; dv of tokens in no sequence is not written.
+ * workspace: at least gdn_chunk_bwd_workspace_size(...) bytes (the checkpoints).
+ */
+size_t gdn_chunk_bwd_workspace_size(int N, int num_seqs, int H, int dk, int dv);
+
+gdn_status_t gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk,
+                           int dv, float scale, gdn_dtype_t in_dtype, const void* dy, gdn_dtype_t dy_dtype,
+                           const float* dS_T, float* dq, float* dk_out, float* dv_out, float* dg,
+                           float* dbeta, float* dS0, void* workspace, size_t workspace_bytes,
+                           gdn_stream_t stream);
+
+/*
  * gdn_decode_step -- one token per row against a resident state, eqs. (1)-(4):
  *   S <- alpha S + beta k e^T with e = v - alpha S^T k, y = scale * S^T q (new S).
  *   q, k [B,H,dk], v [B,H,dv]: in_dtype.  g, beta [B,H] fp32.

@@ -1,0 +1,189 @@
+// bwd.cuh -- reverse-mode derivative of eqs. (1)-(4) of "On the design of Qwen3.8-Next
+// architecture", section 2.1.1, token-sequential in fp32 on the CUDA cores.
+//
+// For a loss L with dL/dy_t = dy_t and dL/dS_T = dS_T, each token step
+//     S~ = alpha S,  e = v - S~^T k,  S_t = S~ + beta k e^T,  y = scale S_t^T q
+// (S = S_{t-1}, alpha = exp(g)) is walked backwards with D = dL/dS_t:
+//     D += scale q dy^T,  dq = scale S_t dy,  de = beta D^T k,  dbeta = k^T D e,
+//     dk = beta D e - S~ de,  dv = de,  D~ = D - k de^T,  dg = alpha <D~, S>,  D <- alpha D~
+// and dS0 is D after the first token.  A forward pass (recurrent_fwd_kernel with checkpoints)
+// stores the state before every kBwdBlk-th token; this kernel walks each sequence's blocks from
+// the last, recomputes the block's states into shared memory and walks them backwards.
+//
+// One CTA per (sequence, head, slab of state columns), laid out as the forward kernel: thread
+// (column jl, row phase r) keeps rows r, r + RS, ... of its column of D and of the block's
+// states.  de, dv and the column's share of dbeta and dg need only the column; dq and dk sum over
+// every column, so each CTA adds its slab's part through a shared-memory transpose and atomicAdd
+// into fp32 outputs the caller has zeroed (the slabs' order of addition is not fixed).
+#pragma once
+#include "common.cuh"
+#include "recurrent.cuh"
+
+namespace gdn {
+
+template <int DK, int DV>
+struct BwdShape {
+    using R = RecShape<DK, DV>;
+    static constexpr int SLAB = R::SLAB, RPT = R::RPT, RS = R::RS, THREADS = R::THREADS;
+    static constexpr int PAD = SLAB + 1;  // row stride of the transposes (bank spread)
+    // shared memory: the block's states, the block's token inputs, two transposes, column sums
+    static constexpr int ST_FLOATS = kBwdBlk * DK * SLAB;
+    static constexpr int TOK_FLOATS = kBwdBlk * (2 * DK + 2 * SLAB + 2);
+    static constexpr int RED_FLOATS = 2 * DK * PAD + 2 * SLAB;
+    static constexpr int BYTES = 4 * (ST_FLOATS + TOK_FLOATS + RED_FLOATS);
+};
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(RecShape<DK, DV>::THREADS)
+recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
+                     const float* __restrict__ g, const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                     int num_seqs, int N, int H, float scale, int in_dt, const void* __restrict__ dy, int dy_dt,
+                     const float* __restrict__ dS_T, const float* __restrict__ ckpt, float* __restrict__ dq,
+                     float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dg,
+                     float* __restrict__ dbeta, float* __restrict__ dS0) {
+    using Sh = BwdShape<DK, DV>;
+    constexpr int NSLAB = DV / Sh::SLAB, SLAB = Sh::SLAB, RPT = Sh::RPT, RS = Sh::RS, NT = Sh::THREADS;
+    constexpr int B = kBwdBlk;
+    extern __shared__ float smem_f[];
+    float* st = smem_f;                                  // [B][DK][SLAB]: S before token tb + i
+    float* sk = st + Sh::ST_FLOATS;                      // [B][DK]
+    float* sq = sk + B * DK;                             // [B][DK]
+    float* sv = sq + B * DK;                             // [B][SLAB]
+    float* sdy = sv + B * SLAB;                          // [B][SLAB]
+    float* sa = sdy + B * SLAB;                          // [B] alpha
+    float* sb = sa + B;                                  // [B] beta
+    float* p_q = sb + B;                                 // [DK][PAD] the slab's terms of dq
+    float* p_k = p_q + DK * Sh::PAD;                     // [DK][PAD] the slab's terms of dk
+    float* c_b = p_k + DK * Sh::PAD;                     // [SLAB] the columns' terms of dbeta
+    float* c_g = c_b + SLAB;                             // [SLAB] the columns' terms of dg / alpha
+    __shared__ int s_bbase;
+
+    const int slab = blockIdx.x % NSLAB;
+    const int h = (blockIdx.x / NSLAB) % H;
+    const int n = blockIdx.x / (NSLAB * H);
+    const int tid = threadIdx.x, jl = tid / RS, r = tid % RS, j = slab * SLAB + jl;
+    int t0, t1;
+    seq_bounds(cu, n, num_seqs, N, t0, t1);
+    if (tid == 0) s_bbase = blocks_before(cu, num_seqs, N, n);
+
+    const size_t sbase = ((size_t)n * H + h) * DK * DV;
+    float D[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) D[m] = dS_T ? dS_T[sbase + (size_t)(r + m * RS) * DV + j] : 0.f;
+    int nb = (t1 - t0 + B - 1) / B;
+    __syncthreads();  // s_bbase
+    if (s_bbase + (long long)nb > bwd_block_bound(N, num_seqs)) {  // malformed cu_seqlens: no block past the workspace
+        if (tid == 0) raise_error(kErrSeqlens);
+        nb = (int)max(0LL, bwd_block_bound(N, num_seqs) - s_bbase);
+    }
+
+    for (int b = nb - 1; b >= 0; --b) {
+        const int tb = t0 + b * B, nt = min(B, t1 - tb);
+        __syncthreads();  // the previous block's token inputs are no longer read (and s_bbase is set)
+        for (int idx = tid; idx < nt * DK; idx += NT) {
+            const int tt = idx / DK, i = idx % DK;
+            const size_t off = ((size_t)(tb + tt) * H + h) * DK + i;
+            sk[tt * DK + i] = ld1(k, in_dt, off);
+            sq[tt * DK + i] = ld1(q, in_dt, off);
+        }
+        for (int idx = tid; idx < nt * SLAB; idx += NT) {
+            const int tt = idx / SLAB, jj = idx % SLAB;
+            const size_t off = ((size_t)(tb + tt) * H + h) * DV + slab * SLAB + jj;
+            sv[tt * SLAB + jj] = ld1(v, in_dt, off);
+            sdy[tt * SLAB + jj] = ld1(dy, dy_dt, off);
+        }
+        for (int tt = tid; tt < nt; tt += NT) {
+            sa[tt] = expf(g[(size_t)(tb + tt) * H + h]);
+            sb[tt] = beta[(size_t)(tb + tt) * H + h];
+        }
+        __syncthreads();
+        // the block's states, recomputed from its checkpoint; each thread keeps the entries it owns
+        {
+            const float* cp = ckpt + ((size_t)(s_bbase + b) * H + h) * DK * DV;
+            float S[RPT];
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) S[m] = cp[(size_t)(r + m * RS) * DV + j];
+            for (int i = 0; i < nt; ++i) {
+                float a = 0.f;
+#pragma unroll
+                for (int m = 0; m < RPT; ++m) {
+                    st[(i * DK + r + m * RS) * SLAB + jl] = S[m];
+                    a += S[m] * sk[i * DK + r + m * RS];
+                }
+#pragma unroll
+                for (int o = 1; o < RS; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                const float e = sv[i * SLAB + jl] - sa[i] * a;
+#pragma unroll
+                for (int m = 0; m < RPT; ++m) S[m] = sa[i] * S[m] + sb[i] * sk[i * DK + r + m * RS] * e;
+            }
+        }
+        for (int i = nt - 1; i >= 0; --i) {
+            const int t = tb + i;
+            const float alpha = sa[i], bt = sb[i], dyj = sdy[i * SLAB + jl];
+            const float* kk = sk + i * DK;
+            const float* qq = sq + i * DK;
+            float Sp[RPT], a = 0.f;
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) {
+                Sp[m] = st[(i * DK + r + m * RS) * SLAB + jl];
+                a += Sp[m] * kk[r + m * RS];
+            }
+#pragma unroll
+            for (int o = 1; o < RS; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            const float e = sv[i * SLAB + jl] - alpha * a;
+            float kd = 0.f;
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) {
+                const int row = r + m * RS;
+                const float St = alpha * Sp[m] + bt * kk[row] * e;    // S_t
+                D[m] += scale * qq[row] * dyj;                          // readout
+                p_q[row * Sh::PAD + jl] = scale * St * dyj;             // dq = scale S_t dy
+                kd += kk[row] * D[m];
+            }
+#pragma unroll
+            for (int o = 1; o < RS; o <<= 1) kd += __shfl_xor_sync(0xffffffffu, kd, o);
+            const float de = bt * kd;                                   // de = beta D^T k
+            float da = 0.f;
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) {
+                const int row = r + m * RS;
+                p_k[row * Sh::PAD + jl] = bt * D[m] * e - alpha * Sp[m] * de;  // dk = beta D e - S~ de
+                D[m] -= kk[row] * de;                                   // D~
+                da += D[m] * Sp[m];
+                D[m] *= alpha;                                          // dL/dS_{t-1}
+            }
+#pragma unroll
+            for (int o = 1; o < RS; o <<= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
+            if (r == 0) {
+                dv[((size_t)t * H + h) * DV + j] = de;
+                c_b[jl] = kd * e;                                       // dbeta = k^T D e
+                c_g[jl] = da;
+            }
+            __syncthreads();
+            for (int row = tid; row < DK; row += NT) {
+                float sq_ = 0.f, sk_ = 0.f;
+#pragma unroll 8
+                for (int c = 0; c < SLAB; ++c) {
+                    sq_ += p_q[row * Sh::PAD + c];
+                    sk_ += p_k[row * Sh::PAD + c];
+                }
+                atomicAdd(dq + ((size_t)t * H + h) * DK + row, sq_);
+                atomicAdd(dk + ((size_t)t * H + h) * DK + row, sk_);
+            }
+            if (tid == 0) {
+                float s1 = 0.f, s2 = 0.f;
+                for (int c = 0; c < SLAB; ++c) {
+                    s1 += c_b[c];
+                    s2 += c_g[c];
+                }
+                atomicAdd(dbeta + (size_t)t * H + h, s1);
+                atomicAdd(dg + (size_t)t * H + h, alpha * s2);
+            }
+            __syncthreads();  // the transposes are read before the next token writes them
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) dS0[sbase + (size_t)(r + m * RS) * DV + j] = D[m];
+}
+
+}  // namespace gdn

@@ -19,6 +19,7 @@
 #include "prep.cuh"
 #include "recurrent.cuh"
 #include "state_map.cuh"
+#include "bwd.cuh"
 #include "chunk_tc.cuh"
 
 namespace {
@@ -124,6 +125,39 @@ struct RecurrentLaunch {
         gdn::recurrent_fwd_kernel<DK, DV><<<grid, Sh::THREADS, 0, st>>>(
             q, k, v, g, beta, S0, cu, num_seqs, N, H, scale, in_dt, y_dt, y, S_T);
         return launched("recurrent_fwd_kernel");
+    }
+};
+
+template <int DK, int DV>
+struct BwdLaunch {
+    static gdn_status_t run(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                            const float* S0, const int32_t* cu, int num_seqs, int N, int H, float scale, int in_dt,
+                            const void* dy, int dy_dt, const float* dS_T, float* ckpt, float* dq, float* dk, float* dv,
+                            float* dg, float* dbeta, float* dS0, cudaStream_t st) {
+        using Sh = gdn::RecShape<DK, DV>;
+        using Bw = gdn::BwdShape<DK, DV>;
+        const unsigned grid = (unsigned)((long long)num_seqs * H * (DV / Sh::SLAB));  // <= 2^31 (host check)
+        if (N > 0) {
+            const size_t nbytes = (size_t)N * H * DK * 4;
+            cudaError_t e = cudaMemsetAsync(dq, 0, nbytes, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nbytes, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(dg, 0, (size_t)N * H * 4, st);
+            if (e == cudaSuccess) e = cudaMemsetAsync(dbeta, 0, (size_t)N * H * 4, st);
+            if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+            gdn::LaunchScope timed(st, "recurrent_fwd_kernel");
+            gdn::recurrent_fwd_kernel<DK, DV><<<grid, Sh::THREADS, 0, st>>>(q, k, v, g, beta, S0, cu, num_seqs, N, H,
+                                                                            scale, in_dt, in_dt, nullptr, nullptr,
+                                                                            ckpt);
+            gdn_status_t r = launched("recurrent_fwd_kernel");
+            if (r != GDN_OK) return r;
+        }
+        cudaError_t e = cudaFuncSetAttribute(gdn::recurrent_bwd_kernel<DK, DV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Bw::BYTES);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "recurrent_bwd_kernel attribute: %s", cudaGetErrorString(e));
+        gdn::LaunchScope timed(st, "recurrent_bwd_kernel");
+        gdn::recurrent_bwd_kernel<DK, DV><<<grid, Sh::THREADS, Bw::BYTES, st>>>(
+            q, k, v, g, beta, cu, num_seqs, N, H, scale, in_dt, dy, dy_dt, dS_T, ckpt, dq, dk, dv, dg, dbeta, dS0);
+        return launched("recurrent_bwd_kernel");
     }
 };
 
@@ -424,6 +458,37 @@ gdn_status_t gdn_chunk_fwd_prep(const void* x_q, const void* x_k, const void* x_
     if (why) return fail(GDN_ERR_CUDA, "chunk_tc: %s", why);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "chunk_tc: %s", cudaGetErrorString(e));
     return GDN_OK;
+}
+
+size_t gdn_chunk_bwd_workspace_size(int N, int num_seqs, int H, int dk, int dv) {
+    if (N <= 0 || num_seqs <= 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
+    return (size_t)gdn::bwd_block_bound(N, num_seqs) * H * dk * dv * 4;
+}
+
+gdn_status_t gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                           const float* S0, const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk, int dv,
+                           float scale, gdn_dtype_t in_dtype, const void* dy, gdn_dtype_t dy_dtype, const float* dS_T,
+                           float* dq, float* dk_out, float* dv_out, float* dg, float* dbeta, float* dS0,
+                           void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
+    REQUIRE(head_dim_ok(dk) && head_dim_ok(dv), "dk=%d dv=%d not in {16,32,64,128}", dk, dv);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(dy_dtype), "bad dtype");
+    REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
+    REQUIRE((long long)N * H * (dk > dv ? dk : dv) < (1LL << 40), "problem too large");
+    REQUIRE((long long)num_seqs * H * 128 <= 0x7fffffffLL, "num_seqs*H too large (%d x %d)", num_seqs, H);
+    OPT_PTR(S0, "S0"); OPT_PTR(dS_T, "dS_T"); OPT_PTR(cu_seqlens, "cu_seqlens");
+    REQUIRE_PTR(dS0, "dS0");
+    if (N > 0) {
+        REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k"); REQUIRE_PTR(v, "v"); REQUIRE_PTR(g, "g"); REQUIRE_PTR(beta, "beta");
+        REQUIRE_PTR(dy, "dy"); REQUIRE_PTR(dq, "dq"); REQUIRE_PTR(dk_out, "dk"); REQUIRE_PTR(dv_out, "dv");
+        REQUIRE_PTR(dg, "dg"); REQUIRE_PTR(dbeta, "dbeta");
+        const size_t need = gdn_chunk_bwd_workspace_size(N, num_seqs, H, dk, dv);
+        REQUIRE_PTR(workspace, "workspace");
+        REQUIRE(workspace_bytes >= need, "workspace of %zu bytes < %zu", workspace_bytes, need);
+    }
+    return dispatch_dims<BwdLaunch>(dk, dv, q, k, v, g, beta, S0, cu_seqlens, num_seqs, N, H, scale, (int)in_dtype, dy,
+                                    (int)dy_dtype, dS_T, reinterpret_cast<float*>(workspace), dq, dk_out, dv_out, dg,
+                                    dbeta, dS0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 gdn_status_t gdn_chunk_fwd_gated(const void* q, const void* k, const void* v, const float* g, const float* beta,

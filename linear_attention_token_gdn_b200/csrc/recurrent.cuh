@@ -13,6 +13,26 @@
 
 namespace gdn {
 
+constexpr int kBwdBlk = 8;  // tokens between the backward's checkpoints
+
+// Upper bound of the checkpoint blocks of all sequences (the workspace's size); it holds for every
+// valid cu_seqlens.
+__host__ __device__ inline long long bwd_block_bound(int N, int num_seqs) {
+    return (N + kBwdBlk - 1) / kBwdBlk + num_seqs;
+}
+
+// Checkpoint blocks of sequences 0 .. n-1 (one thread; CTAs of these kernels may be narrower
+// than a warp).
+__device__ __forceinline__ int blocks_before(const int32_t* cu, int num_seqs, int N, int n) {
+    int s = 0;
+    for (int m = 0; m < n; ++m) {
+        int a, b;
+        seq_bounds(cu, m, num_seqs, N, a, b);
+        s += (b - a + kBwdBlk - 1) / kBwdBlk;
+    }
+    return s;
+}
+
 template <int DK, int DV>
 struct RecShape {
     static constexpr int SLAB = DV < 32 ? DV : 32;         // state columns per CTA
@@ -27,7 +47,8 @@ __global__ void __launch_bounds__(RecShape<DK, DV>::THREADS)
 recurrent_fwd_kernel(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
                      const float* __restrict__ g, const float* __restrict__ beta,
                      const float* __restrict__ S0, const int32_t* __restrict__ cu, int num_seqs, int N,
-                     int H, float scale, int in_dt, int y_dt, void* __restrict__ y, float* __restrict__ S_T) {
+                     int H, float scale, int in_dt, int y_dt, void* __restrict__ y, float* __restrict__ S_T,
+                     float* __restrict__ ckpt = nullptr) {
     using Sh = RecShape<DK, DV>;
     constexpr int NSLAB = DV / Sh::SLAB;
     const int slab = blockIdx.x % NSLAB;
@@ -43,6 +64,13 @@ recurrent_fwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
 
     int t0, t1;
     seq_bounds(cu, n, num_seqs, N, t0, t1);
+    // ckpt (the backward's checkpoints): the state before every kBwdBlk-th token of the sequence,
+    // [block of all sequences in order][H][DK][DV]; y may then be NULL
+    __shared__ int s_bbase;
+    if (ckpt != nullptr) {
+        if (tid == 0) s_bbase = blocks_before(cu, num_seqs, N, n);
+        __syncthreads();
+    }
 
     float S[Sh::RPT];
     const size_t sbase = ((size_t)n * H + h) * DK * DV;
@@ -69,6 +97,13 @@ recurrent_fwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
         __syncthreads();
 
         for (int tt = 0; tt < nt; ++tt) {
+            const long long blk = (long long)s_bbase + (tb + tt - t0) / kBwdBlk;
+            // (malformed cu_seqlens, already flagged, could describe more blocks than the workspace)
+            if (ckpt != nullptr && (tb + tt - t0) % kBwdBlk == 0 && blk < bwd_block_bound(N, num_seqs)) {
+                float* cp = ckpt + ((size_t)blk * H + h) * DK * DV;
+#pragma unroll
+                for (int m = 0; m < Sh::RPT; ++m) cp[(size_t)(r + m * Sh::RS) * DV + j] = S[m];
+            }
             const float alpha = s_a[tt], bt = s_b[tt];
             float a = 0.f;
 #pragma unroll
@@ -85,7 +120,7 @@ recurrent_fwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
             }
 #pragma unroll
             for (int o = 1; o < Sh::RS; o <<= 1) yb += __shfl_xor_sync(0xffffffffu, yb, o);
-            if (r == 0) st1(y, y_dt, ((size_t)(tb + tt) * H + h) * DV + j, scale * yb);
+            if (r == 0 && y != nullptr) st1(y, y_dt, ((size_t)(tb + tt) * H + h) * DV + j, scale * yb);
         }
     }
     if (S_T) {

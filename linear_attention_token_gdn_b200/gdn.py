@@ -42,6 +42,9 @@ SIGNATURES = {
     "gdn_out_gate": ([_P, _P, _P, _F, _I, _I, _I, _I, _I, _P, _P], _I),
     "gdn_state_map_apply": ([_P, _P, _P, _P, _I, _I, _I, _P], _I),
     "gdn_chunk_fwd_prep_workspace_size": ([_I, _I, _I, _I, _I, _I], ctypes.c_size_t),
+    "gdn_chunk_bwd_workspace_size": ([_I, _I, _I, _I, _I], ctypes.c_size_t),
+    "gdn_chunk_bwd": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                       ctypes.c_size_t, _P], _I),
     "gdn_chunk_fwd_prep": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _F, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                             _I, _P, _P, _P, ctypes.c_size_t, _P], _I),
     "gdn_timing_start": ([_I], _I),
@@ -288,6 +291,31 @@ def chunk_fwd_prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log,
                                     _DT[qkv_dtype], _DT[y_dtype], _ptr(y), _ptr(S_T), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)))
     return y, S_T
+
+
+def chunk_bwd(q, k, v, g, beta, dy, S0=None, dS_T=None, cu_seqlens=None, num_seqs=None, scale=1.0, out=None,
+              workspace=None, stream=None):
+    """gdn_chunk_bwd: gradients through eqs. (1)-(4).  Returns dict(dq, dk, dv, dg, dbeta, dS0),
+    fp32 (dg: with respect to g = log alpha)."""
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    elif num_seqs is None:
+        num_seqs = 1
+    dev = q.device
+    if out is None:
+        out = dict(dq=torch.empty(N, H, dk, device=dev), dk=torch.empty(N, H, dk, device=dev),
+                   dv=torch.zeros(N, H, dv, device=dev), dg=torch.empty(N, H, device=dev),
+                   dbeta=torch.empty(N, H, device=dev), dS0=torch.empty(num_seqs, H, dk, dv, device=dev))
+    if workspace is None:
+        nbytes = lib().gdn_chunk_bwd_workspace_size(N, num_seqs, H, dk, dv)
+        workspace = torch.empty(max(nbytes, 16), device=dev, dtype=torch.uint8)
+    _check(lib().gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(cu_seqlens), num_seqs,
+                               N, H, dk, dv, float(scale), _dt(q), _ptr(dy), _dt(dy), _ptr(dS_T), _ptr(out["dq"]),
+                               _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbeta"]), _ptr(out["dS0"]),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
 
 
 def state_map_apply(M, B, S_in, S_out=None, stream=None):

@@ -210,3 +210,19 @@ def test_chunk_fwd_prep_is_tensor_core_only(L, over):
 def test_chunk_fwd_prep_workspace_holds_records_and_q_k(L):
     rec = L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64)
     assert L.gdn_chunk_fwd_prep_workspace_size(8192, 2, 16, 128, 128, 64) == rec + 2 * 8192 * 16 * 128 * 2
+
+
+@pytest.mark.parametrize("over", [dict(dk=48), dict(ws=None), dict(ws_bytes=16), dict(dy=None), dict(dS0=None),
+                                  dict(in_dt=9)])
+def test_chunk_bwd_rejects_bad_arguments(L, over):
+    a = dict(dk=128, ws=A, ws_bytes=1 << 30, dy=A, dS0=A, in_dt=gdn.BF16)
+    a.update(over)
+    st = L.gdn_chunk_bwd(A, A, A, A, A, None, None, 2, 64, 2, a["dk"], 128, 1.0, a["in_dt"], a["dy"], gdn.F32, None,
+                         A, A, A, A, A, a["dS0"], a["ws"], a["ws_bytes"], None)
+    assert st == gdn.GDN_ERR_INVALID_ARG
+    assert gdn.last_error_message() != ""
+
+
+def test_chunk_bwd_workspace_holds_a_checkpoint_per_eight_tokens(L):
+    assert L.gdn_chunk_bwd_workspace_size(8192, 2, 16, 128, 128) == (1024 + 2) * 16 * 128 * 128 * 4
+    assert L.gdn_chunk_bwd_workspace_size(0, 2, 16, 128, 128) == 0
