@@ -211,8 +211,8 @@ gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v, 
 /*
  * gdn_chunk_fwd_prep -- gdn_prep (eqs. (6)-(10)) fused into gdn_chunk_fwd's chunked pass: the
  * projection outputs x_q, x_k, x_v go through ShortConv -> SiLU (-> L2Norm) inside the chunk
- * kernel, and q, k, v, g, beta never reach HBM (q and k are kept in the workspace for the
- * sequential pass).  Arguments as gdn_prep and gdn_chunk_fwd:
+ * kernel, and q, k, v, g, beta are never stored as tensors (the per-chunk records carry what the
+ * sequential pass needs).  Arguments as gdn_prep and gdn_chunk_fwd:
  *   x_q, x_k, x_v [N,H,128], beta_logit, alpha_logit [N,H]: in_dtype (BF16 or F16).
  *   conv_w_* [H*128, conv_width] fp32, conv_width in [1, 8]; A_log, alpha_bias [H] fp32.
  *   qkv_dtype (BF16 or F16): the format q, k, v are rounded to before eqs. (1)-(4), as

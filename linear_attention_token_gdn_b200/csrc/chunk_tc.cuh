@@ -102,7 +102,9 @@ constexpr int kRecU = 24576;       // U~: four 32-column dv slabs, each [64 rows
                                    // (16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3))
 constexpr int kRecUSlab = 4096;
 constexpr int kRecG = 40960;       // Gamma_r = exp(gamma_r) [64] then f_r = exp(gamma_C - gamma_r) [64], fp32
-constexpr int kRecBytes = 41472;
+constexpr int kRecK = 41472;       // K, fp16, two dk halves [64 rows x 128 B] 128B-swizzled K-major
+constexpr int kRecQ = 57856;       // Q, fp16, the same layout
+constexpr int kRecBytes = 74240;
 
 // Upper bound of the number of 64-token chunks over all sequences (the records the workspace
 // holds); it holds for every valid cu_seqlens.
@@ -234,7 +236,6 @@ struct PrepIn {
     const float *A_log, *alpha_bias;     // [H]
     float l2_eps;
     int raw_dt;                          // x_q, x_k, x_v and the logits: bf16 or fp16
-    void *q_out, *k_out;                 // [N, H, 128] q and k in the operand format (for the chain)
 };
 
 // Shared-memory byte offset of 16-byte chunk c of row r in a [rows x 128 B] 128B-swizzled tile.
@@ -388,8 +389,6 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
             meta[1] = t0;
             meta[2] = min(kChunk, te - t0);
             meta[3] = j == 0;
-            // the end of the last sequence: tokens from there to N belong to no sequence
-            meta[4] = a.cu ? min(max(a.cu[a.num_seqs], 0), a.N) : a.N;
             if (found) {
                 // with PREP the maps cover the raw projection outputs, 64 + W - 1 rows from the conv
                 // history on (a load before token 0 reads zeros)
@@ -416,7 +415,6 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
     const int t0 = meta[1], L = meta[2];
     uint8_t* rec = reinterpret_cast<uint8_t*>(a.workspace) + ((size_t)v * H + h) * kRecBytes;
     const bool first = meta[3] != 0;  // the chunk starts its sequence (PREP: a zero conv history)
-    const int stop = meta[4];
     auto drain = [&]() {  // a copy did not land in time: flag it and let every copy finish
         if (tid == 0) {
             raise_error(kErrTimeout);
@@ -488,8 +486,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
         //      half w & 1, all 64 rows.  For q and k pass one sums each row's squares over this half
         //      (the L2Norm needs both halves, exchanged through shared memory between the two warps
         //      of the tensor); pass two recomputes the conv, normalises, rounds to the operand format
-        //      and writes each row over its raw row, and to q_out / k_out for the chain.  v: one
-        //      pass, no norm. --------------------------------------------------------------------
+        //      and writes each row over its raw row.  v: one pass, no norm. ------------------------
         bool okv = true;
         if (warp < 6) {
             const int ten = warp >> 1, hf = warp & 1;
@@ -503,18 +500,9 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
                     if (lane == 0) pss[hf * 64 + r] = ss;
                 });
                 tc::bar_sync(2 + ten, 64);
-                uint16_t* gout = reinterpret_cast<uint16_t*>(ten ? p.k_out : p.q_out);
                 conv_silu_half(half, p.W, wl, first, lane, p.raw_dt, [&](int r, float y0, float y1) {
                     const float inv = rsqrtf(pss[r] + pss[64 + r] + p.l2_eps);
-                    const uint32_t o = pack2<BF>(y0 * inv, y1 * inv);
-                    put_row(half, r, lane, o);
-                    // rows of this sequence; zeros for tokens of no sequence (the chain reads them in
-                    // its last chunk, against zero coefficients); rows of the next sequence are its
-                    // own CTA's
-                    uint32_t* gp =
-                        reinterpret_cast<uint32_t*>(gout + ((size_t)(t0 + r) * H + h) * 128 + 64 * hf + 2 * lane);
-                    if (r < L) *gp = o;
-                    else if (t0 + r >= stop && t0 + r < a.N) *gp = 0u;
+                    put_row(half, r, lane, pack2<BF>(y0 * inv, y1 * inv));
                 });
             } else {
                 okv = tc::mbar_wait_bounded(bar_v, 0, a.budget);
@@ -597,7 +585,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
                         *reinterpret_cast<float2*>(fA + (16 * R + g8 + 8 * hh) * LD + 8 * strip[si] + 2 * t4) =
                             make_float2(acc[R][si][2 * hh], acc[R][si][2 * hh + 1]);
         } else {
-            tc::bar_sync(1, 128);  // every Q-row warp has finished reading Q
+            // M straight from the registers to the record (its upper blocks as zeros)
 #pragma unroll
             for (int R = 0; R < 4; ++R)
 #pragma unroll
@@ -605,14 +593,9 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const int r = 16 * R + g8 + 8 * hh;
-                        sts32(Qt + sw128(r, strip[si]) + 4 * t4, pack2<false>(acc[R][si][2 * hh], acc[R][si][2 * hh + 1]));
+                        *reinterpret_cast<uint32_t*>(rec + kRecM + sw128(r, strip[si]) + 4 * t4) =
+                            pack2<false>(acc[R][si][2 * hh], acc[R][si][2 * hh + 1]);
                     }
-            tc::fence_async_smem();
-            tc::bar_sync(1, 128);
-            if (tid == 128) {
-                tc::bulk_s2g(rec + kRecM, Qt, 8192);
-                tc::bulk_commit();
-            }
         }
     }
     __syncthreads();
@@ -642,6 +625,24 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
             __syncwarp(0x0000ffffu);
 #pragma unroll
             for (int r = 0; r < 16; ++r) fA[(b0 + r) * LD + b0 + jc] = xs[r];
+        }
+    } else {
+        // meanwhile K and Q in fp16 to the record (the chain's operands), converted in place (exact
+        // for |x| >= 2^-14); W = T_w K then reads K as is
+        if constexpr (BF) {
+            to_f16_block<128, 8192>(Kt, tid - 128);
+            to_f16_block<128, 8192>(Kt + Cf::HS, tid - 128);
+            to_f16_block<128, 8192>(Qt, tid - 128);
+            to_f16_block<128, 8192>(Qt + Cf::HS, tid - 128);
+        }
+        tc::fence_async_smem();
+        tc::bar_sync(1, 128);
+        if (tid == 128) {
+            tc::bulk_s2g(rec + kRecK, Kt, 8192);
+            tc::bulk_s2g(rec + kRecK + 8192, Kt + Cf::HS, 8192);
+            tc::bulk_s2g(rec + kRecQ, Qt, 8192);
+            tc::bulk_s2g(rec + kRecQ + 8192, Qt + Cf::HS, 8192);
+            tc::bulk_commit();
         }
     }
     __syncthreads();
@@ -686,7 +687,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
             wm::mma_split(d, ah, al, bh, bl);
         }
         wm::store_c(x2, LD, 16 * mt, 8 * nt, d);
-        if (tid == 128) tc::bulk_wait_read0();  // M has left the Q tile, which [T_w; T_u] overwrites
+        if (tid == 128) tc::bulk_wait_read0();  // Q and K have left their tiles ([T_w; T_u], -W overwrite them)
         __syncthreads();
         float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -741,7 +742,7 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t bv[4];
                 wm::ldsm_x4_t(bopnd + hf * Cf::HS + sw128(16 * kk + rr + 8 * (mi & 1), cb + (mi >> 1)), bv);
-                if constexpr (BF) {
+                if (BF && isU) {  // V as stored; K is fp16 by now
 #pragma unroll
                     for (int e = 0; e < 4; ++e) bv[e] = wm::bf2_to_h2(bv[e]);
                 }
@@ -1259,21 +1260,22 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
         auto rec_ptr = [&](int ci) {
             return reinterpret_cast<const uint8_t*>(a.workspace) + ((size_t)(rec_base + ci) * H + h) * kRecBytes;
         };
-        // K of chunk ci -> stage ci % 3; Q of ci -> rows 0-63 of [Q;-W] stage ci % 3; from the record:
-        // -W -> rows 64-127, this slab's U~ -> U~ stage, the gates -> gate stage
+        // Everything of chunk ci from its record, already fp16 in the operand layouts: K -> stage
+        // ci % 3; Q -> rows 0-63 and -W -> rows 64-127 of [Q;-W] stage ci % 3; this slab's U~ -> U~
+        // stage; the gates -> gate stage
         auto issue_stage = [&](int ci) {
             st_issued = ci;
             if (it != kIssuer) return;
-            const int c0 = t_begin + ci * kChunk, s = ci % 3;
+            const int s = ci % 3;
             uint64_t* bk = bar_kv + s;
-            tc::mbar_arrive_expect_tx(bk, Cf::K_TX);
-            tc::tma_load_3d(smem + Koff(s), &maps.k, 0, h, c0, bk);
-            tc::tma_load_3d(smem + Koff(s) + Cf::K_HALF, &maps.k, 64, h, c0, bk);
-            uint8_t* qw = smem + QWoff(s);
             const uint8_t* rp = rec_ptr(ci);
+            tc::mbar_arrive_expect_tx(bk, Cf::K_TX);
+            tc::bulk_g2s(smem + Koff(s), rp + kRecK, 8192, bk);
+            tc::bulk_g2s(smem + Koff(s) + Cf::K_HALF, rp + kRecK + 8192, 8192, bk);
+            uint8_t* qw = smem + QWoff(s);
             tc::mbar_arrive_expect_tx(bar_q + s, Cf::OP_TX);
-            tc::tma_load_3d(qw, &maps.q, 0, h, c0, bar_q + s);
-            tc::tma_load_3d(qw + Cf::QW_HALF, &maps.q, 64, h, c0, bar_q + s);
+            tc::bulk_g2s(qw, rp + kRecQ, 8192, bar_q + s);
+            tc::bulk_g2s(qw + Cf::QW_HALF, rp + kRecQ + 8192, 8192, bar_q + s);
             tc::bulk_g2s(qw + 64 * 128, rp + kRecW, 8192, bar_q + s);
             tc::bulk_g2s(qw + Cf::QW_HALF + 64 * 128, rp + kRecW + 8192, 8192, bar_q + s);
             tc::bulk_g2s(smem + Cf::OFF_UT + s * 64 * Cf::ROWB, rp + kRecU + slab * kRecUSlab, 64 * Cf::ROWB,
@@ -1289,7 +1291,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 tc::tma_load_3d(smem + Cf::OFF_ZS + bb * 64 * Cf::ROWB, &maps.z, slab * NS, h, t_begin + ci * kChunk,
                                 bar_m + bb);
         };
-        // chunk ci landed -> bf16 K and Q to fp16 in place -> handed to the chain (full[ci & 1])
+        // chunk ci landed -> handed to the chain (full[ci & 1])
         auto finish = [&](int ci) -> bool {
             const int s = ci % 3;
             bool w = tc::mbar_wait_bounded(bar_kv + s, (ci / 3) & 1, a.budget);
@@ -1299,24 +1301,12 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
                 return false;
             }
             st_landed = ci;
-            if constexpr (BF) {
-                // bf16 -> fp16 is exact for |x| >= 2^-14; the smaller entries of a unit-norm key or
-                // query lose at most 2^-25 absolute
-                to_f16_block<128, 2 * Cf::K_HALF>(smem + Koff(s), it);
-                to_f16_block<128, 64 * 128>(smem + QWoff(s), it);               // Q rows of half 0
-                to_f16_block<128, 64 * 128>(smem + QWoff(s) + Cf::QW_HALF, it);  // Q rows of half 1
-            }
-            tc::fence_async_smem();
             tc::tc_fence_before();
             tc::bar_sync(BID, 128);
             if (it == 0) tc::mbar_arrive(bar_full + (ci & 1));
             return true;
         };
-        if (it == kIssuer) {
-            tc::prefetch_tmap(&maps.k);
-            tc::prefetch_tmap(&maps.q);
-            if constexpr (GATED) tc::prefetch_tmap(&maps.z);
-        }
+        if (it == kIssuer && GATED) tc::prefetch_tmap(&maps.z);
         if (nchunks > 0) issue_stage(0);
         if (nchunks > 1) issue_stage(1);
         if (nchunks > 0) ok = finish(0);
@@ -1436,8 +1426,8 @@ inline cudaError_t chunk_tc_launch(const ChunkArgs& a, cudaStream_t st, const ch
 }
 
 // The chunked path with eqs. (6)-(10) fused into chunk_ut_kernel: x_q, x_k, x_v (p.raw_dt) are
-// the projection outputs; a.in_dt is the operand format q, k, v are rounded to (bf16 or fp16), in
-// which p.q_out / p.k_out receive q and k for the chain.  a.q, a.k, a.v, a.g, a.beta are unused.
+// the projection outputs; a.in_dt is the operand format q, k, v are rounded to (bf16 or fp16).
+// a.q, a.k, a.v, a.g, a.beta are unused.
 inline cudaError_t chunk_tc_prep_launch(const ChunkArgs& a, const PrepIn& p, const void* x_q, const void* x_k,
                                         const void* x_v, cudaStream_t st, const char** why) {
     *why = nullptr;
@@ -1447,13 +1437,11 @@ inline cudaError_t chunk_tc_prep_launch(const ChunkArgs& a, const PrepIn& p, con
     }
     constexpr int NS = 32;
     const CUtensorMapSwizzle yswz = a.y_dt == kF32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    ChainMaps raw = {}, maps = {};
+    ChainMaps raw = {}, maps = {};  // the chain reads K and Q from the records
     const uint32_t rows = 64 + p.W - 1;
     if (!encode_map_3d(&raw.k, x_k, p.raw_dt, a.N, a.H, 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !encode_map_3d(&raw.q, x_q, p.raw_dt, a.N, a.H, 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !encode_map_3d(&raw.v, x_v, p.raw_dt, a.N, a.H, 128, 64, rows, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_map_3d(&maps.k, p.k_out, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_map_3d(&maps.q, p.q_out, a.in_dt, a.N, a.H, 128, 64, kChunk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_map_3d(&maps.y, a.y, a.y_dt, a.N, a.H, 128, NS, kChunk, yswz)) {
         *why = "cuTensorMapEncodeTiled failed";
         return cudaSuccess;

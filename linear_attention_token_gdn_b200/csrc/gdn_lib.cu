@@ -412,8 +412,7 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v, const fl
 }
 
 size_t gdn_chunk_fwd_prep_workspace_size(int N, int num_seqs, int H, int dk, int dv, int chunk) {
-    const size_t rec = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
-    return rec == 0 ? 0 : rec + 2 * (size_t)N * H * dk * 2;  // + q and k in the operand format
+    return gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
 }
 
 gdn_status_t gdn_chunk_fwd_prep(const void* x_q, const void* x_k, const void* x_v, const float* conv_w_q,
@@ -445,11 +444,8 @@ gdn_status_t gdn_chunk_fwd_prep(const void* x_q, const void* x_k, const void* x_
     const size_t need = gdn_chunk_fwd_prep_workspace_size(N, num_seqs, H, dk, dv, chunk);
     REQUIRE_PTR(workspace, "workspace");
     REQUIRE(workspace_bytes >= need, "workspace of %zu bytes < %zu", workspace_bytes, need);
-    const size_t rec = gdn::chunk_tc_workspace_bytes(N, num_seqs, H, dk, dv, chunk);
-    uint8_t* q_out = reinterpret_cast<uint8_t*>(workspace) + rec;
-    uint8_t* k_out = q_out + (size_t)N * H * dk * 2;
     gdn::PrepIn p{conv_w_q, conv_w_k, conv_w_v, conv_width, beta_logit, alpha_logit, A_log, alpha_bias, l2_eps,
-                  (int)in_dtype, q_out, k_out};
+                  (int)in_dtype};
     gdn::ChunkArgs a{nullptr, nullptr, nullptr, nullptr, nullptr, S0, cu_seqlens, num_seqs, N, H, chunk, scale,
                      (int)qkv_dtype, (int)y_dtype, y, S_T, workspace, wait_budget()};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

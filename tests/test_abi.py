@@ -101,9 +101,9 @@ def test_workspace_size_is_zero_without_records(L):
 
 
 def test_workspace_size_covers_every_chunk(L):
-    # one 40.5 KB record per (64-token chunk, head); packed sequences add one partial chunk each
-    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 41472
-    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 41472
+    # one 72.5 KB record per (64-token chunk, head); packed sequences add one partial chunk each
+    assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64) == (128 + 2) * 16 * 74240
+    assert L.gdn_chunk_fwd_workspace_size(100, 3, 4, 128, 128, 64) == (2 + 3) * 4 * 74240
     assert L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 0) == 0
 
 
@@ -207,9 +207,9 @@ def test_chunk_fwd_prep_is_tensor_core_only(L, over):
     assert prep_call(L, **over) == gdn.GDN_ERR_UNSUPPORTED
 
 
-def test_chunk_fwd_prep_workspace_holds_records_and_q_k(L):
+def test_chunk_fwd_prep_workspace_is_the_records(L):
     rec = L.gdn_chunk_fwd_workspace_size(8192, 2, 16, 128, 128, 64)
-    assert L.gdn_chunk_fwd_prep_workspace_size(8192, 2, 16, 128, 128, 64) == rec + 2 * 8192 * 16 * 128 * 2
+    assert L.gdn_chunk_fwd_prep_workspace_size(8192, 2, 16, 128, 128, 64) == rec
 
 
 @pytest.mark.parametrize("over", [dict(dk=48), dict(ws=None), dict(ws_bytes=16), dict(dy=None), dict(dS0=None),
