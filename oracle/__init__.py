@@ -13,6 +13,8 @@ Every function follows "On the design of Qwen3.8-Next architecture"
 * :func:`decode_step` -- the same four equations for one token per row,
   against a state updated in place.
 * :func:`prep`        -- eqs. (6)-(10) ("GDN parameterisation").
+* :func:`in_proj_prep` -- the input projections W_q x, W_k x, W_v x, W_beta x, W_alpha x
+  and W_z x of eqs. (6)-(11), then eqs. (6)-(10).
 * :func:`out_gate`    -- eq. (11) without the output projection W_o.
 * :func:`mixer`       -- prep -> recurrence -> out_gate in fp64 (optionally with q, k, v
   rounded once to a 16-bit storage format between prep and the recurrence,
@@ -199,6 +201,28 @@ def prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bia
                         H, dk, dv, float(eps), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                         int(nthreads))
     return q, k, v, g, beta
+
+
+def in_proj_prep(x, w, H, d, conv_q, conv_k, conv_v, A_log, alpha_bias, cu_seqlens=None, num_seqs=1,
+                 eps=1e-6, nthreads=0):
+    """The mixer's input side from the normalised residual stream x_t: the projections that
+    eqs. (6)-(11) apply to x_t, then eqs. (6)-(10).
+
+    x [N, D]; w [4*H*d + 2*H, D] stacks, as rows (out_features x in_features), W_q, W_k, W_v,
+    W_z (H*d rows each, row c = h*d + i) and W_beta, W_alpha (H rows each).  conv_* [H*d, W]
+    are the ShortConv taps.  The projections are one fp64 matrix product; their outputs go
+    to prep() unrounded.  Returns (q, k, v, g, beta, z) in float64, z = W_z x [N, H, d].
+    """
+    x, w = _f64(x), _f64(w)
+    N, D = x.shape
+    hd = H * d
+    assert w.shape == (4 * hd + 2 * H, D)
+    p = x @ w.T                                            # [N, 4*H*d + 2*H]
+    xq, xk, xv, z = (p[:, j * hd:(j + 1) * hd].reshape(N, H, d) for j in range(4))
+    bl, al = p[:, 4 * hd:4 * hd + H], p[:, 4 * hd + H:]
+    q, k, v, g, beta = prep(xq, xk, xv, conv_q, conv_k, conv_v, bl, al, A_log, alpha_bias,
+                            cu_seqlens, num_seqs, eps, nthreads)
+    return q, k, v, g, beta, z.copy()
 
 
 # significant bits and smallest exponent step of the 16-bit storage formats

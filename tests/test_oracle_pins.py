@@ -407,6 +407,60 @@ def test_mixer_composes_the_three_stages():
     assert np.array_equal(out, oracle.out_gate(y2, z, nw))
 
 
+def _in_proj_case(rng, lengths, H, d, D, W=4):
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    N = int(cu[-1])
+    return dict(x=rng.standard_normal((N, D)), H=H, d=d,
+                conv_q=rng.standard_normal((H * d, W)) * 0.5, conv_k=rng.standard_normal((H * d, W)) * 0.5,
+                conv_v=rng.standard_normal((H * d, W)) * 0.5, A_log=np.log(rng.uniform(1, 16, H)),
+                alpha_bias=rng.standard_normal(H) * 0.5, cu_seqlens=cu)
+
+
+def test_in_proj_prep_with_one_hot_rows_is_prep_of_the_selected_columns():
+    """With every weight row one-hot, W x_t picks columns of x exactly, so the projection step
+    reduces to indexing and in_proj_prep must equal prep (pinned above) of those columns.  Each
+    block (W_q, W_k, W_v, W_z, W_beta, W_alpha) picks its own random columns, so a block taken
+    from the wrong rows, a transposed operand or a projection applied after the conv fails."""
+    rng = np.random.default_rng(41)
+    H, d, D = 2, 4, 13
+    c = _in_proj_case(rng, [5, 1, 9], H, d, D)
+    hd = H * d
+    sel = rng.integers(0, D, size=4 * hd + 2 * H)
+    w = np.zeros((4 * hd + 2 * H, D))
+    w[np.arange(w.shape[0]), sel] = 1.0
+    q, k, v, g, beta, z = oracle.in_proj_prep(w=w, **c)
+    x, N = c["x"], c["x"].shape[0]
+    cols = [c["x"][:, sel[j * hd:(j + 1) * hd]].reshape(N, H, d) for j in range(4)]
+    ref = oracle.prep(cols[0], cols[1], cols[2], c["conv_q"], c["conv_k"], c["conv_v"],
+                      x[:, sel[4 * hd:4 * hd + H]], x[:, sel[4 * hd + H:]], c["A_log"], c["alpha_bias"],
+                      cu_seqlens=c["cu_seqlens"])
+    for a, b in zip((q, k, v, g, beta), ref):
+        assert np.array_equal(a, b)
+    assert np.array_equal(z, cols[3])
+
+
+def test_in_proj_prep_projections_by_explicit_sums():
+    """The projections themselves, summed term by term in Python: z_t[c] = sum_j W_z[c, j] x_t[j],
+    beta_t = logistic(sum_j W_beta[h, j] x_t[j]) (eq. 9) and
+    g_t = -exp(A_h) softplus(sum_j W_alpha[h, j] x_t[j] + b_h) (eq. 10)."""
+    rng = np.random.default_rng(42)
+    H, d, D = 2, 2, 5
+    c = _in_proj_case(rng, [3], H, d, D)
+    w = rng.standard_normal((4 * H * d + 2 * H, D)) / math.sqrt(D)
+    q, k, v, g, beta, z = oracle.in_proj_prep(w=w, **c)
+    x, hd = c["x"], H * d
+    for t in range(x.shape[0]):
+        for h in range(H):
+            for i in range(d):
+                zz = sum(w[3 * hd + h * d + i, j] * x[t, j] for j in range(D))
+                assert abs(z[t, h, i] - zz) < 1e-12
+            lb = sum(w[4 * hd + h, j] * x[t, j] for j in range(D))
+            la = sum(w[4 * hd + H + h, j] * x[t, j] for j in range(D)) + c["alpha_bias"][h]
+            assert abs(beta[t, h] - 1.0 / (1.0 + math.exp(-lb))) < 1e-12
+            sp = math.log1p(math.exp(la)) if la < 30 else la
+            assert abs(g[t, h] + math.exp(c["A_log"][h]) * sp) < 1e-12
+
+
 # IEEE 754 binary16: p = 11, emin = -14; bfloat16: p = 8, emin = -126.  The subnormal spacing
 # is 2^(emin - p + 1).
 @pytest.mark.parametrize("fmt,bits,emin", [("bf16", 8, -126), ("fp16", 11, -14)])
