@@ -127,6 +127,30 @@ gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const f
                       void* q, void* k, void* v, float* g_out, float* beta_out, gdn_stream_t stream);
 
 /*
+ * gdn_inproj_prep -- the mixer's input projections fused with eqs. (6)-(10): from the
+ * normalised residual stream x_t (section 2.1.1, "GDN parameterisation") the six products
+ * W_q x_t, W_k x_t, W_v x_t, W_z x_t, W_beta x_t, W_alpha x_t as one tensor-core matrix
+ * product, then, on its fp32 results, exactly gdn_prep's steps (ShortConv -> SiLU -> L2Norm
+ * for q and k, ShortConv -> SiLU for v, eqs. (9)-(10) for beta and g).  The raw projections
+ * are never stored; z = W_z x_t (the input of eq. (11)'s gate) is stored as is.
+ *   x [N, D] in_dtype (BF16 or F16), row-major; D a multiple of 64.
+ *   w [4*H*d + 2*H, D] in_dtype: the rows (out_features x in_features) of W_q, W_k, W_v, W_z
+ *     (H*d rows each, row h*d + i is channel i of head h), then W_beta and W_alpha (H rows each).
+ *   conv_w_*, conv_width, A_log, alpha_bias, cu_seqlens, num_seqs, l2_eps as in gdn_prep.
+ *   q, k, v [N,H,d] and z [N,H,d] (NULL: W_z is not applied): out_dtype (BF16 or F16).
+ *   g_out, beta_out [N,H] fp32.
+ * Built for dk = dv = d = 128 and H a multiple of 16 up to 128 (others: GDN_ERR_UNSUPPORTED).
+ * q, k, v of tokens at index >= cu_seqlens[num_seqs] are left untouched; z, g and beta are
+ * written for all N tokens.  Nothing is allocated; asynchronous on the stream.
+ */
+gdn_status_t gdn_inproj_prep(const void* x, const void* w, int D, const float* conv_w_q,
+                             const float* conv_w_k, const float* conv_w_v, int conv_width,
+                             const float* A_log, const float* alpha_bias, const int32_t* cu_seqlens,
+                             int num_seqs, int N, int H, int dk, int dv, float l2_eps,
+                             gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* q, void* k, void* v,
+                             void* z, float* g_out, float* beta_out, gdn_stream_t stream);
+
+/*
  * gdn_chunk_fwd -- prefill: eqs. (1)-(4) over every token of every packed sequence.
  *   q, k [N,H,dk], v [N,H,dv]: in_dtype.  g = log alpha, beta [N,H]: fp32.
  *   S0 [num_seqs,H,dk,dv] fp32 or NULL (zero initial state).

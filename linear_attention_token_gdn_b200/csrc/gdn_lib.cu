@@ -21,6 +21,7 @@
 #include "state_map.cuh"
 #include "bwd.cuh"
 #include "chunk_tc.cuh"
+#include "inproj.cuh"
 
 namespace {
 
@@ -282,6 +283,27 @@ void launch_out_gate(const void* y, const void* z, const float* w, float eps, lo
     if (yt == gdn::kF32) launch_out_gate_y<DV, gdn::kF32>(y, z, w, eps, rows, zt, out, st);
     else if (yt == gdn::kBF16) launch_out_gate_y<DV, gdn::kBF16>(y, z, w, eps, rows, zt, out, st);
     else launch_out_gate_y<DV, gdn::kF16>(y, z, w, eps, rows, zt, out, st);
+}
+
+}  // namespace
+
+namespace {
+
+template <bool BF, int TAPS>
+gdn_status_t inproj_go(const gdn::InprojMaps& maps, const gdn::InprojArgs& a, cudaStream_t st) {
+    using Cf = gdn::IpCfg<TAPS>;
+    const int bytes = Cf::BYTES + Cf::ALIGN;
+    cudaError_t e = cudaFuncSetAttribute(gdn::inproj_prep_kernel<BF, TAPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         bytes);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "inproj_prep_kernel smem: %s", cudaGetErrorString(e));
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
+    const long long grid = a.n_tiles < sms ? a.n_tiles : sms;  // persistent: one CTA per SM
+    gdn::LaunchScope timed(st, "inproj_prep_kernel");
+    gdn::inproj_prep_kernel<BF, TAPS><<<(unsigned)grid, Cf::THREADS, bytes, st>>>(maps, a);
+    return launched("inproj_prep_kernel");
 }
 
 }  // namespace
@@ -565,6 +587,52 @@ gdn_status_t gdn_prep(const void* x_q, const void* x_k, const void* x_v, const f
                                      alpha_logit, A_log, alpha_bias, cu_seqlens, num_seqs, N, H, l2_eps,
                                      (int)in_dtype, (int)out_dtype, q, k, v, g_out, beta_out,
                                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+gdn_status_t gdn_inproj_prep(const void* x, const void* w, int D, const float* conv_w_q, const float* conv_w_k,
+                             const float* conv_w_v, int conv_width, const float* A_log, const float* alpha_bias,
+                             const int32_t* cu_seqlens, int num_seqs, int N, int H, int dk, int dv, float l2_eps,
+                             gdn_dtype_t in_dtype, gdn_dtype_t out_dtype, void* q, void* k, void* v, void* z,
+                             float* g_out, float* beta_out, gdn_stream_t stream) {
+    REQUIRE(N >= 0 && H >= 1 && num_seqs >= 1, "bad sizes N=%d H=%d num_seqs=%d", N, H, num_seqs);
+    REQUIRE(dtype_ok(in_dtype) && dtype_ok(out_dtype), "bad dtype");
+    REQUIRE(conv_width >= 1 && conv_width <= 8, "conv_width=%d not in [1, 8]", conv_width);
+    REQUIRE(cu_seqlens != nullptr || N % num_seqs == 0, "N=%d not a multiple of num_seqs=%d", N, num_seqs);
+    REQUIRE(l2_eps >= 0.f, "l2_eps < 0");
+    REQUIRE(D >= 64 && D % 64 == 0, "D=%d not a positive multiple of 64", D);
+    if (dk != 128 || dv != 128 || H % 16 != 0 || H > 128 || in_dtype == GDN_F32 || out_dtype == GDN_F32)
+        return fail(GDN_ERR_UNSUPPORTED,
+                    "gdn_inproj_prep is built for dk = dv = 128, H a multiple of 16 up to 128 and 16-bit x, w and "
+                    "outputs (dk=%d dv=%d H=%d)", dk, dv, H);
+    REQUIRE((long long)N * D < (1LL << 40), "N * D too large");
+    if (N == 0) return GDN_OK;
+    REQUIRE_PTR(x, "x"); REQUIRE_PTR(w, "w");
+    REQUIRE_PTR(conv_w_q, "conv_w_q"); REQUIRE_PTR(conv_w_k, "conv_w_k"); REQUIRE_PTR(conv_w_v, "conv_w_v");
+    REQUIRE_PTR(A_log, "A_log"); REQUIRE_PTR(alpha_bias, "alpha_bias");
+    REQUIRE_PTR(q, "q"); REQUIRE_PTR(k, "k"); REQUIRE_PTR(v, "v"); OPT_PTR(z, "z");
+    REQUIRE_PTR(g_out, "g_out"); REQUIRE_PTR(beta_out, "beta_out"); OPT_PTR(cu_seqlens, "cu_seqlens");
+    const int taps = conv_width <= 4 ? 4 : 8;
+    const int rows_out = 128 - (taps - 1);
+    gdn::InprojArgs a;
+    a.N = N; a.D = D; a.H = H; a.W = conv_width;
+    a.nq = H * 128 / 256;
+    a.has_z = z != nullptr;
+    a.n_tiles_n = (3 + a.has_z) * a.nq + 1;
+    a.n_tiles = (long long)((N + rows_out - 1) / rows_out) * a.n_tiles_n;
+    a.conv_q = conv_w_q; a.conv_k = conv_w_k; a.conv_v = conv_w_v;
+    a.A_log = A_log; a.alpha_bias = alpha_bias;
+    a.cu = cu_seqlens; a.num_seqs = num_seqs; a.eps = l2_eps; a.out_dt = (int)out_dtype;
+    a.q = q; a.k = k; a.v = v; a.z = z; a.g = g_out; a.beta = beta_out;
+    a.budget = wait_budget();
+    const bool bf = in_dtype == GDN_BF16;
+    const long long wrows = 4LL * H * 128 + 2 * H;
+    gdn::InprojMaps maps;
+    if (!gdn::encode_map_2d(&maps.x, x, bf, N, D, 64, 128) || !gdn::encode_map_2d(&maps.w, w, bf, wrows, D, 64, 256) ||
+        !gdn::encode_map_2d(&maps.wg, w, bf, wrows, D, 64, (uint32_t)(2 * H)))
+        return fail(GDN_ERR_CUDA, "inproj: cuTensorMapEncodeTiled failed");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (bf) return taps == 4 ? inproj_go<true, 4>(maps, a, st) : inproj_go<true, 8>(maps, a, st);
+    return taps == 4 ? inproj_go<false, 4>(maps, a, st) : inproj_go<false, 8>(maps, a, st);
 }
 
 gdn_status_t gdn_out_gate(const void* y, const void* z, const float* norm_w, float eps, int N, int H, int dv,

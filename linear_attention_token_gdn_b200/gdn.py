@@ -30,6 +30,8 @@ SIGNATURES = {
     "gdn_set_wait_budget": ([_U64], None),
     "gdn_prep": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I,
                   _P, _P, _P, _P, _P, _P], _I),
+    "gdn_inproj_prep": ([_P, _P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P, _P,
+                         _P, _P, _P], _I),
     "gdn_chunk_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
     "gdn_chunk_fwd": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P,
                        _Z, _P], _I),
@@ -163,6 +165,29 @@ def prep(x_q, x_k, x_v, w_q, w_k, w_v, beta_logit, alpha_logit, A_log, alpha_bia
                           num_seqs, N, H, dk, dv, float(eps), _dt(x_q), _DT[out_dtype], _ptr(q), _ptr(k),
                           _ptr(v), _ptr(g), _ptr(beta), _stream(stream)))
     return q, k, v, g, beta
+
+
+def inproj_prep(x, w, H, conv_q, conv_k, conv_v, A_log, alpha_bias, cu_seqlens=None, num_seqs=1, eps=1e-6,
+                out_dtype=None, with_z=True, out=None, stream=None):
+    """gdn_inproj_prep: the input projections of x [N, D] by the stacked rows
+    w = [W_q; W_k; W_v; W_z; W_beta; W_alpha] fused with eqs. (6)-(10).
+    Returns (q, k, v, g, beta, z) (z None when with_z is False)."""
+    N, D = x.shape
+    d = 128
+    if cu_seqlens is not None:
+        num_seqs = cu_seqlens.numel() - 1
+    out_dtype = x.dtype if out_dtype is None else out_dtype
+    if out is None:
+        dev = x.device
+        out = tuple(torch.empty(N, H, d, device=dev, dtype=out_dtype) for _ in range(3)) + (
+            torch.empty(N, H, device=dev), torch.empty(N, H, device=dev),
+            torch.empty(N, H, d, device=dev, dtype=out_dtype) if with_z else None)
+    q, k, v, g, beta, z = out
+    _check(lib().gdn_inproj_prep(_ptr(x), _ptr(w), D, _ptr(conv_q), _ptr(conv_k), _ptr(conv_v), conv_q.shape[1],
+                                 _ptr(A_log), _ptr(alpha_bias), _ptr(cu_seqlens), num_seqs, N, H, d, d, float(eps),
+                                 _dt(x), _DT[out_dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(g), _ptr(beta),
+                                 _stream(stream)))
+    return q, k, v, g, beta, z
 
 
 def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, num_seqs=None, chunk=64, scale=1.0, y_dtype=None,

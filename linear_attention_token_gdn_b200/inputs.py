@@ -20,6 +20,11 @@ Workloads (every tensor is token-major: [N, H, d] with d contiguous):
    bf16 projection outputs ~ N(0,1), conv taps ~ N(0, 0.5) width 4, beta/alpha
    logits ~ N(0,1), A = log U(1,16), b_alpha ~ N(0, 0.5), z ~ N(0,1),
    norm weight ~ N(0, 0.02), eps 1e-6.
+5. input projections + prep: the mixer's lengths, H=16, d=128, from the normalised
+   residual stream x ~ N(0,1) of width D = H*d = 2048 (bf16) and the stacked weight rows
+   [W_q; W_k; W_v; W_z; W_beta; W_alpha] ~ N(0, 1/D) (standard deviation D^-1/2, so each
+   projection output is about N(0,1), the mixer's distribution), conv taps, A and b_alpha
+   as in the mixer.
 
 q and k are drawn N(0,1) and scaled to unit L2 norm per head (in fp32) before
 the cast to the storage dtype; v ~ N(0,1); beta = sigmoid(N(0,1)).
@@ -32,7 +37,7 @@ import torch
 SEED_BASE = 20261202
 
 # workload keys (each workload's seed is SEED_BASE + its key)
-TINY, PREFILL, LONG_PREFILL, DECODE, MIXER = 0, 1, 2, 3, 4
+TINY, PREFILL, LONG_PREFILL, DECODE, MIXER, INPROJ = 0, 1, 2, 3, 4, 5
 
 WORKLOAD_SPECS = {
     TINY: dict(name="tiny_fp32_B1_H2_T64_d16", kind="prefill", B=1, H=2, T=64, d=16, dtype=torch.float32,
@@ -46,6 +51,8 @@ WORKLOAD_SPECS = {
     MIXER: dict(name="mixer_4seq_H16_d128_N<=32768", kind="mixer", nseq=4, H=16, d=128, L=(1024, 8192),
             dtype=torch.bfloat16, W=4, conv_std=0.5, norm_std=0.02, expA=(1.0, 16.0), ba_std=0.5,
             eps=1e-6),
+    INPROJ: dict(name="inproj_prep_4seq_H16_d128_D2048", kind="inproj", nseq=4, H=16, d=128, D=2048,
+            L=(1024, 8192), dtype=torch.bfloat16, W=4, conv_std=0.5, expA=(1.0, 16.0), ba_std=0.5, eps=1e-6),
 }
 
 
@@ -159,4 +166,31 @@ def make_mixer(cfg=MIXER, device="cpu", seed=None, lengths=None, **over):
         A_log=torch.log(expA).to(torch.float32), alpha_bias=randn(H, std=c["ba_std"]),
         z=randn(N, H, d).to(dt), norm_w=randn(d, std=c["norm_std"]),
         cu_seqlens=torch.from_numpy(cu).to(device), num_seqs=len(lengths), N=N, H=H, d=d, W=W,
+        eps=c["eps"], lengths=list(lengths))
+
+
+def make_inproj(cfg=INPROJ, device="cpu", seed=None, lengths=None, **over):
+    """Residual-stream rows x [N, D] and the stacked projection weights w [4*H*d + 2*H, D] with
+    the prep parameters, for the fused input projections."""
+    c = dict(WORKLOAD_SPECS[cfg])
+    c.update(over)
+    H, d, D, W = c["H"], c["d"], c["D"], c["W"]
+    if lengths is None:
+        lengths = mixer_lengths(MIXER, seed)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    N = int(cu[-1])
+    gen = _gen(device, SEED_BASE + cfg if seed is None else seed)
+    dt = c["dtype"]
+
+    def randn(*shape, std=1.0):
+        return torch.randn(*shape, generator=gen, device=device, dtype=torch.float32) * std
+
+    lo, hi = c["expA"]
+    expA = torch.empty(H, device=device, dtype=torch.float64).uniform_(lo, hi, generator=gen)
+    return dict(
+        x=randn(N, D).to(dt), w=randn(4 * H * d + 2 * H, D, std=D ** -0.5).to(dt),
+        conv_q=randn(H * d, W, std=c["conv_std"]), conv_k=randn(H * d, W, std=c["conv_std"]),
+        conv_v=randn(H * d, W, std=c["conv_std"]),
+        A_log=torch.log(expA).to(torch.float32), alpha_bias=randn(H, std=c["ba_std"]),
+        cu_seqlens=torch.from_numpy(cu).to(device), num_seqs=len(lengths), N=N, H=H, d=d, D=D, W=W,
         eps=c["eps"], lengths=list(lengths))

@@ -226,3 +226,24 @@ def test_chunk_bwd_rejects_bad_arguments(L, over):
 def test_chunk_bwd_workspace_holds_a_checkpoint_per_eight_tokens(L):
     assert L.gdn_chunk_bwd_workspace_size(8192, 2, 16, 128, 128) == (1024 + 2) * 16 * 128 * 128 * 4
     assert L.gdn_chunk_bwd_workspace_size(0, 2, 16, 128, 128) == 0
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(D=96), gdn.GDN_ERR_INVALID_ARG), (dict(D=0), gdn.GDN_ERR_INVALID_ARG),
+    (dict(W=0), gdn.GDN_ERR_INVALID_ARG), (dict(W=9), gdn.GDN_ERR_INVALID_ARG),
+    (dict(x=None), gdn.GDN_ERR_INVALID_ARG), (dict(w=MIS), gdn.GDN_ERR_INVALID_ARG),
+    (dict(eps=-1.0), gdn.GDN_ERR_INVALID_ARG), (dict(q=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(H=8), gdn.GDN_ERR_UNSUPPORTED), (dict(H=144), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(dk=64), gdn.GDN_ERR_UNSUPPORTED), (dict(io=0), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_inproj_prep_rejects_bad_arguments(L, over, status):
+    a = dict(D=256, W=4, x=A, w=A, eps=1e-6, q=A, H=16, dk=128, io=1)
+    a.update(over)
+    st = L.gdn_inproj_prep(a["x"], a["w"], a["D"], A, A, A, a["W"], A, A, None, 1, 16, a["H"], a["dk"], 128,
+                           a["eps"], a["io"], 1, a["q"], A, A, None, A, A, None)
+    assert st == status
+
+
+def test_inproj_prep_with_no_tokens_is_a_no_op(L):
+    assert L.gdn_inproj_prep(None, None, 256, None, None, None, 4, None, None, None, 1, 0, 16, 128, 128, 1e-6, 1, 1,
+                             None, None, None, None, None, None, None) == gdn.GDN_OK
