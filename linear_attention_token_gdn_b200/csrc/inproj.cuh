@@ -15,15 +15,20 @@
 // t-(TAPS-1) .. t, so a tile's first TAPS-1 rows are a halo: they are recomputed by the tile
 // before, and each tile outputs 128-(TAPS-1) tokens.
 //   warp 0      TMA producer: x and W tiles, 64 channels of D (one 128-byte swizzle row) per
-//               stage, four stages in flight
+//               stage, three stages in flight
 //   warp 1      allocates TMEM; one lane issues the MMAs (M = 128, N = 256 or 2H, K = 16) into
 //               one of two TMEM accumulators, so the epilogue of a tile overlaps the next
 //               tile's products
-//   warps 2-5   epilogue: one token per thread (its TMEM lane).  Conv tiles stage 32 columns
-//               at a time in shared memory, where each thread reads its token's TAPS-1
-//               predecessors; then SiLU, and for q and k the L2Norm over the head's 128
-//               channels, held in registers.  v: conv and SiLU.  z: stored as is.  Gate tile:
-//               beta = sigmoid (eq. 9), g = -exp(A_h) softplus(. + b_h) (eq. 10).
+//   warps 2-9   epilogue, two groups of four warps (two warps per SM sub-partition, so one
+//               hides the other's latency).  A thread owns one token (its TMEM lane) and, in
+//               group g, channels [64 g, 64 g + 64) of each head.  Conv tiles stage those 64
+//               columns in shared memory, where each thread reads its token's TAPS-1
+//               predecessors four columns at a time; then SiLU, and for q and k the L2Norm
+//               over the head's 128 channels, whose sum of squares the two groups exchange
+//               through shared memory.  v: conv and SiLU.  z: stored as is.  Results go back
+//               through the staging rows in 16-bit form so that each warp stores whole 128-byte
+//               row segments.  Gate tile: beta = sigmoid (eq. 9), g = -exp(A_h) softplus(. + b_h)
+//               (eq. 10).
 // Every wait is bounded: a wait that runs out flags kErrTimeout and then waits for the
 // hardware event (a TMA copy or an MMA always completes), so every role walks the same tiles
 // and the CTA always reaches its teardown.
@@ -36,21 +41,23 @@ namespace gdn {
 
 template <int TAPS>
 struct IpCfg {
-    static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+    static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
     static constexpr int HALO = TAPS - 1, ROWS_OUT = BM - HALO;
     static constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2, STAGE = A_BYTES + B_BYTES;
-    static constexpr int XLD = 33;                                // staging row stride (floats)
-    static constexpr int OFF_X = STAGES * STAGE;                  // [BM][XLD] fp32
-    static constexpr int OFF_TAPS = OFF_X + BM * XLD * 4;         // [BN][TAPS] fp32, right-aligned
-    static constexpr int OFF_BAR = OFF_TAPS + BN * TAPS * 4;      // full[S], empty[S], accf[2], acce[2]
+    static constexpr int XC = 64, XLD = XC + 4;                   // staged columns, row stride (floats)
+    static constexpr int OFF_X = STAGES * STAGE;                  // per group [BM][XLD] fp32
+    static constexpr int OFF_TAPS = OFF_X + 2 * BM * XLD * 4;     // [BN][TAPS] fp32, right-aligned
+    static constexpr int OFF_SS = OFF_TAPS + BN * TAPS * 4;       // [2 heads][2 groups][BM] sums of squares
+    static constexpr int OFF_BAR = OFF_SS + 4 * BM * 4;           // full[S], empty[S], accf[2], acce[2]
     static constexpr int NBAR = 2 * STAGES + 4;
     static constexpr int OFF_SLOT = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_SLOT + 16;
     static constexpr int ALIGN = 1024;                            // 128-byte swizzle atoms
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 320;
+    static constexpr int EPI_WARPS = 8;
     static constexpr int TMEM_COLS = 512;                         // two 256-column accumulators
     static_assert(BYTES + ALIGN <= 232448, "shared memory");
-    static_assert(OFF_X % 16 == 0 && OFF_TAPS % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
+    static_assert(OFF_X % 16 == 0 && OFF_TAPS % 16 == 0 && OFF_SS % 16 == 0 && OFF_BAR % 8 == 0, "alignment");
 };
 
 struct InprojArgs {
@@ -91,6 +98,41 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, in
             tc::smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(tc::smem_u32(bar))
         : "memory");
+}
+
+// Warp-wide load of 16 consecutive fp32 columns of the warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// The same load without the wait, so that several can be in flight; tmem_wait() completes them.
+__device__ __forceinline__ void tmem_ld16_nw(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 64 consecutive accumulator columns of the warp's lanes into v.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+    uint32_t u[64];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld16_nw(taddr + 16 * c, u + 16 * c);
+    tmem_wait();
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(u[i]);
 }
 
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
@@ -152,7 +194,7 @@ inproj_prep_kernel(const __grid_constant__ InprojMaps maps, const InprojArgs a) 
     const int KB = a.D / Cf::BK;
 
     if (tid == 0) {
-        for (int i = 0; i < Cf::NBAR; ++i) tc::mbar_init(bars + i, i >= 2 * Cf::STAGES + 2 ? 4 : 1);
+        for (int i = 0; i < Cf::NBAR; ++i) tc::mbar_init(bars + i, i >= 2 * Cf::STAGES + 2 ? Cf::EPI_WARPS : 1);
         tc::fence_mbar_init();
         tc::prefetch_tmap(&maps.x);
         tc::prefetch_tmap(&maps.w);
@@ -225,12 +267,15 @@ inproj_prep_kernel(const __grid_constant__ InprojMaps maps, const InprojArgs a) 
         }
     } else {
         // ================================ epilogue ====================================
+        const int grp = (warp - 2) >> 2;           // column group: channels [64 grp, 64 grp + 64) of a head
         const int quad = warp & 3;                 // TMEM lanes 32 quad .. 32 quad + 31
         const int r = quad * 32 + lane;            // this thread's tile row
-        const int et = tid - 64;                   // 0..127 over the epilogue warps
-        constexpr int BID = 1;                     // named barrier of the 128 epilogue threads
-        float* X = reinterpret_cast<float*>(smem + Cf::OFF_X);
+        const int gt = (warp - 2 - 4 * grp) * 32 + lane;  // 0..127 within the group
+        const int BIDG = 1 + grp;                  // named barrier of the group's 128 threads
+        constexpr int BID_PAIR = 3;                // both groups (the sum-of-squares exchange)
+        float* X = reinterpret_cast<float*>(smem + Cf::OFF_X) + grp * Cf::BM * Cf::XLD;
         float* taps = reinterpret_cast<float*>(smem + Cf::OFF_TAPS);
+        float* ssx = reinterpret_cast<float*>(smem + Cf::OFF_SS);
         const int stop = a.cu ? min(max(a.cu[a.num_seqs], 0), a.N) : (a.N / a.num_seqs) * a.num_seqs;
         const bool bf_out = a.out_dt == kBF16;
         const size_t HD = (size_t)a.H * 128;
@@ -252,15 +297,43 @@ inproj_prep_kernel(const __grid_constant__ InprojMaps maps, const InprojArgs a) 
             const bool row_out = r >= Cf::HALO && t < a.N;          // this tile outputs token t
             const bool conv_out = row_out && t < stop;               // ... and t lies in a sequence
             const uint32_t tcol = tmem + ((uint32_t)(quad * 32) << 16) + buf * 256;
+            auto release = [&]() {  // every TMEM load of the tile is done: the accumulator is free
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(acce + buf);
+            };
+
+            // A warp's 32 rows of 64 16-bit results, written by their owners into the first 128 bytes
+            // of their staging rows, leave as whole 128-byte row segments: instruction k stores rows
+            // 4k .. 4k+3 of the warp, eight lanes per row.
+            auto store_rows = [&](void* base, int col0, int row_end) {  // columns [col0, col0 + 64)
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int rr = quad * 32 + 4 * k + (lane >> 3), tt = tok0 + rr;
+                    const uint4 u = *reinterpret_cast<const uint4*>(X + rr * Cf::XLD + 4 * (lane & 7));
+                    if (rr >= Cf::HALO && tt < row_end)
+                        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(base) +
+                                                  ((size_t)tt * HD + (size_t)local * Cf::BN + col0 + 8 * (lane & 7)) * 2) = u;
+                }
+                __syncwarp();
+            };
+            auto stage_out = [&](const float* o) {  // this row's 64 results, 16-bit, into its staging row
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8) *reinterpret_cast<uint4*>(X + r * Cf::XLD + 4 * c8) = ip::pack8(o + 8 * c8, bf_out);
+            };
 
             if (kind <= ip::kV) {
-                // taps of the tile's 256 channels, right-aligned to TAPS (zeros before)
+                // the taps of the group's 128 channels, right-aligned to TAPS (zeros before)
                 const float* cw = kind == ip::kQ ? a.conv_q : kind == ip::kK ? a.conv_k : a.conv_v;
-                tc::bar_sync(BID, 128);  // the previous tile's taps are no longer read
-                for (int e = et; e < Cf::BN * TAPS; e += 128) {
-                    const int c = e / TAPS, i = e - c * TAPS, j = i - (TAPS - a.W);
-                    taps[e] = j >= 0 ? __ldg(cw + (size_t)(local * Cf::BN + c) * a.W + j) : 0.f;
+                tc::bar_sync(BIDG, 128);  // the group's previous tile no longer reads taps or X
+                for (int e = gt; e < 128 * TAPS; e += 128) {
+                    const int lc = e / TAPS, i = e - lc * TAPS, j = i - (TAPS - a.W);
+                    const int c = (lc >> 6) * 128 + grp * 64 + (lc & 63);
+                    taps[c * TAPS + i] = j >= 0 ? __ldg(cw + (size_t)(local * Cf::BN + c) * a.W + j) : 0.f;
                 }
+            } else if (kind == ip::kZ) {
+                tc::bar_sync(BIDG, 128);  // the group's previous tile no longer reads X
             }
             ip::wait(accf + buf, use & 1u, a.budget);
             tc::tc_fence_after();
@@ -271,88 +344,88 @@ inproj_prep_kernel(const __grid_constant__ InprojMaps maps, const InprojArgs a) 
                     const int s0 = seq_start_of(a.cu, a.num_seqs, a.N, t);
                     nmask = min(max(s0 - t + Cf::HALO, 0), TAPS);
                 }
+                const bool clean = __all_sync(0xffffffffu, nmask == 0);  // no masked tap in this warp
                 void* outp = kind == ip::kQ ? a.q : kind == ip::kK ? a.k : a.v;
                 const bool norm = kind != ip::kV;
+                const float* xr = X + (conv_out ? r - Cf::HALO : 0) * Cf::XLD;  // rows t-(TAPS-1) .. t
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
-                    float acc[128];
+                    const int col0 = hh * 128 + grp * 64;
+                    float v[64];
+                    ip::tmem_ld64(tcol + col0, v);
+                    if (hh == 1) release();
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        float vv[32];
-                        tc::tmem_ld32(tcol + hh * 128 + cc * 32, vv);
-                        if (hh == 1 && cc == 3) {  // the accumulator is free for the next tile
-                            tc::tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) tc::mbar_arrive(acce + buf);
+                    for (int c4 = 0; c4 < 16; ++c4)
+                        *reinterpret_cast<float4*>(X + r * Cf::XLD + 4 * c4) = make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+                    tc::bar_sync(BIDG, 128);  // the group's rows are staged
+                    const float* tp = taps + col0 * TAPS;
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        float x[TAPS][4];  // rows t-(TAPS-1) .. t of columns 4 c4 .. 4 c4 + 3
+#pragma unroll
+                        for (int i = 0; i < TAPS - 1; ++i) {
+                            const float4 x4 = *reinterpret_cast<const float4*>(xr + i * Cf::XLD + 4 * c4);
+                            const bool m = clean || i >= nmask;
+                            x[i][0] = m ? x4.x : 0.f; x[i][1] = m ? x4.y : 0.f; x[i][2] = m ? x4.z : 0.f; x[i][3] = m ? x4.w : 0.f;
                         }
-                        tc::bar_sync(BID, 128);  // X of the previous chunk is read (and taps are written)
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) X[r * Cf::XLD + j] = vv[j];
-                        tc::bar_sync(BID, 128);
-                        const float* tp = taps + (hh * 128 + cc * 32) * TAPS;
+                        for (int j = 0; j < 4; ++j) x[TAPS - 1][j] = v[4 * c4 + j];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
+                        for (int j = 0; j < 4; ++j) {
                             float s = 0.f;
-                            if (conv_out) {
 #pragma unroll
-                                for (int i = 0; i < TAPS; ++i) {
-                                    const float xv = i >= nmask ? X[(r - Cf::HALO + i) * Cf::XLD + j] : 0.f;
-                                    s = fmaf(tp[j * TAPS + i], xv, s);
-                                }
+                            for (int i = 0; i < TAPS; i += 4) {
+                                const float4 w4 = *reinterpret_cast<const float4*>(tp + (4 * c4 + j) * TAPS + i);
+                                s = fmaf(w4.x, x[i][j], s);
+                                s = fmaf(w4.y, x[i + 1][j], s);
+                                s = fmaf(w4.z, x[i + 2][j], s);
+                                s = fmaf(w4.w, x[i + 3][j], s);
                             }
-                            acc[cc * 32 + j] = __fdividef(s, 1.0f + __expf(-s));  // SiLU
+                            v[4 * c4 + j] = __fdividef(s, 1.0f + __expf(-s));  // SiLU
                         }
                     }
-                    if (conv_out) {
-                        float inv = 1.f;
-                        if (norm) {
-                            float ss = 0.f;
+                    float inv = 1.f;
+                    if (norm) {  // L2Norm over the head's 128 channels: this group's 64 plus the other's
+                        float ss = 0.f;
 #pragma unroll
-                            for (int j = 0; j < 128; ++j) ss = fmaf(acc[j], acc[j], ss);
-                            inv = rsqrtf(ss + a.eps);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 128; ++j) acc[j] *= inv;
-                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(outp) +
-                                                              ((size_t)t * HD + (size_t)local * Cf::BN + hh * 128) * 2);
-#pragma unroll
-                        for (int c8 = 0; c8 < 16; ++c8) dst[c8] = ip::pack8(acc + 8 * c8, bf_out);
+                        for (int j = 0; j < 64; ++j) ss = fmaf(v[j], v[j], ss);
+                        ssx[(hh * 2 + grp) * Cf::BM + r] = ss;
+                        tc::bar_sync(BID_PAIR, 256);  // also: every row of X has been read by its successors
+                        ss += ssx[(hh * 2 + (grp ^ 1)) * Cf::BM + r];
+                        inv = rsqrtf(ss + a.eps);
+                    } else {
+                        tc::bar_sync(BIDG, 128);  // every row of X has been read by its successors
                     }
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) v[j] *= inv;
+                    stage_out(v);
+                    store_rows(outp, hh * 128 + grp * 64, stop);
                 }
             } else if (kind == ip::kZ) {
 #pragma unroll 1
-                for (int cc = 0; cc < 8; ++cc) {
-                    float vv[32];
-                    tc::tmem_ld32(tcol + cc * 32, vv);
-                    if (cc == 7) {
-                        tc::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(acce + buf);
-                    }
-                    if (row_out) {
-                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(a.z) +
-                                                              ((size_t)t * HD + (size_t)local * Cf::BN + cc * 32) * 2);
-#pragma unroll
-                        for (int c8 = 0; c8 < 4; ++c8) dst[c8] = ip::pack8(vv + 8 * c8, bf_out);
-                    }
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int col0 = grp * 128 + hh * 64;
+                    float v[64];
+                    ip::tmem_ld64(tcol + col0, v);
+                    if (hh == 1) release();
+                    stage_out(v);
+                    store_rows(a.z, col0, a.N);
                 }
             } else {
-                // gate tile: columns [0, H) beta logits, [H, 2H) alpha logits
-                const int nchunk = (2 * a.H) / 32;
+                // gate tile: columns [0, H) beta logits, [H, 2H) alpha logits; group g takes the
+                // 16-column chunks g, g + 2, ...
+                const int nchunk = (2 * a.H) / 16;
+                if (grp >= nchunk) release();
 #pragma unroll 1
-                for (int cc = 0; cc < nchunk; ++cc) {
-                    float vv[32];
-                    tc::tmem_ld32(tcol + cc * 32, vv);
-                    if (cc == nchunk - 1) {
-                        tc::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) tc::mbar_arrive(acce + buf);
-                    }
+                for (int cc = grp; cc < nchunk; cc += 2) {
+                    float vv[16];
+                    ip::tmem_ld16(tcol + cc * 16, vv);
+                    if (cc + 2 >= nchunk) release();
                     if (row_out) {
                         // four columns at a time, all beta or all alpha logits (H is a multiple of 16)
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const int c = cc * 32 + 4 * q4;
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int c = cc * 16 + 4 * q4;
                             float o[4];
                             if (c < a.H) {
 #pragma unroll
