@@ -8,7 +8,8 @@ chunk 64 -- one launch of the tensor-core chunked kernel per step, inputs reside
 three input sets rotated so that every step reads from DRAM (3 x 137 MB > 126 MB L2).
 Secondary workloads measured in the same run (``other_workloads``): decode (256 x 32
 heads, 100 in-place steps), long prefill (T=32768, H=32, S0 != 0), full mixer (4 packed
-sequences, prep -> chunk -> out gate).
+sequences, prep -> chunk -> out gate), full-mixer decode step, backward, and the input
+projections fused with prep (gdn_inproj_prep, D = 2048).
 
 N > 1: one process per GPU (torchrun), every rank runs its own batch (independent
 sequences, no data-path collective: weak scaling); time = max over ranks.
@@ -611,8 +612,65 @@ def wl_backward(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
             "gpu_launches": sum(k["launches"] for k in kb)}
 
 
+def wl_inproj(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
+    """input projections + prep on the mixer's 4 packed sequences from a D = 2048 residual
+    stream: gdn_inproj_prep (one tcgen05 GEMM, eqs. (6)-(10) in its epilogue).  Beside it, as
+    context only: the same FLOPs as one cuBLAS GEMM (x @ w^T, bf16 out), and the unfused path
+    of six cuBLAS GEMMs (one per projection) followed by gdn_prep."""
+    m = inputs.make_inproj(inputs.INPROJ, "cuda", seed=rank_seed(inputs.SEED_BASE + inputs.INPROJ, rank))
+    N, H, D, d = m["N"], m["H"], m["D"], m["d"]
+    x, w = m["x"], m["w"]
+    R = w.shape[0]
+    hd = H * d
+    out = tuple(torch.empty(N, H, d, device="cuda", dtype=torch.bfloat16) for _ in range(3)) + (
+        torch.empty(N, H, device="cuda"), torch.empty(N, H, device="cuda"),
+        torch.empty(N, H, d, device="cuda", dtype=torch.bfloat16))
+    args_ip = (x, w, H, m["conv_q"], m["conv_k"], m["conv_v"], m["A_log"], m["alpha_bias"], m["cu_seqlens"])
+
+    def fused(i):
+        gdn.inproj_prep(*args_ip, eps=m["eps"], out=out)
+
+    pw = torch.empty(N, R, device="cuda", dtype=torch.bfloat16)
+
+    def gemm_only(i):
+        torch.matmul(x, w.t(), out=pw)
+
+    blocks = [w[j * hd:(j + 1) * hd] for j in range(4)] + [w[4 * hd:4 * hd + H], w[4 * hd + H:]]
+    raw = [torch.empty(N, hd, device="cuda", dtype=torch.bfloat16) for _ in range(4)] + [
+        torch.empty(N, H, device="cuda", dtype=torch.bfloat16) for _ in range(2)]
+    pbuf = tuple(torch.empty(N, H, d, device="cuda", dtype=torch.bfloat16) for _ in range(3)) + (
+        torch.empty(N, H, device="cuda"), torch.empty(N, H, device="cuda"))
+
+    def unfused(i):
+        for b, o in zip(blocks, raw):
+            torch.matmul(x, b.t(), out=o)
+        gdn.prep(raw[0].view(N, H, d), raw[1].view(N, H, d), raw[2].view(N, H, d), m["conv_q"], m["conv_k"],
+                 m["conv_v"], raw[4], raw[5], m["A_log"], m["alpha_bias"], m["cu_seqlens"], eps=m["eps"], out=pbuf)
+
+    barrier(torch, dist, world)
+    n_i = 10
+    dt = max_over_ranks(torch, dist, timed(torch, fused, n_i, 3, stream, on_start=lambda: gdn.timing_start(64)),
+                        world) / n_i
+    ki = kernel_table(gdn.timing_stop(), n_i)
+    dt_gemm = max_over_ranks(torch, dist, timed(torch, gemm_only, n_i, 3, stream), world) / n_i
+    dt_unf = max_over_ranks(torch, dist, timed(torch, unfused, n_i, 3, stream), world) / n_i
+    flops = 2.0 * N * D * R
+    _, tf_peak, src = peaks()
+    ach = flops / (ki[0]["avg_us"] * 1e-6) / 1e12 if ki else flops / dt / 1e12
+    return {"workload": inputs.WORKLOAD_SPECS[inputs.INPROJ]["name"], "lengths": m["lengths"],
+            "value": N * H * world / dt, "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
+            "context_ms_cublas_gemm_same_flops": dt_gemm * 1e3,
+            "context_ms_six_cublas_gemms_then_gdn_prep": dt_unf * 1e3,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": tf_peak, "unit": "TFLOP/s", "frac": ach / tf_peak,
+                         "peak_source": f"{src} bf16_tflops (burst)", "kernel": "inproj_prep_kernel",
+                         "alg_flops_per_launch": flops,
+                         "note": "flops = 2 N D (4 H d + 2 H); the conv halo rows recomputed per tile are not counted",
+                         "kernels": ki},
+            "gpu_launches": sum(k["launches"] for k in ki)}
+
+
 WORKLOADS = {"decode": wl_decode, "long": wl_long, "mixer": wl_mixer, "mixer_decode": wl_mixer_decode,
-             "backward": wl_backward}
+             "backward": wl_backward, "inproj": wl_inproj}
 
 
 def extra_workloads(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
@@ -630,7 +688,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extra", action="store_true")
-    ap.add_argument("--only", choices=["decode", "long", "mixer", "mixer_decode", "backward"], default=None,
+    ap.add_argument("--only", choices=["decode", "long", "mixer", "mixer_decode", "backward", "inproj"], default=None,
                     help="run one secondary workload alone and print its line (profiling aid)")
     ap.add_argument("--cpu-s", type=float, default=12.0, help="target seconds of the CPU-baseline sample")
     ap.add_argument("--ref-step-s", type=float, default=8.0)
