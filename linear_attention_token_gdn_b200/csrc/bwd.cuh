@@ -10,9 +10,8 @@
 // stores the state before every kBwdBlk-th token; this kernel walks each sequence's blocks from
 // the last, recomputes the block's states into shared memory and walks them backwards.
 //
-// One CTA per (sequence, head, slab of state columns), laid out as the forward kernel: thread
-// (column jl, row phase r) keeps rows r, r + RS, ... of its column of D and of the block's
-// states.  de, dv and the column's share of dbeta and dg need only the column; dq and dk sum over
+// One CTA per (sequence, head, slab of state columns): thread (column jl, row phase r) keeps rows
+// r, r + RS, ... of its column of D and of the block's states.  de, dv and the column's share of dbeta and dg need only the column; dq and dk sum over
 // every column, so each CTA adds its slab's part through a shared-memory transpose and atomicAdd
 // into fp32 outputs the caller has zeroed (the slabs' order of addition is not fixed).
 #pragma once
@@ -23,8 +22,11 @@ namespace gdn {
 
 template <int DK, int DV>
 struct BwdShape {
-    using R = RecShape<DK, DV>;
-    static constexpr int SLAB = R::SLAB, RPT = R::RPT, RS = R::RS, THREADS = R::THREADS;
+    // the forward kernel's column slabs, with twice its threads per column (rows split finer)
+    static constexpr int SLAB = RecShape<DK, DV>::SLAB;
+    static constexpr int RS = 2 * RecShape<DK, DV>::RS;           // threads per column (2, 4 or 8)
+    static constexpr int RPT = DK / RS;                           // rows per thread
+    static constexpr int THREADS = SLAB * RS;
     static constexpr int PAD = SLAB + 1;  // row stride of the transposes (bank spread)
     // shared memory: the block's states, the block's token inputs, two transposes, column sums
     static constexpr int ST_FLOATS = kBwdBlk * DK * SLAB;
@@ -34,7 +36,7 @@ struct BwdShape {
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(RecShape<DK, DV>::THREADS)
+__global__ void __launch_bounds__(BwdShape<DK, DV>::THREADS)
 recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
                      const float* __restrict__ g, const float* __restrict__ beta, const int32_t* __restrict__ cu,
                      int num_seqs, int N, int H, float scale, int in_dt, const void* __restrict__ dy, int dy_dt,
@@ -160,24 +162,27 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
                 c_g[jl] = da;
             }
             __syncthreads();
-            for (int row = tid; row < DK; row += NT) {
-                float sq_ = 0.f, sk_ = 0.f;
-#pragma unroll 8
-                for (int c = 0; c < SLAB; ++c) {
-                    sq_ += p_q[row * Sh::PAD + c];
-                    sk_ += p_k[row * Sh::PAD + c];
-                }
-                atomicAdd(dq + ((size_t)t * H + h) * DK + row, sq_);
-                atomicAdd(dk + ((size_t)t * H + h) * DK + row, sk_);
+            // the slab's column terms: a row of dq or dk per thread (four partial sums), dbeta and
+            // dg by one warp
+            for (int e = tid; e < 2 * DK; e += NT) {
+                const int row = e < DK ? e : e - DK;
+                const float* pr = (e < DK ? p_q : p_k) + row * Sh::PAD;
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < SLAB; ++c) s4[c & 3] += pr[c];
+                atomicAdd((e < DK ? dq : dk) + ((size_t)t * H + h) * DK + row, (s4[0] + s4[1]) + (s4[2] + s4[3]));
             }
-            if (tid == 0) {
-                float s1 = 0.f, s2 = 0.f;
-                for (int c = 0; c < SLAB; ++c) {
-                    s1 += c_b[c];
-                    s2 += c_g[c];
+            if (tid < 32) {
+                float s1 = tid < SLAB ? c_b[tid] : 0.f, s2 = tid < SLAB ? c_g[tid] : 0.f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
                 }
-                atomicAdd(dbeta + (size_t)t * H + h, s1);
-                atomicAdd(dg + (size_t)t * H + h, alpha * s2);
+                if (tid == 0) {
+                    atomicAdd(dbeta + (size_t)t * H + h, s1);
+                    atomicAdd(dg + (size_t)t * H + h, alpha * s2);
+                }
             }
             __syncthreads();  // the transposes are read before the next token writes them
         }

@@ -156,7 +156,7 @@ struct BwdLaunch {
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, Bw::BYTES);
         if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "recurrent_bwd_kernel attribute: %s", cudaGetErrorString(e));
         gdn::LaunchScope timed(st, "recurrent_bwd_kernel");
-        gdn::recurrent_bwd_kernel<DK, DV><<<grid, Sh::THREADS, Bw::BYTES, st>>>(
+        gdn::recurrent_bwd_kernel<DK, DV><<<grid, Bw::THREADS, Bw::BYTES, st>>>(
             q, k, v, g, beta, cu, num_seqs, N, H, scale, in_dt, dy, dy_dt, dS_T, ckpt, dq, dk, dv, dg, dbeta, dS0);
         return launched("recurrent_bwd_kernel");
     }
