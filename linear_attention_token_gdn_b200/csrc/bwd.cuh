@@ -27,7 +27,10 @@ struct BwdShape {
     static constexpr int RS = 2 * RecShape<DK, DV>::RS;           // threads per column (2, 4 or 8)
     static constexpr int RPT = DK / RS;                           // rows per thread
     static constexpr int THREADS = SLAB * RS;
-    static constexpr int PAD = SLAB + 1;  // row stride of the transposes (bank spread)
+    // row stride of the transposes: a warp writes RS rows x 32/RS columns, and with a stride of
+    // 4 (mod 32) words those land in 32 distinct banks; the readers rotate their start column by
+    // lane so that a warp's 32 rows also read 32 distinct banks
+    static constexpr int PAD = SLAB + 4;
     // shared memory: the block's states, the block's token inputs, two transposes, column sums
     static constexpr int ST_FLOATS = kBwdBlk * DK * SLAB;
     static constexpr int TOK_FLOATS = kBwdBlk * (2 * DK + 2 * SLAB + 2);
@@ -47,7 +50,7 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
     constexpr int NSLAB = DV / Sh::SLAB, SLAB = Sh::SLAB, RPT = Sh::RPT, RS = Sh::RS, NT = Sh::THREADS;
     constexpr int B = kBwdBlk;
     extern __shared__ float smem_f[];
-    float* st = smem_f;                                  // [B][DK][SLAB]: S before token tb + i
+    float* st = smem_f;                                  // [B][RPT][THREADS]: S before token tb + i, thread-major
     float* sk = st + Sh::ST_FLOATS;                      // [B][DK]
     float* sq = sk + B * DK;                             // [B][DK]
     float* sv = sq + B * DK;                             // [B][SLAB]
@@ -109,7 +112,7 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
                 float a = 0.f;
 #pragma unroll
                 for (int m = 0; m < RPT; ++m) {
-                    st[(i * DK + r + m * RS) * SLAB + jl] = S[m];
+                    st[(i * RPT + m) * NT + tid] = S[m];
                     a += S[m] * sk[i * DK + r + m * RS];
                 }
 #pragma unroll
@@ -122,13 +125,17 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
         for (int i = nt - 1; i >= 0; --i) {
             const int t = tb + i;
             const float alpha = sa[i], bt = sb[i], dyj = sdy[i * SLAB + jl];
-            const float* kk = sk + i * DK;
-            const float* qq = sq + i * DK;
+            float kk[RPT], qq[RPT];  // this thread's rows of k_t and q_t
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) {
+                kk[m] = sk[i * DK + r + m * RS];
+                qq[m] = sq[i * DK + r + m * RS];
+            }
             float Sp[RPT], a = 0.f;
 #pragma unroll
             for (int m = 0; m < RPT; ++m) {
-                Sp[m] = st[(i * DK + r + m * RS) * SLAB + jl];
-                a += Sp[m] * kk[r + m * RS];
+                Sp[m] = st[(i * RPT + m) * NT + tid];
+                a += Sp[m] * kk[m];
             }
 #pragma unroll
             for (int o = 1; o < RS; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -137,10 +144,10 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
 #pragma unroll
             for (int m = 0; m < RPT; ++m) {
                 const int row = r + m * RS;
-                const float St = alpha * Sp[m] + bt * kk[row] * e;    // S_t
-                D[m] += scale * qq[row] * dyj;                          // readout
+                const float St = alpha * Sp[m] + bt * kk[m] * e;      // S_t
+                D[m] += scale * qq[m] * dyj;                            // readout
                 p_q[row * Sh::PAD + jl] = scale * St * dyj;             // dq = scale S_t dy
-                kd += kk[row] * D[m];
+                kd += kk[m] * D[m];
             }
 #pragma unroll
             for (int o = 1; o < RS; o <<= 1) kd += __shfl_xor_sync(0xffffffffu, kd, o);
@@ -150,7 +157,7 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
             for (int m = 0; m < RPT; ++m) {
                 const int row = r + m * RS;
                 p_k[row * Sh::PAD + jl] = bt * D[m] * e - alpha * Sp[m] * de;  // dk = beta D e - S~ de
-                D[m] -= kk[row] * de;                                   // D~
+                D[m] -= kk[m] * de;                                     // D~
                 da += D[m] * Sp[m];
                 D[m] *= alpha;                                          // dL/dS_{t-1}
             }
@@ -169,7 +176,7 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
                 const float* pr = (e < DK ? p_q : p_k) + row * Sh::PAD;
                 float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < SLAB; ++c) s4[c & 3] += pr[c];
+                for (int c = 0; c < SLAB; ++c) s4[c & 3] += pr[(c + tid) & (SLAB - 1)];
                 atomicAdd((e < DK ? dq : dk) + ((size_t)t * H + h) * DK + row, (s4[0] + s4[1]) + (s4[2] + s4[3]));
             }
             if (tid < 32) {
