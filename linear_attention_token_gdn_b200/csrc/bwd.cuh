@@ -22,9 +22,9 @@ namespace gdn {
 
 template <int DK, int DV>
 struct BwdShape {
-    // the forward kernel's column slabs, with twice its threads per column (rows split finer)
+    // the forward kernel's column slabs; 16 rows per thread (8 for dk = 16)
     static constexpr int SLAB = RecShape<DK, DV>::SLAB;
-    static constexpr int RS = 2 * RecShape<DK, DV>::RS;           // threads per column (2, 4 or 8)
+    static constexpr int RS = DK >= 32 ? DK / 16 : 2;             // threads per column (2, 4 or 8)
     static constexpr int RPT = DK / RS;                           // rows per thread
     static constexpr int THREADS = SLAB * RS;
     // row stride of the transposes: a warp writes RS rows x 32/RS columns, and with a stride of

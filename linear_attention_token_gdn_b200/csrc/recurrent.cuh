@@ -36,8 +36,8 @@ __device__ __forceinline__ int blocks_before(const int32_t* cu, int num_seqs, in
 template <int DK, int DV>
 struct RecShape {
     static constexpr int SLAB = DV < 32 ? DV : 32;         // state columns per CTA
-    static constexpr int RPT = DK < 32 ? DK : 32;          // rows per thread
-    static constexpr int RS = DK / RPT;                    // threads per column (1, 2 or 4)
+    static constexpr int RPT = DK < 16 ? DK : 16;          // rows per thread
+    static constexpr int RS = DK / RPT;                    // threads per column (1, 2, 4 or 8)
     static constexpr int THREADS = SLAB * RS;
     static constexpr int TILE = 32;                        // tokens staged per refill
 };
