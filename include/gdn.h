@@ -67,6 +67,14 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1, GDN_F16 = 2 } gdn_dtype_t;
 /* Library version, major*10000 + minor*100 + patch. */
 int gdn_version(void);
 
+/* 1 for the bounds-checking build (libgdn_debug.so, compiled with -DGDN_BOUNDS_CHECK), else 0.
+ * In that build the kernels test their computed global indices (state blocks of decode slots,
+ * chunk records and token rows, checkpoint blocks, output rows) against the tensors' extents
+ * that the call's sizes imply; an index outside them is not accessed, and
+ * gdn_check_device_error then returns GDN_ERR_INVALID_ARG naming the bounds check.  Results of
+ * a call that trips no check are those of the release build. */
+int gdn_bounds_checked(void);
+
 /* Static string naming a status code. */
 const char* gdn_status_string(gdn_status_t status);
 

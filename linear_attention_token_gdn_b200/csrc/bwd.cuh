@@ -84,6 +84,10 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
 
     for (int b = nb - 1; b >= 0; --b) {
         const int tb = t0 + b * B, nt = min(B, t1 - tb);
+        // (bounds-checking build) the block's tokens and checkpoint lie inside their tensors;
+        // uniform over the CTA
+        if (!in_bounds(tb, N) || !in_bounds(tb + nt - 1, N) || !in_bounds(s_bbase + b, bwd_block_bound(N, num_seqs)))
+            break;
         __syncthreads();  // the previous block's token inputs are no longer read (and s_bbase is set)
         for (int idx = tid; idx < nt * DK; idx += NT) {
             const int tt = idx / DK, i = idx % DK;

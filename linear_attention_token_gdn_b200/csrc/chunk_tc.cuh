@@ -385,11 +385,15 @@ __global__ void __launch_bounds__(UtCfg::THREADS, 3) chunk_ut_kernel(const __gri
         const bool found = locate_chunk(a.cu, a.num_seqs, a.N, v, n, j, tb, te);
         if (lane == 0) {
             const int t0 = tb + j * kChunk;
-            meta[0] = found;
+            // (bounds-checking build) the record and the chunk's tokens lie inside their tensors;
+            // a chunk that fails is skipped before any copy is issued
+            const bool use = found && in_bounds(v, chunk_count_bound(a.N, a.num_seqs, a.cu != nullptr)) &&
+                             in_bounds(t0, a.N) && in_bounds(te - 1, a.N);
+            meta[0] = use;
             meta[1] = t0;
             meta[2] = min(kChunk, te - t0);
             meta[3] = j == 0;
-            if (found) {
+            if (use) {
                 // with PREP the maps cover the raw projection outputs, 64 + W - 1 rows from the conv
                 // history on (a load before token 0 reads zeros)
                 const int row0 = PREP ? t0 - (p.W - 1) : t0;
@@ -1024,7 +1028,7 @@ __global__ void __launch_bounds__(256, 1) chunk_chain_kernel(const __grid_consta
 #pragma unroll
                     for (int cc = 0; cc < NS / 8; ++cc) st16(ys + tc::swz_off(tid, cc, 2 * NS), pack8<false>(t + 8 * cc));
                 }
-            } else if (tid < py_L) {
+            } else if (tid < py_L && in_bounds(py_c0 + tid, a.N)) {
                 void* dst = reinterpret_cast<uint8_t*>(GATED ? a.out : a.y) +
                             (((size_t)(py_c0 + tid) * H + h) * 128 + slab * NS) * (dt == kF32 ? 4 : 2);
 #pragma unroll

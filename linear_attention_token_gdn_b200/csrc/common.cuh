@@ -16,11 +16,29 @@ enum ErrBits : unsigned {
     kErrTimeout = 1u,      // a bounded wait ran out
     kErrSeqlens = 2u,      // cu_seqlens not non-decreasing / out of [0, N]
     kErrSlot = 4u,         // a decode row named a state slot out of range
+    kErrBounds = 8u,       // bounds-checking build: a computed global index fell outside its tensor
 };
 
 __device__ unsigned int g_error_word;
 
 __device__ __forceinline__ void raise_error(unsigned bits) { atomicOr(&g_error_word, bits); }
+
+// The bounds-checking build (compiled with -DGDN_BOUNDS_CHECK into libgdn_debug.so) tests the
+// computed global indices of the kernels against their tensors' extents: in_bounds(i, n) is
+// 0 <= i < n, and otherwise flags kErrBounds so that the caller skips the access.  In the
+// release build every check is the constant true.
+__device__ __forceinline__ bool in_bounds(long long i, long long n) {
+#ifdef GDN_BOUNDS_CHECK
+    if (i < 0 || i >= n) {
+        raise_error(kErrBounds);
+        return false;
+    }
+#else
+    (void)i;
+    (void)n;
+#endif
+    return true;
+}
 
 // ---- scalar / vector loads and stores in any of the three element types -------------
 

@@ -45,6 +45,10 @@ decode_step_kernel(const void* __restrict__ q, const void* __restrict__ k, const
         if (tid == 0) raise_error(kErrSlot);
         return;
     }
+    // (bounds-checking build) the state block and the token row lie inside their tensors
+    if (!in_bounds(((long long)s * H + h + 1) * DK * DV - 1, (long long)num_slots * H * DK * DV) ||
+        !in_bounds(bh, (long long)gridDim.x))
+        return;
     float* S = state + ((size_t)s * H + h) * DK * DV;
 
     // Issue the state loads first: they are the only traffic that matters.

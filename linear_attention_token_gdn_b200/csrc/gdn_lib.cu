@@ -312,6 +312,14 @@ extern "C" {
 
 int gdn_version(void) { return 100; }
 
+int gdn_bounds_checked(void) {
+#ifdef GDN_BOUNDS_CHECK
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 const char* gdn_status_string(gdn_status_t s) {
     switch (s) {
         case GDN_OK: return "GDN_OK";
@@ -340,6 +348,8 @@ gdn_status_t gdn_check_device_error(gdn_stream_t stream) {
         if (word & gdn::kErrTimeout) return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (word 0x%x)", word);
         if (word & gdn::kErrSeqlens) return fail(GDN_ERR_INVALID_ARG, "cu_seqlens out of order or range (word 0x%x)", word);
         if (word & gdn::kErrSlot) return fail(GDN_ERR_INVALID_ARG, "state_slot out of range (word 0x%x)", word);
+        if (word & gdn::kErrBounds)
+            return fail(GDN_ERR_INVALID_ARG, "a device-side bounds check failed: an index outside its tensor (word 0x%x)", word);
         return fail(GDN_ERR_CUDA, "device error word 0x%x", word);
     }
     g_msg[0] = 0;

@@ -312,7 +312,7 @@ inproj_prep_kernel(const __grid_constant__ InprojMaps maps, const InprojArgs a) 
                 for (int k = 0; k < 8; ++k) {
                     const int rr = quad * 32 + 4 * k + (lane >> 3), tt = tok0 + rr;
                     const uint4 u = *reinterpret_cast<const uint4*>(X + rr * Cf::XLD + 4 * (lane & 7));
-                    if (rr >= Cf::HALO && tt < row_end)
+                    if (rr >= Cf::HALO && tt < row_end && in_bounds(tt, a.N))
                         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(base) +
                                                   ((size_t)tt * HD + (size_t)local * Cf::BN + col0 + 8 * (lane & 7)) * 2) = u;
                 }

@@ -59,6 +59,8 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 
         if (tid == 0) raise_error(kErrSlot);
         return;
     }
+    // (bounds-checking build) the slot's state block lies inside the state tensor
+    if (!in_bounds(((long long)s * H + h + 1) * DK * DV - 1, (long long)a.num_slots * H * DK * DV)) return;
     float* S = a.state + ((size_t)s * H + h) * DK * DV;
 
     // the state loads first: they are the traffic that matters
@@ -78,6 +80,10 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 
     const int W = a.W, HW = W - 1;
     const size_t hist_stride = (size_t)H * CH;  // elements between history entries of a slot
     const size_t hist0 = (size_t)s * HW * hist_stride + (size_t)h * CH;
+    // (bounds-checking build) the slot's conv history lies inside its tensor; uniform over the CTA
+    if (HW > 0 && !in_bounds((long long)hist0 + (long long)(HW - 1) * hist_stride + CH - 1,
+                             (long long)a.num_slots * HW * hist_stride))
+        return;
     float xw[CPT][HMAX], taps[CPT][HMAX];       // history oldest first, and its taps
     float xcur[CPT], tcur[CPT];                 // the current input and tap W-1
     float bl = 0.f, al = 0.f, Ah = 0.f, bh_ = 0.f;

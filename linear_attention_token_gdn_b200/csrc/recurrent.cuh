@@ -79,6 +79,8 @@ recurrent_fwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
 
     for (int tb = t0; tb < t1; tb += Sh::TILE) {
         const int nt = min(Sh::TILE, t1 - tb);
+        // (bounds-checking build) the tile's tokens lie inside [0, N); uniform over the CTA
+        if (!in_bounds(tb, N) || !in_bounds(tb + nt - 1, N)) break;
         __syncthreads();
         for (int idx = tid; idx < nt * DK; idx += Sh::THREADS) {
             const int tt = idx / DK, i = idx % DK;

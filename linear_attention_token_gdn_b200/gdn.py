@@ -8,6 +8,7 @@ compute calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -15,6 +16,7 @@ import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgdn.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libgdn_debug.so")  # the bounds-checking build
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = range(5)
 F32, BF16, F16 = 0, 1, 2
@@ -30,6 +32,7 @@ SIGNATURES = {
     "gdn_set_wait_budget": ([_U64], None),
     "gdn_prep": ([_P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I,
                   _P, _P, _P, _P, _P, _P], _I),
+    "gdn_bounds_checked": ([], _I),
     "gdn_inproj_prep": ([_P, _P, _I, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _P, _P, _P, _P,
                          _P, _P, _P], _I),
     "gdn_chunk_fwd_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
@@ -63,19 +66,37 @@ class GDNError(RuntimeError):
         self.status = status
 
 
+def load(path):
+    """ctypes.CDLL of a built libgdn with every declared signature bound.  Raises if it is missing."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: run `python -m linear_attention_token_gdn_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
 def lib():
     """The loaded libgdn.so (ctypes.CDLL with argtypes set).  Raises if it was never built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m linear_attention_token_gdn_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        for name, (args, res) in SIGNATURES.items():
-            fn = getattr(L, name)
-            fn.argtypes = args
-            fn.restype = res
-        _lib = L
+        _lib = load(LIB_PATH)
     return _lib
+
+
+@contextlib.contextmanager
+def using(L):
+    """Route this module's calls through another loaded build (e.g. load(DEBUG_LIB_PATH), the
+    bounds-checking one) inside the block."""
+    global _lib
+    prev = lib()
+    _lib = L
+    try:
+        yield L
+    finally:
+        _lib = prev
 
 
 def status_string(s: int) -> str:

@@ -247,3 +247,12 @@ def test_inproj_prep_rejects_bad_arguments(L, over, status):
 def test_inproj_prep_with_no_tokens_is_a_no_op(L):
     assert L.gdn_inproj_prep(None, None, 256, None, None, None, 4, None, None, None, 1, 0, 16, 128, 128, 1e-6, 1, 1,
                              None, None, None, None, None, None, None) == gdn.GDN_OK
+
+
+def test_bounds_checking_build_exports_every_symbol_and_says_so(L):
+    gbuild.build(debug=True)
+    D = gdn.load(gdn.DEBUG_LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(D, n), n
+    assert D.gdn_bounds_checked() == 1 and L.gdn_bounds_checked() == 0
+    assert D.gdn_version() == L.gdn_version()
