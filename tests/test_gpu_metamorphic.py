@@ -6,7 +6,9 @@ section 2.1.1) fixes that they agree:
 * splitting a sequence and passing S_T of the first part as S0 of the second equals one call
   (the state after a prefix is all the recurrence carries);
 * packing sequences with cu_seqlens equals one call per sequence (sequences never interact);
-* T decode steps equal one prefill over the same T tokens.
+* T decode steps equal one prefill over the same T tokens;
+* permuting the heads permutes every output (heads never interact);
+* the chunkwise form (chunk = 64) equals the token-sequential recurrence (chunk = 0).
 """
 import numpy as np
 import pytest
@@ -111,3 +113,35 @@ def test_decode_steps_equal_one_prefill():
     y_ref, S_ref = oracle.recurrence(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], num_seqs=B)
     assert excess_rel_err(ys.cpu().numpy(), y_ref, 0.0) < 1e-4
     assert excess_rel_err(state.cpu().numpy(), S_ref, 0.0) < 1e-4
+
+
+@pytest.mark.parametrize("chunk", [64, 0])
+def test_permuting_heads_permutes_outputs(chunk):
+    """Heads are independent recurrences: a permutation of the heads of q, k, v, g, beta and S0
+    gives the same permutation of y and S_T, bit for bit (each head's arithmetic is unchanged)."""
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=17, lengths=[300, 77], H=8)
+    perm = torch.tensor([5, 2, 7, 0, 3, 6, 1, 4], device="cuda")
+    S0 = torch.randn(2, 8, 128, 128, device="cuda") * 0.02
+    y, S_T = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], S0, x["cu_seqlens"], chunk=chunk,
+                           y_dtype=torch.float32)
+    px = {n: x[n][:, perm].contiguous() for n in ("q", "k", "v", "g", "beta")}
+    yp, S_Tp = gdn.chunk_fwd(px["q"], px["k"], px["v"], px["g"], px["beta"], S0[:, perm].contiguous(),
+                             x["cu_seqlens"], chunk=chunk, y_dtype=torch.float32)
+    gdn.check_device_error()
+    assert torch.equal(yp, y[:, perm]) and torch.equal(S_Tp, S_T[:, perm])
+
+
+def test_chunkwise_form_equals_token_sequential():
+    """gdn_chunk_fwd with chunk = 64 (the tensor-core UT form derived from eq. (5)) against chunk = 0
+    (eqs. (1)-(4) token by token in fp32) on the same bf16 inputs, ragged sequences and S0 != 0:
+    the tensor-core bound on y and S_T."""
+    x = inputs.make_prefill(inputs.LONG_PREFILL, "cuda", seed=23, lengths=[1, 200, 0, 777], H=4)
+    S0 = torch.randn(4, 4, 128, 128, device="cuda") * 0.02
+    y64, S64 = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], S0, x["cu_seqlens"], chunk=64,
+                             y_dtype=torch.float32)
+    y0, S0_ = gdn.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], S0, x["cu_seqlens"], chunk=0,
+                            y_dtype=torch.float32)
+    gdn.check_device_error()
+    ey, es = rel(y64, y0), rel(S64, S0_)
+    print(f"chunk 64 vs chunk 0: y {ey:.2e}, S_T {es:.2e}")
+    assert ey < TOL_16 and es < TOL_16

@@ -177,6 +177,18 @@ def test_contraction_bound_unit_keys():
 
 # -------------------------------------------------------- hand-worked case
 
+def test_permuting_heads_permutes_outputs():
+    """Heads never interact (each runs its own recurrence): permuting the heads of every input
+    permutes y and S_T exactly."""
+    rng = np.random.default_rng(61)
+    q, k, v, g, beta, S0 = rand_inputs(rng, 13, 4, 5, 3, nseq=2)
+    cu = np.array([0, 6, 13])
+    perm = np.array([2, 0, 3, 1])
+    y, S_T = oracle.recurrence(q, k, v, g, beta, S0, cu)
+    yp, S_Tp = oracle.recurrence(q[:, perm], k[:, perm], v[:, perm], g[:, perm], beta[:, perm], S0[:, perm], cu)
+    assert np.array_equal(yp, y[:, perm]) and np.array_equal(S_Tp, S_T[:, perm])
+
+
 def test_hand_worked_two_token_example():
     rows, S_rows = [], []
     with open(os.path.join(GOLDEN, "hand_worked_two_tokens.txt")) as f:
