@@ -108,9 +108,15 @@ template <int DK, int DV>
 struct MixerDecodeLaunch {
     static gdn_status_t run(const gdn::MixerDecodeArgs& args, int B, cudaStream_t st) {
         using Sh = gdn::DecodeShape<DK, DV>;
+        constexpr int bytes = DK * DV * 4;  // the state block, staged in shared memory
+        cudaError_t e = args.W <= 4 ? cudaFuncSetAttribute(gdn::mixer_decode_kernel<DK, DV, 4>,
+                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)
+                                    : cudaFuncSetAttribute(gdn::mixer_decode_kernel<DK, DV, 8>,
+                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "mixer_decode_kernel smem: %s", cudaGetErrorString(e));
         gdn::LaunchScope timed(st, "mixer_decode_kernel");
-        if (args.W <= 4) gdn::mixer_decode_kernel<DK, DV, 4><<<(unsigned)(B * args.H), Sh::THREADS, 0, st>>>(args);
-        else gdn::mixer_decode_kernel<DK, DV, 8><<<(unsigned)(B * args.H), Sh::THREADS, 0, st>>>(args);
+        if (args.W <= 4) gdn::mixer_decode_kernel<DK, DV, 4><<<(unsigned)(B * args.H), Sh::THREADS, bytes, st>>>(args);
+        else gdn::mixer_decode_kernel<DK, DV, 8><<<(unsigned)(B * args.H), Sh::THREADS, bytes, st>>>(args);
         return launched("mixer_decode_kernel");
     }
 };
@@ -396,7 +402,8 @@ gdn_status_t gdn_mixer_decode_step(const void* x_q, const void* x_k, const void*
     OPT_PTR(state_slot, "state_slot");
     const gdn::MixerDecodeArgs args{x_q, x_k, x_v, conv_w_q, conv_w_k, conv_w_v, conv_width, beta_logit,
                                     alpha_logit, A_log, alpha_bias, z, norm_w, l2_eps, rms_eps, conv_state,
-                                    state, state_slot, num_slots, H, scale, (int)in_dtype, (int)out_dtype, out};
+                                    state, state_slot, num_slots, H, scale, (int)in_dtype, (int)out_dtype, out,
+                                    wait_budget()};
     return dispatch_dims<MixerDecodeLaunch>(dk, dv, args, B, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -8,13 +8,16 @@
 // place, the current input appended.  Nothing between the steps goes to memory: q, k, v stay
 // fp32 in shared memory.
 //
-// One CTA per (row, head), the state read and written once with 128-bit streaming accesses
-// (as in decode_step_kernel): the state loads are issued before the prep arithmetic, so the
-// prep work hides under them.  HBM-bound: dk x dv x 8 bytes of state per (row, head), plus
+// One CTA per (row, head).  Thread 0 brings the slot's whole state block into shared memory with
+// one bulk copy before the prep arithmetic starts, so the prep work hides under it; the updated
+// state is written back with 128-bit streaming stores.  Holding the state in shared memory rather
+// than registers lets three CTAs share an SM, so that one CTA's prep and reductions overlap the
+// others' state traffic.  HBM-bound: dk x dv x 8 bytes of state per (row, head), plus
 // 2 (W-1) (2 dk + dv) bytes of conv history and the token's inputs and output.
 #pragma once
 #include "common.cuh"
 #include "decode.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdn {
 
@@ -34,12 +37,13 @@ struct MixerDecodeArgs {
     float scale;
     int in_dt, out_dt;
     void* out;
+    unsigned long long budget;  // clock cycles a wait may take before it is reported
 };
 
 // TAPS: the largest conv width the instantiation takes (4 or 8), so that the window lives in
 // registers with static indices.
 template <int DK, int DV, int TAPS>
-__global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 1)
+__global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 3 : 2)
     mixer_decode_kernel(const MixerDecodeArgs a) {
     using Sh = DecodeShape<DK, DV>;
     constexpr int NT = Sh::THREADS, CH = 2 * DK + DV;  // channels of one head's conv input
@@ -63,12 +67,16 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 
     if (!in_bounds(((long long)s * H + h + 1) * DK * DV - 1, (long long)a.num_slots * H * DK * DV)) return;
     float* S = a.state + ((size_t)s * H + h) * DK * DV;
 
-    // the state loads first: they are the traffic that matters
-    float4 st[Sh::RPT];
-#pragma unroll
-    for (int m = 0; m < Sh::RPT; ++m) {
-        const int i = rg + m * Sh::RG;
-        st[m] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)i * DV) + cq);
+    // the state first: it is the traffic that matters.  One bulk copy of the dk x dv block; the
+    // barrier's initialisation is visible to the other threads after the first __syncthreads below,
+    // before any of them waits on it.
+    extern __shared__ __align__(16) float s_st[];  // [DK][DV]
+    __shared__ __align__(8) uint64_t s_bar;
+    if (tid == 0) {
+        tc::mbar_init(&s_bar, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(&s_bar, DK * DV * 4);
+        tc::bulk_g2s(s_st, S, DK * DV * 4, &s_bar);
     }
 
     // ---- eqs. (6)-(8): ShortConv over [history, current] then SiLU, one channel per thread; the
@@ -163,13 +171,19 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 
 
     // ---- eqs. (1)-(4): a = S^T k and b = S^T q from one sweep, e = v - alpha a,
     //      S <- alpha S + beta k e^T, y = scale (alpha b + beta (k.q) e) ----------------------------
+    if (!tc::mbar_wait_bounded(&s_bar, 0, a.budget)) {  // flag it, and let the copy land
+        if (tid == 0) raise_error(kErrTimeout);
+        tc::mbar_wait_bounded(&s_bar, 0, 4000000000ull);
+    }
+    const float4* st = reinterpret_cast<const float4*>(s_st);  // row i, float4 column cq: st[i * CPR + cq]
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
 #pragma unroll
     for (int m = 0; m < Sh::RPT; ++m) {
         const int i = rg + m * Sh::RG;
         const float ki = sk[i], qi = sq[i];
-        pa.x += st[m].x * ki; pa.y += st[m].y * ki; pa.z += st[m].z * ki; pa.w += st[m].w * ki;
-        pb.x += st[m].x * qi; pb.y += st[m].y * qi; pb.z += st[m].z * qi; pb.w += st[m].w * qi;
+        const float4 sv4 = st[i * Sh::CPR + cq];
+        pa.x += sv4.x * ki; pa.y += sv4.y * ki; pa.z += sv4.z * ki; pa.w += sv4.w * ki;
+        pb.x += sv4.x * qi; pb.y += sv4.y * qi; pb.z += sv4.z * qi; pb.w += sv4.w * qi;
     }
     s_red_a[rg][cq] = pa;
     s_red_b[rg][cq] = pb;
@@ -192,11 +206,12 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, TAPS == 4 ? 2 : 
     for (int m = 0; m < Sh::RPT; ++m) {
         const int i = rg + m * Sh::RG;
         const float wk = bt * sk[i];
+        const float4 sv4 = st[i * Sh::CPR + cq];
         float4 o;
-        o.x = alpha * st[m].x + wk * e4.x;
-        o.y = alpha * st[m].y + wk * e4.y;
-        o.z = alpha * st[m].z + wk * e4.z;
-        o.w = alpha * st[m].w + wk * e4.w;
+        o.x = alpha * sv4.x + wk * e4.x;
+        o.y = alpha * sv4.y + wk * e4.y;
+        o.z = alpha * sv4.z + wk * e4.z;
+        o.w = alpha * sv4.w + wk * e4.w;
         __stcs(reinterpret_cast<float4*>(S + (size_t)i * DV) + cq, o);
     }
 
