@@ -7,10 +7,14 @@
 //   e = v - alpha a                      (eq. 2 with S~ = alpha S, eq. 1)
 //   S <- alpha S + beta k e^T            (eq. 3), written back in place
 //   y = scale (alpha b + beta (k.q) e)   (eq. 4: S_t^T q expanded, no second pass)
-// The kernel is HBM-bound (about 0.9 FLOP per byte): one CTA per (row, head), every
-// thread keeps RPT rows x 4 columns of S in registers, 128-bit streaming loads/stores.
+// The kernel is HBM-bound (about 0.9 FLOP per byte): one CTA per (row, head).  Thread 0 brings
+// the state block into shared memory with one bulk copy first; every thread then reads RPT rows
+// x 4 columns of it twice (the two dot products, then the update) and streams the new state out
+// with 128-bit stores.  With the state in shared memory rather than registers, three CTAs share
+// an SM, so one CTA's reductions overlap the others' state traffic.
 #pragma once
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdn {
 
@@ -24,11 +28,11 @@ struct DecodeShape {
 };
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS)
+__global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS, 3)
 decode_step_kernel(const void* __restrict__ q, const void* __restrict__ k, const void* __restrict__ v,
                    const float* __restrict__ g, const float* __restrict__ beta, float* __restrict__ state,
                    const int32_t* __restrict__ slot, int num_slots, int H, float scale, int in_dt,
-                   int y_dt, void* __restrict__ y) {
+                   int y_dt, void* __restrict__ y, unsigned long long budget) {
     using Sh = DecodeShape<DK, DV>;
     const int bh = blockIdx.x;  // row * H + head
     const int b = bh / H, h = bh - b * H;
@@ -51,12 +55,16 @@ decode_step_kernel(const void* __restrict__ q, const void* __restrict__ k, const
         return;
     float* S = state + ((size_t)s * H + h) * DK * DV;
 
-    // Issue the state loads first: they are the only traffic that matters.
-    float4 st[Sh::RPT];
-#pragma unroll
-    for (int m = 0; m < Sh::RPT; ++m) {
-        const int i = rg + m * Sh::RG;
-        st[m] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)i * DV) + cq);
+    // The state first: it is the only traffic that matters.  One bulk copy of the dk x dv block;
+    // the barrier's initialisation is visible to the other threads after the __syncthreads
+    // below, before any of them waits on it.
+    extern __shared__ __align__(16) float s_st[];  // [DK][DV]
+    __shared__ __align__(8) uint64_t s_bar;
+    if (tid == 0) {
+        tc::mbar_init(&s_bar, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(&s_bar, DK * DV * 4);
+        tc::bulk_g2s(s_st, S, DK * DV * 4, &s_bar);
     }
 
     for (int i = tid; i < DK; i += Sh::THREADS) {
@@ -75,13 +83,19 @@ decode_step_kernel(const void* __restrict__ q, const void* __restrict__ k, const
         if (tid == 0) s_kq = p;
     }
 
+    if (!tc::mbar_wait_bounded(&s_bar, 0, budget)) {  // flag it, and let the copy land
+        if (tid == 0) raise_error(kErrTimeout);
+        tc::mbar_wait_bounded(&s_bar, 0, 4000000000ull);
+    }
+    const float4* st = reinterpret_cast<const float4*>(s_st);  // row i, float4 column cq: st[i * CPR + cq]
     float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
 #pragma unroll
     for (int m = 0; m < Sh::RPT; ++m) {
         const int i = rg + m * Sh::RG;
         const float ki = s_k[i], qi = s_q[i];
-        pa.x += st[m].x * ki; pa.y += st[m].y * ki; pa.z += st[m].z * ki; pa.w += st[m].w * ki;
-        pb.x += st[m].x * qi; pb.y += st[m].y * qi; pb.z += st[m].z * qi; pb.w += st[m].w * qi;
+        const float4 sv4 = st[i * Sh::CPR + cq];
+        pa.x += sv4.x * ki; pa.y += sv4.y * ki; pa.z += sv4.z * ki; pa.w += sv4.w * ki;
+        pb.x += sv4.x * qi; pb.y += sv4.y * qi; pb.z += sv4.z * qi; pb.w += sv4.w * qi;
     }
     s_red_a[rg][cq] = pa;
     s_red_b[rg][cq] = pb;
@@ -106,11 +120,12 @@ decode_step_kernel(const void* __restrict__ q, const void* __restrict__ k, const
     for (int m = 0; m < Sh::RPT; ++m) {
         const int i = rg + m * Sh::RG;
         const float w = bt * s_k[i];
+        const float4 sv4 = st[i * Sh::CPR + cq];
         float4 o;
-        o.x = alpha * st[m].x + w * e4.x;
-        o.y = alpha * st[m].y + w * e4.y;
-        o.z = alpha * st[m].z + w * e4.z;
-        o.w = alpha * st[m].w + w * e4.w;
+        o.x = alpha * sv4.x + w * e4.x;
+        o.y = alpha * sv4.y + w * e4.y;
+        o.z = alpha * sv4.z + w * e4.z;
+        o.w = alpha * sv4.w + w * e4.w;
         __stcs(reinterpret_cast<float4*>(S + (size_t)i * DV) + cq, o);
     }
 }

@@ -97,9 +97,13 @@ struct DecodeLaunch {
                             float* state, const int32_t* slot, int num_slots, int B, int H, float scale,
                             int in_dt, int y_dt, void* y, cudaStream_t st) {
         using Sh = gdn::DecodeShape<DK, DV>;
+        constexpr int bytes = DK * DV * 4;  // the state block, staged in shared memory
+        cudaError_t e = cudaFuncSetAttribute(gdn::decode_step_kernel<DK, DV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "decode_step_kernel smem: %s", cudaGetErrorString(e));
         gdn::LaunchScope timed(st, "decode_step_kernel");
-        gdn::decode_step_kernel<DK, DV><<<(unsigned)(B * H), Sh::THREADS, 0, st>>>(
-            q, k, v, g, beta, state, slot, num_slots, H, scale, in_dt, y_dt, y);
+        gdn::decode_step_kernel<DK, DV><<<(unsigned)(B * H), Sh::THREADS, bytes, st>>>(
+            q, k, v, g, beta, state, slot, num_slots, H, scale, in_dt, y_dt, y, wait_budget());
         return launched("decode_step_kernel");
     }
 };
