@@ -31,10 +31,14 @@ struct BwdShape {
     // 4 (mod 32) words those land in 32 distinct banks; the readers rotate their start column by
     // lane so that a warp's 32 rows also read 32 distinct banks
     static constexpr int PAD = SLAB + 4;
-    // shared memory: the block's states, the block's token inputs, two transposes, column sums
+    // tokens walked between two reductions: each has its own transposes and column sums, so that
+    // one pair of barriers serves them all
+    static constexpr int NP = 2;
+    // shared memory: the block's states, the block's token inputs, NP x (two transposes, column sums)
     static constexpr int ST_FLOATS = kBwdBlk * DK * SLAB;
     static constexpr int TOK_FLOATS = kBwdBlk * (2 * DK + 2 * SLAB + 2);
-    static constexpr int RED_FLOATS = 2 * DK * PAD + 2 * SLAB;
+    static constexpr int RED_ONE = 2 * DK * PAD + 2 * SLAB;
+    static constexpr int RED_FLOATS = NP * RED_ONE;
     static constexpr int BYTES = 4 * (ST_FLOATS + TOK_FLOATS + RED_FLOATS);
 };
 
@@ -57,10 +61,9 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
     float* sdy = sv + B * SLAB;                          // [B][SLAB]
     float* sa = sdy + B * SLAB;                          // [B] alpha
     float* sb = sa + B;                                  // [B] beta
-    float* p_q = sb + B;                                 // [DK][PAD] the slab's terms of dq
-    float* p_k = p_q + DK * Sh::PAD;                     // [DK][PAD] the slab's terms of dk
-    float* c_b = p_k + DK * Sh::PAD;                     // [SLAB] the columns' terms of dbeta
-    float* c_g = c_b + SLAB;                             // [SLAB] the columns' terms of dg / alpha
+    // NP slots of: [DK][PAD] the slab's terms of dq, [DK][PAD] of dk, [SLAB] the columns' terms of
+    // dbeta, [SLAB] of dg / alpha
+    float* p_q0 = sb + B;
     __shared__ int s_bbase;
 
     const int slab = blockIdx.x % NSLAB;
@@ -126,76 +129,91 @@ recurrent_bwd_kernel(const void* __restrict__ q, const void* __restrict__ k, con
                 for (int m = 0; m < RPT; ++m) S[m] = sa[i] * S[m] + sb[i] * sk[i * DK + r + m * RS] * e;
             }
         }
-        for (int i = nt - 1; i >= 0; --i) {
-            const int t = tb + i;
-            const float alpha = sa[i], bt = sb[i], dyj = sdy[i * SLAB + jl];
-            float kk[RPT], qq[RPT];  // this thread's rows of k_t and q_t
+        // tokens i, i - 1, ... (NP of them) are walked back to back, each into its own transposes;
+        // one barrier, then their column sums, then a barrier before the next group overwrites them
+        for (int i0 = nt - 1; i0 >= 0; i0 -= Sh::NP) {
+            const int np = min(Sh::NP, i0 + 1);
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) {
-                kk[m] = sk[i * DK + r + m * RS];
-                qq[m] = sq[i * DK + r + m * RS];
-            }
-            float Sp[RPT], a = 0.f;
+            for (int sl = 0; sl < Sh::NP; ++sl) {
+                if (sl >= np) break;  // uniform
+                const int i = i0 - sl, t = tb + i;
+                float* p_q = p_q0 + sl * Sh::RED_ONE;
+                float* p_k = p_q + DK * Sh::PAD;
+                float* c_b = p_k + DK * Sh::PAD;
+                float* c_g = c_b + SLAB;
+                const float alpha = sa[i], bt = sb[i], dyj = sdy[i * SLAB + jl];
+                float kk[RPT], qq[RPT];  // this thread's rows of k_t and q_t
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) {
-                Sp[m] = st[(i * RPT + m) * NT + tid];
-                a += Sp[m] * kk[m];
-            }
+                for (int m = 0; m < RPT; ++m) {
+                    kk[m] = sk[i * DK + r + m * RS];
+                    qq[m] = sq[i * DK + r + m * RS];
+                }
+                float Sp[RPT], a = 0.f;
 #pragma unroll
-            for (int o = 1; o < RS; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            const float e = sv[i * SLAB + jl] - alpha * a;
-            float kd = 0.f;
+                for (int m = 0; m < RPT; ++m) {
+                    Sp[m] = st[(i * RPT + m) * NT + tid];
+                    a += Sp[m] * kk[m];
+                }
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) {
-                const int row = r + m * RS;
-                const float St = alpha * Sp[m] + bt * kk[m] * e;      // S_t
-                D[m] += scale * qq[m] * dyj;                            // readout
-                p_q[row * Sh::PAD + jl] = scale * St * dyj;             // dq = scale S_t dy
-                kd += kk[m] * D[m];
-            }
+                for (int o = 1; o < RS; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                const float e = sv[i * SLAB + jl] - alpha * a;
+                float kd = 0.f;
 #pragma unroll
-            for (int o = 1; o < RS; o <<= 1) kd += __shfl_xor_sync(0xffffffffu, kd, o);
-            const float de = bt * kd;                                   // de = beta D^T k
-            float da = 0.f;
+                for (int m = 0; m < RPT; ++m) {
+                    const int row = r + m * RS;
+                    const float St = alpha * Sp[m] + bt * kk[m] * e;      // S_t
+                    D[m] += scale * qq[m] * dyj;                            // readout
+                    p_q[row * Sh::PAD + jl] = scale * St * dyj;             // dq = scale S_t dy
+                    kd += kk[m] * D[m];
+                }
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) {
-                const int row = r + m * RS;
-                p_k[row * Sh::PAD + jl] = bt * D[m] * e - alpha * Sp[m] * de;  // dk = beta D e - S~ de
-                D[m] -= kk[m] * de;                                     // D~
-                da += D[m] * Sp[m];
-                D[m] *= alpha;                                          // dL/dS_{t-1}
-            }
+                for (int o = 1; o < RS; o <<= 1) kd += __shfl_xor_sync(0xffffffffu, kd, o);
+                const float de = bt * kd;                                   // de = beta D^T k
+                float da = 0.f;
 #pragma unroll
-            for (int o = 1; o < RS; o <<= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
-            if (r == 0) {
-                dv[((size_t)t * H + h) * DV + j] = de;
-                c_b[jl] = kd * e;                                       // dbeta = k^T D e
-                c_g[jl] = da;
+                for (int m = 0; m < RPT; ++m) {
+                    const int row = r + m * RS;
+                    p_k[row * Sh::PAD + jl] = bt * D[m] * e - alpha * Sp[m] * de;  // dk = beta D e - S~ de
+                    D[m] -= kk[m] * de;                                     // D~
+                    da += D[m] * Sp[m];
+                    D[m] *= alpha;                                          // dL/dS_{t-1}
+                }
+#pragma unroll
+                for (int o = 1; o < RS; o <<= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
+                if (r == 0) {
+                    dv[((size_t)t * H + h) * DV + j] = de;
+                    c_b[jl] = kd * e;                                       // dbeta = k^T D e
+                    c_g[jl] = da;
+                }
             }
             __syncthreads();
-            // the slab's column terms: a row of dq or dk per thread (four partial sums), dbeta and
-            // dg by one warp
-            for (int e = tid; e < 2 * DK; e += NT) {
-                const int row = e < DK ? e : e - DK;
-                const float* pr = (e < DK ? p_q : p_k) + row * Sh::PAD;
+            // the slab's column terms: a row of dq or dk of one token per thread (four partial
+            // sums), and dbeta, dg of each token by one warp
+            for (int e = tid; e < np * 2 * DK; e += NT) {
+                const int sl = e / (2 * DK), re = e - sl * 2 * DK;
+                const int row = re < DK ? re : re - DK, t = tb + i0 - sl;
+                const float* pr = p_q0 + sl * Sh::RED_ONE + (re < DK ? 0 : DK * Sh::PAD) + row * Sh::PAD;
                 float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < SLAB; ++c) s4[c & 3] += pr[(c + tid) & (SLAB - 1)];
-                atomicAdd((e < DK ? dq : dk) + ((size_t)t * H + h) * DK + row, (s4[0] + s4[1]) + (s4[2] + s4[3]));
+                atomicAdd((re < DK ? dq : dk) + ((size_t)t * H + h) * DK + row, (s4[0] + s4[1]) + (s4[2] + s4[3]));
             }
-            if (tid < 32) {
-                float s1 = tid < SLAB ? c_b[tid] : 0.f, s2 = tid < SLAB ? c_g[tid] : 0.f;
+            for (int sl = tid >> 5; sl < np; sl += NT / 32) {  // (warp-uniform; NT is a multiple of 32)
+                const int l = tid & 31, t = tb + i0 - sl;
+                const float* c_b = p_q0 + sl * Sh::RED_ONE + 2 * DK * Sh::PAD;
+                const float* c_g = c_b + SLAB;
+                float s1 = l < SLAB ? c_b[l] : 0.f, s2 = l < SLAB ? c_g[l] : 0.f;
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
                     s1 += __shfl_xor_sync(0xffffffffu, s1, o);
                     s2 += __shfl_xor_sync(0xffffffffu, s2, o);
                 }
-                if (tid == 0) {
+                if (l == 0) {
                     atomicAdd(dbeta + (size_t)t * H + h, s1);
-                    atomicAdd(dg + (size_t)t * H + h, alpha * s2);
+                    atomicAdd(dg + (size_t)t * H + h, sa[i0 - sl] * s2);
                 }
             }
-            __syncthreads();  // the transposes are read before the next token writes them
+            __syncthreads();  // the transposes are read before the next group writes them
         }
     }
 #pragma unroll
