@@ -89,7 +89,8 @@ def lib():
 @contextlib.contextmanager
 def using(L):
     """Route this module's calls through another loaded build (e.g. load(DEBUG_LIB_PATH), the
-    bounds-checking one) inside the block."""
+    bounds-checking one) inside the block.  The module-level handle is swapped, so the switch
+    applies to every thread of the process while the block runs."""
     global _lib
     prev = lib()
     _lib = L
