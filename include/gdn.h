@@ -167,12 +167,14 @@ gdn_status_t gdn_inproj_prep(const void* x, const void* w, int D, const float* c
  * chunk selects the algorithm:
  *   chunk = 0: token-sequential fp32 recurrence on CUDA cores (any supported
  *              shape and dtype; exact up to fp32 rounding order).
- *   chunk = 64: chunkwise-parallel form on the tcgen05 tensor cores
+ *   chunk = 64: chunkwise-parallel form on the tensor cores
  *              (requires dk = dv = 128 and in_dtype BF16 or F16; other shapes and
  *              chunk sizes return GDN_ERR_UNSUPPORTED).  It is derived
  *              from eq. (5): within a chunk, the UT transform T = (I + A)^-1 with
  *              A[r,s] = beta_r exp(gamma_r - gamma_s) k_r.k_s turns the token loop
- *              into dense products; between chunks the state is carried in fp32.
+ *              into dense products (one kernel per (chunk, head), warp-level mma);
+ *              between chunks a second kernel carries the fp32 state through tcgen05
+ *              products with TMEM accumulators.
  * workspace: device scratch of at least gdn_chunk_fwd_workspace_size(...) bytes
  * (may be NULL when that size is 0).  Tokens at index >= cu_seqlens[num_seqs] are
  * neither read nor written.  N = 0 (every sequence empty): nothing is done without S_T;
