@@ -124,6 +124,15 @@ def timed(torch, fn, steps, warmup, stream, on_start=None):
     return e0.elapsed_time(e1) / 1e3  # seconds
 
 
+def kernel_split(torch, gdn, fn, steps, stream, max_launches=64):
+    """Per-kernel device times from a separate pass with the library's launch timing on.  Its
+    events bracket every launch, which cancels the programmatic dependent launch between the
+    chunked pass's two kernels, so the reported times come from un-instrumented passes and this
+    table only splits a call into its kernels."""
+    timed(torch, fn, steps, 0, stream, on_start=lambda: gdn.timing_start(max_launches))
+    return kernel_table(gdn.timing_stop(), steps)
+
+
 def kernel_table(per_kernel, steps):
     """{name: (launches, total ms)} from gdn.timing_stop -> per-kernel averages and shares."""
     tot = sum(ms for _, ms in per_kernel.values()) or 1.0
@@ -290,9 +299,8 @@ def run_ours(args):
 
     barrier(torch, dist, world)
     with ClockSampler(torch.cuda.current_device()) as clk:
-        # every launch inside the timed region is bracketed by CUDA events on its stream
-        dt = timed(torch, step, args.steps, args.warmup, stream, on_start=lambda: gdn.timing_start(4 * args.steps + 8))
-        per_kernel = gdn.timing_stop()
+        # the timed region runs the calls back to back, as a caller would (no launch events)
+        dt = timed(torch, step, args.steps, args.warmup, stream)
         barrier(torch, dist, world)
         if dt < 0.5:  # keep the GPU busy long enough for the clock sampler to see it
             soak = timed(torch, step, max(1, int(args.steps * 0.6 / max(dt, 1e-6))), 0, stream)
@@ -302,9 +310,11 @@ def run_ours(args):
     work = N * H  # token-heads per rank per step
     value = aggregate(work, world, per_step)
     alg_bytes = prefill_bytes(N, H, nseq)
-    kern = kernel_table(per_kernel, args.steps)
-    op_s = sum(k["avg_us"] for k in kern) / 1e6  # device time of one gdn_chunk_fwd call
-    achieved = alg_bytes / op_s / 1e9
+    # the per-kernel split (and the launch count per call) from a separate instrumented pass
+    n_split = min(args.steps, 20)
+    kern = kernel_split(torch, gdn, step, n_split, stream, 4 * n_split + 8)
+    launches_per_call = sum(k["launches"] for k in kern) / n_split
+    achieved = alg_bytes / per_step / 1e9  # one gdn_chunk_fwd call per step, timed over the region
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -316,8 +326,12 @@ def run_ours(args):
                          "frac": achieved / hbm_peak, "traffic": traffic_per_call(), "kernel":
                          "gdn_chunk_fwd = chunk_ut_kernel + chunk_chain_kernel (per call)",
                          "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": alg_bytes,
-                         "kernels": kern},
-            "gpu_launches": sum(k["launches"] for k in kern), "clocks": clk.summary()}
+                         "achieved_from": "the call's device time over the timed region (CUDA events, no "
+                                          "launch instrumentation)",
+                         "kernels": kern,
+                         "kernels_note": "per-kernel split from a separate pass with launch events, which "
+                                         "serialise the two kernels (no programmatic overlap there)"},
+            "gpu_launches": int(round(launches_per_call * args.steps)), "clocks": clk.summary()}
 
     # ---- end to end through the public API with pinned host buffers ----------------------
     # Each sequence is split into P segments of T/P tokens chained through S_T -> S0 (identical to
@@ -455,17 +469,16 @@ def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
     barrier(torch, dist, world)
     n_lp = 3
-    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 1, stream, on_start=lambda: gdn.timing_start(64)),
-                        world) / n_lp
-    kl = kernel_table(gdn.timing_stop(), n_lp)
-    op_s = sum(k["avg_us"] for k in kl) / 1e6
+    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 1, stream), world) / n_lp
+    kl = kernel_split(torch, gdn, lp, n_lp, stream)
     bl = prefill_bytes(N, H, nseq, S0=True)
     return {"workload": inputs.WORKLOAD_SPECS[inputs.LONG_PREFILL]["name"], "value": N * H * world / dt, "unit": UNIT,
                 "ms_per_step": dt * 1e3,
-                "roofline": {"bound": "hbm", "achieved": bl / op_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
-                             "frac": bl / op_s / 1e9 / hbm_peak,
+                "roofline": {"bound": "hbm", "achieved": bl / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                             "frac": bl / dt / 1e9 / hbm_peak,
                              "kernel": "gdn_chunk_fwd = chunk_ut_kernel + chunk_chain_kernel (per call)",
-                             "alg_bytes_per_launch": bl, "kernels": kl},
+                             "alg_bytes_per_launch": bl, "kernels": kl,
+                             "kernels_note": "per-kernel split from a separate instrumented pass"},
                 "gpu_launches": sum(k["launches"] for k in kl), "l2": "1.1 GB working set > L2"}
 
 
@@ -509,12 +522,10 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
     barrier(torch, dist, world)
     n_m = 5
     dt_fused = max_over_ranks(torch, dist, timed(torch, mix_fused, n_m, 1, stream), world) / n_m
-    dt_prep = max_over_ranks(torch, dist, timed(torch, mix_prep_fused, n_m, 1, stream,
-                                                 on_start=lambda: gdn.timing_start(64)), world) / n_m
-    kp = kernel_table(gdn.timing_stop(), n_m)
-    dt = max_over_ranks(torch, dist, timed(torch, mix, n_m, 1, stream, on_start=lambda: gdn.timing_start(64)),
-                        world) / n_m
-    km = kernel_table(gdn.timing_stop(), n_m)
+    dt_prep = max_over_ranks(torch, dist, timed(torch, mix_prep_fused, n_m, 1, stream), world) / n_m
+    kp = kernel_split(torch, gdn, mix_prep_fused, n_m, stream)
+    dt = max_over_ranks(torch, dist, timed(torch, mix, n_m, 1, stream), world) / n_m
+    km = kernel_split(torch, gdn, mix, n_m, stream)
     fused_min = N * (H * 3 * 128 * 2 + H * 2 * 2 + H * 128 * 2 + H * 128 * 2)
     return {"workload": inputs.WORKLOAD_SPECS[inputs.MIXER]["name"], "lengths": m["lengths"], "value": N * H * world / dt,
                 "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
@@ -523,7 +534,8 @@ def wl_mixer(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
                 "roofline": {"bound": "hbm", "achieved": fused_min / dt / 1e9, "peak": hbm_peak, "unit": "GB/s",
                              "frac": fused_min / dt / 1e9 / hbm_peak, "kernel": "prep+chunk+out_gate",
                              "alg_bytes_per_step": fused_min,
-                             "note": "bytes = fused minimum (read projections, logits, z; write out)",
+                             "note": "bytes = fused minimum (read projections, logits, z; write out); per-kernel "
+                                     "split from a separate instrumented pass",
                              "kernels": km},
                 "gpu_launches": sum(k["launches"] for k in km)}
 
