@@ -468,8 +468,8 @@ def wl_long(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
                       workspace=ws)
 
     barrier(torch, dist, world)
-    n_lp = 3
-    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 1, stream), world) / n_lp
+    n_lp = 5
+    dt = max_over_ranks(torch, dist, timed(torch, lp, n_lp, 2, stream), world) / n_lp
     kl = kernel_split(torch, gdn, lp, n_lp, stream)
     bl = prefill_bytes(N, H, nseq, S0=True)
     return {"workload": inputs.WORKLOAD_SPECS[inputs.LONG_PREFILL]["name"], "value": N * H * world / dt, "unit": UNIT,
