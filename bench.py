@@ -611,9 +611,8 @@ def wl_backward(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
     barrier(torch, dist, world)
     n_b = 3
-    dt = max_over_ranks(torch, dist, timed(torch, bwd, n_b, 1, stream, on_start=lambda: gdn.timing_start(64)),
-                        world) / n_b
-    kb = kernel_table(gdn.timing_stop(), n_b)
+    dt = max_over_ranks(torch, dist, timed(torch, bwd, n_b, 1, stream), world) / n_b
+    kb = kernel_split(torch, gdn, bwd, n_b, stream)
     # read q, k, v, dy (bf16), g, beta; write dq, dk, dv (fp32), dg, dbeta; dS_T in, dS0 out
     alg = N * H * (3 * 128 * 2 + 128 * 2 + 8 + 3 * 128 * 4 + 8) + 2 * nseq * H * 128 * 128 * 4
     return {"workload": "backward_prefill_B2_H16_T4096_d128", "value": N * H * world / dt, "unit": UNIT,
@@ -661,14 +660,13 @@ def wl_inproj(torch, dist, gdn, inputs, args, rank, world, stream, hbm_peak):
 
     barrier(torch, dist, world)
     n_i = 10
-    dt = max_over_ranks(torch, dist, timed(torch, fused, n_i, 3, stream, on_start=lambda: gdn.timing_start(64)),
-                        world) / n_i
-    ki = kernel_table(gdn.timing_stop(), n_i)
+    dt = max_over_ranks(torch, dist, timed(torch, fused, n_i, 3, stream), world) / n_i
+    ki = kernel_split(torch, gdn, fused, n_i, stream)
     dt_gemm = max_over_ranks(torch, dist, timed(torch, gemm_only, n_i, 3, stream), world) / n_i
     dt_unf = max_over_ranks(torch, dist, timed(torch, unfused, n_i, 3, stream), world) / n_i
     flops = 2.0 * N * D * R
     _, tf_peak, src = peaks()
-    ach = flops / (ki[0]["avg_us"] * 1e-6) / 1e12 if ki else flops / dt / 1e12
+    ach = flops / dt / 1e12  # one launch per step, timed over the region
     return {"workload": inputs.WORKLOAD_SPECS[inputs.INPROJ]["name"], "lengths": m["lengths"],
             "value": N * H * world / dt, "unit": UNIT, "tokens_per_s": N * world / dt, "ms_per_step": dt * 1e3,
             "context_ms_cublas_gemm_same_flops": dt_gemm * 1e3,
